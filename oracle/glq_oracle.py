@@ -1,0 +1,202 @@
+"""ctypes wrapper around the fp64 CPU oracle in ``glq_oracle.c``.
+
+TEST INFRASTRUCTURE ONLY: the test-suite, the package entry point's smoke
+check and the benchmark's CPU-baseline leg are the only callers.  The CUDA
+library never imports this module and this module never imports the CUDA
+library.
+
+Every function here is a thin marshalling layer over the C oracle; the
+arithmetic lives in ``glq_oracle.c`` and follows the GLQ project pages cited
+there (glq 0.5.1 PyPI page: "How it works", "Bit widths", "Inference
+kernels").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "glq_oracle.c")
+_LIB = os.path.join(_HERE, "libglq_oracle.so")
+
+CODEBOOK_ENTRIES = 65536
+
+
+def build(force: bool = False) -> str:
+    """Compiles the oracle into ``libglq_oracle.so`` beside its source."""
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    tmp = _LIB + f".tmp{os.getpid()}"
+    # -ffp-contract=off: no silent a*b+c fusion; the one fused step is the
+    # explicit fmaf() of the residual reconstruction.
+    subprocess.check_call([
+        "gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+        "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build())
+    c_i64, c_int, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
+    lib.glq_oracle_f16_to_double.restype = ctypes.c_double
+    lib.glq_oracle_f16_to_double.argtypes = [ctypes.c_uint16]
+    lib.glq_oracle_bf16_to_double.restype = ctypes.c_double
+    lib.glq_oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
+    lib.glq_oracle_e8_points.restype = c_i64
+    lib.glq_oracle_e8_points.argtypes = [c_int, vp, c_i64]
+    lib.glq_oracle_hadamard_blocks.restype = c_int
+    lib.glq_oracle_hadamard_blocks.argtypes = [c_i64, vp, c_int]
+    lib.glq_oracle_hadamard_matrix.restype = None
+    lib.glq_oracle_hadamard_matrix.argtypes = [c_i64, vp]
+    lib.glq_oracle_hadamard_apply.restype = None
+    lib.glq_oracle_hadamard_apply.argtypes = [c_i64, vp, vp, c_int]
+    lib.glq_oracle_decode_rows.restype = c_int
+    lib.glq_oracle_decode_rows.argtypes = [
+        c_i64, c_i64, c_int, vp, vp, vp, vp, ctypes.c_float, ctypes.c_float,
+        c_i64, c_i64, vp]
+    lib.glq_oracle_linear.restype = c_int
+    lib.glq_oracle_linear.argtypes = [
+        c_i64, c_i64, c_int, vp, vp, vp, vp, ctypes.c_float, ctypes.c_float,
+        vp, vp, vp, c_int, c_i64, vp]
+    _lib = lib
+    return lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def f16_bits_to_double(bits) -> float:
+    return _load().glq_oracle_f16_to_double(int(bits))
+
+
+def bf16_bits_to_double(bits) -> float:
+    return _load().glq_oracle_bf16_to_double(int(bits))
+
+
+def e8_points(max_norm: int = 12, max_entries: int = 200000):
+    """All E8 points of squared norm <= max_norm, sorted by (norm, x0..x7).
+
+    Returns (points[k][8] float64, total) with k = min(total, max_entries).
+    """
+    out = np.zeros((max_entries, 8), dtype=np.float64)
+    total = _load().glq_oracle_e8_points(int(max_norm), _ptr(out), int(max_entries))
+    if total < 0:
+        raise RuntimeError("oracle E8 enumeration failed")
+    return out[:min(total, max_entries)].copy(), int(total)
+
+
+_codebook_cache = None
+
+
+def e8_codebook() -> np.ndarray:
+    """The 65,536 x 8 E8 shell codebook (float64, every value a multiple of 1/2)."""
+    global _codebook_cache
+    if _codebook_cache is None:
+        cb, total = e8_points(12, CODEBOOK_ENTRIES)
+        if total < CODEBOOK_ENTRIES:
+            raise RuntimeError("fewer than 65,536 E8 points of norm <= 12")
+        cb.setflags(write=False)
+        _codebook_cache = cb
+    return _codebook_cache
+
+
+def hadamard_blocks(n: int):
+    sizes = np.zeros(64, dtype=np.int64)
+    nb = _load().glq_oracle_hadamard_blocks(int(n), _ptr(sizes), 64)
+    if nb < 0:
+        raise ValueError(f"bad size {n}")
+    return [int(s) for s in sizes[:nb]]
+
+
+def hadamard_matrix(n: int) -> np.ndarray:
+    H = np.zeros((n, n), dtype=np.float64)
+    _load().glq_oracle_hadamard_matrix(int(n), _ptr(H))
+    return H
+
+
+def hadamard_apply(v, force_dense: bool = False) -> np.ndarray:
+    """H_n v for a 1-D vector (block-diagonal normalised Hadamard)."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.empty_like(v)
+    _load().glq_oracle_hadamard_apply(v.shape[0], _ptr(v), _ptr(out), int(bool(force_dense)))
+    return out
+
+
+def _residual_table(bpw: int, cb2):
+    if bpw == 2:
+        return None
+    if bpw == 4:
+        return e8_codebook() if cb2 is None else np.ascontiguousarray(cb2, dtype=np.float64)
+    if cb2 is None:
+        raise ValueError("bpw 3 needs the 256-entry residual codebook")
+    cb2 = np.asarray(cb2)
+    if cb2.dtype == np.uint16:  # fp16 bits
+        cb2 = f16_table_to_double(cb2)
+    return np.ascontiguousarray(cb2, dtype=np.float64).reshape(256, 8)
+
+
+def f16_table_to_double(bits) -> np.ndarray:
+    """fp16 bit patterns -> float64 through the oracle's own binary16 decoder."""
+    bits = np.asarray(bits, dtype=np.uint16)
+    lib = _load()
+    flat = [lib.glq_oracle_f16_to_double(int(b)) for b in bits.reshape(-1)]
+    return np.array(flat, dtype=np.float64).reshape(bits.shape)
+
+
+def _check_idx(m, n, bpw, idx1, idx2):
+    G = n // 8
+    idx1 = np.ascontiguousarray(idx1, dtype=np.uint16).reshape(m, G)
+    if bpw == 3:
+        idx2 = np.ascontiguousarray(idx2, dtype=np.uint8).reshape(m, G)
+    elif bpw == 4:
+        idx2 = np.ascontiguousarray(idx2, dtype=np.uint16).reshape(m, G)
+    else:
+        idx2 = None
+    return idx1, idx2
+
+
+def decode_rows(m, n, bpw, idx1, idx2, ws, rs, r0=0, r1=None, cb2=None) -> np.ndarray:
+    """Explicit W^ rows [r0, r1) as float64 arrays holding fp32 values."""
+    r1 = m if r1 is None else r1
+    idx1, idx2 = _check_idx(m, n, bpw, idx1, idx2)
+    cb1 = e8_codebook()
+    cb2 = _residual_table(bpw, cb2)
+    w = np.zeros((r1 - r0, n), dtype=np.float64)
+    rc = _load().glq_oracle_decode_rows(m, n, bpw, _ptr(idx1), _ptr(idx2), _ptr(cb1),
+                                        _ptr(cb2), float(ws), float(rs), r0, r1, _ptr(w))
+    if rc != 0:
+        raise ValueError("oracle decode rejected its arguments")
+    return w
+
+
+def linear(m, n, bpw, idx1, idx2, ws, rs, s_in, s_out, x_bits, x_is_bf16, cb2=None) -> np.ndarray:
+    """y[B][m] (float64) = S_out . H_m . W^ . H_n . (S_in . x).
+
+    x_bits: uint16 [B][n] holding fp16 (x_is_bf16 False) or bf16 bit patterns.
+    """
+    idx1, idx2 = _check_idx(m, n, bpw, idx1, idx2)
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16).reshape(-1, n)
+    B = x_bits.shape[0]
+    s_in = np.ascontiguousarray(s_in, dtype=np.int8)
+    s_out = np.ascontiguousarray(s_out, dtype=np.int8)
+    cb1 = e8_codebook()
+    cb2 = _residual_table(bpw, cb2)
+    y = np.zeros((B, m), dtype=np.float64)
+    rc = _load().glq_oracle_linear(m, n, bpw, _ptr(idx1), _ptr(idx2), _ptr(cb1), _ptr(cb2),
+                                   float(ws), float(rs), _ptr(s_in), _ptr(s_out),
+                                   _ptr(x_bits), int(bool(x_is_bf16)), B, _ptr(y))
+    if rc != 0:
+        raise ValueError("oracle linear rejected its arguments")
+    return y
