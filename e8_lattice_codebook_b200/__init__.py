@@ -1,0 +1,286 @@
+"""glq-b200: B200-native (sm_100a) GLQ compressed-weight linear layer.
+
+    y = S_out . H_m . W^ . H_n . (S_in . x)
+
+W^ is stored as 16-bit indices into a 65,536-entry E8 lattice codebook (one
+per 8 weights), optionally refined by a uint8 (256-entry) or uint16 (E8)
+residual index times a residual scale, times a per-layer weight scale; H is
+a normalised (block-diagonal) Walsh-Hadamard transform and S_in / S_out are
+random +-1 signs (GLQ project pages: glq 0.5.1 PyPI page, "How it works",
+"Bit widths", "Inference kernels"; GLQ v0.3.2 release notes).
+
+This module is argument marshalling over the C ABI of ``libglq_b200.so``
+(declared in include/glq.h): every step of the layer runs in the library's
+CUDA kernels.  PyTorch is used only for device memory and streams.  There is
+no CPU fallback: if the library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libglq_b200.so")
+
+GLQ_F16, GLQ_BF16, GLQ_F32 = 0, 1, 2
+
+STATUS = {
+    0: "GLQ_OK", 1: "GLQ_ERR_INVALID_ARG", 2: "GLQ_ERR_SHAPE", 3: "GLQ_ERR_DTYPE",
+    4: "GLQ_ERR_BPW", 5: "GLQ_ERR_NO_CODEBOOK", 6: "GLQ_ERR_OOM", 7: "GLQ_ERR_CUDA",
+    8: "GLQ_ERR_DEVICE_CHECK", 9: "GLQ_ERR_TIMEOUT", 10: "GLQ_ERR_UNSUPPORTED",
+}
+
+# every symbol include/glq.h declares
+EXPORTS = (
+    "glq_status_str", "glq_version", "glq_e8_codebook", "glq_codebook_upload",
+    "glq_codebook_destroy", "glq_layer_create", "glq_layer_destroy", "glq_layer_reserve",
+    "glq_linear", "glq_dequant_reference", "glq_rht_input", "glq_rht_output",
+    "glq_layer_check", "glq_layer_info",
+)
+
+
+class GlqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what} failed: {STATUS.get(status, status)}")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m e8_lattice_codebook_b200.build` "
+        "(the GLQ layer has no CPU fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp, _i64, _i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+
+
+def _sig(name, args, res=ctypes.c_int):
+    f = getattr(_lib, name)
+    f.argtypes = args
+    f.restype = res
+    return f
+
+
+_lib_status_str = _sig("glq_status_str", [ctypes.c_int], ctypes.c_char_p)
+_lib_version = _sig("glq_version", [], ctypes.c_char_p)
+_lib_e8 = _sig("glq_e8_codebook", [_vp])
+_lib_cb_upload = _sig("glq_codebook_upload", [_vp, _i32, _i32, ctypes.POINTER(_vp)])
+_lib_cb_destroy = _sig("glq_codebook_destroy", [_vp])
+_lib_layer_create = _sig("glq_layer_create", [
+    _i64, _i64, _i32, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float, _vp, _vp,
+    ctypes.POINTER(_vp)])
+_lib_layer_destroy = _sig("glq_layer_destroy", [_vp])
+_lib_layer_reserve = _sig("glq_layer_reserve", [_vp, _i64])
+_lib_linear = _sig("glq_linear", [_vp, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, _vp])
+_lib_dequant = _sig("glq_dequant_reference", [_vp, _vp, _vp])
+_lib_rht_in = _sig("glq_rht_input", [_vp, _vp, ctypes.c_int, _vp, _i64, _vp])
+_lib_rht_out = _sig("glq_rht_output", [_vp, _vp, _vp, ctypes.c_int, _i64, _vp])
+_lib_check = _sig("glq_layer_check", [_vp, _vp])
+_lib_info = _sig("glq_layer_info", [
+    _vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i32),
+    ctypes.POINTER(ctypes.c_size_t)])
+
+
+def _ok(st: int, what: str):
+    if st != 0:
+        raise GlqError(st, what)
+
+
+# ---------------------------------------------------------------------------
+# C-ABI mirrors (same names, same arguments; raw pointers and sizes)
+# ---------------------------------------------------------------------------
+
+def glq_status_str(status: int) -> str:
+    return _lib_status_str(status).decode()
+
+
+def glq_version() -> str:
+    return _lib_version().decode()
+
+
+def glq_e8_codebook() -> np.ndarray:
+    """The library's 65,536 x 8 E8 codebook as fp16 bit patterns (uint16)."""
+    out = np.zeros((65536, 8), dtype=np.uint16)
+    _ok(_lib_e8(out.ctypes.data), "glq_e8_codebook")
+    return out
+
+
+def glq_codebook_upload(fp16_bits: np.ndarray) -> int:
+    a = np.ascontiguousarray(fp16_bits, dtype=np.uint16)
+    if a.ndim != 2:
+        raise ValueError("codebook must be [entries][8]")
+    h = _vp()
+    _ok(_lib_cb_upload(a.ctypes.data, a.shape[0], a.shape[1], ctypes.byref(h)), "glq_codebook_upload")
+    return h.value
+
+
+def glq_codebook_destroy(handle: int) -> None:
+    _ok(_lib_cb_destroy(handle), "glq_codebook_destroy")
+
+
+def glq_layer_create(m, n, bpw, idx1, idx2, primary, residual, weight_scale, resid_scale,
+                     s_in, s_out) -> int:
+    idx1 = np.ascontiguousarray(idx1, dtype=np.uint16)
+    if idx2 is not None:
+        idx2 = np.ascontiguousarray(idx2, dtype=np.uint8 if bpw == 3 else np.uint16)
+    s_in = np.ascontiguousarray(s_in, dtype=np.int8)
+    s_out = np.ascontiguousarray(s_out, dtype=np.int8)
+    if idx1.size != m * (n // 8) or s_in.size != n or s_out.size != m:
+        raise ValueError("array sizes do not match m, n")
+    if idx2 is not None and idx2.size != idx1.size:
+        raise ValueError("idx2 size does not match idx1")
+    h = _vp()
+    _ok(_lib_layer_create(m, n, bpw, idx1.ctypes.data, None if idx2 is None else idx2.ctypes.data,
+                          primary, residual, float(weight_scale), float(resid_scale),
+                          s_in.ctypes.data, s_out.ctypes.data, ctypes.byref(h)),
+        "glq_layer_create")
+    return h.value
+
+
+def glq_layer_destroy(handle: int) -> None:
+    _ok(_lib_layer_destroy(handle), "glq_layer_destroy")
+
+
+def glq_layer_reserve(handle: int, max_B: int) -> None:
+    _ok(_lib_layer_reserve(handle, max_B), "glq_layer_reserve")
+
+
+def glq_linear(handle, x_ptr, x_dtype, y_ptr, y_dtype, B, stream) -> None:
+    _ok(_lib_linear(handle, x_ptr, x_dtype, y_ptr, y_dtype, B, stream), "glq_linear")
+
+
+def glq_dequant_reference(handle, w_ptr, stream) -> None:
+    _ok(_lib_dequant(handle, w_ptr, stream), "glq_dequant_reference")
+
+
+def glq_rht_input(handle, x_ptr, x_dtype, xr_ptr, B, stream) -> None:
+    _ok(_lib_rht_in(handle, x_ptr, x_dtype, xr_ptr, B, stream), "glq_rht_input")
+
+
+def glq_rht_output(handle, z_ptr, y_ptr, y_dtype, B, stream) -> None:
+    _ok(_lib_rht_out(handle, z_ptr, y_ptr, y_dtype, B, stream), "glq_rht_output")
+
+
+def glq_layer_check(handle, stream) -> None:
+    _ok(_lib_check(handle, stream), "glq_layer_check")
+
+
+def glq_layer_info(handle):
+    m, n, bpw, nb = _i64(), _i64(), _i32(), ctypes.c_size_t()
+    _ok(_lib_info(handle, ctypes.byref(m), ctypes.byref(n), ctypes.byref(bpw), ctypes.byref(nb)),
+        "glq_layer_info")
+    return m.value, n.value, bpw.value, nb.value
+
+
+# ---------------------------------------------------------------------------
+# torch convenience (device memory and streams only)
+# ---------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def dtype_code(dt) -> int:
+    torch = _torch()
+    if dt == torch.float16:
+        return GLQ_F16
+    if dt == torch.bfloat16:
+        return GLQ_BF16
+    if dt == torch.float32:
+        return GLQ_F32
+    raise ValueError(f"unsupported dtype {dt}")
+
+
+def _stream_ptr(stream):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+class Codebook:
+    """A device codebook (65,536 x 8 E8 or 256 x 8 residual), fp16 bits on the host."""
+
+    def __init__(self, fp16_bits: np.ndarray):
+        self.entries = int(np.asarray(fp16_bits).shape[0])
+        self.handle = glq_codebook_upload(fp16_bits)
+
+    @classmethod
+    def e8(cls) -> "Codebook":
+        return cls(glq_e8_codebook())
+
+    def close(self):
+        if self.handle:
+            glq_codebook_destroy(self.handle)
+            self.handle = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class GlqLinear:
+    """One compressed linear layer on the current CUDA device."""
+
+    def __init__(self, m, n, bpw, idx1, idx2, primary: Codebook, residual: Codebook | None,
+                 weight_scale, resid_scale, s_in, s_out):
+        self.m, self.n, self.bpw = int(m), int(n), int(bpw)
+        self._cbs = (primary, residual)  # keep codebooks alive
+        self.handle = glq_layer_create(
+            self.m, self.n, self.bpw, idx1, idx2, primary.handle,
+            0 if residual is None else residual.handle, weight_scale, resid_scale, s_in, s_out)
+
+    def reserve(self, max_B: int):
+        glq_layer_reserve(self.handle, max_B)
+
+    def forward(self, x, out=None, out_dtype=None, stream=None):
+        torch = _torch()
+        if x.dim() != 2 or x.shape[1] != self.n or not x.is_cuda or not x.is_contiguous():
+            raise ValueError("x must be a contiguous CUDA tensor [B][n]")
+        B = x.shape[0]
+        odt = out_dtype or x.dtype
+        if out is None:
+            out = torch.empty((B, self.m), dtype=odt, device=x.device)
+        glq_linear(self.handle, x.data_ptr(), dtype_code(x.dtype), out.data_ptr(),
+                   dtype_code(out.dtype), B, _stream_ptr(stream))
+        return out
+
+    __call__ = forward
+
+    def dequant(self, stream=None):
+        torch = _torch()
+        w = torch.empty((self.m, self.n), dtype=torch.float32, device="cuda")
+        glq_dequant_reference(self.handle, w.data_ptr(), _stream_ptr(stream))
+        return w
+
+    def rht_input(self, x, stream=None):
+        torch = _torch()
+        xr = torch.empty((x.shape[0], self.n), dtype=torch.float32, device=x.device)
+        glq_rht_input(self.handle, x.data_ptr(), dtype_code(x.dtype), xr.data_ptr(), x.shape[0],
+                      _stream_ptr(stream))
+        return xr
+
+    def rht_output(self, z, out_dtype=None, stream=None):
+        torch = _torch()
+        y = torch.empty((z.shape[0], self.m), dtype=out_dtype or torch.float32, device=z.device)
+        glq_rht_output(self.handle, z.data_ptr(), y.data_ptr(), dtype_code(y.dtype), z.shape[0],
+                       _stream_ptr(stream))
+        return y
+
+    def check(self, stream=None):
+        glq_layer_check(self.handle, _stream_ptr(stream))
+
+    def close(self):
+        if self.handle:
+            glq_layer_destroy(self.handle)
+            self.handle = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,202 @@
+/*
+ * glq.h -- C ABI of glq-b200, a B200 (sm_100a) library for GLQ's fused
+ * compressed-weight linear layer
+ *
+ *     y = S_out . H_m . W^ . H_n . (S_in . x)
+ *
+ * Definitions (GLQ project pages):
+ *   - glq 0.5.1 PyPI page, "How it works" 1: each 8-weight group of W^ is a
+ *     16-bit index into a 65,536-entry E8 lattice codebook (the first shells
+ *     of E8); 3-8 bpw add 8-bit (256-entry) or 16-bit (E8) residual stages.
+ *   - same page, "How it works" 2: the Randomized Hadamard Transform is a
+ *     random sign flip followed by a fast Walsh-Hadamard transform.
+ *   - same page, "Bit widths": one global scale per layer; a size that is not
+ *     a power of two uses a block-diagonal Hadamard over its binary
+ *     decomposition (2688 = 2048 + 512 + 128).
+ *   - same page, "Inference kernels": Y = X . dequant(W)^T computed against
+ *     the indices without materialising W; residual index, residual codebook
+ *     and inverse residual scale are arguments of the matmul.
+ *   - GLQ v0.3.2 release notes, "What changed": the linear path is the three
+ *     ops input_rht -> fused linear -> output_rht.
+ *
+ * Conventions fixed by this library where the pages leave them open:
+ *   - codeword of group g in row r covers input columns 8g..8g+7; index
+ *     arrays are row-major [m][n/8];
+ *   - w^[r][8g+j] = ws * (cb1[idx1][j] + rs * cb2[idx2][j]) where rs is the
+ *     multiplier applied at decode (the pages' inverse residual scale);
+ *   - H_k[i][j] = (-1)^popcount(i & j) / sqrt(k) per block, blocks of the
+ *     binary decomposition of n in descending size at increasing offsets;
+ *   - input side: sign then H_n; output side: H_m then sign.
+ *
+ * Threading and ordering: every call that takes a cudaStream_t is
+ * asynchronous and stream-ordered.  Calls on one layer must be serialised
+ * (one stream, or explicit events): a layer owns one device workspace.
+ * Handles are not thread-safe; distinct layers may be used concurrently on
+ * distinct streams.  Every function returns a status and never throws.
+ */
+#ifndef GLQ_B200_H
+#define GLQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GLQ_API __attribute__((visibility("default")))
+#else
+#define GLQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GLQ_OK = 0,
+    GLQ_ERR_INVALID_ARG = 1,  /* null pointer, bad sign value, bad scale */
+    GLQ_ERR_SHAPE = 2,        /* m, n not positive multiples of 8; B < 0; size limits */
+    GLQ_ERR_DTYPE = 3,        /* unsupported dtype combination */
+    GLQ_ERR_BPW = 4,          /* bpw not in {2,3,4} or inconsistent residual */
+    GLQ_ERR_NO_CODEBOOK = 5,  /* missing or wrong-sized codebook handle */
+    GLQ_ERR_OOM = 6,          /* device or host allocation failed */
+    GLQ_ERR_CUDA = 7,         /* a CUDA runtime call or launch failed */
+    GLQ_ERR_DEVICE_CHECK = 8, /* a device-side check recorded a fault */
+    GLQ_ERR_TIMEOUT = 9,      /* a bounded device-side wait gave up */
+    GLQ_ERR_UNSUPPORTED = 10  /* codebook contents the kernels cannot hold */
+} glq_status;
+
+typedef enum { GLQ_F16 = 0, GLQ_BF16 = 1, GLQ_F32 = 2 } glq_dtype;
+
+/* Opaque handles; `void*` stream arguments are cudaStream_t (0 = legacy). */
+typedef struct glq_codebook_s *glq_codebook;
+typedef struct glq_layer_s *glq_layer;
+
+/* Human-readable name of a status.  Never NULL; static storage. */
+GLQ_API const char *glq_status_str(glq_status s);
+
+/* Library version string, static storage. */
+GLQ_API const char *glq_version(void);
+
+/*
+ * glq_e8_codebook -- the library's E8 shell codebook (host only, no GPU).
+ * Definition: glq 0.5.1 PyPI page, "How it works" 1 ("65,536 vectors from
+ * the first seven shells of the E8 lattice").  The subset is fixed by this
+ * library: every E8 point x (all coordinates integers, or all integers plus
+ * 1/2, with an even coordinate sum) of squared norm <= 12, sorted by
+ * (squared norm, x0, x1, ..., x7) ascending, first 65,536 kept.
+ * out_fp16_bits: caller-owned host array of 65536*8 uint16 receiving the
+ * IEEE binary16 bit patterns, row-major [65536][8] (every value is exact).
+ * Errors: GLQ_ERR_INVALID_ARG if out_fp16_bits is NULL.
+ */
+GLQ_API glq_status glq_e8_codebook(uint16_t *out_fp16_bits);
+
+/*
+ * glq_codebook_upload -- copy a codebook to the current CUDA device.
+ * Definition: glq 0.5.1 PyPI page, "How it works" 1 and "Bit widths".
+ * host_fp16_bits: caller-owned host array [entries][dim] of fp16 bit
+ *   patterns, read during the call only.
+ * entries: 65536 (a 16-bit primary / residual table) or 256 (an 8-bit
+ *   residual table); dim must be 8.
+ * A 65,536-entry table must hold values k/2 with |k| <= 6 whose
+ *   negation-folded size fits the on-chip table (true for glq_e8_codebook's
+ *   table); otherwise GLQ_ERR_UNSUPPORTED.  A 256-entry table may hold any
+ *   finite fp16 values of magnitude below 4094 (the kernels keep coordinates
+ *   2, 3, 6, 7 scaled by 16 in fp16); otherwise GLQ_ERR_UNSUPPORTED.
+ * out: receives a library-owned handle; release with glq_codebook_destroy
+ *   after every layer that uses it has been destroyed.
+ * Errors: GLQ_ERR_INVALID_ARG (NULL pointers, non-finite values),
+ *   GLQ_ERR_SHAPE (entries/dim), GLQ_ERR_UNSUPPORTED, GLQ_ERR_OOM,
+ *   GLQ_ERR_CUDA.  Synchronous.
+ */
+GLQ_API glq_status glq_codebook_upload(const uint16_t *host_fp16_bits, int32_t entries, int32_t dim,
+                               glq_codebook *out);
+GLQ_API glq_status glq_codebook_destroy(glq_codebook cb);
+
+/*
+ * glq_layer_create -- build a compressed linear layer on the current device.
+ * Definition: glq 0.5.1 PyPI page, "How it works" 1-2, "Bit widths",
+ * "Inference kernels" (Qidxs, Qidxs2, codebook2, Wscale, inv_resid_scale).
+ * m, n: output / input features, positive multiples of 8, each <= 32768
+ *   (the largest Hadamard row the one-CTA-per-row transforms hold).
+ * bpw: 2 (primary only), 3 (primary + uint8 residual into a 256-entry
+ *   table) or 4 (primary + uint16 residual into the E8 table).
+ * idx1: host uint16 [m][n/8]; idx2: host uint8 [m][n/8] (bpw 3), host
+ *   uint16 [m][n/8] (bpw 4) or NULL (bpw 2).  Both are read during the call
+ *   only (copied and re-laid-out for the kernels).
+ * primary: a 65,536-entry codebook handle.  residual: a 256-entry handle
+ *   for bpw 3; for bpw 4 NULL or the primary handle itself (the E8 table);
+ *   NULL for bpw 2.
+ * weight_scale: ws, finite.  resid_scale: rs, finite (ignored for bpw 2).
+ * s_in [n], s_out [m]: host int8, every entry +1 or -1.
+ * out: receives the layer handle (library-owned; glq_layer_destroy).
+ * Errors: GLQ_ERR_INVALID_ARG, GLQ_ERR_SHAPE, GLQ_ERR_BPW,
+ *   GLQ_ERR_NO_CODEBOOK, GLQ_ERR_OOM, GLQ_ERR_CUDA.  Synchronous.
+ */
+GLQ_API glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *idx1,
+                            const void *idx2, glq_codebook primary, glq_codebook residual,
+                            float weight_scale, float resid_scale, const int8_t *s_in,
+                            const int8_t *s_out, glq_layer *out);
+GLQ_API glq_status glq_layer_destroy(glq_layer layer);
+
+/*
+ * glq_layer_reserve -- size the layer's device workspace for batches up to
+ * max_B so that later glq_linear calls with B <= max_B allocate nothing
+ * (and may be captured in a CUDA graph).  glq_linear grows the workspace
+ * on demand otherwise (a synchronous allocation).  Errors: GLQ_ERR_SHAPE,
+ * GLQ_ERR_OOM, GLQ_ERR_CUDA.
+ */
+GLQ_API glq_status glq_layer_reserve(glq_layer layer, int64_t max_B);
+
+/*
+ * glq_linear -- y = S_out . H_m . W^ . H_n . (S_in . x).
+ * Definition: the layer formula above (glq 0.5.1 PyPI page, "How it works",
+ * "Inference kernels"; GLQ v0.3.2 release notes, input_rht ->
+ * fused_linear_block_diag -> output_rht).
+ * x_dev: device [B][n] row-major, dtype x_dtype (GLQ_F16 or GLQ_BF16).
+ * y_dev: device [B][m] row-major, dtype y_dtype (== x_dtype, or GLQ_F32).
+ * B >= 0 (B == 0 is a no-op).  stream: cudaStream_t.
+ * Paths: B <= 16 runs the decode kernels (input RHT, codebook GEMV on the
+ *   legacy warp MMA with an on-chip codebook, output RHT); B > 16 runs the
+ *   tensor-core path (input RHT, tcgen05/TMEM GEMM with a dequantising
+ *   producer, output RHT).  Accumulation is fp32 on every path.
+ * Errors: GLQ_ERR_INVALID_ARG, GLQ_ERR_DTYPE, GLQ_ERR_SHAPE, GLQ_ERR_OOM
+ *   (workspace growth), GLQ_ERR_CUDA (launch failure).  Asynchronous.
+ */
+GLQ_API glq_status glq_linear(glq_layer layer, const void *x_dev, glq_dtype x_dtype, void *y_dev,
+                      glq_dtype y_dtype, int64_t B, void *stream);
+
+/*
+ * glq_dequant_reference -- materialise W^ (fp32, no Hadamards, ws included)
+ * into w_dev [m][n] row-major, using the same on-chip decode the GEMV uses.
+ * Each value is fp32(ws * fma_f32(rs, cb2, cb1)) (single roundings).
+ * Errors: GLQ_ERR_INVALID_ARG, GLQ_ERR_CUDA.  Asynchronous.
+ */
+GLQ_API glq_status glq_dequant_reference(glq_layer layer, float *w_dev, void *stream);
+
+/*
+ * glq_rht_input / glq_rht_output -- the two Hadamard stages alone, for
+ * testing and composition (GLQ v0.3.2 release notes: input_rht,
+ * output_rht).  glq_rht_input: xr[B][n] (fp32, device) = H_n (S_in . x).
+ * glq_rht_output: y[B][m] (device, y_dtype) = S_out . H_m z, z fp32 device
+ * [B][m].  Errors as glq_linear.  Asynchronous.
+ */
+GLQ_API glq_status glq_rht_input(glq_layer layer, const void *x_dev, glq_dtype x_dtype, float *xr_dev,
+                         int64_t B, void *stream);
+GLQ_API glq_status glq_rht_output(glq_layer layer, const float *z_dev, void *y_dev, glq_dtype y_dtype,
+                          int64_t B, void *stream);
+
+/*
+ * glq_layer_check -- synchronise `stream`, then read and clear the layer's
+ * device error word (set by bounded device-side waits and checks).
+ * Returns GLQ_OK, GLQ_ERR_TIMEOUT, GLQ_ERR_DEVICE_CHECK or GLQ_ERR_CUDA.
+ */
+GLQ_API glq_status glq_layer_check(glq_layer layer, void *stream);
+
+/* Layer geometry, for callers sizing buffers.  Any output may be NULL. */
+GLQ_API glq_status glq_layer_info(glq_layer layer, int64_t *m, int64_t *n, int32_t *bpw,
+                          size_t *device_bytes);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GLQ_B200_H */

@@ -1,0 +1,162 @@
+"""GPU parity of the CUDA path against the fp64 oracle, through the C ABI.
+
+* glq_dequant_reference: bit-exact against the oracle's explicit decode;
+* glq_rht_input / glq_rht_output: against the oracle's dense Hadamard;
+* glq_linear (fp32 output): max |y - y_oracle| <= 2e-3 (||y_oracle||_inf + 1),
+  on small shapes spanning several tiles with ragged tails, and on every
+  synthetic workload at full size (sampled tokens, all outputs);
+* production dtype output: the same bound plus one output unit roundoff;
+* run-to-run bitwise determinism and per-token batch invariance.
+"""
+import numpy as np
+import pytest
+
+import glq_inputs as gi
+from gpu_helpers import Device, production_tolerance, to_torch_x, tolerance
+from oracle import glq_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return Device()
+
+
+def oracle_y(L, xbits, xdt):
+    return orc.linear(L.m, L.n, L.bpw, L.idx1, L.idx2, L.weight_scale, L.resid_scale, L.s_in,
+                      L.s_out, xbits, xdt == "bf16", cb2=L.cb2_f16)
+
+
+def x_to_f64(xbits, xdt):
+    if xdt == "f16":
+        return xbits.view(np.float16).astype(np.float64)
+    return (xbits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+SMALL = [  # m, n, bpw, B, x dtype -- several tiles, ragged row / column tails
+    (16, 128, 2, 1, "f16"), (40, 200, 2, 3, "f16"), (272, 264, 4, 5, "bf16"),
+    (64, 1024, 3, 8, "f16"), (1000, 968, 4, 9, "bf16"), (24, 56, 3, 16, "bf16"),
+    (520, 136, 2, 16, "f16"), (8, 8, 4, 2, "f16"), (264, 520, 3, 13, "bf16"),
+]
+
+
+@pytest.mark.parametrize("m,n,bpw,B,xdt", SMALL)
+def test_dequant_bit_exact_small(dev, m, n, bpw, B, xdt):
+    L = gi.make_layer(m + n, 3, m, n, bpw)
+    lay = dev.layer(L)
+    w = lay.dequant().cpu().numpy().astype(np.float64)
+    ref = orc.decode_rows(m, n, bpw, L.idx1, L.idx2, L.weight_scale, L.resid_scale, cb2=L.cb2_f16)
+    np.testing.assert_array_equal(w, ref)
+
+
+@pytest.mark.parametrize("m,n,bpw,B,xdt", SMALL)
+def test_linear_small(dev, m, n, bpw, B, xdt):
+    L = gi.make_layer(m * 7 + n, 1, m, n, bpw)
+    xb = gi.make_x(m * 7 + n, 1, B, n, xdt)
+    lay = dev.layer(L)
+    x = to_torch_x(xb, xdt)
+    y = lay(x, out_dtype=torch.float32).cpu().numpy().astype(np.float64)
+    ref = oracle_y(L, xb, xdt)
+    err = np.max(np.abs(y - ref))
+    assert err <= tolerance(ref), (err, tolerance(ref))
+    # production dtype
+    yp = lay(x).float().cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(yp - ref) <= production_tolerance(ref, xdt))
+
+
+@pytest.mark.parametrize("n", [8, 24, 56, 64, 200, 960, 1024, 2560, 5120, 11008, 14336, 32768])
+def test_rht_input_matches_dense_hadamard(dev, n):
+    m = 8
+    L = gi.make_layer(n, 0, m, n, 2)
+    xb = gi.make_x(n, 0, 3, n, "bf16")
+    lay = dev.layer(L)
+    xr = lay.rht_input(to_torch_x(xb, "bf16")).cpu().numpy().astype(np.float64)
+    xf = x_to_f64(xb, "bf16") * L.s_in
+    for b in range(3):
+        ref = orc.hadamard_apply(xf[b])
+        np.testing.assert_allclose(xr[b], ref, rtol=0, atol=1e-5 * (np.abs(ref).max() + 1))
+
+
+@pytest.mark.parametrize("m", [8, 24, 56, 64, 200, 960, 2048, 11008, 14336, 32768])
+def test_rht_output_matches_dense_hadamard(dev, m):
+    n = 8
+    L = gi.make_layer(m, 0, m, n, 2)
+    rng = np.random.default_rng(m)
+    z = rng.standard_normal((2, m)).astype(np.float32)
+    lay = dev.layer(L)
+    y = lay.rht_output(torch.from_numpy(z).cuda()).cpu().numpy().astype(np.float64)
+    for b in range(2):
+        ref = orc.hadamard_apply(z[b].astype(np.float64)) * L.s_out
+        np.testing.assert_allclose(y[b], ref, rtol=0, atol=1e-5 * (np.abs(ref).max() + 1))
+
+
+def _workload_cases():
+    cases = []
+    for key, wl in gi.WORKLOADS.items():
+        for li, spec in enumerate(wl.layers):
+            cases.append((key, li))
+    return cases
+
+
+@pytest.mark.parametrize("key,li", _workload_cases())
+def test_linear_workloads_full_size(dev, key, li):
+    """Every layer of every workload at full size, at the largest batch of the
+    workload that the decode kernels take plus, for prefill, 512 tokens;
+    the oracle checks a seeded sample of tokens (all m outputs each)."""
+    wl = gi.WORKLOADS[key]
+    L = gi.workload_layer(wl, li)
+    lay = dev.layer(L)
+    B = max(wl.batches) if max(wl.batches) <= 16 else min(wl.batches)
+    xb = gi.workload_x(wl, li, B)
+    x = to_torch_x(xb, wl.x_dtype)
+    y = lay(x, out_dtype=torch.float32).cpu().numpy().astype(np.float64)
+    rng = np.random.default_rng(li)
+    sample = sorted(set([0, B - 1] + list(rng.choice(B, size=min(B, 2), replace=False))))
+    ref = oracle_y(L, xb[sample], wl.x_dtype)
+    err = np.max(np.abs(y[sample] - ref))
+    print(f"\nPARITY {key} layer {li} ({L.m}x{L.n}) B={B}: max err {err:.3e} "
+          f"tol {tolerance(ref):.3e} ratio {err / tolerance(ref):.3f}")
+    assert err <= tolerance(ref), (err, tolerance(ref))
+    # dequantised codewords, sampled rows: bit-exact
+    w = lay.dequant()
+    rows = sorted(set([0, L.m - 1] + list(rng.choice(L.m, size=8, replace=False))))
+    wr = w[rows].cpu().numpy().astype(np.float64)
+    for i, r in enumerate(rows):
+        ref_w = orc.decode_rows(L.m, L.n, L.bpw, L.idx1, L.idx2, L.weight_scale, L.resid_scale,
+                                r, r + 1, cb2=L.cb2_f16)
+        np.testing.assert_array_equal(wr[i], ref_w[0])
+
+
+def test_determinism_and_batch_invariance(dev):
+    wl = gi.WORKLOADS["24b-decode-4bpw"]
+    L = gi.workload_layer(wl, 0)
+    lay = dev.layer(L)
+    xb = gi.workload_x(wl, 0, 16)
+    x = to_torch_x(xb, "bf16")
+    y1 = lay(x, out_dtype=torch.float32)
+    y2 = lay(x, out_dtype=torch.float32)
+    assert torch.equal(y1, y2)
+    for B in (1, 2, 4, 8):
+        yb = lay(x[:B].contiguous(), out_dtype=torch.float32)
+        assert torch.equal(yb, y1[:B]), B
+
+
+def test_empty_batch_and_errors(dev):
+    import e8_lattice_codebook_b200 as glq
+    L = gi.make_layer(0, 0, 64, 64, 2)
+    lay = dev.layer(L)
+    x = torch.zeros((0, 64), dtype=torch.float16, device="cuda")
+    y = lay(x)
+    assert y.shape == (0, 64)
+    xx = torch.zeros((2, 64), dtype=torch.float16, device="cuda")
+    yy = torch.zeros((2, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(glq.GlqError) as e:
+        glq.glq_linear(lay.handle, xx.data_ptr(), glq.GLQ_F16, yy.data_ptr(), glq.GLQ_BF16, 2,
+                       torch.cuda.current_stream().cuda_stream)
+    assert e.value.status == 3  # DTYPE
+    lay.check()
