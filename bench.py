@@ -1,0 +1,524 @@
+#!/usr/bin/env python
+"""Benchmark of the GLQ compressed-weight linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl glq|reference]
+
+A step is one pass of the decode hot path (input RHT -> codebook GEMV ->
+output RHT) over the five projections of the SmolLM3-3B-shaped workload
+(q, o 2048x2048; gate, up 11008x2048; down 2048x11008; 4 bpw = uint16 E8
+index + uint16 E8 residual, residual scale 1/8) for one token (B = 1), bf16
+activations.  Indices are HBM-resident: 8 copies of the five layers rotate
+(310 MB > the 126 MB L2).  Steps are CUDA-graph replays.
+
+value = algorithmic bytes per step (index bytes + activations in/out +
+bit-packed signs) / step time, in GB/s, summed over replicas.  Extra keys
+report the per-layer times, the 24B-class decode sweep, prefill TFLOP/s, the
+kernel roofline, the end-to-end number through host buffers, the fp64
+oracle on the host cores and the SM clocks seen while timing.
+
+Multi-GPU: the layer does not shard (one GPU per layer); --gpus N runs N
+independent replicas under torchrun, one per rank (weak scaling, no
+collective on the data path), and reports the max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import glq_inputs as gi  # noqa: E402
+
+METRIC = "glq_linear achieved HBM GB/s + µs/layer at B=1; prefill TFLOP/s; % roofline"
+MAIN_WORKLOAD = "smollm3-3b-4bpw"
+NCOPY = 8
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def layer_bytes(m: int, n: int, bpw: int, B: int, out_bytes: int = 2) -> int:
+    """Algorithmic HBM bytes of one layer call: indices + x + y + signs."""
+    return m * n * bpw // 8 + 2 * B * n + out_bytes * B * m + (m + 7) // 8 + (n + 7) // 8
+
+
+def gemv_bytes(m: int, n: int, bpw: int, B: int) -> int:
+    """Algorithmic bytes of the GEMV kernel alone: indices + fp16 xr + fp32 z."""
+    return m * n * bpw // 8 + 2 * B * n + 4 * B * m
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get(
+            "bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples (200 ms period) with wall times."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 100):
+        self.samples = []
+        self.proc = None
+        self.thread = None
+        self.gpu_index = gpu_index
+        self.period_ms = period_ms
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", f"-lms={self.period_ms}"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._reader, daemon=True)
+        self.thread.start()
+
+    def _reader(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0: float, t1: float):
+        inside = [p for (t, p) in self.samples if t0 <= t <= t1]
+        note = "samples inside the timed region"
+        if not inside:
+            inside = [p for (t, p) in self.samples if t0 - 2.0 <= t <= t1 + 0.5]
+            note = ("timed region shorter than the sampling period: samples from the identical "
+                    "replays around it")
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "no samples"}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+
+        sm = [num(p[1]) for p in inside if num(p[1]) is not None]
+        smax = [num(p[2]) for p in inside if num(p[2]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for p in inside:
+            for name, v in zip(names, p[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(inside), "note": note}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a float over all ranks (the job time is the slowest rank's)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# the GLQ arm
+# ---------------------------------------------------------------------------
+
+class WorkloadSet:
+    """ncopy device copies of the layers of a workload, with their x / y."""
+
+    def __init__(self, glq, torch, key: str, B: int, ncopy: int, out_dtype=None):
+        self.wl = gi.WORKLOADS[key]
+        self.B = B
+        self.torch = torch
+        self.e8 = glq.Codebook.e8()
+        xdt = torch.bfloat16 if self.wl.x_dtype == "bf16" else torch.float16
+        self.out_dtype = out_dtype or xdt
+        self.host = [gi.workload_layer(self.wl, i) for i in range(len(self.wl.layers))]
+        self.xbits = [gi.workload_x(self.wl, i, B) for i in range(len(self.wl.layers))]
+        self.copies = []
+        for c in range(ncopy):
+            layers = []
+            for i, L in enumerate(self.host):
+                res = None
+                if L.bpw == 3:
+                    res = glq.Codebook(L.cb2_f16.reshape(256, 8))
+                elif L.bpw == 4:
+                    res = self.e8
+                lay = glq.GlqLinear(L.m, L.n, L.bpw, L.idx1, L.idx2, self.e8, res,
+                                    L.weight_scale, L.resid_scale, L.s_in, L.s_out)
+                lay.reserve(min(B, 16))
+                x = torch.from_numpy(self.xbits[i].view(np.int16).copy()).cuda().view(xdt)
+                y = torch.empty((B, L.m), dtype=self.out_dtype, device="cuda")
+                layers.append((lay, x, y))
+            self.copies.append(layers)
+
+    def step(self, c: int, stream=None, B=None):
+        B = self.B if B is None else B
+        for lay, x, y in self.copies[c]:
+            lay(x[:B], out=y[:B], stream=stream)
+
+    def step_bytes(self, B=None) -> int:
+        B = self.B if B is None else B
+        ob = 4 if self.out_dtype == self.torch.float32 else 2
+        return sum(layer_bytes(L.m, L.n, L.bpw, B, ob) for L in self.host)
+
+    def step_flops(self, B=None) -> int:
+        B = self.B if B is None else B
+        return sum(2 * B * L.m * L.n for L in self.host)
+
+
+def capture_graphs(torch, fn_per_copy, ncopy):
+    graphs = []
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for c in range(ncopy):  # warm the launch paths outside capture
+            fn_per_copy(c)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    for c in range(ncopy):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn_per_copy(c)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    return graphs
+
+
+def time_replays(torch, graphs, reps: int, warm: int = 3) -> float:
+    """Mean ms per replay over `reps` replays rotating the graphs."""
+    for i in range(warm):
+        graphs[i % len(graphs)].replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(reps):
+        graphs[i % len(graphs)].replay()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def per_layer_times(torch, ws: WorkloadSet, reps: int, B=None):
+    B = ws.B if B is None else B
+    out = {}
+    for i, spec in enumerate(ws.wl.layers):
+        def fn(c, i=i):
+            lay, x, y = ws.copies[c][i]
+            lay(x[:B], out=y[:B])
+        graphs = capture_graphs(torch, fn, len(ws.copies))
+        ms = time_replays(torch, graphs, reps)
+        L = ws.host[i]
+        b = layer_bytes(L.m, L.n, L.bpw, B, 2)
+        out[f"{spec.name} {L.m}x{L.n}"] = {"us": round(ms * 1e3, 3),
+                                           "GBps": round(b / (ms * 1e-3) / 1e9, 1)}
+        del graphs
+    return out
+
+
+def gemv_kernel_time(torch, ws: WorkloadSet, layer_index: int, reps: int, B=None) -> float:
+    """Mean ms of the GEMV kernel alone (events on its stream, rotating copies)."""
+    B = min(ws.B if B is None else B, 16)
+    stream = torch.cuda.current_stream()
+    for c in range(len(ws.copies)):
+        lay, x, y = ws.copies[c][layer_index]
+        lay(x[:B], out=y[:B])
+    torch.cuda.synchronize()
+    for i in range(3):
+        ws.copies[i % len(ws.copies)][layer_index][0].gemv_replay(B, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(reps):
+        ws.copies[i % len(ws.copies)][layer_index][0].gemv_replay(B, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def oracle_step_seconds(ws_host, xbits, bpw, x_bf16) -> float:
+    from oracle import glq_oracle as orc
+    t0 = time.perf_counter()
+    for L, xb in zip(ws_host, xbits):
+        orc.linear(L.m, L.n, L.bpw, L.idx1, L.idx2, L.weight_scale, L.resid_scale, L.s_in,
+                   L.s_out, xb[:1], x_bf16, cb2=L.cb2_f16)
+    return time.perf_counter() - t0
+
+
+def run_glq(args):
+    import torch
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    import e8_lattice_codebook_b200 as glq
+
+    hbm_peak, tc_peak, tc_peak_sus, peak_src = read_peaks()
+    B = 1
+    ws = WorkloadSet(glq, torch, MAIN_WORKLOAD, B, NCOPY)
+    graphs = capture_graphs(torch, ws.step, NCOPY)
+    bytes_step = ws.step_bytes()
+
+    # clocks: the sampler runs through warm-up and the timed steps
+    sampler = ClockSampler(local)
+    sampler.start()
+    soak_end = time.time() + 1.0
+    i = 0
+    while time.time() < soak_end:  # ~1 s of identical replays for the clock sampler
+        graphs[i % NCOPY].replay()
+        i += 1
+        if i % 256 == 0:
+            torch.cuda.synchronize()
+    for i in range(args.warmup):
+        graphs[i % NCOPY].replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    torch.cuda.nvtx.range_push("timed")
+    e0.record()
+    for i in range(args.steps):
+        graphs[i % NCOPY].replay()
+    e1.record()
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world)
+    time.sleep(0.25)
+    sampler.stop()
+    ms_total = e0.elapsed_time(e1)
+    ms_total = max_over_ranks(ms_total, world, device=torch.device("cuda", local))
+    ms_step = ms_total / args.steps
+    value = world * bytes_step / (ms_step * 1e-3) / 1e9
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16 MMA operands, fp32 accumulate (bf16 activations in/out)",
+        "data": "synthetic (seeded uniform indices, Rademacher signs, N(0,1) activations)",
+        "config": {
+            "workload": ("smollm3-3b-4bpw decode: q,o 2048x2048, gate,up 11008x2048, "
+                         "down 2048x11008 @ 4 bpw (u16 E8 + u16 E8 residual, rs 1/8), B=1, bf16"),
+            "global_batch": B * world, "parallelism": f"replicas x{world}",
+            "l2": f"{NCOPY} rotating copies of the layer set "
+                  f"({NCOPY * sum(L.m * L.n // 2 for L in ws.host) / 1e6:.0f} MB > 126 MB L2)",
+            "timing": "CUDA-graph replay, CUDA events, max over ranks",
+        },
+        "gpu_launches": 3 * len(ws.host) * args.steps,
+        "clocks": clocks,
+    }
+    if rank != 0:
+        return None
+
+    # ---- extra measurements (rank 0) -------------------------------------
+    result["layers_us"] = per_layer_times(torch, ws, reps=400)
+
+    # roofline of the GEMV (the largest layer of the step: gate 11008x2048)
+    li = 2
+    L = ws.host[li]
+    ms_k = gemv_kernel_time(torch, ws, li, reps=400)
+    achieved = gemv_bytes(L.m, L.n, L.bpw, B) / (ms_k * 1e-3) / 1e9
+    result["roofline"] = {
+        "kernel": f"gemv_kernel<4,1> gate {L.m}x{L.n} B=1",
+        "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+        "frac": round(achieved / hbm_peak, 4), "peak_source": f"{peak_src} hbm_gbs (burst)",
+        "traffic": None, "kernel_us": round(ms_k * 1e3, 3),
+        "algorithmic_bytes": gemv_bytes(L.m, L.n, L.bpw, B),
+    }
+
+    # e2e through the public API with host buffers (eager, pinned copies)
+    xdt = torch.bfloat16
+    hx = [torch.from_numpy(xb.view(np.int16).copy()).view(xdt).pin_memory() for xb in ws.xbits]
+    hy = [torch.empty((B, Lh.m), dtype=xdt).pin_memory() for Lh in ws.host]
+    h2d = sum(t.numel() * 2 for t in hx)
+    d2h = sum(t.numel() * 2 for t in hy)
+
+    def e2e_step(c):
+        for (lay, x, y), hxi, hyi in zip(ws.copies[c], hx, hy):
+            x.copy_(hxi, non_blocking=True)
+            lay(x, out=y)
+            hyi.copy_(y, non_blocking=True)
+
+    for c in range(NCOPY):
+        e2e_step(c)
+    torch.cuda.synchronize()
+    reps = max(50, min(args.steps, 2000))
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for i in range(reps):
+        e2e_step(i % NCOPY)
+    f1.record()
+    torch.cuda.synchronize()
+    ms_e2e = f0.elapsed_time(f1) / reps
+    result["e2e"] = {"value": round(bytes_step / (ms_e2e * 1e-3) / 1e9, 2), "unit": "GB/s",
+                     "ms_per_step": round(ms_e2e, 6), "h2d_bytes_per_step": h2d,
+                     "d2h_bytes_per_step": d2h,
+                     "how": "glq_linear eager per layer + pinned H2D of x and D2H of y, events"}
+
+    # 24B-class decode sweep
+    if not args.quick:
+        sweep = {}
+        w24 = WorkloadSet(glq, torch, "24b-decode-4bpw", 16, 2)
+        for Bd in (1, 2, 4, 8, 16):
+            g24 = capture_graphs(torch, lambda c, Bd=Bd: w24.step(c, B=Bd), 2)
+            ms24 = time_replays(torch, g24, reps=100)
+            b24 = w24.step_bytes(Bd)
+            entry = {"ms_per_step": round(ms24, 4), "GBps": round(b24 / (ms24 * 1e-3) / 1e9, 1),
+                     "frac_hbm": round(b24 / (ms24 * 1e-3) / 1e9 / hbm_peak, 4)}
+            if Bd == 1:
+                entry["layers_us"] = per_layer_times(torch, w24, reps=100, B=1)
+                mk = gemv_kernel_time(torch, w24, 2, reps=100, B=1)
+                Lg = w24.host[2]
+                ach = gemv_bytes(Lg.m, Lg.n, Lg.bpw, 1) / (mk * 1e-3) / 1e9
+                entry["gemv_gate_us"] = round(mk * 1e3, 3)
+                entry["gemv_gate_frac_hbm"] = round(ach / hbm_peak, 4)
+            sweep[f"B={Bd}"] = entry
+            del g24
+        del w24
+        torch.cuda.empty_cache()
+        result["decode_24b"] = sweep
+
+        pre = {}
+        wp = WorkloadSet(glq, torch, "prefill-8b-mlp-4bpw", 8192, 1)
+        for Bp in (512, 2048, 8192):
+            wp.step(0, B=Bp)
+            torch.cuda.synchronize()
+            reps = 3
+            p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            p0.record()
+            for _ in range(reps):
+                wp.step(0, B=Bp)
+            p1.record()
+            torch.cuda.synchronize()
+            msp = p0.elapsed_time(p1) / reps
+            tf = wp.step_flops(Bp) / (msp * 1e-3) / 1e12
+            pre[f"B={Bp}"] = {"ms_per_step": round(msp, 3), "TFLOPs": round(tf, 2),
+                              "frac_bf16_peak": round(tf / tc_peak, 4)}
+        del wp
+        torch.cuda.empty_cache()
+        result["prefill"] = pre
+
+    # fp64 oracle on the host cores (one decode step, 1 token, 5 layers)
+    if world == 1 and not args.no_cpu:
+        secs = oracle_step_seconds(ws.host, ws.xbits, 4, True)
+        result["cpu_baseline"] = {
+            "value": round(bytes_step / secs / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle", "seconds": round(secs, 3),
+            "sample": "one full step: 1 token through q,o,gate,up,down (fp64, single thread)"}
+    return result
+
+
+# ---------------------------------------------------------------------------
+# the reference arm: the fp64 oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    world, rank, local = dist_setup()
+    if world > 1 and rank != 0:
+        return None
+    wl = gi.WORKLOADS[MAIN_WORKLOAD]
+    host = [gi.workload_layer(wl, i) for i in range(len(wl.layers))]
+    xbits = [gi.workload_x(wl, i, 1) for i in range(len(wl.layers))]
+    bytes_step = sum(layer_bytes(L.m, L.n, L.bpw, 1, 2) for L in host)
+    for _ in range(args.warmup if args.warmup <= 1 else 1):
+        oracle_step_seconds(host, xbits, 4, True)
+    budget = 150.0
+    t_step = None
+    times = []
+    t_start = time.perf_counter()
+    for i in range(args.steps):
+        times.append(oracle_step_seconds(host, xbits, 4, True))
+        if time.perf_counter() - t_start > budget:
+            break
+    t_step = sum(times) / len(times)
+    value = bytes_step / t_step / 1e9
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": len(times), "warmup": args.warmup,
+        "ms_per_step": round(t_step * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": ("smollm3-3b-4bpw decode: q,o 2048x2048, gate,up 11008x2048, "
+                                "down 2048x11008 @ 4 bpw, B=1, bf16"),
+                   "global_batch": 1, "parallelism": "single host thread"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{len(times)} full steps (1 token, 5 layers) of the fp64 oracle"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["glq", "reference"], default="glq")
+    ap.add_argument("--quick", action="store_true", help="skip the 24B sweep and prefill")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    res = run_reference(args) if args.impl == "reference" else run_glq(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1 and args.impl == "glq":
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

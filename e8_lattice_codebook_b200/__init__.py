@@ -12,7 +12,7 @@ random +-1 signs (GLQ project pages: glq 0.5.1 PyPI page, "How it works",
 This module is argument marshalling over the C ABI of ``libglq_b200.so``
 (declared in include/glq.h): every step of the layer runs in the library's
 CUDA kernels.  PyTorch is used only for device memory and streams.  There is
-no CPU fallback: if the library is missing, importing this module raises.
+no CPU fallback: if the library is missing, the first call raises.
 """
 from __future__ import annotations
 
@@ -37,7 +37,7 @@ EXPORTS = (
     "glq_status_str", "glq_version", "glq_e8_codebook", "glq_codebook_upload",
     "glq_codebook_destroy", "glq_layer_create", "glq_layer_destroy", "glq_layer_reserve",
     "glq_linear", "glq_dequant_reference", "glq_rht_input", "glq_rht_output",
-    "glq_layer_check", "glq_layer_info",
+    "glq_layer_check", "glq_layer_info", "glq_gemv_replay",
 )
 
 
@@ -47,40 +47,47 @@ class GlqError(RuntimeError):
         self.status = status
 
 
-if not os.path.exists(LIB_PATH):
-    raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m e8_lattice_codebook_b200.build` "
-        "(the GLQ layer has no CPU fallback)")
-
-_lib = ctypes.CDLL(LIB_PATH)
 _vp, _i64, _i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
 
+# argument / result types of every exported function
+_SIGNATURES = {
+    "glq_status_str": ([ctypes.c_int], ctypes.c_char_p),
+    "glq_version": ([], ctypes.c_char_p),
+    "glq_e8_codebook": ([_vp], ctypes.c_int),
+    "glq_codebook_upload": ([_vp, _i32, _i32, ctypes.POINTER(_vp)], ctypes.c_int),
+    "glq_codebook_destroy": ([_vp], ctypes.c_int),
+    "glq_layer_create": ([_i64, _i64, _i32, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float,
+                          _vp, _vp, ctypes.POINTER(_vp)], ctypes.c_int),
+    "glq_layer_destroy": ([_vp], ctypes.c_int),
+    "glq_layer_reserve": ([_vp, _i64], ctypes.c_int),
+    "glq_linear": ([_vp, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, _vp], ctypes.c_int),
+    "glq_dequant_reference": ([_vp, _vp, _vp], ctypes.c_int),
+    "glq_rht_input": ([_vp, _vp, ctypes.c_int, _vp, _i64, _vp], ctypes.c_int),
+    "glq_rht_output": ([_vp, _vp, _vp, ctypes.c_int, _i64, _vp], ctypes.c_int),
+    "glq_layer_check": ([_vp, _vp], ctypes.c_int),
+    "glq_gemv_replay": ([_vp, _i64, _vp], ctypes.c_int),
+    "glq_layer_info": ([_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i32),
+                        ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
+}
 
-def _sig(name, args, res=ctypes.c_int):
-    f = getattr(_lib, name)
-    f.argtypes = args
-    f.restype = res
-    return f
+_lib = None
 
 
-_lib_status_str = _sig("glq_status_str", [ctypes.c_int], ctypes.c_char_p)
-_lib_version = _sig("glq_version", [], ctypes.c_char_p)
-_lib_e8 = _sig("glq_e8_codebook", [_vp])
-_lib_cb_upload = _sig("glq_codebook_upload", [_vp, _i32, _i32, ctypes.POINTER(_vp)])
-_lib_cb_destroy = _sig("glq_codebook_destroy", [_vp])
-_lib_layer_create = _sig("glq_layer_create", [
-    _i64, _i64, _i32, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float, _vp, _vp,
-    ctypes.POINTER(_vp)])
-_lib_layer_destroy = _sig("glq_layer_destroy", [_vp])
-_lib_layer_reserve = _sig("glq_layer_reserve", [_vp, _i64])
-_lib_linear = _sig("glq_linear", [_vp, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, _vp])
-_lib_dequant = _sig("glq_dequant_reference", [_vp, _vp, _vp])
-_lib_rht_in = _sig("glq_rht_input", [_vp, _vp, ctypes.c_int, _vp, _i64, _vp])
-_lib_rht_out = _sig("glq_rht_output", [_vp, _vp, _vp, ctypes.c_int, _i64, _vp])
-_lib_check = _sig("glq_layer_check", [_vp, _vp])
-_lib_info = _sig("glq_layer_info", [
-    _vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i32),
-    ctypes.POINTER(ctypes.c_size_t)])
+def _L():
+    """The loaded library (loaded on first use; raises if it is missing)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m e8_lattice_codebook_b200.build` "
+                "(the GLQ layer has no CPU fallback)")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGNATURES.items():
+            f = getattr(lib, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = lib
+    return _lib
 
 
 def _ok(st: int, what: str):
@@ -93,17 +100,17 @@ def _ok(st: int, what: str):
 # ---------------------------------------------------------------------------
 
 def glq_status_str(status: int) -> str:
-    return _lib_status_str(status).decode()
+    return _L().glq_status_str(status).decode()
 
 
 def glq_version() -> str:
-    return _lib_version().decode()
+    return _L().glq_version().decode()
 
 
 def glq_e8_codebook() -> np.ndarray:
     """The library's 65,536 x 8 E8 codebook as fp16 bit patterns (uint16)."""
     out = np.zeros((65536, 8), dtype=np.uint16)
-    _ok(_lib_e8(out.ctypes.data), "glq_e8_codebook")
+    _ok(_L().glq_e8_codebook(out.ctypes.data), "glq_e8_codebook")
     return out
 
 
@@ -112,12 +119,12 @@ def glq_codebook_upload(fp16_bits: np.ndarray) -> int:
     if a.ndim != 2:
         raise ValueError("codebook must be [entries][8]")
     h = _vp()
-    _ok(_lib_cb_upload(a.ctypes.data, a.shape[0], a.shape[1], ctypes.byref(h)), "glq_codebook_upload")
+    _ok(_L().glq_codebook_upload(a.ctypes.data, a.shape[0], a.shape[1], ctypes.byref(h)), "glq_codebook_upload")
     return h.value
 
 
 def glq_codebook_destroy(handle: int) -> None:
-    _ok(_lib_cb_destroy(handle), "glq_codebook_destroy")
+    _ok(_L().glq_codebook_destroy(handle), "glq_codebook_destroy")
 
 
 def glq_layer_create(m, n, bpw, idx1, idx2, primary, residual, weight_scale, resid_scale,
@@ -132,7 +139,7 @@ def glq_layer_create(m, n, bpw, idx1, idx2, primary, residual, weight_scale, res
     if idx2 is not None and idx2.size != idx1.size:
         raise ValueError("idx2 size does not match idx1")
     h = _vp()
-    _ok(_lib_layer_create(m, n, bpw, idx1.ctypes.data, None if idx2 is None else idx2.ctypes.data,
+    _ok(_L().glq_layer_create(m, n, bpw, idx1.ctypes.data, None if idx2 is None else idx2.ctypes.data,
                           primary, residual, float(weight_scale), float(resid_scale),
                           s_in.ctypes.data, s_out.ctypes.data, ctypes.byref(h)),
         "glq_layer_create")
@@ -140,36 +147,40 @@ def glq_layer_create(m, n, bpw, idx1, idx2, primary, residual, weight_scale, res
 
 
 def glq_layer_destroy(handle: int) -> None:
-    _ok(_lib_layer_destroy(handle), "glq_layer_destroy")
+    _ok(_L().glq_layer_destroy(handle), "glq_layer_destroy")
 
 
 def glq_layer_reserve(handle: int, max_B: int) -> None:
-    _ok(_lib_layer_reserve(handle, max_B), "glq_layer_reserve")
+    _ok(_L().glq_layer_reserve(handle, max_B), "glq_layer_reserve")
 
 
 def glq_linear(handle, x_ptr, x_dtype, y_ptr, y_dtype, B, stream) -> None:
-    _ok(_lib_linear(handle, x_ptr, x_dtype, y_ptr, y_dtype, B, stream), "glq_linear")
+    _ok(_L().glq_linear(handle, x_ptr, x_dtype, y_ptr, y_dtype, B, stream), "glq_linear")
 
 
 def glq_dequant_reference(handle, w_ptr, stream) -> None:
-    _ok(_lib_dequant(handle, w_ptr, stream), "glq_dequant_reference")
+    _ok(_L().glq_dequant_reference(handle, w_ptr, stream), "glq_dequant_reference")
 
 
 def glq_rht_input(handle, x_ptr, x_dtype, xr_ptr, B, stream) -> None:
-    _ok(_lib_rht_in(handle, x_ptr, x_dtype, xr_ptr, B, stream), "glq_rht_input")
+    _ok(_L().glq_rht_input(handle, x_ptr, x_dtype, xr_ptr, B, stream), "glq_rht_input")
 
 
 def glq_rht_output(handle, z_ptr, y_ptr, y_dtype, B, stream) -> None:
-    _ok(_lib_rht_out(handle, z_ptr, y_ptr, y_dtype, B, stream), "glq_rht_output")
+    _ok(_L().glq_rht_output(handle, z_ptr, y_ptr, y_dtype, B, stream), "glq_rht_output")
+
+
+def glq_gemv_replay(handle, B, stream) -> None:
+    _ok(_L().glq_gemv_replay(handle, B, stream), "glq_gemv_replay")
 
 
 def glq_layer_check(handle, stream) -> None:
-    _ok(_lib_check(handle, stream), "glq_layer_check")
+    _ok(_L().glq_layer_check(handle, stream), "glq_layer_check")
 
 
 def glq_layer_info(handle):
     m, n, bpw, nb = _i64(), _i64(), _i32(), ctypes.c_size_t()
-    _ok(_lib_info(handle, ctypes.byref(m), ctypes.byref(n), ctypes.byref(bpw), ctypes.byref(nb)),
+    _ok(_L().glq_layer_info(handle, ctypes.byref(m), ctypes.byref(n), ctypes.byref(bpw), ctypes.byref(nb)),
         "glq_layer_info")
     return m.value, n.value, bpw.value, nb.value
 
@@ -270,6 +281,9 @@ class GlqLinear:
         glq_rht_output(self.handle, z.data_ptr(), y.data_ptr(), dtype_code(y.dtype), z.shape[0],
                        _stream_ptr(stream))
         return y
+
+    def gemv_replay(self, B, stream=None):
+        glq_gemv_replay(self.handle, B, _stream_ptr(stream))
 
     def check(self, stream=None):
         glq_layer_check(self.handle, _stream_ptr(stream))

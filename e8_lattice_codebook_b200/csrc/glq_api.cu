@@ -44,6 +44,7 @@ struct glq_layer_s {
     int bands = 0, splits = 0, cps = 0, grid = 0;
     // workspace
     int64_t cap_rows = 0;  // rows of xr / info
+    int64_t last_B = 0;    // batch of the last decode slice (glq_gemv_replay)
     __half *d_xr = nullptr;
     glq_rowinfo *d_info = nullptr;
     float *d_part = nullptr;
@@ -455,6 +456,7 @@ glq_status glq_linear(glq_layer L, const void *x_dev, glq_dtype x_dtype, void *y
 
         glq::GemvParams pg = gemv_params(L, L->d_xr, L->d_info, nb);
         if (glq::launch_gemv(pg, L->bpw, L->grid, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+        L->last_B = nb;
 
         glq::RhtOutParams pout{};
         pout.m = (int)L->m;
@@ -537,6 +539,16 @@ glq_status glq_rht_output(glq_layer L, const float *z_dev, void *y_dev, glq_dtyp
     p.y_dtype = (int)y_dtype;
     return glq::launch_rht_out(p, static_cast<cudaStream_t>(stream), false) == cudaSuccess ? GLQ_OK
                                                                                           : GLQ_ERR_CUDA;
+}
+
+glq_status glq_gemv_replay(glq_layer L, int64_t B, void *stream) {
+    if (!L) return GLQ_ERR_INVALID_ARG;
+    if (B < 1 || B > L->last_B) return GLQ_ERR_SHAPE;
+    DeviceGuard guard(L->device);
+    glq::GemvParams pg = gemv_params(L, L->d_xr, L->d_info, (int)B);
+    return glq::launch_gemv(pg, L->bpw, L->grid, static_cast<cudaStream_t>(stream), false) == cudaSuccess
+               ? GLQ_OK
+               : GLQ_ERR_CUDA;
 }
 
 glq_status glq_layer_check(glq_layer L, void *stream) {

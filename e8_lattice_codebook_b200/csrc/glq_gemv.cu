@@ -197,12 +197,14 @@ __global__ void __launch_bounds__(GEMV_WARPS * 32, 1) gemv_kernel(GemvParams p) 
 template <int BPW, int NT>
 cudaError_t launch_t(const GemvParams &p, int grid, cudaStream_t s, bool pdl) {
     size_t smem = gemv_smem_bytes(p.table_words, BPW);
-    static size_t configured = 0;
-    if (configured < smem) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<BPW, NT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // raised once to the largest table the library accepts (never lowered:
+    // captured graphs replay against the attribute value at replay time)
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<BPW, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)gemv_smem_bytes(GLQ_TABLE_MAX_WORDS, BPW));
         if (e != cudaSuccess) return e;
-        configured = smem;
+        configured = true;
     }
     GemvParams q = p;
     void *args[] = {&q};

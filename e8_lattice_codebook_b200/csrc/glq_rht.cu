@@ -130,10 +130,23 @@ __global__ void __launch_bounds__(RHT_THREADS) rht_out_kernel(RhtOutParams p) {
 
 }  // namespace
 
+// The dynamic shared memory limit of each kernel is raised once, to the
+// largest row any layer can have: a graph captured over several layers
+// replays every node against the attribute value current at replay time.
+cudaError_t ensure_rht_smem() {
+    static bool done = false;
+    if (done) return cudaSuccess;
+    const int bytes = GLQ_RHT_MAX_N * (int)sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(rht_in_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(rht_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done = true;
+    return e;
+}
+
 cudaError_t launch_rht_in(const RhtInParams &p, cudaStream_t s, bool pdl) {
     size_t smem = (size_t)p.n * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(rht_in_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = ensure_rht_smem();
     if (e != cudaSuccess) return e;
     RhtInParams q = p;
     void *args[] = {&q};
@@ -142,8 +155,7 @@ cudaError_t launch_rht_in(const RhtInParams &p, cudaStream_t s, bool pdl) {
 
 cudaError_t launch_rht_out(const RhtOutParams &p, cudaStream_t s, bool pdl) {
     size_t smem = (size_t)p.m * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(rht_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e = ensure_rht_smem();
     if (e != cudaSuccess) return e;
     RhtOutParams q = p;
     void *args[] = {&q};

@@ -185,6 +185,18 @@ GLQ_API glq_status glq_rht_output(glq_layer layer, const float *z_dev, void *y_d
                           int64_t B, void *stream);
 
 /*
+ * glq_gemv_replay -- measurement entry point: re-launches only the codebook
+ * GEMV of the most recent glq_linear call on this layer (same activations
+ * already in the layer's workspace, batch B <= min(16, that call's B)),
+ * writing the same split-K partial sums.  Lets a caller time the GEMV kernel
+ * alone with events on `stream`.  The decode path's GEMV is the one of
+ * "Inference kernels" on the glq 0.5.1 PyPI page (matmul against indices).
+ * Errors: GLQ_ERR_INVALID_ARG, GLQ_ERR_SHAPE (B out of range or no previous
+ * call), GLQ_ERR_CUDA.  Asynchronous.
+ */
+GLQ_API glq_status glq_gemv_replay(glq_layer layer, int64_t B, void *stream);
+
+/*
  * glq_layer_check -- synchronise `stream`, then read and clear the layer's
  * device error word (set by bounded device-side waits and checks).
  * Returns GLQ_OK, GLQ_ERR_TIMEOUT, GLQ_ERR_DEVICE_CHECK or GLQ_ERR_CUDA.
