@@ -37,7 +37,7 @@ EXPORTS = (
     "glq_status_str", "glq_version", "glq_e8_codebook", "glq_codebook_upload",
     "glq_codebook_destroy", "glq_layer_create", "glq_layer_destroy", "glq_layer_reserve",
     "glq_linear", "glq_dequant_reference", "glq_rht_input", "glq_rht_output",
-    "glq_layer_check", "glq_layer_info", "glq_gemv_replay",
+    "glq_layer_check", "glq_layer_info", "glq_gemv_replay", "glq_linear_noalloc",
 )
 
 
@@ -61,6 +61,7 @@ _SIGNATURES = {
     "glq_layer_destroy": ([_vp], ctypes.c_int),
     "glq_layer_reserve": ([_vp, _i64], ctypes.c_int),
     "glq_linear": ([_vp, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, _vp], ctypes.c_int),
+    "glq_linear_noalloc": ([_vp, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, _vp], ctypes.c_int),
     "glq_dequant_reference": ([_vp, _vp, _vp], ctypes.c_int),
     "glq_rht_input": ([_vp, _vp, ctypes.c_int, _vp, _i64, _vp], ctypes.c_int),
     "glq_rht_output": ([_vp, _vp, _vp, ctypes.c_int, _i64, _vp], ctypes.c_int),
@@ -156,6 +157,12 @@ def glq_layer_reserve(handle: int, max_B: int) -> None:
 
 def glq_linear(handle, x_ptr, x_dtype, y_ptr, y_dtype, B, stream) -> None:
     _ok(_L().glq_linear(handle, x_ptr, x_dtype, y_ptr, y_dtype, B, stream), "glq_linear")
+
+
+def glq_linear_noalloc(handle, x_ptr, x_dtype, y_ptr, y_dtype, B, stream) -> None:
+    """glq_linear without device allocation (B <= 16; fixed 8 MiB device scratch)."""
+    _ok(_L().glq_linear_noalloc(handle, x_ptr, x_dtype, y_ptr, y_dtype, B, stream),
+        "glq_linear_noalloc")
 
 
 def glq_dequant_reference(handle, w_ptr, stream) -> None:

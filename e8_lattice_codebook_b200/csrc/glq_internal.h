@@ -60,6 +60,12 @@
 // decode batch limit (the GEMV handles up to two 8-column MMA tiles)
 #define GLQ_DECODE_MAX_B 16
 
+// size of the fixed device scratch array of glq_linear_noalloc (the public
+// header states the same value)
+#ifndef GLQ_NOALLOC_SCRATCH_BYTES
+#define GLQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+#endif
+
 // largest Hadamard block handled by the one-CTA-per-row RHT kernels
 #define GLQ_RHT_MAX_N 32768
 #define GLQ_MAX_BLOCKS 32

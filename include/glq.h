@@ -197,6 +197,31 @@ GLQ_API glq_status glq_rht_output(glq_layer layer, const float *z_dev, void *y_d
 GLQ_API glq_status glq_gemv_replay(glq_layer layer, int64_t B, void *stream);
 
 /*
+ * glq_linear_noalloc -- glq_linear for a batch of at most 16 tokens that
+ * allocates no device memory, for callers that cannot call cudaMalloc at
+ * call time: code running while a CUDA graph is captured, in host
+ * callbacks, or under a framework that owns every device allocation.  (The
+ * GLQ pages have no counterpart: this is a property of this library's
+ * workspace handling.)
+ * Instead of the layer's workspace it uses one fixed device array of
+ * GLQ_NOALLOC_SCRATCH_BYTES (8 MiB) that the library defines at file scope;
+ * every GPU that loads the library holds it until the process exits.
+ * x_dev, y_dev, x_dtype, y_dtype, stream: as glq_linear; 0 <= B <= 16.
+ * The first call on a device resolves the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Calls share the array and it keeps the last call's contents: two calls
+ * whose work overlaps on the GPU (other streams, unordered layers) race.
+ * Results equal glq_linear's up to the order of fp32 sums (the split-K
+ * plan is narrowed when its partial sums would not fit the array).
+ * Errors: GLQ_ERR_INVALID_ARG, GLQ_ERR_DTYPE, GLQ_ERR_SHAPE (B > 16, or a
+ *   layer whose activations plus one split of partial sums exceed the
+ *   array), GLQ_ERR_CUDA.  Asynchronous.
+ */
+#define GLQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+GLQ_API glq_status glq_linear_noalloc(glq_layer layer, const void *x_dev, glq_dtype x_dtype,
+                                      void *y_dev, glq_dtype y_dtype, int64_t B, void *stream);
+
+/*
  * glq_layer_check -- synchronise `stream`, then read and clear the layer's
  * device error word (set by bounded device-side waits and checks).
  * Returns GLQ_OK, GLQ_ERR_TIMEOUT, GLQ_ERR_DEVICE_CHECK or GLQ_ERR_CUDA.
