@@ -264,22 +264,25 @@ def per_layer_times(torch, ws: WorkloadSet, reps: int, B=None):
 
 
 def gemv_kernel_time(torch, ws: WorkloadSet, layer_index: int, reps: int, B=None) -> float:
-    """Mean ms of the GEMV kernel alone (events on its stream, rotating copies)."""
+    """Mean ms of the GEMV kernel alone: CUDA graphs of 20 back-to-back
+    launches (no host launch cost between them), rotating the weight copies,
+    timed with events on the stream the kernels run on."""
     B = min(ws.B if B is None else B, 16)
-    stream = torch.cuda.current_stream()
     for c in range(len(ws.copies)):
         lay, x, y = ws.copies[c][layer_index]
         lay(x[:B], out=y[:B])
     torch.cuda.synchronize()
-    for i in range(3):
-        ws.copies[i % len(ws.copies)][layer_index][0].gemv_replay(B, stream)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(reps):
-        ws.copies[i % len(ws.copies)][layer_index][0].gemv_replay(B, stream)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / reps
+    per_graph = 20
+
+    def fn(c):
+        for i in range(per_graph):
+            ws.copies[(c + i) % len(ws.copies)][layer_index][0].gemv_replay(B)
+
+    graphs = capture_graphs(torch, fn, len(ws.copies))
+    n = max(1, reps // per_graph)
+    ms = time_replays(torch, graphs, n)
+    del graphs
+    return ms / per_graph
 
 
 def oracle_step_seconds(ws_host, xbits, bpw, x_bf16) -> float:

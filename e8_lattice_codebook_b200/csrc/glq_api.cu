@@ -34,22 +34,6 @@ struct DeviceGuard {
     }
 };
 
-glq_blocks make_blocks(int64_t n) {
-    glq_blocks b{};
-    int off = 0;
-    for (int bit = 30; bit >= 0; --bit) {
-        if (n & (int64_t(1) << bit)) {
-            int k = 1 << bit;
-            b.size[b.count] = k;
-            b.offset[b.count] = off;
-            b.inv_sqrt[b.count] = (float)(1.0 / std::sqrt((double)k));
-            off += k;
-            ++b.count;
-        }
-    }
-    return b;
-}
-
 bool all_signs(const int8_t *s, int64_t k) {
     for (int64_t i = 0; i < k; ++i)
         if (s[i] != 1 && s[i] != -1) return false;
@@ -75,6 +59,20 @@ glq_status dmalloc(T **p, size_t bytes, size_t *total) {
     return GLQ_OK;
 }
 
+void free_workspace(glq_layer L) {
+    cudaFree(L->wsp.xq);
+    cudaFree(L->wsp.xh);
+    cudaFree(L->wsp.info);
+    cudaFree(L->wsp.part);
+    cudaFree(L->wsp.z);
+    L->wsp.xq = nullptr;
+    L->wsp.xh = nullptr;
+    L->wsp.info = nullptr;
+    L->wsp.part = nullptr;
+    L->wsp.z = nullptr;
+    L->cap_rows = 0;
+}
+
 void free_layer(glq_layer L) {
     if (!L) return;
     cudaFree(L->d_idx1);
@@ -82,83 +80,94 @@ void free_layer(glq_layer L) {
     cudaFree(L->d_sin);
     cudaFree(L->d_sout);
     cudaFree(L->d_err);
-    cudaFree(L->d_r8);
-    cudaFree(L->d_xr);
-    cudaFree(L->d_info);
-    cudaFree(L->d_part);
+    cudaFree(L->wsp.cnt);
+    free_workspace(L);
     delete L;
-}
-
-// Chooses the split of the chunk range so that (bands x splits) tasks spread
-// over the persistent grid with the least makespan (in chunks per CTA).
-void plan_gemv(glq_layer L) {
-    L->bands = (L->RT + glq::GEMV_WARPS - 1) / glq::GEMV_WARPS;
-    int best_s = 1;
-    double best = 1e30;
-    for (int s = 1; s <= L->KC; ++s) {
-        int cps = (L->KC + s - 1) / s;
-        int used = (L->KC + cps - 1) / cps;  // splits actually populated
-        if (used != s) continue;
-        int64_t tasks = (int64_t)L->bands * s;
-        int64_t waves = (tasks + L->num_sms - 1) / L->num_sms;
-        double cost = (double)waves * cps + 0.02 * s;
-        if (cost < best) {
-            best = cost;
-            best_s = s;
-        }
-    }
-    L->splits = best_s;
-    L->cps = (L->KC + best_s - 1) / best_s;
-    int64_t tasks = (int64_t)L->bands * L->splits;
-    L->grid = (int)std::min<int64_t>(tasks, L->num_sms);
 }
 
 glq_status grow_workspace(glq_layer L, int64_t rows) {
     if (rows <= L->cap_rows) return GLQ_OK;
     cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return GLQ_ERR_CUDA;
-    cudaFree(L->d_xr);
-    cudaFree(L->d_info);
-    cudaFree(L->d_part);
-    L->d_xr = nullptr;
-    L->d_info = nullptr;
-    L->d_part = nullptr;
-    L->cap_rows = 0;
-    size_t dummy = 0;
-    int64_t dec_rows = std::min<int64_t>(rows, GLQ_DECODE_MAX_B);
-    glq_status st = dmalloc(&L->d_xr, (size_t)rows * L->n_pad * sizeof(__half), &dummy);
-    if (st == GLQ_OK) st = dmalloc(&L->d_info, (size_t)rows * sizeof(glq_rowinfo), &dummy);
-    if (st == GLQ_OK)
-        st = dmalloc(&L->d_part, (size_t)L->splits * dec_rows * L->m_pad * sizeof(float), &dummy);
-    if (st != GLQ_OK) return st;
+    free_workspace(L);
+    glq_status st = dmalloc(&L->wsp.xq, (size_t)rows * L->n_pad * 2, nullptr);
+    if (st == GLQ_OK && L->bpw == 3) st = dmalloc(&L->wsp.xh, (size_t)rows * L->n_pad * sizeof(__half), nullptr);
+    if (st == GLQ_OK) st = dmalloc(&L->wsp.info, (size_t)rows * sizeof(glq_rowinfo), nullptr);
+    const int max_splits = std::max(L->plan[0].splits, L->plan[1].splits);
+    if (st == GLQ_OK && max_splits > 1)
+        st = dmalloc(&L->wsp.part, (size_t)max_splits * rows * L->m_pad * sizeof(double), nullptr);
+    if (st == GLQ_OK) st = dmalloc(&L->wsp.z, (size_t)rows * L->m_pad * sizeof(float), nullptr);
+    if (st != GLQ_OK) {
+        free_workspace(L);
+        return st;
+    }
     L->cap_rows = rows;
     return GLQ_OK;
 }
 
-glq::GemvParams gemv_params(glq_layer L, const __half *xr, const glq_rowinfo *, int B) {
-    glq::GemvParams p{};
+}  // namespace
+
+namespace glq {
+
+GemvParams gemv_params(glq_layer L, const glq_workspace &w, const GemvPlan &plan, int nb) {
+    GemvParams p{};
     p.idx1 = L->d_idx1;
     p.idx2 = L->d_idx2;
     p.table = L->primary->d_table;
     p.table_words = L->primary->table_words;
-    p.fold = glq::FoldParams{L->primary->fold.nb, L->primary->fold.neg_base};
-    p.res8 = (L->bpw == 3) ? reinterpret_cast<const uint4 *>(L->d_r8) : nullptr;
-    p.xr = xr;
-    p.B = B;
+    p.fold = FoldParams{L->primary->fold.nb, L->primary->fold.neg_base};
+    p.res8 = (L->bpw == 3) ? reinterpret_cast<const uint4 *>(L->residual->d_fp16) : nullptr;
+    p.xq = w.xq;
+    p.xh = w.xh;
+    p.info = w.info;
+    p.B = nb;
     p.n_pad = (int)L->n_pad;
     p.KC = L->KC;
     p.RT = L->RT;
-    p.bands = L->bands;
-    p.splits = L->splits;
-    p.cps = L->cps;
-    p.rs_acc = L->bpw == 3 ? L->rs / GLQ_ACC_SCALE : L->rs;
-    p.partials = L->d_part;
+    p.bands = plan.bands;
+    p.splits = plan.splits;
+    p.cps = plan.cps;
+    p.rs_d = L->bpw == 3 ? 2.0 * (double)L->rs : (double)L->rs;
+    p.corr_mult = L->bpw == 4 ? 1.0 + (double)L->rs : 1.0;
+    p.ws = L->ws;
+    p.partials = w.part;
+    p.counters = w.cnt;
+    p.z = w.z;
     p.m_pad = (int)L->m_pad;
     p.err = L->d_err;
     return p;
 }
 
-}  // namespace
+cudaError_t run_decode(glq_layer L, const glq_workspace &w, const GemvPlan &plan, const void *x, bool x_bf16,
+                       void *y, int y_dtype, int nb, cudaStream_t s) {
+    RhtInParams pin{};
+    pin.x = x;
+    pin.x_bf16 = x_bf16 ? 1 : 0;
+    pin.n = (int)L->n;
+    pin.n_pad = (int)L->n_pad;
+    pin.B = nb;
+    pin.sign_bits = L->d_sin;
+    pin.plan = L->plan_n;
+    pin.xq = w.xq;
+    pin.xh = w.xh;
+    pin.info = w.info;
+    cudaError_t e = launch_rht_in(pin, s, true);
+    if (e != cudaSuccess) return e;
+    e = launch_gemv(gemv_params(L, w, plan, nb), L->bpw, plan.grid, s, true);
+    if (e != cudaSuccess) return e;
+    RhtOutParams pout{};
+    pout.m = (int)L->m;
+    pout.B = nb;
+    pout.z = w.z;
+    pout.z_ld = (int)L->m_pad;
+    pout.sign_bits = L->d_sout;
+    pout.plan = L->plan_m;
+    pout.y = y;
+    pout.y_dtype = y_dtype;
+    return launch_rht_out(pout, s, true);
+}
+
+}  // namespace glq
 
 extern "C" {
 
@@ -198,16 +207,6 @@ glq_status glq_codebook_upload(const uint16_t *host_fp16_bits, int32_t entries, 
     glq_codebook cb = new (std::nothrow) glq_codebook_s;
     if (!cb) return GLQ_ERR_OOM;
     cb->entries = entries;
-    if (entries == GLQ_CB8_ENTRIES) {
-        cb->host.assign(host_fp16_bits, host_fp16_bits + (size_t)entries * dim);
-        // the decode kernels hold columns 2,3,6,7 scaled by 16 in fp16
-        for (int e = 0; e < entries; ++e)
-            for (int j : {2, 3, 6, 7})
-                if (std::fabs(glq::half_bits_to_float(host_fp16_bits[e * dim + j])) >= 4094.0f) {
-                    delete cb;
-                    return GLQ_ERR_UNSUPPORTED;
-                }
-    }
     if (entries == GLQ_CB_ENTRIES) {
         int rc = glq::fold_table(host_fp16_bits, &cb->fold);
         if (rc != 0) {
@@ -297,11 +296,13 @@ glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *i
     L->residual = bpw == 4 ? primary : residual;
     L->ws = weight_scale;
     L->rs = bpw == 2 ? 0.f : resid_scale;
-    L->bn = make_blocks(n);
-    L->bm = make_blocks(m);
+    L->plan_n = glq::make_rht_plan((int)n);
+    L->plan_m = glq::make_rht_plan((int)m);
     cudaDeviceGetAttribute(&L->num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (L->num_sms <= 0) L->num_sms = 1;
-    plan_gemv(L);
+    L->plan[0] = glq::plan_gemv(L->RT, L->KC, L->num_sms, glq::gemv_warps(1));
+    L->plan[1] = glq::plan_gemv(L->RT, L->KC, L->num_sms, glq::gemv_warps(2));
+    const int max_bands = std::max(L->plan[0].bands, L->plan[1].bands);
 
     // fragment-native index streams (layout: glq_internal.h)
     const FoldedTable &F = primary->fold;
@@ -329,13 +330,6 @@ glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *i
         }
     }
     std::vector<uint32_t> sin_bits = pack_signs(s_in, n), sout_bits = pack_signs(s_out, m);
-    std::vector<uint16_t> r8;
-    if (bpw == 3) {
-        r8 = residual->host;
-        for (int e = 0; e < GLQ_CB8_ENTRIES; ++e)
-            for (int j : {2, 3, 6, 7}) r8[e * 8 + j] = glq::half_bits_times16(r8[e * 8 + j]);
-    }
-
     size_t total = 0;
     L->idx1_bytes = s1.size() * sizeof(uint16_t);
     L->idx2_bytes = bpw == 4 ? s2u16.size() * 2 : (bpw == 3 ? s2u8.size() : 0);
@@ -344,7 +338,7 @@ glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *i
     if (st == GLQ_OK) st = dmalloc(&L->d_sin, sin_bits.size() * 4, &total);
     if (st == GLQ_OK) st = dmalloc(&L->d_sout, sout_bits.size() * 4, &total);
     if (st == GLQ_OK) st = dmalloc(&L->d_err, sizeof(unsigned), &total);
-    if (st == GLQ_OK && bpw == 3) st = dmalloc(&L->d_r8, r8.size() * 2, &total);
+    if (st == GLQ_OK) st = dmalloc(&L->wsp.cnt, (size_t)max_bands * sizeof(unsigned), &total);
     if (st == GLQ_OK) {
         bool ok = cudaMemcpy(L->d_idx1, s1.data(), L->idx1_bytes, cudaMemcpyHostToDevice) == cudaSuccess;
         if (ok && bpw == 4)
@@ -356,8 +350,7 @@ glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *i
         ok = ok && cudaMemcpy(L->d_sout, sout_bits.data(), sout_bits.size() * 4, cudaMemcpyHostToDevice) ==
                        cudaSuccess;
         ok = ok && cudaMemset(L->d_err, 0, sizeof(unsigned)) == cudaSuccess;
-        if (ok && bpw == 3)
-            ok = cudaMemcpy(L->d_r8, r8.data(), r8.size() * 2, cudaMemcpyHostToDevice) == cudaSuccess;
+        ok = ok && cudaMemset(L->wsp.cnt, 0, (size_t)max_bands * sizeof(unsigned)) == cudaSuccess;
         if (!ok) st = GLQ_ERR_CUDA;
     }
     if (st != GLQ_OK) {
@@ -408,36 +401,14 @@ glq_status glq_linear(glq_layer L, const void *x_dev, glq_dtype x_dtype, void *y
     const size_t xe = 2, ye = y_dtype == GLQ_F32 ? 4 : 2;
     for (int64_t b0 = 0; b0 < B; b0 += GLQ_DECODE_MAX_B) {
         const int nb = (int)std::min<int64_t>(GLQ_DECODE_MAX_B, B - b0);
-        glq::RhtInParams pin{};
-        pin.x = static_cast<const char *>(x_dev) + (size_t)b0 * L->n * xe;
-        pin.x_bf16 = x_dtype == GLQ_BF16;
-        pin.n = (int)L->n;
-        pin.n_pad = (int)L->n_pad;
-        pin.B = nb;
-        pin.sign_bits = L->d_sin;
-        pin.blocks = L->bn;
-        pin.xr_h = L->d_xr;
-        pin.info = L->d_info;
-        if (glq::launch_rht_in(pin, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
-
-        glq::GemvParams pg = gemv_params(L, L->d_xr, L->d_info, nb);
-        if (glq::launch_gemv(pg, L->bpw, L->grid, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+        const void *x = static_cast<const char *>(x_dev) + (size_t)b0 * L->n * xe;
+        void *y = static_cast<char *>(y_dev) + (size_t)b0 * L->m * ye;
+        if (glq::run_decode(L, L->wsp, glq::plan_for(L, nb), x, x_dtype == GLQ_BF16, y, (int)y_dtype, nb, s) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return GLQ_ERR_CUDA;
+        }
         L->last_B = nb;
-
-        glq::RhtOutParams pout{};
-        pout.m = (int)L->m;
-        pout.m_pad = (int)L->m_pad;
-        pout.B = nb;
-        pout.partials = L->d_part;
-        pout.splits = L->splits;
-        pout.info = L->d_info;
-        pout.ws = L->ws;
-        pout.corr_mult = L->bpw == 4 ? 1.f + L->rs : 1.f;
-        pout.sign_bits = L->d_sout;
-        pout.blocks = L->bm;
-        pout.y = static_cast<char *>(y_dev) + (size_t)b0 * L->m * ye;
-        pout.y_dtype = (int)y_dtype;
-        if (glq::launch_rht_out(pout, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
     }
     return GLQ_OK;
 }
@@ -478,7 +449,7 @@ glq_status glq_rht_input(glq_layer L, const void *x_dev, glq_dtype x_dtype, floa
     p.n_pad = (int)L->n_pad;
     p.B = (int)B;
     p.sign_bits = L->d_sin;
-    p.blocks = L->bn;
+    p.plan = L->plan_n;
     p.xr_f32 = xr_dev;
     return glq::launch_rht_in(p, static_cast<cudaStream_t>(stream), false) == cudaSuccess ? GLQ_OK
                                                                                          : GLQ_ERR_CUDA;
@@ -495,12 +466,11 @@ glq_status glq_rht_output(glq_layer L, const float *z_dev, void *y_dev, glq_dtyp
     DeviceGuard guard(L->device);
     glq::RhtOutParams p{};
     p.m = (int)L->m;
-    p.m_pad = (int)L->m_pad;
     p.B = (int)B;
     p.z = z_dev;
     p.z_ld = (int)L->m;
     p.sign_bits = L->d_sout;
-    p.blocks = L->bm;
+    p.plan = L->plan_m;
     p.y = y_dev;
     p.y_dtype = (int)y_dtype;
     return glq::launch_rht_out(p, static_cast<cudaStream_t>(stream), false) == cudaSuccess ? GLQ_OK
@@ -511,8 +481,9 @@ glq_status glq_gemv_replay(glq_layer L, int64_t B, void *stream) {
     if (!L) return GLQ_ERR_INVALID_ARG;
     if (B < 1 || B > L->last_B) return GLQ_ERR_SHAPE;
     DeviceGuard guard(L->device);
-    glq::GemvParams pg = gemv_params(L, L->d_xr, L->d_info, (int)B);
-    return glq::launch_gemv(pg, L->bpw, L->grid, static_cast<cudaStream_t>(stream), false) == cudaSuccess
+    const glq::GemvPlan &plan = glq::plan_for(L, (int)B);
+    glq::GemvParams pg = glq::gemv_params(L, L->wsp, plan, (int)B);
+    return glq::launch_gemv(pg, L->bpw, plan.grid, static_cast<cudaStream_t>(stream), false) == cudaSuccess
                ? GLQ_OK
                : GLQ_ERR_CUDA;
 }

@@ -100,21 +100,6 @@ float half_bits_to_float(uint16_t h) {
     return f;
 }
 
-uint16_t half_bits_times16(uint16_t h) {
-    uint16_t sign = h & 0x8000u, exp = (h >> 10) & 0x1fu, mant = h & 0x3ffu;
-    if (exp == 0) {
-        if (mant == 0) return h;
-        // subnormal: value mant * 2^-24; times 16 = mant * 2^-20
-        uint32_t v = (uint32_t)mant << 4;  // in units of 2^-24, < 2^14
-        if (v < 0x400u) return (uint16_t)(sign | v);  // still subnormal
-        int e = 0;
-        while ((v >> (10 + e)) > 1) ++e;  // v in [2^(10+e), 2^(11+e))
-        // value = v 2^-24 = (v / 2^(10+e)) 2^(e-14): exponent field e + 1
-        return (uint16_t)(sign | ((uint16_t)(e + 1) << 10) | (uint16_t)((v >> e) & 0x3ffu));
-    }
-    return (uint16_t)(sign | ((uint16_t)(exp + 4) << 10) | mant);
-}
-
 int fold_table(const uint16_t *fp16_bits, FoldedTable *out) {
     // doubled coordinates of every entry, validated to lie in [-6, 6]
     std::vector<std::array<int8_t, 8>> ys(GLQ_CB_ENTRIES);
@@ -163,7 +148,7 @@ int fold_table(const uint16_t *fp16_bits, FoldedTable *out) {
     for (int e = 0; e < GLQ_CB_ENTRIES; ++e) {
         if (pos[e] >= 0) {
             uint32_t w = 0;
-            static const int shift[8] = {0, 16, 4, 20, 8, 24, 12, 28};
+            static const int shift[8] = {0, 8, 16, 24, 4, 12, 20, 28};
             for (int j = 0; j < 8; ++j) w |= (uint32_t)(ys[e][j] + 6) << shift[j];
             out->words[(size_t)pos[e]] = w;
             out->code[e] = (uint16_t)pos[e];

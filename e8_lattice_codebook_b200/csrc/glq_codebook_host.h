@@ -13,9 +13,6 @@ void build_e8_codebook(uint16_t *out_fp16_bits);
 // IEEE binary16 bits -> float (exact).
 float half_bits_to_float(uint16_t h);
 
-// Bits of 16 * h for a finite h with |16 h| <= 65504 (exact).
-uint16_t half_bits_times16(uint16_t h);
-
 struct FoldedTable {
     int nb = 0;                   // words in the on-chip table
     int neg_base = 0;             // code e >= nb reads words[e - neg_base] negated

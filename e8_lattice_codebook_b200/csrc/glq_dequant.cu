@@ -29,11 +29,11 @@ __global__ void dequant_kernel(DequantParams p) {
     const uint32_t *w1 = reinterpret_cast<const uint32_t *>(p.idx1 + slot);
     uint32_t code1 = (w1[s] >> (16 * hi)) & 0xFFFFu;
     float c1[8], c2[8];
-    unpack_exact(table_word(p.table, code1, p.fold), c1);
+    unpack_exact(table_word_global(p.table, code1, p.fold), c1);
     if (p.bpw == 4) {
         const uint32_t *w2 = reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint4 *>(p.idx2) + slot);
         uint32_t code2 = (w2[s] >> (16 * hi)) & 0xFFFFu;
-        unpack_exact(table_word(p.table, code2, p.fold), c2);
+        unpack_exact(table_word_global(p.table, code2, p.fold), c2);
     } else if (p.bpw == 3) {
         const uint8_t *b2 = reinterpret_cast<const uint8_t *>(reinterpret_cast<const uint2 *>(p.idx2) + slot);
         uint32_t i2 = b2[2 * s + hi];

@@ -20,44 +20,72 @@ struct FoldParams {
 };
 
 // Table word of code e (a 16-bit value), negation applied.
-// T is a shared-memory (or global) array of nibble words.
+// T is a shared-memory array of nibble words (address space shared).
 __device__ __forceinline__ uint32_t table_word(const uint32_t *T, uint32_t e, FoldParams f) {
-    bool neg = e >= (uint32_t)f.nb;
-    uint32_t pos = neg ? e - (uint32_t)f.neg_base : e;
-    uint32_t w = T[pos];
+    uint32_t w;
+    asm("{\n"
+        " .reg .pred p;\n"
+        " .reg .u32 c, a;\n"
+        " setp.ge.u32 p, %1, %2;\n"
+        " mov.u32 c, %1;\n"
+        " @p sub.u32 c, %1, %3;\n"
+        " shl.b32 a, c, 2;\n"
+        " add.u32 a, a, %4;\n"
+        " ld.shared.u32 %0, [a];\n"
+        " @p sub.u32 %0, 0xCCCCCCCC, %0;\n"
+        "}\n"
+        : "=r"(w)
+        : "r"(e), "r"((uint32_t)f.nb), "r"((uint32_t)f.neg_base),
+          "r"((uint32_t)__cvta_generic_to_shared(T)));
+    return w;
+}
+
+// The same lookup from a global-memory table (reference decode).
+__device__ __forceinline__ uint32_t table_word_global(const uint32_t *T, uint32_t e, FoldParams f) {
+    const bool neg = e >= (uint32_t)f.nb;
+    const uint32_t w = T[neg ? e - (uint32_t)f.neg_base : e];
     return neg ? 0xCCCCCCCCu - w : w;
 }
 
-// Unpacks a nibble word into four fp16x2 registers of exact subnormals:
-//   h[0] = (v0, v1) 2^-24,     h[1] = (v2, v3) 16 * 2^-24,
-//   h[2] = (v4, v5) 2^-24,     h[3] = (v6, v7) 16 * 2^-24,
-// with v_j = 2 x_j + 6 (layout: glq_internal.h).
-__device__ __forceinline__ void unpack_sub(uint32_t w, uint32_t h[4]) {
-    uint32_t w8 = w >> 8;
-    h[0] = w & 0x000F000Fu;
-    h[1] = w & 0x00F000F0u;
-    h[2] = w8 & 0x000F000Fu;
-    h[3] = w8 & 0x00F000F0u;
-}
+// The two A-fragment registers of one codeword for the integer MMA:
+// lo = (v0, v1, v2, v3), hi = (v4, v5, v6, v7) as u8, v = 2x + 6.
+__device__ __forceinline__ uint32_t nib_lo(uint32_t w) { return w & 0x0F0F0F0Fu; }
+__device__ __forceinline__ uint32_t nib_hi(uint32_t w) { return (w >> 4) & 0x0F0F0F0Fu; }
 
-// Exact float coordinates x0..x7 of a nibble word: the same unpack, then
-// x = h * 2^23 - 3 (x 2^19 for the h[1], h[3] pairs), exact in fp32.
+// Exact float coordinates x0..x7 of a table word (reference decode): the
+// same byte unpack, then x = v/2 - 3.
 __device__ __forceinline__ void unpack_exact(uint32_t w, float x[8]) {
-    uint32_t h[4];
-    unpack_sub(w, h);
+    const uint32_t lo = nib_lo(w), hi = nib_hi(w);
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        __half2 v = *reinterpret_cast<__half2 *>(&h[p]);
-        float mul = (p & 1) ? 524288.0f : 8388608.0f;  // 2^19 : 2^23
-        x[2 * p] = __low2float(v) * mul - 3.0f;
-        x[2 * p + 1] = __high2float(v) * mul - 3.0f;
+    for (int j = 0; j < 4; ++j) {
+        x[j] = 0.5f * (float)((lo >> (8 * j)) & 0xFFu) - 3.0f;
+        x[4 + j] = 0.5f * (float)((hi >> (8 * j)) & 0xFFu) - 3.0f;
     }
 }
 
 // ---------------------------------------------------------------------------
-// Warp MMA  D = A(16x16, f16, row) . B(16x8, f16, col) + D (f32)
+// Warp MMAs
 // ---------------------------------------------------------------------------
 
+// D(16x8, s32) += A(16x32, u8, row) . B(32x8, s8, col)
+__device__ __forceinline__ void mma_u8s8(int d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D(16x8, s32) += A(16x32, u8, row) . B(32x8, u8, col)
+__device__ __forceinline__ void mma_u8u8(int d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D(16x8, f32) += A(16x16, f16, row) . B(16x8, f16, col)
 __device__ __forceinline__ void mma_16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
@@ -93,6 +121,12 @@ __device__ __forceinline__ uint4 ldg_v4(const void *p) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
+}
+
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned *p, unsigned v) {
+    unsigned old;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
 }
 
 // ---------------------------------------------------------------------------

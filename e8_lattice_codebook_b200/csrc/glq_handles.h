@@ -1,8 +1,10 @@
 // glq_handles.h -- the opaque handle types of the C ABI (include/glq.h):
-// what a codebook and a layer own on the host and on the device.
+// what a codebook and a layer own on the host and on the device, and the
+// decode launch sequence shared by glq_linear and glq_linear_noalloc.
 #pragma once
 
 #include <cuda_fp16.h>
+#include <cuda_runtime.h>
 #include <stdint.h>
 
 #include <vector>
@@ -10,9 +12,9 @@
 #include "../../include/glq.h"
 #include "glq_codebook_host.h"
 #include "glq_internal.h"
+#include "glq_kernels.cuh"
 
 struct glq_codebook_s {
-    std::vector<uint16_t> host;  // fp16 bits (256-entry tables)
     int entries = 0;
     int device = 0;
     uint16_t *d_fp16 = nullptr;  // [entries][8]
@@ -20,6 +22,16 @@ struct glq_codebook_s {
     glq::FoldedTable fold;
     uint32_t *d_table = nullptr;  // table_words words
     int table_words = 0;          // nb rounded up to a multiple of 4
+};
+
+// Device buffers one decode call works in (B <= 16 tokens).
+struct glq_workspace {
+    uint8_t *xq = nullptr;        // [B][n_pad * 2] activations, high / low bytes per group
+    __half *xh = nullptr;         // [B][n_pad] fp16 activations (3 bpw only)
+    glq_rowinfo *info = nullptr;  // [B]
+    double *part = nullptr;       // [splits][B][m_pad] split-K partial sums
+    float *z = nullptr;           // [B][m_pad]
+    unsigned *cnt = nullptr;      // [bands], zero between calls
 };
 
 struct glq_layer_s {
@@ -32,17 +44,26 @@ struct glq_layer_s {
     void *d_idx2 = nullptr;
     size_t idx1_bytes = 0, idx2_bytes = 0;
     uint32_t *d_sin = nullptr, *d_sout = nullptr;
-    uint16_t *d_r8 = nullptr;  // 3 bpw residual table, columns 2,3,6,7 x 16
-    glq_blocks bn{}, bm{};
+    glq::RhtPlan plan_n{}, plan_m{};
     unsigned *d_err = nullptr;
-    // GEMV work split
-    int bands = 0, splits = 0, cps = 0, grid = 0;
-    // workspace
-    int64_t cap_rows = 0;  // rows of xr / info
-    int64_t last_B = 0;    // batch of the last decode slice (glq_gemv_replay)
-    __half *d_xr = nullptr;
-    glq_rowinfo *d_info = nullptr;
-    float *d_part = nullptr;
+    // GEMV work split for B <= 8 (plan[0]) and B <= 16 (plan[1])
+    glq::GemvPlan plan[2]{};
+    // workspace (sized by glq_layer_reserve / on first use)
+    int64_t cap_rows = 0;
+    int64_t last_B = 0;  // batch of the last decode slice (glq_gemv_replay)
+    glq_workspace wsp;
     size_t device_bytes = 0;
 };
 
+namespace glq {
+
+// Input RHT -> codebook GEMV -> output RHT for nb <= 16 tokens, in the
+// buffers of `w`, with the GEMV split plan (splits, cps, grid).
+cudaError_t run_decode(glq_layer L, const glq_workspace &w, const GemvPlan &plan, const void *x,
+                       bool x_bf16, void *y, int y_dtype, int nb, cudaStream_t s);
+
+GemvParams gemv_params(glq_layer L, const glq_workspace &w, const GemvPlan &plan, int nb);
+
+inline const GemvPlan &plan_for(glq_layer L, int nb) { return L->plan[nb > 8 ? 1 : 0]; }
+
+}  // namespace glq

@@ -27,20 +27,19 @@
 //     creation; glq_dequant_reference inverts nothing, it decodes codes.
 //
 //   * A table word packs the 8 coordinates as nibbles v = 2x + 6 in [0, 12]:
-//     bits 0-3 x0, 16-19 x1, 4-7 x2, 20-23 x3, 8-11 x4, 24-27 x5,
-//     12-15 x6, 28-31 x7.  A 16-bit half whose only set bits are a nibble
-//     at bits 0-3 is the fp16 subnormal v * 2^-24 (at bits 4-7: 16 v * 2^-24),
-//     so one AND per coordinate pair turns a word into exact MMA operands
-//     with no exponent offset.  Columns k with k mod 8 in {2,3,6,7} (the
-//     bits 4-7 nibbles) carry the factor 16, which the input RHT removes by
-//     storing those activations divided by 16.  The MMA then yields
-//     2^-24 sum_k v_k X_k with v = 2x + 6, so
-//         sum_k x_k X_k = 2^23 acc - 3 sum_k X_k,
-//     and the row-independent term 3 sum_k X_k is formed once per token in
-//     fp64.  (A large per-column offset would not do: the warp MMA's fp32
-//     accumulation truncates, and a bias common to every row becomes one
-//     sqrt(m)-sized spike after the output Hadamard.)  Negation is
-//     v -> 12 - v per nibble, i.e. word -> 0xCCCCCCCC - word.
+//     x0..x3 in the low nibbles of bytes 0..3, x4..x7 in the high nibbles.
+//     w & 0x0F0F0F0F and (w >> 4) & 0x0F0F0F0F are then exactly the two
+//     32-bit A-fragment registers (four u8 values each) one lane of the
+//     integer mma.m16n8k32 needs for one row: a whole codeword per lane.
+//     Negation is v -> 12 - v per nibble, i.e. word -> 0xCCCCCCCC - word.
+//
+//   * Activations for the integer MMA: per token the input RHT writes
+//     X = round(xr * 2^e) (|X| <= 2^14, e per token from max |xr|) as
+//     16 bytes per group of 8 columns: 8 high bytes (X >> 8, signed) then 8
+//     low bytes (X & 255).  The MMA accumulates sum v X exactly in int32
+//     (u8 x s8 and u8 x u8), and sum x X = (sum v X - 6 sum X) / 2 with the
+//     exact integer row sum sum X.  Exact integer accumulation makes the
+//     result independent of summation order and of the batch size.
 #pragma once
 
 #include <stdint.h>
@@ -66,13 +65,16 @@
 #define GLQ_NOALLOC_SCRATCH_BYTES (8u << 20)
 #endif
 
-// largest Hadamard block handled by the one-CTA-per-row RHT kernels
+// largest row of the RHT kernels (8 parts of 4096 in one cluster)
 #define GLQ_RHT_MAX_N 32768
 #define GLQ_MAX_BLOCKS 32
+#define GLQ_RHT_SEG 4096
+#define GLQ_RHT_THREADS 1024
+#define GLQ_RHT_MAX_PARTS 8
+#define GLQ_RHT_MAX_PIECES 32
 
-// the nibble decode: operand = v * 2^-24 (x 16 on columns k mod 8 in {2,3,6,7})
-#define GLQ_ACC_SCALE 8388608.0f  // 2^23: sum x X = 2^23 acc - 3 sum X
-#define GLQ_NIB_OFFSET 3.0        // x = v/2 - 3
+// x = v/2 - 3 for a table nibble v
+#define GLQ_NIB_OFFSET 6  // sum x X = (sum v X - 6 sum X) / 2
 
 // device error word bits
 #define GLQ_DEVERR_TIMEOUT 1u
@@ -85,11 +87,10 @@ struct glq_blocks {
     float inv_sqrt[GLQ_MAX_BLOCKS];  // 1/sqrt(size), computed on the host in double
 };
 
-// Row info written by the input RHT for every token: the activations X are
-// xr * 2^scale_exp (stored /16 on columns k mod 8 in {2,3,6,7});
-// inv_scale = 2^-scale_exp; corr = 3 sum_k X_k (fp64).
+// Row info written by the input RHT for every token: X = round(xr 2^e),
+// inv_scale = 2^-e, sum_x = exact sum over the row of X.
 struct glq_rowinfo {
-    double corr;
+    long long sum_x;
     float inv_scale;
     float pad;
 };

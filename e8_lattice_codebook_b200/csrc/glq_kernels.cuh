@@ -11,30 +11,42 @@
 
 namespace glq {
 
+// One piece of a part of the RHT row plan: `len` values at row offset
+// `off`, belonging to a Hadamard block of size K split over C parts (this is
+// part q; the block's parts are cluster ranks rank0 .. rank0+C-1).
+struct RhtPiece {
+    int off, len, K, C, q, rank0;
+    float norm;  // 1/sqrt(K), computed on the host in double
+};
+
+struct RhtPlan {
+    int parts, npieces, clustered;
+    int first_piece[GLQ_RHT_MAX_PARTS + 1];
+    RhtPiece piece[GLQ_RHT_MAX_PIECES];
+};
+
+RhtPlan make_rht_plan(int N);
+
 struct RhtInParams {
     const void *x;  // [B][n] fp16 / bf16
     int x_bf16;
     int n, n_pad;
     int B;
     const uint32_t *sign_bits;  // bit k set: S_in[k] = -1
-    glq_blocks blocks;
-    __half *xr_h;          // [B][n_pad] scaled fp16 (product path) or null
-    glq_rowinfo *info;     // [B] (product path) or null
-    float *xr_f32;         // [B][n] unscaled fp32 (test entry point) or null
+    RhtPlan plan;
+    uint8_t *xq;        // [B][n_pad/8][16]: high bytes, low bytes of X (product path)
+    __half *xh;         // [B][n_pad] fp16 X (3 bpw residual stage) or null
+    glq_rowinfo *info;  // [B] (product path)
+    float *xr_f32;      // [B][n] unscaled fp32 (test entry point) or null
 };
 
 struct RhtOutParams {
-    int m, m_pad, B;
-    const float *partials;  // [splits][B][m_pad] (decode path) or null
-    int splits;
-    const float *z;         // [B][z_ld] fp32 (tensor path / test entry point) or null
+    int m, B;
+    const float *z;  // [B][z_ld] fp32
     int z_ld;
-    const glq_rowinfo *info;  // used with partials
-    float ws;
-    float corr_mult;
     const uint32_t *sign_bits;  // bit r set: S_out[r] = -1
-    glq_blocks blocks;
-    void *y;  // [B][m]
+    RhtPlan plan;
+    void *y;      // [B][m]
     int y_dtype;  // 0 f16, 1 bf16, 2 f32
 };
 
@@ -44,13 +56,18 @@ struct GemvParams {
     const uint32_t *table; // folded nibble table (global), table_words (multiple of 4)
     int table_words;
     FoldParams fold;
-    const uint4 *res8;     // 3 bpw: [256] x 8 fp16, columns 2,3,6,7 scaled by 16
-    const __half *xr;      // [B][n_pad]
+    const uint4 *res8;     // 3 bpw: [256] x 8 fp16
+    const uint8_t *xq;     // [B][n_pad/8][16]
+    const __half *xh;      // [B][n_pad] (3 bpw)
+    const glq_rowinfo *info;
     int B, n_pad, KC, RT;
     int bands, splits, cps;
-    float rs_acc;          // residual weight of acc2 in the partial sum: rs (4 bpw),
-                           // rs * 2^-23 (3 bpw: acc2 holds unscaled fp16 products)
-    float *partials;       // [splits][B][m_pad]
+    double rs_d;           // weight of the residual sum in a partial: rs (4 bpw) or 2 rs (3 bpw)
+    double corr_mult;      // (1 + rs) for 4 bpw, 1 otherwise
+    float ws;
+    double *partials;      // [splits][B][m_pad]
+    unsigned *counters;    // [bands], zero between launches
+    float *z;              // [B][m_pad]
     int m_pad;
     unsigned *err;
 };
@@ -89,10 +106,18 @@ inline cudaError_t launch_ex(const void *fn, dim3 grid, dim3 block, size_t smem,
 cudaError_t launch_rht_in(const RhtInParams &p, cudaStream_t s, bool pdl);
 cudaError_t launch_rht_out(const RhtOutParams &p, cudaStream_t s, bool pdl);
 cudaError_t launch_gemv(const GemvParams &p, int bpw, int grid, cudaStream_t s, bool pdl);
+
+// GEMV work split: bands of row tiles x splits of the chunk range.
+struct GemvPlan {
+    int bands, splits, cps, grid;
+};
+GemvPlan plan_gemv(int RT, int KC, int num_sms, int warps);
 cudaError_t launch_dequant(const DequantParams &p, cudaStream_t s);
 
-constexpr int GEMV_WARPS = 16;
-constexpr int GEMV_PREFETCH = 4;
+// warps per GEMV CTA (one 16-row tile each): 24 for one 8-column MMA tile
+// (B <= 8), 16 for two (B <= 16, more live registers per lane)
+__host__ __device__ constexpr int gemv_warps(int nt) { return nt == 1 ? 24 : 16; }
+constexpr int GEMV_PREFETCH = 2;
 size_t gemv_smem_bytes(int table_words, int bpw);
 
 }  // namespace glq

@@ -23,11 +23,11 @@
 #include "glq_internal.h"
 #include "glq_kernels.cuh"
 
-// The scratch array: activations (fp16), per-token row info and split-K
-// partial sums of one call.  Every GPU that loads the library holds it
-// until the process exits.  Calls share it: two calls whose kernels overlap
-// on the GPU (different streams, or different layers without ordering)
-// race on it.
+// The scratch array: activations, per-token row info, the output of the
+// GEMV, the per-band counters and the split-K partial sums of one call.
+// Every GPU that loads the library holds it until the process exits.  Calls
+// share it: two calls whose kernels overlap on the GPU (different streams,
+// or different layers without ordering) race on it.
 static __device__ __align__(256) unsigned char g_glq_noalloc_scratch[GLQ_NOALLOC_SCRATCH_BYTES];
 
 namespace {
@@ -78,84 +78,47 @@ extern "C" glq_status glq_linear_noalloc(glq_layer L, const void *x_dev, glq_dty
         cudaGetLastError();
         return GLQ_ERR_CUDA;
     }
-    glq_status st = GLQ_OK;
     void *base = nullptr;
-    st = scratch_address(L->device, &base);
+    glq_status st = scratch_address(L->device, &base);
 
-    // carve the array: xr [B][n_pad] fp16 | info [B] | partials [splits][B][m_pad]
-    const size_t xr_bytes = align256((size_t)B * L->n_pad * sizeof(__half));
-    const size_t info_bytes = align256((size_t)B * sizeof(glq_rowinfo));
-    const size_t per_split = (size_t)B * L->m_pad * sizeof(float);
-    int splits = L->splits, cps = L->cps;
+    // carve the array: xq | xh | info | z | counters | partials
+    const size_t xq_b = align256((size_t)B * L->n_pad * 2);
+    const size_t xh_b = L->bpw == 3 ? align256((size_t)B * L->n_pad * sizeof(__half)) : 0;
+    const size_t info_b = align256((size_t)B * sizeof(glq_rowinfo));
+    const size_t z_b = align256((size_t)B * L->m_pad * sizeof(float));
+    glq::GemvPlan plan = glq::plan_for(L, (int)B);
+    const size_t cnt_b = align256((size_t)plan.bands * sizeof(unsigned));
+    const size_t fixed = xq_b + xh_b + info_b + z_b + cnt_b;
+    const size_t per_split = (size_t)B * L->m_pad * sizeof(double);
     if (st == GLQ_OK) {
-        if (xr_bytes + info_bytes + per_split > GLQ_NOALLOC_SCRATCH_BYTES) {
-            st = GLQ_ERR_SHAPE;  // even one split does not fit the array
+        if (fixed > GLQ_NOALLOC_SCRATCH_BYTES) {
+            st = GLQ_ERR_SHAPE;  // the activations and outputs alone do not fit
         } else {
-            // narrow the split-K plan until its partial sums fit
-            const size_t room = GLQ_NOALLOC_SCRATCH_BYTES - xr_bytes - info_bytes;
-            while ((size_t)splits * per_split > room) {
-                cps = cps + 1;
-                splits = (L->KC + cps - 1) / cps;
+            // narrow the split-K plan until its partial sums fit (one split
+            // needs none: the GEMV then writes z directly)
+            const size_t room = GLQ_NOALLOC_SCRATCH_BYTES - fixed;
+            while (plan.splits > 1 && (size_t)plan.splits * per_split > room) {
+                plan.cps = plan.cps + 1;
+                plan.splits = (L->KC + plan.cps - 1) / plan.cps;
             }
+            plan.grid = (int)std::min<int64_t>((int64_t)plan.bands * plan.splits, L->num_sms);
         }
     }
     if (st == GLQ_OK) {
         char *p = static_cast<char *>(base);
-        __half *xr = reinterpret_cast<__half *>(p);
-        glq_rowinfo *info = reinterpret_cast<glq_rowinfo *>(p + xr_bytes);
-        float *part = reinterpret_cast<float *>(p + xr_bytes + info_bytes);
+        glq_workspace w;
+        w.xq = reinterpret_cast<uint8_t *>(p);
+        w.xh = L->bpw == 3 ? reinterpret_cast<__half *>(p + xq_b) : nullptr;
+        w.info = reinterpret_cast<glq_rowinfo *>(p + xq_b + xh_b);
+        w.z = reinterpret_cast<float *>(p + xq_b + xh_b + info_b);
+        w.cnt = reinterpret_cast<unsigned *>(p + xq_b + xh_b + info_b + z_b);
+        w.part = plan.splits > 1 ? reinterpret_cast<double *>(p + fixed) : nullptr;
         cudaStream_t s = static_cast<cudaStream_t>(stream);
-        const int nb = (int)B;
-
-        glq::RhtInParams pin{};
-        pin.x = x_dev;
-        pin.x_bf16 = x_dtype == GLQ_BF16;
-        pin.n = (int)L->n;
-        pin.n_pad = (int)L->n_pad;
-        pin.B = nb;
-        pin.sign_bits = L->d_sin;
-        pin.blocks = L->bn;
-        pin.xr_h = xr;
-        pin.info = info;
-
-        glq::GemvParams pg{};
-        pg.idx1 = L->d_idx1;
-        pg.idx2 = L->d_idx2;
-        pg.table = L->primary->d_table;
-        pg.table_words = L->primary->table_words;
-        pg.fold = glq::FoldParams{L->primary->fold.nb, L->primary->fold.neg_base};
-        pg.res8 = (L->bpw == 3) ? reinterpret_cast<const uint4 *>(L->d_r8) : nullptr;
-        pg.xr = xr;
-        pg.B = nb;
-        pg.n_pad = (int)L->n_pad;
-        pg.KC = L->KC;
-        pg.RT = L->RT;
-        pg.bands = L->bands;
-        pg.splits = splits;
-        pg.cps = cps;
-        pg.rs_acc = L->bpw == 3 ? L->rs / GLQ_ACC_SCALE : L->rs;
-        pg.partials = part;
-        pg.m_pad = (int)L->m_pad;
-        pg.err = L->d_err;
-        const int grid = (int)std::min<int64_t>((int64_t)L->bands * splits, L->num_sms);
-
-        glq::RhtOutParams pout{};
-        pout.m = (int)L->m;
-        pout.m_pad = (int)L->m_pad;
-        pout.B = nb;
-        pout.partials = part;
-        pout.splits = splits;
-        pout.info = info;
-        pout.ws = L->ws;
-        pout.corr_mult = L->bpw == 4 ? 1.f + L->rs : 1.f;
-        pout.sign_bits = L->d_sout;
-        pout.blocks = L->bm;
-        pout.y = y_dev;
-        pout.y_dtype = (int)y_dtype;
-
-        if (glq::launch_rht_in(pin, s, true) != cudaSuccess ||
-            glq::launch_gemv(pg, L->bpw, grid, s, true) != cudaSuccess ||
-            glq::launch_rht_out(pout, s, true) != cudaSuccess) {
+        // the band counters must start at zero (the array keeps whatever the
+        // previous call, of any layer, left there)
+        if (cudaMemsetAsync(w.cnt, 0, (size_t)plan.bands * sizeof(unsigned), s) != cudaSuccess ||
+            glq::run_decode(L, w, plan, x_dev, x_dtype == GLQ_BF16, y_dev, (int)y_dtype, (int)B, s) !=
+                cudaSuccess) {
             cudaGetLastError();
             st = GLQ_ERR_CUDA;
         }

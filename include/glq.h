@@ -99,8 +99,7 @@ GLQ_API glq_status glq_e8_codebook(uint16_t *out_fp16_bits);
  * A 65,536-entry table must hold values k/2 with |k| <= 6 whose
  *   negation-folded size fits the on-chip table (true for glq_e8_codebook's
  *   table); otherwise GLQ_ERR_UNSUPPORTED.  A 256-entry table may hold any
- *   finite fp16 values of magnitude below 4094 (the kernels keep coordinates
- *   2, 3, 6, 7 scaled by 16 in fp16); otherwise GLQ_ERR_UNSUPPORTED.
+ *   finite fp16 values.
  * out: receives a library-owned handle; release with glq_codebook_destroy
  *   after every layer that uses it has been destroyed.
  * Errors: GLQ_ERR_INVALID_ARG (NULL pointers, non-finite values),
