@@ -1,6 +1,8 @@
 // glq_api.cu -- the C ABI of glq-b200 (include/glq.h): argument checks,
 // the host-side re-layout of index arrays into the kernels' fragment-native
 // streams, device memory ownership and kernel dispatch.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -73,8 +75,16 @@ void free_workspace(glq_layer L) {
     L->cap_rows = 0;
 }
 
+void free_prefill_ws(glq_layer L) {
+    cudaFree(L->pws.xh);
+    cudaFree(L->pws.info);
+    cudaFree(L->pws.z);
+    L->pws = glq_prefill_ws{};
+}
+
 void free_layer(glq_layer L) {
     if (!L) return;
+    free_prefill_ws(L);
     cudaFree(L->d_idx1);
     cudaFree(L->d_idx2);
     cudaFree(L->d_sin);
@@ -102,6 +112,106 @@ glq_status grow_workspace(glq_layer L, int64_t rows) {
         return st;
     }
     L->cap_rows = rows;
+    return GLQ_OK;
+}
+
+glq_status grow_prefill_ws(glq_layer L, int64_t rows) {
+    if (rows <= L->pws.cap) return GLQ_OK;
+    if (cudaDeviceSynchronize() != cudaSuccess) return GLQ_ERR_CUDA;
+    free_prefill_ws(L);
+    glq_status st = dmalloc(&L->pws.xh, (size_t)rows * L->n_pad * sizeof(__half), nullptr);
+    if (st == GLQ_OK) st = dmalloc(&L->pws.info, (size_t)rows * sizeof(glq_rowinfo), nullptr);
+    if (st == GLQ_OK) st = dmalloc(&L->pws.z, (size_t)rows * L->m_pad * sizeof(float), nullptr);
+    if (st != GLQ_OK) {
+        free_prefill_ws(L);
+        return st;
+    }
+    L->pws.cap = rows;
+    return GLQ_OK;
+}
+
+// TMA descriptor of the fp16 activations [B][n_pad]: boxes of 64 columns x
+// 256 tokens, 128-byte swizzle, zero fill past the last token.
+bool encode_x_map(CUtensorMap *map, const __half *xh, int64_t n_pad, int64_t B) {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        cudaDriverEntryPointQueryResult q;
+        void *fn = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn) {
+            cudaGetLastError();
+            return false;
+        }
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const cuuint64_t dims[2] = {(cuuint64_t)n_pad, (cuuint64_t)B};
+    const cuuint64_t strides[1] = {(cuuint64_t)n_pad * sizeof(__half)};
+    const cuuint32_t box[2] = {64, 256};
+    const cuuint32_t estr[2] = {1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half *>(xh), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor-core path for B > 16 tokens: input RHT (fp16 activations), tcgen05
+// GEMM with the dequantising producer, output RHT.
+glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_dtype, int64_t B, cudaStream_t s) {
+    glq_status st = grow_prefill_ws(L, B);
+    if (st != GLQ_OK) return st;
+    for (int64_t b0 = 0; b0 < B;) {
+        const int nb = (int)std::min<int64_t>(B - b0, 65535);  // RHT grid.y limit
+        glq::RhtInParams pin{};
+        pin.x = static_cast<const char *>(x) + (size_t)b0 * L->n * 2;
+        pin.x_bf16 = x_bf16 ? 1 : 0;
+        pin.n = (int)L->n;
+        pin.n_pad = (int)L->n_pad;
+        pin.B = nb;
+        pin.sign_bits = L->d_sin;
+        pin.plan = L->plan_n;
+        pin.xh = L->pws.xh + (size_t)b0 * L->n_pad;
+        pin.info = L->pws.info + b0;
+        pin.xh_only = 1;
+        if (glq::launch_rht_in(pin, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+        b0 += nb;
+    }
+    CUtensorMap xmap;
+    if (!encode_x_map(&xmap, L->pws.xh, L->n_pad, B)) return GLQ_ERR_CUDA;
+    glq::PrefillParams pp{};
+    pp.idx1 = L->d_idx1;
+    pp.idx2 = L->d_idx2;
+    pp.cb_f16 = L->primary->d_table_f16;
+    pp.fold = glq::FoldParams{L->primary->fold.nb, L->primary->fold.neg_base};
+    pp.res8 = L->bpw == 3 ? reinterpret_cast<const uint4 *>(L->residual->d_fp16) : nullptr;
+    pp.bpw = L->bpw;
+    const __half2 rs2 = __floats2half2_rn(L->rs, L->rs);
+    pp.rs_h2 = *reinterpret_cast<const uint32_t *>(&rs2);
+    pp.info = L->pws.info;
+    pp.ws = L->ws;
+    pp.z = L->pws.z;
+    pp.B = (int)B;
+    pp.m_pad = (int)L->m_pad;
+    pp.KC = L->KC;
+    pp.RT = L->RT;
+    const int tiles_m = (int)((L->m_pad + 127) / 128);
+    pp.tiles_tok = (int)((B + glq::prefill_tile_tokens() - 1) / glq::prefill_tile_tokens());
+    pp.ntiles = tiles_m * pp.tiles_tok;
+    pp.err = L->d_err;
+    const int grid = std::min(pp.ntiles, L->num_sms);
+    if (glq::launch_prefill(pp, xmap, grid, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+    for (int64_t b0 = 0; b0 < B;) {
+        const int nb = (int)std::min<int64_t>(B - b0, 65535);
+        glq::RhtOutParams pout{};
+        pout.m = (int)L->m;
+        pout.B = nb;
+        pout.z = L->pws.z + (size_t)b0 * L->m_pad;
+        pout.z_ld = (int)L->m_pad;
+        pout.sign_bits = L->d_sout;
+        pout.plan = L->plan_m;
+        pout.y = static_cast<char *>(y) + (size_t)b0 * L->m * (y_dtype == GLQ_F32 ? 4 : 2);
+        pout.y_dtype = y_dtype;
+        if (glq::launch_rht_out(pout, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+        b0 += nb;
+    }
     return GLQ_OK;
 }
 
@@ -227,6 +337,23 @@ glq_status glq_codebook_upload(const uint16_t *host_fp16_bits, int32_t entries, 
     if (st == GLQ_OK && cudaMemcpy(cb->d_fp16, host_fp16_bits, bytes, cudaMemcpyHostToDevice) != cudaSuccess)
         st = GLQ_ERR_CUDA;
     if (st == GLQ_OK && cb->folded) {
+        // the folded table as fp16 codewords (x = v/2 - 3, exact) for the
+        // tensor-core path's gathers
+        std::vector<uint16_t> f16((size_t)cb->table_words * 8, 0);
+        for (int i = 0; i < cb->fold.nb; ++i) {
+            const uint32_t w = cb->fold.words[(size_t)i];
+            static const int shift[8] = {0, 8, 16, 24, 4, 12, 20, 28};
+            for (int j = 0; j < 8; ++j) {
+                const int y2 = (int)((w >> shift[j]) & 0xF) - 6;  // 2x
+                f16[(size_t)i * 8 + j] = glq::half_bits_of_half_integer(y2);
+            }
+        }
+        st = dmalloc(&cb->d_table_f16, f16.size() * 2, nullptr);
+        if (st == GLQ_OK && cudaMemcpy(cb->d_table_f16, f16.data(), f16.size() * 2, cudaMemcpyHostToDevice) !=
+                                cudaSuccess)
+            st = GLQ_ERR_CUDA;
+    }
+    if (st == GLQ_OK && cb->folded) {
         st = dmalloc(&cb->d_table, (size_t)cb->table_words * 4, nullptr);
         if (st == GLQ_OK && cudaMemcpy(cb->d_table, cb->fold.words.data(), (size_t)cb->table_words * 4,
                                        cudaMemcpyHostToDevice) != cudaSuccess)
@@ -235,6 +362,7 @@ glq_status glq_codebook_upload(const uint16_t *host_fp16_bits, int32_t entries, 
     if (st != GLQ_OK) {
         cudaFree(cb->d_fp16);
         cudaFree(cb->d_table);
+        cudaFree(cb->d_table_f16);
         delete cb;
         return st;
     }
@@ -247,6 +375,7 @@ glq_status glq_codebook_destroy(glq_codebook cb) {
     DeviceGuard guard(cb->device);
     cudaFree(cb->d_fp16);
     cudaFree(cb->d_table);
+    cudaFree(cb->d_table_f16);
     delete cb;
     return GLQ_OK;
 }
@@ -395,9 +524,10 @@ glq_status glq_linear(glq_layer L, const void *x_dev, glq_dtype x_dtype, void *y
     if (B == 0) return GLQ_OK;
     if (!x_dev || !y_dev) return GLQ_ERR_INVALID_ARG;
     DeviceGuard guard(L->device);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (B > GLQ_DECODE_MAX_B) return run_prefill(L, x_dev, x_dtype == GLQ_BF16, y_dev, (int)y_dtype, B, s);
     glq_status st = grow_workspace(L, std::min<int64_t>(B, GLQ_DECODE_MAX_B));
     if (st != GLQ_OK) return st;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t xe = 2, ye = y_dtype == GLQ_F32 ? 4 : 2;
     for (int64_t b0 = 0; b0 < B; b0 += GLQ_DECODE_MAX_B) {
         const int nb = (int)std::min<int64_t>(GLQ_DECODE_MAX_B, B - b0);

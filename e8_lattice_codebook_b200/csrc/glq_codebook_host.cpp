@@ -44,6 +44,8 @@ void grow(int depth, int parity, int budget, int ysum, Point &cur, std::vector<P
     }
 }
 
+}  // namespace
+
 uint16_t half_bits_of_half_integer(int y2) {
     // exact binary16 of y2 / 2 for |y2| <= 12
     if (y2 == 0) return 0;
@@ -56,8 +58,6 @@ uint16_t half_bits_of_half_integer(int y2) {
     uint16_t mant = (uint16_t)((a - (1 << e)) << (10 - e));
     return (uint16_t)(sign | (exp_field << 10) | mant);
 }
-
-}  // namespace
 
 void build_e8_codebook(uint16_t *out_fp16_bits) {
     std::vector<Point> pts;

@@ -10,6 +10,9 @@ namespace glq {
 // The library's 65,536 x 8 E8 shell codebook as fp16 bit patterns.
 void build_e8_codebook(uint16_t *out_fp16_bits);
 
+// Exact binary16 bits of y2 / 2 for an integer |y2| <= 12.
+uint16_t half_bits_of_half_integer(int y2);
+
 // IEEE binary16 bits -> float (exact).
 float half_bits_to_float(uint16_t h);
 

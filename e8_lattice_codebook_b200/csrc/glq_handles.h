@@ -22,6 +22,15 @@ struct glq_codebook_s {
     glq::FoldedTable fold;
     uint32_t *d_table = nullptr;  // table_words words
     int table_words = 0;          // nb rounded up to a multiple of 4
+    uint4 *d_table_f16 = nullptr; // the folded table as fp16 codewords [nb][8] (tensor-core path)
+};
+
+// Device buffers of the tensor-core path (B > 16 tokens).
+struct glq_prefill_ws {
+    int64_t cap = 0;
+    __half *xh = nullptr;         // [cap][n_pad]
+    glq_rowinfo *info = nullptr;  // [cap]
+    float *z = nullptr;           // [cap][m_pad]
 };
 
 // Device buffers one decode call works in (B <= 16 tokens).
@@ -52,6 +61,7 @@ struct glq_layer_s {
     int64_t cap_rows = 0;
     int64_t last_B = 0;  // batch of the last decode slice (glq_gemv_replay)
     glq_workspace wsp;
+    glq_prefill_ws pws;
     size_t device_bytes = 0;
 };
 

@@ -1,6 +1,7 @@
 // glq_kernels.cuh -- kernel parameter blocks and launchers of glq-b200.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -38,6 +39,7 @@ struct RhtInParams {
     __half *xh;         // [B][n_pad] fp16 X (3 bpw residual stage) or null
     glq_rowinfo *info;  // [B] (product path)
     float *xr_f32;      // [B][n] unscaled fp32 (test entry point) or null
+    int xh_only;        // tensor-core path: write xh = fp16(xr 2^e) only (no xq, no sum)
 };
 
 struct RhtOutParams {
@@ -69,6 +71,22 @@ struct GemvParams {
     unsigned *counters;    // [bands], zero between launches
     float *z;              // [B][m_pad]
     int m_pad;
+    unsigned *err;
+};
+
+struct PrefillParams {
+    const uint4 *idx1;       // [RT][KC][32] 16 B, fragment-native codes
+    const void *idx2;        // 4 bpw: 16 B / 3 bpw: 8 B per slot
+    const uint4 *cb_f16;     // folded E8 table as fp16 codewords [nb][8]
+    FoldParams fold;
+    const uint4 *res8;       // 3 bpw: [256][8] fp16
+    int bpw;
+    uint32_t rs_h2;          // residual scale as fp16x2
+    const glq_rowinfo *info; // [B]: inv_scale per token
+    float ws;
+    float *z;                // [B][m_pad]
+    int B, m_pad, KC, RT;
+    int tiles_tok, ntiles;
     unsigned *err;
 };
 
@@ -113,6 +131,9 @@ struct GemvPlan {
 };
 GemvPlan plan_gemv(int RT, int KC, int num_sms, int warps);
 cudaError_t launch_dequant(const DequantParams &p, cudaStream_t s);
+cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &xmap, int grid, cudaStream_t s, bool pdl);
+size_t prefill_smem_bytes();
+int prefill_tile_tokens();
 
 // warps per GEMV CTA (one 16-row tile each): 24 for one 8-column MMA tile
 // (B <= 8), 16 for two (B <= 16, more live registers per lane)

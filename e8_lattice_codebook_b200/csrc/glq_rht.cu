@@ -308,8 +308,19 @@ __global__ void __launch_bounds__(THREADS) rht_in_kernel(RhtInParams p) {
         frexpf(rowmax, &e);  // rowmax < 2^e
         scale = ldexpf(1.f, 14 - e);
     }
-    uint8_t *xq = p.xq + (size_t)b * p.n_pad * 2;  // per group: 8 high bytes, 8 low bytes
     __half *xh = p.xh ? p.xh + (size_t)b * p.n_pad : nullptr;
+    if (p.xh_only) {  // tensor-core path: fp16 activations, one rounding
+#pragma unroll
+        for (int r = 0; r < VPT; ++r)
+            if (o.idx[r] >= 0) xh[o.idx[r]] = __float2half_rn(o.v[r] * scale);
+        if (part == 0) {
+            for (int k = p.n + threadIdx.x; k < p.n_pad; k += THREADS) xh[k] = __float2half(0.f);
+            if (threadIdx.x == 0) p.info[b] = glq_rowinfo{0, 1.f / scale, 0.f};
+        }
+        if (p.plan.clustered) cluster.sync();  // peers may still read this CTA's shared memory
+        return;
+    }
+    uint8_t *xq = p.xq + (size_t)b * p.n_pad * 2;  // per group: 8 high bytes, 8 low bytes
     long long sum = 0;
 #pragma unroll
     for (int r = 0; r < VPT; ++r) {

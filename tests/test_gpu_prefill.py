@@ -1,0 +1,98 @@
+"""GPU parity of the tensor-core (prefill, B > 16 tokens) path of glq_linear
+against the fp64 oracle, through the C ABI.
+
+The path rounds the rotated activations and the reconstructed codewords
+(cb1 + rs cb2) to fp16 once each and accumulates in fp32 on the tensor
+cores, so it keeps the same bound as the decode path:
+max |y - y_oracle| <= 2e-3 (||y_oracle||_inf + 1).
+
+* small shapes: every token of batches that span one and several 512-token
+  tiles, with ragged row, column and token tails, all three bit rates;
+* full-size prefill workload at its largest batch: sampled tokens, the last
+  (ragged) token tile included;
+* run-to-run determinism, and per-token independence of the batch size
+  within the tensor-core path.
+"""
+import numpy as np
+import pytest
+
+import glq_inputs as gi
+from gpu_helpers import Device, production_tolerance, to_torch_x, tolerance
+from oracle import glq_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return Device()
+
+
+def oracle_y(L, xbits, xdt):
+    return orc.linear(L.m, L.n, L.bpw, L.idx1, L.idx2, L.weight_scale, L.resid_scale, L.s_in,
+                      L.s_out, xbits, xdt == "bf16", cb2=L.cb2_f16)
+
+
+PREFILL_SMALL = [  # m, n, bpw, B, x dtype
+    (16, 128, 2, 17, "f16"),        # one row tile, one column chunk, smallest prefill batch
+    (272, 264, 4, 40, "bf16"),      # ragged rows (3 row tiles) and columns
+    (1000, 968, 3, 33, "f16"),      # 8 row tiles, 3 bpw residual table
+    (136, 1024, 2, 600, "bf16"),    # second token tile has one live accumulator
+    (264, 520, 4, 777, "f16"),      # second token tile: one full and one ragged accumulator
+    (200, 2560, 3, 300, "bf16"),    # long K (40 steps), ragged accumulator
+    (8, 8, 4, 20, "f16"),           # tiny layer, most of the tile is padding
+    (1024, 1024, 2, 1100, "bf16"),  # three token tiles
+]
+
+
+@pytest.mark.parametrize("m,n,bpw,B,xdt", PREFILL_SMALL)
+def test_prefill_small_all_tokens(dev, m, n, bpw, B, xdt):
+    L = gi.make_layer(m * 11 + n, 7, m, n, bpw)
+    xb = gi.make_x(m * 11 + n, 7, B, n, xdt)
+    lay = dev.layer(L)
+    x = to_torch_x(xb, xdt)
+    y = lay(x, out_dtype=torch.float32).cpu().numpy().astype(np.float64)
+    ref = oracle_y(L, xb, xdt)
+    err = np.max(np.abs(y - ref))
+    print(f"\nPREFILL {m}x{n} bpw {bpw} B={B}: max err {err:.3e} tol {tolerance(ref):.3e} "
+          f"ratio {err / tolerance(ref):.3f}")
+    assert err <= tolerance(ref), (err, tolerance(ref))
+    yp = lay(x).float().cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(yp - ref) <= production_tolerance(ref, xdt))
+
+
+@pytest.mark.parametrize("li", [0, 1])
+def test_prefill_workload_largest_batch(dev, li):
+    wl = gi.WORKLOADS["prefill-8b-mlp-4bpw"]
+    L = gi.workload_layer(wl, li)
+    lay = dev.layer(L)
+    B = max(wl.batches)
+    xb = gi.workload_x(wl, li, B)
+    x = to_torch_x(xb, wl.x_dtype)
+    y = lay(x, out_dtype=torch.float32).cpu().numpy().astype(np.float64)
+    rng = np.random.default_rng(100 + li)
+    sample = sorted(set([0, 511, 512, B - 1] + list(rng.choice(B, size=3, replace=False))))
+    ref = oracle_y(L, xb[sample], wl.x_dtype)
+    err = np.max(np.abs(y[sample] - ref))
+    print(f"\nPARITY prefill layer {li} ({L.m}x{L.n}) B={B}: max err {err:.3e} "
+          f"tol {tolerance(ref):.3e} ratio {err / tolerance(ref):.3f}")
+    assert err <= tolerance(ref), (err, tolerance(ref))
+    assert np.all(np.isfinite(y))
+
+
+def test_prefill_determinism_and_batch_independence(dev):
+    m, n, bpw = 520, 1032, 4
+    L = gi.make_layer(5, 5, m, n, bpw)
+    lay = dev.layer(L)
+    xb = gi.make_x(5, 5, 700, n, "bf16")
+    x = to_torch_x(xb, "bf16")
+    y1 = lay(x, out_dtype=torch.float32)
+    y2 = lay(x, out_dtype=torch.float32)
+    assert torch.equal(y1, y2)
+    for B in (17, 300, 512, 513):
+        yb = lay(x[:B].contiguous(), out_dtype=torch.float32)
+        assert torch.equal(yb, y1[:B]), B
