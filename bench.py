@@ -285,6 +285,52 @@ def gemv_kernel_time(torch, ws: WorkloadSet, layer_index: int, reps: int, B=None
     return ms / per_graph
 
 
+def prefill_section(glq, torch, tc_peak, peak_src, batches=(512, 2048, 8192), reps=5) -> dict:
+    """8B-class MLP prefill (14336x4096 and 4096x14336 at 4 bpw): the whole
+    glq_linear step (input RHT, tensor-core GEMM, output RHT) per batch, and
+    the GEMM kernel alone (glq_prefill_replay) per layer, timed with events
+    on the stream the kernels run on.  The inputs (x 8192 x 14336 bf16 is
+    235 MB) exceed L2."""
+    pre = {}
+    wp = WorkloadSet(glq, torch, "prefill-8b-mlp-4bpw", max(batches), 1)
+    for Bp in batches:
+        wp.step(0, B=Bp)
+        torch.cuda.synchronize()
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record()
+        for _ in range(reps):
+            wp.step(0, B=Bp)
+        p1.record()
+        torch.cuda.synchronize()
+        msp = p0.elapsed_time(p1) / reps
+        tf = wp.step_flops(Bp) / (msp * 1e-3) / 1e12
+        entry = {"ms_per_step": round(msp, 3), "TFLOPs": round(tf, 2),
+                 "frac_bf16_peak": round(tf / tc_peak, 4)}
+        gemm = {}
+        for li, (lay, x, y) in enumerate(wp.copies[0]):
+            L = wp.host[li]
+            lay(x[:Bp], out=y[:Bp])  # leaves this batch's activations in the workspace
+            torch.cuda.synchronize()
+            lay.prefill_replay(Bp)
+            k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            k0.record()
+            for _ in range(reps):
+                lay.prefill_replay(Bp)
+            k1.record()
+            torch.cuda.synchronize()
+            mk = k0.elapsed_time(k1) / reps
+            tk = 2.0 * Bp * L.m * L.n / (mk * 1e-3) / 1e12
+            gemm[f"{L.m}x{L.n}"] = {"kernel_us": round(mk * 1e3, 1), "TFLOPs": round(tk, 1),
+                                    "frac": round(tk / tc_peak, 4)}
+        entry["gemm_kernel"] = gemm
+        pre[f"B={Bp}"] = entry
+    pre["peak"] = {"TFLOPs": tc_peak, "source": peak_src,
+                   "note": "fp16 operands: measured cuBLAS bf16 peak (same nominal rate)"}
+    del wp
+    torch.cuda.empty_cache()
+    return pre
+
+
 def oracle_step_seconds(ws_host, xbits, bpw, x_bf16) -> float:
     from oracle import glq_oracle as orc
     t0 = time.perf_counter()
@@ -433,25 +479,7 @@ def run_glq(args):
         torch.cuda.empty_cache()
         result["decode_24b"] = sweep
 
-        pre = {}
-        wp = WorkloadSet(glq, torch, "prefill-8b-mlp-4bpw", 8192, 1)
-        for Bp in (512, 2048, 8192):
-            wp.step(0, B=Bp)
-            torch.cuda.synchronize()
-            reps = 3
-            p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            p0.record()
-            for _ in range(reps):
-                wp.step(0, B=Bp)
-            p1.record()
-            torch.cuda.synchronize()
-            msp = p0.elapsed_time(p1) / reps
-            tf = wp.step_flops(Bp) / (msp * 1e-3) / 1e12
-            pre[f"B={Bp}"] = {"ms_per_step": round(msp, 3), "TFLOPs": round(tf, 2),
-                              "frac_bf16_peak": round(tf / tc_peak, 4)}
-        del wp
-        torch.cuda.empty_cache()
-        result["prefill"] = pre
+        result["prefill"] = prefill_section(glq, torch, tc_peak, peak_src)
 
     # fp64 oracle on the host cores (one decode step, 1 token, 5 layers)
     if world == 1 and not args.no_cpu:
@@ -502,6 +530,17 @@ def run_reference(args):
     }
 
 
+def run_prefill_only(args):
+    """The prefill timings alone, one JSON object (not the bench line)."""
+    import torch
+    import e8_lattice_codebook_b200 as glq
+    torch.cuda.set_device(0)
+    _, tc_peak, _, peak_src = read_peaks()
+    batches = (args.prefill_batch,) if args.prefill_batch else (512, 2048, 8192)
+    return {"section": "prefill", "prefill": prefill_section(glq, torch, tc_peak, peak_src, batches,
+                                                            reps=max(1, min(args.steps, 20)))}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -510,10 +549,17 @@ def main():
     ap.add_argument("--impl", choices=["glq", "reference"], default="glq")
     ap.add_argument("--quick", action="store_true", help="skip the 24B sweep and prefill")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle baseline")
+    ap.add_argument("--section", choices=["all", "prefill"], default="all",
+                    help="prefill: time only the prefill workload (profiling runs)")
+    ap.add_argument("--prefill-batch", type=int, default=0,
+                    help="with --section prefill: one batch instead of 512, 2048, 8192")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    res = run_reference(args) if args.impl == "reference" else run_glq(args)
+    if args.section == "prefill":
+        res = run_prefill_only(args)
+    else:
+        res = run_reference(args) if args.impl == "reference" else run_glq(args)
     if res is not None:
         print(json.dumps(res), flush=True)
     if int(os.environ.get("WORLD_SIZE", "1")) > 1 and args.impl == "glq":

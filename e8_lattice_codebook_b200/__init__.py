@@ -38,6 +38,7 @@ EXPORTS = (
     "glq_codebook_destroy", "glq_layer_create", "glq_layer_destroy", "glq_layer_reserve",
     "glq_linear", "glq_dequant_reference", "glq_rht_input", "glq_rht_output",
     "glq_layer_check", "glq_layer_info", "glq_gemv_replay", "glq_linear_noalloc",
+    "glq_prefill_replay",
 )
 
 
@@ -67,6 +68,7 @@ _SIGNATURES = {
     "glq_rht_output": ([_vp, _vp, _vp, ctypes.c_int, _i64, _vp], ctypes.c_int),
     "glq_layer_check": ([_vp, _vp], ctypes.c_int),
     "glq_gemv_replay": ([_vp, _i64, _vp], ctypes.c_int),
+    "glq_prefill_replay": ([_vp, _i64, _vp], ctypes.c_int),
     "glq_layer_info": ([_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i32),
                         ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
 }
@@ -181,6 +183,10 @@ def glq_gemv_replay(handle, B, stream) -> None:
     _ok(_L().glq_gemv_replay(handle, B, stream), "glq_gemv_replay")
 
 
+def glq_prefill_replay(handle, B, stream) -> None:
+    _ok(_L().glq_prefill_replay(handle, B, stream), "glq_prefill_replay")
+
+
 def glq_layer_check(handle, stream) -> None:
     _ok(_L().glq_layer_check(handle, stream), "glq_layer_check")
 
@@ -291,6 +297,9 @@ class GlqLinear:
 
     def gemv_replay(self, B, stream=None):
         glq_gemv_replay(self.handle, B, _stream_ptr(stream))
+
+    def prefill_replay(self, B, stream=None):
+        glq_prefill_replay(self.handle, B, _stream_ptr(stream))
 
     def check(self, stream=None):
         glq_layer_check(self.handle, _stream_ptr(stream))

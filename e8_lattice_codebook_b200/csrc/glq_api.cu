@@ -153,6 +153,34 @@ bool encode_x_map(CUtensorMap *map, const __half *xh, int64_t n_pad, int64_t B) 
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The tcgen05 GEMM of the tensor-core path on the layer's prefill
+// workspace: z[0..B) from xh[0..B).
+cudaError_t launch_prefill_gemm(glq_layer L, int64_t B, cudaStream_t s, bool pdl) {
+    CUtensorMap xmap;
+    if (!encode_x_map(&xmap, L->pws.xh, L->n_pad, B)) return cudaErrorInvalidValue;
+    glq::PrefillParams pp{};
+    pp.idx1 = L->d_idx1;
+    pp.idx2 = L->d_idx2;
+    pp.cb_f16 = L->primary->d_table_f16;
+    pp.res8 = L->bpw == 3 ? reinterpret_cast<const uint4 *>(L->residual->d_fp16) : nullptr;
+    pp.bpw = L->bpw;
+    const __half2 rs2 = __floats2half2_rn(L->rs, L->rs);
+    pp.rs_h2 = *reinterpret_cast<const uint32_t *>(&rs2);
+    pp.info = L->pws.info;
+    pp.ws = L->ws;
+    pp.z = L->pws.z;
+    pp.B = (int)B;
+    pp.m_pad = (int)L->m_pad;
+    pp.KC = L->KC;
+    pp.RT = L->RT;
+    const int tiles_m = (int)((L->m_pad + 127) / 128);
+    pp.tiles_tok = (int)((B + glq::prefill_tile_tokens() - 1) / glq::prefill_tile_tokens());
+    pp.ntiles = tiles_m * pp.tiles_tok;
+    pp.err = L->d_err;
+    const int grid = std::min(pp.ntiles, L->num_sms);
+    return glq::launch_prefill(pp, xmap, grid, s, pdl);
+}
+
 // Tensor-core path for B > 16 tokens: input RHT (fp16 activations), tcgen05
 // GEMM with the dequantising producer, output RHT.
 glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_dtype, int64_t B, cudaStream_t s) {
@@ -174,30 +202,8 @@ glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_d
         if (glq::launch_rht_in(pin, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
         b0 += nb;
     }
-    CUtensorMap xmap;
-    if (!encode_x_map(&xmap, L->pws.xh, L->n_pad, B)) return GLQ_ERR_CUDA;
-    glq::PrefillParams pp{};
-    pp.idx1 = L->d_idx1;
-    pp.idx2 = L->d_idx2;
-    pp.cb_f16 = L->primary->d_table_f16;
-    pp.fold = glq::FoldParams{L->primary->fold.nb, L->primary->fold.neg_base};
-    pp.res8 = L->bpw == 3 ? reinterpret_cast<const uint4 *>(L->residual->d_fp16) : nullptr;
-    pp.bpw = L->bpw;
-    const __half2 rs2 = __floats2half2_rn(L->rs, L->rs);
-    pp.rs_h2 = *reinterpret_cast<const uint32_t *>(&rs2);
-    pp.info = L->pws.info;
-    pp.ws = L->ws;
-    pp.z = L->pws.z;
-    pp.B = (int)B;
-    pp.m_pad = (int)L->m_pad;
-    pp.KC = L->KC;
-    pp.RT = L->RT;
-    const int tiles_m = (int)((L->m_pad + 127) / 128);
-    pp.tiles_tok = (int)((B + glq::prefill_tile_tokens() - 1) / glq::prefill_tile_tokens());
-    pp.ntiles = tiles_m * pp.tiles_tok;
-    pp.err = L->d_err;
-    const int grid = std::min(pp.ntiles, L->num_sms);
-    if (glq::launch_prefill(pp, xmap, grid, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+    if (launch_prefill_gemm(L, B, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+    L->last_prefill_B = B;
     for (int64_t b0 = 0; b0 < B;) {
         const int nb = (int)std::min<int64_t>(B - b0, 65535);
         glq::RhtOutParams pout{};
@@ -337,17 +343,20 @@ glq_status glq_codebook_upload(const uint16_t *host_fp16_bits, int32_t entries, 
     if (st == GLQ_OK && cudaMemcpy(cb->d_fp16, host_fp16_bits, bytes, cudaMemcpyHostToDevice) != cudaSuccess)
         st = GLQ_ERR_CUDA;
     if (st == GLQ_OK && cb->folded) {
-        // the folded table as fp16 codewords (x = v/2 - 3, exact) for the
-        // tensor-core path's gathers
-        std::vector<uint16_t> f16((size_t)cb->table_words * 8, 0);
-        for (int i = 0; i < cb->fold.nb; ++i) {
-            const uint32_t w = cb->fold.words[(size_t)i];
-            static const int shift[8] = {0, 8, 16, 24, 4, 12, 20, 28};
+        // fp16 codewords indexed by folded code (x = v/2 - 3, exact; codes
+        // past nb are the negated words), for the tensor-core path's gathers
+        const size_t ncodes = (size_t)cb->fold.neg_base + (size_t)cb->fold.nb;
+        std::vector<uint16_t> f16(ncodes * 8, 0);
+        static const int shift[8] = {0, 8, 16, 24, 4, 12, 20, 28};
+        for (size_t e = 0; e < ncodes; ++e) {
+            const bool neg = e >= (size_t)cb->fold.nb;
+            const uint32_t w = cb->fold.words[neg ? e - (size_t)cb->fold.neg_base : e];
             for (int j = 0; j < 8; ++j) {
                 const int y2 = (int)((w >> shift[j]) & 0xF) - 6;  // 2x
-                f16[(size_t)i * 8 + j] = glq::half_bits_of_half_integer(y2);
+                f16[e * 8 + j] = glq::half_bits_of_half_integer(neg ? -y2 : y2);
             }
         }
+        cb->code_f16_entries = (int)ncodes;
         st = dmalloc(&cb->d_table_f16, f16.size() * 2, nullptr);
         if (st == GLQ_OK && cudaMemcpy(cb->d_table_f16, f16.data(), f16.size() * 2, cudaMemcpyHostToDevice) !=
                                 cudaSuccess)
@@ -616,6 +625,14 @@ glq_status glq_gemv_replay(glq_layer L, int64_t B, void *stream) {
     return glq::launch_gemv(pg, L->bpw, plan.grid, static_cast<cudaStream_t>(stream), false) == cudaSuccess
                ? GLQ_OK
                : GLQ_ERR_CUDA;
+}
+
+glq_status glq_prefill_replay(glq_layer L, int64_t B, void *stream) {
+    if (!L) return GLQ_ERR_INVALID_ARG;
+    if (B <= GLQ_DECODE_MAX_B || B > L->last_prefill_B) return GLQ_ERR_SHAPE;
+    DeviceGuard guard(L->device);
+    return launch_prefill_gemm(L, B, static_cast<cudaStream_t>(stream), false) == cudaSuccess ? GLQ_OK
+                                                                                            : GLQ_ERR_CUDA;
 }
 
 glq_status glq_layer_check(glq_layer L, void *stream) {

@@ -22,7 +22,8 @@ struct glq_codebook_s {
     glq::FoldedTable fold;
     uint32_t *d_table = nullptr;  // table_words words
     int table_words = 0;          // nb rounded up to a multiple of 4
-    uint4 *d_table_f16 = nullptr; // the folded table as fp16 codewords [nb][8] (tensor-core path)
+    uint4 *d_table_f16 = nullptr; // fp16 codewords by folded code [code_f16_entries][8] (tensor-core path)
+    int code_f16_entries = 0;
 };
 
 // Device buffers of the tensor-core path (B > 16 tokens).
@@ -59,7 +60,8 @@ struct glq_layer_s {
     glq::GemvPlan plan[2]{};
     // workspace (sized by glq_layer_reserve / on first use)
     int64_t cap_rows = 0;
-    int64_t last_B = 0;  // batch of the last decode slice (glq_gemv_replay)
+    int64_t last_B = 0;          // batch of the last decode slice (glq_gemv_replay)
+    int64_t last_prefill_B = 0;  // batch of the last tensor-core call (glq_prefill_replay)
     glq_workspace wsp;
     glq_prefill_ws pws;
     size_t device_bytes = 0;

@@ -77,8 +77,7 @@ struct GemvParams {
 struct PrefillParams {
     const uint4 *idx1;       // [RT][KC][32] 16 B, fragment-native codes
     const void *idx2;        // 4 bpw: 16 B / 3 bpw: 8 B per slot
-    const uint4 *cb_f16;     // folded E8 table as fp16 codewords [nb][8]
-    FoldParams fold;
+    const uint4 *cb_f16;     // E8 codewords as fp16 [folded code][8] (negated entries included)
     const uint4 *res8;       // 3 bpw: [256][8] fp16
     int bpw;
     uint32_t rs_h2;          // residual scale as fp16x2

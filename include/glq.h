@@ -196,6 +196,19 @@ GLQ_API glq_status glq_rht_output(glq_layer layer, const float *z_dev, void *y_d
 GLQ_API glq_status glq_gemv_replay(glq_layer layer, int64_t B, void *stream);
 
 /*
+ * glq_prefill_replay -- measurement entry point: re-launches only the
+ * tensor-core GEMM of the most recent glq_linear call with B > 16 on this
+ * layer (its fp16 rotated activations are still in the layer's workspace),
+ * for 16 < B <= that call's B, rewriting the same pre-rotation outputs z.
+ * Lets a caller time the GEMM kernel alone with events on `stream`.  The
+ * GEMM is the tensor-core path of "Inference kernels" on the glq 0.5.1 PyPI
+ * page (matmul against codebook-reconstructed weights, W never stored).
+ * Errors: GLQ_ERR_INVALID_ARG, GLQ_ERR_SHAPE (B out of range or no previous
+ * call), GLQ_ERR_CUDA.  Asynchronous.
+ */
+GLQ_API glq_status glq_prefill_replay(glq_layer layer, int64_t B, void *stream);
+
+/*
  * glq_linear_noalloc -- glq_linear for a batch of at most 16 tokens that
  * allocates no device memory, for callers that cannot call cudaMalloc at
  * call time: code running while a CUDA graph is captured, in host
