@@ -285,6 +285,25 @@ def gemv_kernel_time(torch, ws: WorkloadSet, layer_index: int, reps: int, B=None
     return ms / per_graph
 
 
+def profiled_traffic(profile: str, source: str):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    recorded in a committed ncu summary under profiles/, or None when the
+    kernel source has changed since that capture (its sha256 differs)."""
+    import hashlib
+    root = os.path.dirname(os.path.abspath(__file__))
+    try:
+        text = open(os.path.join(root, "profiles", profile)).read()
+        src = open(os.path.join(root, "e8_lattice_codebook_b200", "csrc", source), "rb").read()
+    except OSError:
+        return None
+    if hashlib.sha256(src).hexdigest() not in text:
+        return None
+    for line in text.splitlines():
+        if line.startswith("traffic_bytes_per_launch"):
+            return int(line.split(":")[1].split()[0])
+    return None
+
+
 def prefill_section(glq, torch, tc_peak, peak_src, batches=(512, 2048, 8192), reps=5) -> dict:
     """8B-class MLP prefill (14336x4096 and 4096x14336 at 4 bpw): the whole
     glq_linear step (input RHT, tensor-core GEMM, output RHT) per batch, and
@@ -423,7 +442,8 @@ def run_glq(args):
         "kernel": f"gemv_kernel<4,1> gate {L.m}x{L.n} B=1",
         "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
         "frac": round(achieved / hbm_peak, 4), "peak_source": f"{peak_src} hbm_gbs (burst)",
-        "traffic": None, "kernel_us": round(ms_k * 1e3, 3),
+        "traffic": profiled_traffic("gemv_smollm3-3b-gate-up-down_4bpw_b1.md", "glq_gemv.cu"),
+        "kernel_us": round(ms_k * 1e3, 3),
         "algorithmic_bytes": gemv_bytes(L.m, L.n, L.bpw, B),
     }
 
