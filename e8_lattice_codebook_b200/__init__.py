@@ -38,7 +38,7 @@ EXPORTS = (
     "glq_codebook_destroy", "glq_layer_create", "glq_layer_destroy", "glq_layer_reserve",
     "glq_linear", "glq_dequant_reference", "glq_rht_input", "glq_rht_output",
     "glq_layer_check", "glq_layer_info", "glq_gemv_replay", "glq_linear_noalloc",
-    "glq_prefill_replay",
+    "glq_prefill_replay", "glq_layer_set_fusion",
 )
 
 
@@ -69,6 +69,7 @@ _SIGNATURES = {
     "glq_layer_check": ([_vp, _vp], ctypes.c_int),
     "glq_gemv_replay": ([_vp, _i64, _vp], ctypes.c_int),
     "glq_prefill_replay": ([_vp, _i64, _vp], ctypes.c_int),
+    "glq_layer_set_fusion": ([_vp, ctypes.c_int32], ctypes.c_int),
     "glq_layer_info": ([_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i32),
                         ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
 }
@@ -187,6 +188,13 @@ def glq_prefill_replay(handle, B, stream) -> None:
     _ok(_L().glq_prefill_replay(handle, B, stream), "glq_prefill_replay")
 
 
+GLQ_FUSE_INPUT, GLQ_FUSE_OUTPUT, GLQ_FUSE_DEFAULT = 1, 2, -1
+
+
+def glq_layer_set_fusion(handle, flags: int) -> None:
+    _ok(_L().glq_layer_set_fusion(handle, int(flags)), "glq_layer_set_fusion")
+
+
 def glq_layer_check(handle, stream) -> None:
     _ok(_L().glq_layer_check(handle, stream), "glq_layer_check")
 
@@ -297,6 +305,14 @@ class GlqLinear:
 
     def gemv_replay(self, B, stream=None):
         glq_gemv_replay(self.handle, B, _stream_ptr(stream))
+
+    def set_fusion(self, flags):
+        """GLQ_FUSE_* bits; True / False mean both / neither."""
+        if flags is True:
+            flags = GLQ_FUSE_INPUT | GLQ_FUSE_OUTPUT
+        elif flags is False:
+            flags = 0
+        glq_layer_set_fusion(self.handle, flags)
 
     def prefill_replay(self, B, stream=None):
         glq_prefill_replay(self.handle, B, _stream_ptr(stream))

@@ -49,6 +49,23 @@ std::vector<uint32_t> pack_signs(const int8_t *s, int64_t k) {
     return bits;
 }
 
+// block-diagonal Hadamard blocks of a size: its binary decomposition,
+// descending powers of two at increasing offsets
+glq_hblocks hadamard_blocks_of(int64_t k) {
+    glq_hblocks hb;
+    int64_t off = 0;
+    for (int bit = 30; bit >= 0; --bit) {
+        const int64_t sz = (int64_t)1 << bit;
+        if (k & sz) {
+            hb.off[hb.count] = (int)off;
+            hb.len[hb.count] = (int)sz;
+            ++hb.count;
+            off += sz;
+        }
+    }
+    return hb;
+}
+
 template <typename T>
 glq_status dmalloc(T **p, size_t bytes, size_t *total) {
     *p = nullptr;
@@ -85,6 +102,7 @@ void free_prefill_ws(glq_layer L) {
 void free_layer(glq_layer L) {
     if (!L) return;
     free_prefill_ws(L);
+    cudaFree(L->d_blk_cnt);
     cudaFree(L->d_idx1);
     cudaFree(L->d_idx2);
     cudaFree(L->d_sin);
@@ -103,7 +121,8 @@ glq_status grow_workspace(glq_layer L, int64_t rows) {
     glq_status st = dmalloc(&L->wsp.xq, (size_t)rows * L->n_pad * 2, nullptr);
     if (st == GLQ_OK && L->bpw == 3) st = dmalloc(&L->wsp.xh, (size_t)rows * L->n_pad * sizeof(__half), nullptr);
     if (st == GLQ_OK) st = dmalloc(&L->wsp.info, (size_t)rows * sizeof(glq_rowinfo), nullptr);
-    const int max_splits = std::max(L->plan[0].splits, L->plan[1].splits);
+    int max_splits = 1;
+    for (int nb = 1; nb <= rows; ++nb) max_splits = std::max(max_splits, glq::max_decode_splits(L, nb));
     if (st == GLQ_OK && max_splits > 1)
         st = dmalloc(&L->wsp.part, (size_t)max_splits * rows * L->m_pad * sizeof(double), nullptr);
     if (st == GLQ_OK) st = dmalloc(&L->wsp.z, (size_t)rows * L->m_pad * sizeof(float), nullptr);
@@ -225,7 +244,68 @@ glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_d
 
 namespace glq {
 
-GemvParams gemv_params(glq_layer L, const glq_workspace &w, const GemvPlan &plan, int nb) {
+// fused transforms: at most this many values (tokens x largest Hadamard
+// block) are folded per task (input) or rotated by one CTA (output)
+constexpr long long FUSED_IN_MAX_VALUES = 32768;
+constexpr long long FUSED_OUT_MAX_VALUES = 32768;
+// Measured on B200 (CUDA graphs, B = 1 and 8): fusing the input transform
+// saves a launch when every CTA has one short task (below); the output
+// transform done by one CTA at the end of the GEMV is slower than the
+// separate, parallel kernel at every size measured, so it is off by default.
+constexpr int FUSE_DEFAULT_FLAGS = GLQ_FUSE_INPUT;
+
+DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y_dtype, int max_splits) {
+    DecodeCfg c;
+    const int nt = nb > 8 ? 2 : 1;
+    const int warps = gemv_warps(nt);
+    const size_t base = gemv_smem_bytes(L->primary->table_words, L->bpw);
+    const bool x_al = (reinterpret_cast<uintptr_t>(x) & 15) == 0;
+    const bool y_al = (reinterpret_cast<uintptr_t>(y) & 15) == 0;
+    (void)y_dtype;
+    const int flags = L->fusion < 0 ? FUSE_DEFAULT_FLAGS : L->fusion;
+    c.fout = (flags & GLQ_FUSE_OUTPUT) && y_al && (long long)nb * L->hb_m.len[0] <= FUSED_OUT_MAX_VALUES &&
+             (size_t)nb * L->hb_m.len[0] * sizeof(float) <= base;
+    if ((flags & GLQ_FUSE_INPUT) && x_al && (long long)nb * L->hb_n.len[0] <= FUSED_IN_MAX_VALUES) {
+        int cap = 1;  // largest power-of-two chunk count whose activations fit shared memory
+        while (cap < L->KC &&
+               gemv_fused_smem_bytes(L->primary->table_words, L->bpw, nb, std::min(cap * 2, L->KC) * GLQ_CHUNK_K) <=
+                   GEMV_SMEM_LIMIT)
+            cap *= 2;
+        const GemvPlan fp = plan_gemv(L->RT, L->KC, L->num_sms, warps, true, cap, max_splits);
+        const size_t need =
+            gemv_fused_smem_bytes(L->primary->table_words, L->bpw, nb, std::min(fp.cps, L->KC) * GLQ_CHUNK_K);
+        // Measured: the fold pays for the launch it saves when every CTA has
+        // one task and a short range (<= 1024 columns, <= 4096 values in
+        // all); a 4096-column range per CTA is slower than the separate
+        // transform kernel.  An explicit setting always fuses.
+        const int klen = std::min(fp.cps, L->KC) * GLQ_CHUNK_K;
+        const bool cheap = (long long)fp.bands * fp.splits <= L->num_sms && klen <= 1024 && nb * klen <= 4096;
+        if (need <= GEMV_SMEM_LIMIT && (cheap || L->fusion >= 0)) {
+            c.fin = true;
+            c.plan = fp;
+        }
+    }
+    if (!c.fin) {
+        c.plan = plan_for(L, nb);
+        if (c.plan.splits > max_splits) c.plan = plan_gemv(L->RT, L->KC, L->num_sms, warps, false, 1 << 30, max_splits);
+    }
+    return c;
+}
+
+int max_decode_splits(glq_layer L, int nb) {
+    const int warps = gemv_warps(nb > 8 ? 2 : 1);
+    int cap = 1;
+    while (cap < L->KC &&
+           gemv_fused_smem_bytes(L->primary->table_words, L->bpw, nb, std::min(cap * 2, L->KC) * GLQ_CHUNK_K) <=
+               GEMV_SMEM_LIMIT)
+        cap *= 2;
+    const GemvPlan f = plan_gemv(L->RT, L->KC, L->num_sms, warps, true, cap);
+    return std::max(plan_for(L, nb).splits, f.splits);
+}
+
+GemvParams gemv_params(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg, int nb, const void *x,
+                       bool x_bf16, void *y, int y_dtype) {
+    const GemvPlan &plan = cfg.plan;
     GemvParams p{};
     p.idx1 = L->d_idx1;
     p.idx2 = L->d_idx2;
@@ -251,26 +331,58 @@ GemvParams gemv_params(glq_layer L, const glq_workspace &w, const GemvPlan &plan
     p.z = w.z;
     p.m_pad = (int)L->m_pad;
     p.err = L->d_err;
+    // fused transforms
+    p.x = x;
+    p.x_bf16 = x_bf16 ? 1 : 0;
+    p.n = (int)L->n;
+    p.sin_bits = L->d_sin;
+    p.nblk_n = L->hb_n.count;
+    for (int i = 0; i < L->hb_n.count; ++i) {
+        p.blk_off_n[i] = L->hb_n.off[i];
+        p.blk_len_n[i] = L->hb_n.len[i];
+    }
+    p.fuse_out = cfg.fout ? 1 : 0;
+    p.y = y;
+    p.y_dtype = y_dtype;
+    p.m = (int)L->m;
+    p.sout_bits = L->d_sout;
+    p.nblk_m = L->hb_m.count;
+    const int band_rows = gemv_warps(nb > 8 ? 2 : 1) * GLQ_ROW_TILE;
+    for (int i = 0; i < L->hb_m.count; ++i) {
+        const int o = L->hb_m.off[i], N = L->hb_m.len[i];
+        p.blk_off_m[i] = o;
+        p.blk_len_m[i] = N;
+        int cnt = 0;
+        for (int band = 0; band < plan.bands; ++band) {
+            const int r0 = band * band_rows, r1 = std::min<int>(r0 + band_rows, (int)L->m);
+            if (r0 < o + N && o < r1) ++cnt;
+        }
+        p.blk_bands[i] = cnt;
+    }
+    p.blk_cnt = L->d_blk_cnt;
     return p;
 }
 
-cudaError_t run_decode(glq_layer L, const glq_workspace &w, const GemvPlan &plan, const void *x, bool x_bf16,
+cudaError_t run_decode(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg, const void *x, bool x_bf16,
                        void *y, int y_dtype, int nb, cudaStream_t s) {
-    RhtInParams pin{};
-    pin.x = x;
-    pin.x_bf16 = x_bf16 ? 1 : 0;
-    pin.n = (int)L->n;
-    pin.n_pad = (int)L->n_pad;
-    pin.B = nb;
-    pin.sign_bits = L->d_sin;
-    pin.plan = L->plan_n;
-    pin.xq = w.xq;
-    pin.xh = w.xh;
-    pin.info = w.info;
-    cudaError_t e = launch_rht_in(pin, s, true);
-    if (e != cudaSuccess) return e;
-    e = launch_gemv(gemv_params(L, w, plan, nb), L->bpw, plan.grid, s, true);
-    if (e != cudaSuccess) return e;
+    cudaError_t e = cudaSuccess;
+    if (!cfg.fin) {
+        RhtInParams pin{};
+        pin.x = x;
+        pin.x_bf16 = x_bf16 ? 1 : 0;
+        pin.n = (int)L->n;
+        pin.n_pad = (int)L->n_pad;
+        pin.B = nb;
+        pin.sign_bits = L->d_sin;
+        pin.plan = L->plan_n;
+        pin.xq = w.xq;
+        pin.xh = w.xh;
+        pin.info = w.info;
+        e = launch_rht_in(pin, s, true);
+        if (e != cudaSuccess) return e;
+    }
+    e = launch_gemv(gemv_params(L, w, cfg, nb, x, x_bf16, y, y_dtype), L->bpw, cfg.plan.grid, s, true, cfg.fin);
+    if (e != cudaSuccess || cfg.fout) return e;
     RhtOutParams pout{};
     pout.m = (int)L->m;
     pout.B = nb;
@@ -441,6 +553,8 @@ glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *i
     L->plan[0] = glq::plan_gemv(L->RT, L->KC, L->num_sms, glq::gemv_warps(1));
     L->plan[1] = glq::plan_gemv(L->RT, L->KC, L->num_sms, glq::gemv_warps(2));
     const int max_bands = std::max(L->plan[0].bands, L->plan[1].bands);
+    L->hb_n = hadamard_blocks_of(n);
+    L->hb_m = hadamard_blocks_of(m);
 
     // fragment-native index streams (layout: glq_internal.h)
     const FoldedTable &F = primary->fold;
@@ -477,6 +591,7 @@ glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *i
     if (st == GLQ_OK) st = dmalloc(&L->d_sout, sout_bits.size() * 4, &total);
     if (st == GLQ_OK) st = dmalloc(&L->d_err, sizeof(unsigned), &total);
     if (st == GLQ_OK) st = dmalloc(&L->wsp.cnt, (size_t)max_bands * sizeof(unsigned), &total);
+    if (st == GLQ_OK) st = dmalloc(&L->d_blk_cnt, GLQ_MAX_BLOCKS * sizeof(unsigned), &total);
     if (st == GLQ_OK) {
         bool ok = cudaMemcpy(L->d_idx1, s1.data(), L->idx1_bytes, cudaMemcpyHostToDevice) == cudaSuccess;
         if (ok && bpw == 4)
@@ -489,6 +604,7 @@ glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *i
                        cudaSuccess;
         ok = ok && cudaMemset(L->d_err, 0, sizeof(unsigned)) == cudaSuccess;
         ok = ok && cudaMemset(L->wsp.cnt, 0, (size_t)max_bands * sizeof(unsigned)) == cudaSuccess;
+        ok = ok && cudaMemset(L->d_blk_cnt, 0, GLQ_MAX_BLOCKS * sizeof(unsigned)) == cudaSuccess;
         if (!ok) st = GLQ_ERR_CUDA;
     }
     if (st != GLQ_OK) {
@@ -515,6 +631,13 @@ glq_status glq_layer_reserve(glq_layer layer, int64_t max_B) {
     return grow_workspace(layer, std::min<int64_t>(std::max<int64_t>(max_B, 1), GLQ_DECODE_MAX_B));
 }
 
+glq_status glq_layer_set_fusion(glq_layer layer, int32_t flags) {
+    if (!layer) return GLQ_ERR_INVALID_ARG;
+    if (flags != GLQ_FUSE_DEFAULT && (flags & ~(GLQ_FUSE_INPUT | GLQ_FUSE_OUTPUT))) return GLQ_ERR_INVALID_ARG;
+    layer->fusion = flags;
+    return GLQ_OK;
+}
+
 glq_status glq_layer_info(glq_layer layer, int64_t *m, int64_t *n, int32_t *bpw, size_t *device_bytes) {
     if (!layer) return GLQ_ERR_INVALID_ARG;
     if (m) *m = layer->m;
@@ -532,6 +655,8 @@ glq_status glq_linear(glq_layer L, const void *x_dev, glq_dtype x_dtype, void *y
     if (y_dtype != x_dtype && y_dtype != GLQ_F32) return GLQ_ERR_DTYPE;
     if (B == 0) return GLQ_OK;
     if (!x_dev || !y_dev) return GLQ_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(x_dev) & 15) || (reinterpret_cast<uintptr_t>(y_dev) & 15))
+        return GLQ_ERR_INVALID_ARG;  // the kernels use 8- and 16-byte accesses
     DeviceGuard guard(L->device);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (B > GLQ_DECODE_MAX_B) return run_prefill(L, x_dev, x_dtype == GLQ_BF16, y_dev, (int)y_dtype, B, s);
@@ -542,12 +667,16 @@ glq_status glq_linear(glq_layer L, const void *x_dev, glq_dtype x_dtype, void *y
         const int nb = (int)std::min<int64_t>(GLQ_DECODE_MAX_B, B - b0);
         const void *x = static_cast<const char *>(x_dev) + (size_t)b0 * L->n * xe;
         void *y = static_cast<char *>(y_dev) + (size_t)b0 * L->m * ye;
-        if (glq::run_decode(L, L->wsp, glq::plan_for(L, nb), x, x_dtype == GLQ_BF16, y, (int)y_dtype, nb, s) !=
-            cudaSuccess) {
+        const glq::DecodeCfg cfg = glq::decode_config(L, nb, x, y, (int)y_dtype);
+        if (glq::run_decode(L, L->wsp, cfg, x, x_dtype == GLQ_BF16, y, (int)y_dtype, nb, s) != cudaSuccess) {
             cudaGetLastError();
             return GLQ_ERR_CUDA;
         }
         L->last_B = nb;
+        L->last_x = x;
+        L->last_y = y;
+        L->last_x_bf16 = x_dtype == GLQ_BF16 ? 1 : 0;
+        L->last_y_dtype = (int)y_dtype;
     }
     return GLQ_OK;
 }
@@ -620,9 +749,11 @@ glq_status glq_gemv_replay(glq_layer L, int64_t B, void *stream) {
     if (!L) return GLQ_ERR_INVALID_ARG;
     if (B < 1 || B > L->last_B) return GLQ_ERR_SHAPE;
     DeviceGuard guard(L->device);
-    const glq::GemvPlan &plan = glq::plan_for(L, (int)B);
-    glq::GemvParams pg = glq::gemv_params(L, L->wsp, plan, (int)B);
-    return glq::launch_gemv(pg, L->bpw, plan.grid, static_cast<cudaStream_t>(stream), false) == cudaSuccess
+    const glq::DecodeCfg cfg = glq::decode_config(L, (int)B, L->last_x, L->last_y, L->last_y_dtype);
+    glq::GemvParams pg = glq::gemv_params(L, L->wsp, cfg, (int)B, L->last_x, L->last_x_bf16 != 0, L->last_y,
+                                          L->last_y_dtype);
+    return glq::launch_gemv(pg, L->bpw, cfg.plan.grid, static_cast<cudaStream_t>(stream), false, cfg.fin) ==
+                   cudaSuccess
                ? GLQ_OK
                : GLQ_ERR_CUDA;
 }

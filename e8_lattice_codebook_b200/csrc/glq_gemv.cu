@@ -23,7 +23,13 @@
 //     fp16 operands with fp32 accumulation;
 //   * per task, partial sums go to a workspace in fp64; the last CTA to
 //     finish a band (atomic counter, no waiting) adds the splits in fixed
-//     order and writes the band's final z.
+//     order and writes the band's final z;
+//   * small batches fuse both transforms (one launch per layer): each task
+//     rotates, scales and quantises its own aligned column range of x in
+//     shared memory (a Hadamard block of size N = 2^a S restricted to an
+//     aligned range of S outputs is H_S applied to the 2^a-term signed fold
+//     of the block), and the last band to finish a Hadamard block of m
+//     transforms that block of z in shared memory and writes y.
 #include "glq_kernels.cuh"
 
 namespace glq {
@@ -59,7 +65,14 @@ __device__ __forceinline__ void stage_int(const uint32_t *T, FoldParams fold, ui
     }
 }
 
-template <int BPW, int NT>
+// 16-byte load of activations: global (read-only path) or shared memory
+template <bool XS>
+__device__ __forceinline__ uint4 ld_x(const void *p) {
+    if (XS) return *reinterpret_cast<const uint4 *>(p);
+    return ldg_v4(p);
+}
+
+template <int BPW, int NT, bool XS>
 __device__ __forceinline__ void process_chunk(const uint32_t *T, const uint4 *R8, FoldParams fold,
                                               const uint4 &q1, const uint4 &q2, const uint4 *xq0,
                                               const uint4 *xq1, const __half *xh0, const __half *xh1,
@@ -70,8 +83,8 @@ __device__ __forceinline__ void process_chunk(const uint32_t *T, const uint4 *R8
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
         uint4 x0 = make_uint4(0, 0, 0, 0), x1 = make_uint4(0, 0, 0, 0);
-        if (has0) x0 = ldg_v4(xq0 + 4 * s);
-        if (NT == 2 && has1) x1 = ldg_v4(xq1 + 4 * s);
+        if (has0) x0 = ld_x<XS>(xq0 + 4 * s);
+        if (NT == 2 && has1) x1 = ld_x<XS>(xq1 + 4 * s);
         stage_int<NT>(T, fold, p1[s], x0, x1, acc1);
         if (BPW == 4) stage_int<NT>(T, fold, p2[s], x0, x1, acc2);
         if (BPW == 3) {
@@ -83,8 +96,8 @@ __device__ __forceinline__ void process_chunk(const uint32_t *T, const uint4 *R8
             const uint32_t lo[4] = {ra.x, rb.x, ra.y, rb.y};
             const uint32_t hi[4] = {ra.z, rb.z, ra.w, rb.w};
             uint4 h0 = make_uint4(0, 0, 0, 0), h1 = make_uint4(0, 0, 0, 0);
-            if (has0) h0 = ldg_v4(xh0 + 32 * s);
-            if (NT == 2 && has1) h1 = ldg_v4(xh1 + 32 * s);
+            if (has0) h0 = ld_x<XS>(xh0 + 32 * s);
+            if (NT == 2 && has1) h1 = ld_x<XS>(xh1 + 32 * s);
             mma_16816(accr[0], lo, h0.x, h0.y);
             mma_16816(accr[0], hi, h0.z, h0.w);
             if (NT == 2) {
@@ -117,21 +130,303 @@ __device__ __forceinline__ float finish_z(const GemvParams &p, int b, double D) 
     return (float)((D - corr) * (0.5 * (double)p.ws * (double)info.inv_scale));
 }
 
-template <int BPW, int NT>
+// ---------------------------------------------------------------------------
+// Fused transforms
+// ---------------------------------------------------------------------------
+
+struct TaskRow {  // per token, over the task's column range
+    int sum_x;        // exact sum of X
+    float inv_scale;  // 2^-e
+};
+
+// 8 consecutive activations (16-byte aligned) as float
+__device__ __forceinline__ void load8_act(const void *x, size_t i, int bf16, float v[8]) {
+    const uint4 r = ldg_v4(static_cast<const uint16_t *>(x) + i);
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        if (bf16) {
+            v[2 * j] = __uint_as_float(w[j] << 16);
+            v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        } else {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[j]));
+            v[2 * j] = f.x;
+            v[2 * j + 1] = f.y;
+        }
+    }
+}
+
+// butterflies of spans 1, 2, 4 on 8 consecutive values (Sylvester order)
+__device__ __forceinline__ void fwht8(float v[8]) {
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if ((i & h) == 0) {
+                const float a = v[i], b = v[i + h];
+                v[i] = a + b;
+                v[i + h] = a - b;
+            }
+}
+
+// A run of one Hadamard transform within a row of a shared-memory buffer:
+// elements [start, start + size), size a power of two >= 8, start a
+// multiple of size; norm = 1/sqrt(size of the whole block).
+struct Seg {
+    int start, size;
+    float norm;
+};
+
+// Butterflies of spans 8 .. size/2 on every segment of every row (rows of
+// `ld` floats), the spans 1, 2, 4 being done already per 8-vector.  Spans up
+// to 128 run in registers across the lanes of a warp (32 consecutive
+// 8-vectors, shuffles); longer spans run in shared memory, one barrier per
+// span.  Every thread of the CTA calls it; it ends with a barrier.
+template <int THREADS>
+__device__ void fwht_segments(float *u, int nrows, int ld, const Seg *segs, int nseg) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int vrow = ld / 8, total = nrows * vrow;
+    int smax = 0;
+    for (int i = 0; i < nseg; ++i) smax = max(smax, segs[i].size);
+    if (smax > 8) {
+        for (int v0 = warp * 32; v0 < total; v0 += THREADS) {
+            const int v = v0 + lane;
+            const bool valid = v < total;
+            const int row = valid ? v / vrow : 0;
+            const int q = valid ? 8 * (v - row * vrow) : 0;
+            int S = 0;
+            for (int i = 0; i < nseg; ++i)
+                if (q >= segs[i].start && q < segs[i].start + segs[i].size) S = segs[i].size;
+            float r[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            float *src = u + (size_t)row * ld + q;
+            if (valid && S > 8) {
+                const float4 a = *reinterpret_cast<const float4 *>(src);
+                const float4 c = *reinterpret_cast<const float4 *>(src + 4);
+                r[0] = a.x; r[1] = a.y; r[2] = a.z; r[3] = a.w;
+                r[4] = c.x; r[5] = c.y; r[6] = c.z; r[7] = c.w;
+            }
+#pragma unroll
+            for (int k = 0; k < 5; ++k) {  // spans 8, 16, 32, 64, 128
+                const int off = 1 << k;
+                const bool act = valid && (8 << k) < S;
+                const bool upper = (lane & off) != 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float o = __shfl_xor_sync(0xffffffffu, r[j], off);
+                    if (act) r[j] = upper ? o - r[j] : r[j] + o;
+                }
+            }
+            if (valid && S > 8) {
+                *reinterpret_cast<float4 *>(src) = make_float4(r[0], r[1], r[2], r[3]);
+                *reinterpret_cast<float4 *>(src + 4) = make_float4(r[4], r[5], r[6], r[7]);
+            }
+        }
+    }
+    __syncthreads();
+    for (int h = 256; h < smax; h <<= 1) {
+        for (int i = 0; i < nseg; ++i) {
+            if (segs[i].size <= h) continue;
+            const int pairs = segs[i].size >> 1;
+            for (int e = threadIdx.x; e < nrows * pairs; e += THREADS) {
+                const int row = e / pairs, q0 = e - row * pairs;
+                float *r = u + (size_t)row * ld + segs[i].start + ((q0 / h) * 2 * h) + (q0 % h);
+                const float a = r[0], c = r[h];
+                r[0] = a + c;
+                r[h] = a - c;
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// The task's activations for columns [k0, k0 + klen): xr = H_n (S_in x)
+// restricted to the range, scaled per token by 2^e (max |xr| 2^e < 2^14 over
+// the range), rounded to X and stored as the GEMV consumes it: xs[b][group]
+// = 8 high bytes, 8 low bytes; xhs[b][col] = X as fp16 (3 bpw).  The range is
+// aligned and a power-of-two multiple of 128 columns, so within each Hadamard
+// block it meets it is either the whole block or an aligned part of size S
+// of a block of size N: then xr = N^-1/2 H_S f with f[j] = sum over the
+// N/S sub-blocks t of (-1)^popc(i t) (S_in x)[t S + j], i the part's index.
+template <int BPW, int THREADS>
+__device__ void fused_input(const GemvParams &p, int k0, int klen, uint4 *xs, __half *xhs, float *u,
+                            TaskRow *rows, unsigned *s_max, Seg *segs) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int B = p.B, k1 = k0 + klen;
+    for (int e = tid; e < B * klen; e += THREADS) u[e] = 0.f;  // columns >= n stay zero
+    if (tid < GLQ_DECODE_MAX_B) {
+        s_max[tid] = 0u;
+        rows[tid].sum_x = 0;
+    }
+    __syncthreads();
+    int nseg = 0;  // the task's segments (identical in every thread)
+    for (int bi = 0; bi < p.nblk_n; ++bi) {
+        const int o = p.blk_off_n[bi], N = p.blk_len_n[bi];
+        const int lo = max(k0, o), hi = min(k1, o + N);
+        if (lo >= hi) continue;
+        if (tid == 0) segs[nseg] = Seg{lo - k0, hi - lo, __frsqrt_rn((float)N)};
+        ++nseg;
+        const int S = hi - lo;  // N or an aligned part of it
+        const int A = N / S, ihi = (lo - o) / S, nv = S / 8;
+        const int items = B * nv;
+        int G = 1;  // lanes sharing one 8-column vector (split over the fold terms)
+        while (G < 32 && 2 * G <= A && items * 2 * G <= THREADS) G *= 2;
+        for (int it0 = 0; it0 < items * G; it0 += THREADS) {
+            const int it = it0 + tid;
+            const bool valid = it < items * G;
+            const int grp = it & (G - 1), item = it / G;
+            const int b = valid ? item / nv : 0, v = valid ? item - b * nv : 0;
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (valid) {
+                for (int jh = grp; jh < A; jh += G) {
+                    const int col = o + jh * S + 8 * v;
+                    float xv[8];
+                    load8_act(p.x, (size_t)b * p.n + col, p.x_bf16, xv);
+                    const uint32_t sb = (p.sin_bits[col >> 5] >> (col & 31)) & 0xFFu;
+                    const uint32_t neg = (__popc(ihi & jh) & 1) ? 0xFFu : 0u;
+                    const uint32_t flip = sb ^ neg;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[j] += ((flip >> j) & 1u) ? -xv[j] : xv[j];
+                }
+            }
+            // fixed-order reduction over the G lanes of a vector
+            for (int off = 1; off < G; off <<= 1)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+            if (valid && grp == 0) {
+                fwht8(acc);
+                float *dst = u + (size_t)b * klen + (lo - k0) + 8 * v;
+                *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                *reinterpret_cast<float4 *>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            }
+        }
+    }
+    __syncthreads();
+    fwht_segments<THREADS>(u, B, klen, segs, nseg);
+    // normalise per block, row max per token
+    const int nvec = klen / 8;
+    for (int e = tid; e < B * nvec; e += THREADS) {
+        const int b = e / nvec, v = e - b * nvec;
+        float nrm = 0.f;
+        for (int i = 0; i < nseg; ++i)
+            if (8 * v >= segs[i].start && 8 * v < segs[i].start + segs[i].size) nrm = segs[i].norm;
+        float *r = u + (size_t)b * klen + 8 * v;
+        float mx = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            r[j] *= nrm;
+            mx = fmaxf(mx, fabsf(r[j]));
+        }
+        atomicMax(s_max + b, __float_as_uint(mx));
+    }
+    __syncthreads();
+    // X = round(xr 2^e), interleaved bytes, exact sum
+    for (int e = tid; e < B * nvec; e += THREADS) {
+        const int b = e / nvec, v = e - b * nvec;
+        const float rowmax = __uint_as_float(s_max[b]);
+        float scale = 1.f;
+        if (rowmax > 0.f && isfinite(rowmax)) {
+            int ex;
+            frexpf(rowmax, &ex);
+            scale = ldexpf(1.f, 14 - ex);
+        }
+        const float *r = u + (size_t)b * klen + 8 * v;
+        uint32_t hb[2] = {0u, 0u}, lb[2] = {0u, 0u};
+        int sum = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int X = __float2int_rn(r[j] * scale);
+            sum += X;
+            hb[j >> 2] |= (uint32_t)((X >> 8) & 0xFF) << (8 * (j & 3));
+            lb[j >> 2] |= (uint32_t)(X & 0xFF) << (8 * (j & 3));
+            if (BPW == 3) xhs[(size_t)b * klen + 8 * v + j] = __int2half_rn(X);
+        }
+        xs[(size_t)b * nvec + v] = make_uint4(hb[0], hb[1], lb[0], lb[1]);
+        atomicAdd(&rows[b].sum_x, sum);
+        if (v == 0) rows[b].inv_scale = 1.f / scale;
+    }
+    (void)lane;
+    __syncthreads();
+}
+
+// y for Hadamard block `blk` of m, all tokens: the block's z (complete in
+// global memory) is transformed in shared memory `buf` (B x N floats).
+template <int THREADS>
+__device__ void fused_output(const GemvParams &p, int blk, float *buf) {
+    const int o = p.blk_off_m[blk], N = p.blk_len_m[blk], B = p.B;
+    const int nvec = N / 8;
+    for (int e = threadIdx.x; e < B * nvec; e += THREADS) {
+        const int b = e / nvec, v = e - b * nvec;
+        const float4 *zp = reinterpret_cast<const float4 *>(p.z + (size_t)b * p.m_pad + o + 8 * v);
+        const float4 a = __ldcg(zp), c = __ldcg(zp + 1);
+        float r[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+        fwht8(r);
+        float *dst = buf + (size_t)b * N + 8 * v;
+        *reinterpret_cast<float4 *>(dst) = make_float4(r[0], r[1], r[2], r[3]);
+        *reinterpret_cast<float4 *>(dst + 4) = make_float4(r[4], r[5], r[6], r[7]);
+    }
+    __syncthreads();
+    const Seg seg{0, N, 0.f};
+    fwht_segments<THREADS>(buf, B, N, &seg, 1);
+    const float nrm = __frsqrt_rn((float)N);
+    for (int e = threadIdx.x; e < B * nvec; e += THREADS) {
+        const int b = e / nvec, v = e - b * nvec;
+        const int col = o + 8 * v;
+        const uint32_t sb = (p.sout_bits[col >> 5] >> (col & 31)) & 0xFFu;
+        const float *r = buf + (size_t)b * N + 8 * v;
+        float y[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) y[j] = ((sb >> j) & 1u) ? -(r[j] * nrm) : r[j] * nrm;
+        const size_t off = (size_t)b * p.m + col;
+        if (p.y_dtype == 2) {  // fp32
+            float4 *yp = reinterpret_cast<float4 *>(static_cast<float *>(p.y) + off);
+            yp[0] = make_float4(y[0], y[1], y[2], y[3]);
+            yp[1] = make_float4(y[4], y[5], y[6], y[7]);
+        } else {
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (p.y_dtype == 1) {  // bf16
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(y[2 * j], y[2 * j + 1]);
+                    w[j] = *reinterpret_cast<const uint32_t *>(&h);
+                } else {
+                    const __half2 h = __floats2half2_rn(y[2 * j], y[2 * j + 1]);
+                    w[j] = *reinterpret_cast<const uint32_t *>(&h);
+                }
+            }
+            *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.y) + off) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
+template <int BPW, int NT, bool FIN>
 __global__ void __launch_bounds__(gemv_warps(NT) * 32, 1) gemv_kernel(GemvParams p) {
     constexpr int WARPS = gemv_warps(NT);
+    constexpr int THREADS = WARPS * 32;
     constexpr int BAND_ROWS = WARPS * GLQ_ROW_TILE;
     extern __shared__ __align__(16) uint4 smem_u4[];
     __shared__ __align__(8) uint64_t bar;
     __shared__ int s_last;
+    __shared__ TaskRow s_rows[GLQ_DECODE_MAX_B];
+    __shared__ unsigned s_max[GLQ_DECODE_MAX_B];
+    __shared__ int s_pending[GLQ_MAX_BLOCKS];
+    __shared__ Seg s_segs[GLQ_MAX_BLOCKS];
+    __shared__ int s_npending;
     uint32_t *T = reinterpret_cast<uint32_t *>(smem_u4);
     uint4 *R8 = smem_u4 + p.table_words / 4;
+    // fused input: [xs: B x klen/8 uint4][xhs: B x klen halves (3 bpw)][u: B x klen floats]
+    const int klen_max = min(p.cps, p.KC) * GLQ_CHUNK_K;
+    uint4 *xs = R8 + (BPW == 3 ? 256 : 0);
+    __half *xhs = reinterpret_cast<__half *>(xs + (size_t)p.B * klen_max / 8);
+    float *ubuf = reinterpret_cast<float *>(xhs + (BPW == 3 ? (size_t)p.B * klen_max : 0));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int ntasks = p.bands * p.splits;
 
     // 1. codebook into shared memory (constant data: before the PDL wait)
-    if (tid == 0) mbar_init(&bar, 1);
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        s_npending = 0;
+    }
     __syncthreads();
     if (tid == 0) {
         const uint32_t tbytes = (uint32_t)p.table_words * 4u;
@@ -178,15 +473,15 @@ __global__ void __launch_bounds__(gemv_warps(NT) * 32, 1) gemv_kernel(GemvParams
         mbar_wait_bounded(&bar, 0, TABLE_WAIT_POLLS);  // let the copy land before exiting
         return;
     }
-    // 3. activations and row info come from the input-RHT kernel
+    // 3. activations (and row info) come from the previous kernel
     pdl_wait();
 
     const bool has0 = g < p.B, has1 = (g + 8) < p.B;
     const size_t xq_row = (size_t)p.n_pad / 8;  // uint4 (one group) per 8 columns
-    const uint4 *xq0 = reinterpret_cast<const uint4 *>(p.xq) + (size_t)g * xq_row + t;
-    const uint4 *xq1 = reinterpret_cast<const uint4 *>(p.xq) + (size_t)(g + 8) * xq_row + t;
-    const __half *xh0 = p.xh ? p.xh + (size_t)g * p.n_pad + 8 * t : nullptr;
-    const __half *xh1 = p.xh ? p.xh + (size_t)(g + 8) * p.n_pad + 8 * t : nullptr;
+    const uint4 *xq0 = FIN ? nullptr : reinterpret_cast<const uint4 *>(p.xq) + (size_t)g * xq_row + t;
+    const uint4 *xq1 = FIN ? nullptr : reinterpret_cast<const uint4 *>(p.xq) + (size_t)(g + 8) * xq_row + t;
+    const __half *xh0 = (!FIN && p.xh) ? p.xh + (size_t)g * p.n_pad + 8 * t : nullptr;
+    const __half *xh1 = (!FIN && p.xh) ? p.xh + (size_t)(g + 8) * p.n_pad + 8 * t : nullptr;
 
     for (bool first = true; task < ntasks; task += gridDim.x, first = false) {
         if (!first) {
@@ -194,6 +489,11 @@ __global__ void __launch_bounds__(gemv_warps(NT) * 32, 1) gemv_kernel(GemvParams
             prefetch();
         }
         const int band = task / p.splits, split = task - band * p.splits;
+        const int klen = (c1 - c0) * GLQ_CHUNK_K;
+        if (FIN) {
+            __syncthreads();  // the previous task's activations and row info are no longer read
+            fused_input<BPW, THREADS>(p, c0 * GLQ_CHUNK_K, klen, xs, xhs, ubuf, s_rows, s_max, s_segs);
+        }
         Acc acc1, acc2;
         zero<NT>(acc1);
         zero<NT>(acc2);
@@ -203,10 +503,19 @@ __global__ void __launch_bounds__(gemv_warps(NT) * 32, 1) gemv_kernel(GemvParams
             const size_t base = ((size_t)rt * p.KC + c0) * 32 + lane;
             const uint4 *pq1 = p.idx1 + base + GEMV_PREFETCH * 32;  // next chunk to load
             const size_t q2_off = base + GEMV_PREFETCH * 32;
-            const uint4 *px0 = xq0 + (size_t)c0 * GLQ_GROUPS_PER_CHUNK;
-            const uint4 *px1 = xq1 + (size_t)c0 * GLQ_GROUPS_PER_CHUNK;
-            const __half *ph0 = xh0 ? xh0 + (size_t)c0 * GLQ_CHUNK_K : nullptr;
-            const __half *ph1 = xh1 ? xh1 + (size_t)c0 * GLQ_CHUNK_K : nullptr;
+            const uint4 *px0, *px1;
+            const __half *ph0, *ph1;
+            if (FIN) {  // the task's range in shared memory, row stride klen
+                px0 = xs + (size_t)g * (klen / 8) + t;
+                px1 = xs + (size_t)(g + 8) * (klen / 8) + t;
+                ph0 = BPW == 3 ? xhs + (size_t)g * klen + 8 * t : nullptr;
+                ph1 = BPW == 3 ? xhs + (size_t)(g + 8) * klen + 8 * t : nullptr;
+            } else {
+                px0 = xq0 + (size_t)c0 * GLQ_GROUPS_PER_CHUNK;
+                px1 = xq1 + (size_t)c0 * GLQ_GROUPS_PER_CHUNK;
+                ph0 = xh0 ? xh0 + (size_t)c0 * GLQ_CHUNK_K : nullptr;
+                ph1 = xh1 ? xh1 + (size_t)c0 * GLQ_CHUNK_K : nullptr;
+            }
             int ahead = c0 + GEMV_PREFETCH;
             for (int c = c0; c < c1; c += GEMV_PREFETCH) {
 #pragma unroll
@@ -219,8 +528,8 @@ __global__ void __launch_bounds__(gemv_warps(NT) * 32, 1) gemv_kernel(GemvParams
                         }
                         pq1 += 32;
                         ++ahead;
-                        process_chunk<BPW, NT>(T, R8, p.fold, q1, q2, px0, px1, ph0, ph1, has0, has1, acc1,
-                                               acc2, accr);
+                        process_chunk<BPW, NT, FIN>(T, R8, p.fold, q1, q2, px0, px1, ph0, ph1, has0, has1,
+                                                    acc1, acc2, accr);
                         px0 += GLQ_GROUPS_PER_CHUNK;
                         px1 += GLQ_GROUPS_PER_CHUNK;
                         if (BPW == 3) {
@@ -242,8 +551,12 @@ __global__ void __launch_bounds__(gemv_warps(NT) * 32, 1) gemv_kernel(GemvParams
                         double D = exact_sum(acc1.hi[nt][j], acc1.lo[nt][j]);
                         if (BPW == 4) D += p.rs_d * exact_sum(acc2.hi[nt][j], acc2.lo[nt][j]);
                         if (BPW == 3) D += p.rs_d * (double)accr[nt][j];
+                        if (FIN) {  // this range's own scale and sum: a partial of x . w
+                            D = (D - (double)GLQ_NIB_OFFSET * p.corr_mult * (double)s_rows[b].sum_x) *
+                                (0.5 * (double)s_rows[b].inv_scale);
+                        }
                         if (p.splits == 1) {
-                            p.z[(size_t)b * p.m_pad + row] = finish_z(p, b, D);
+                            p.z[(size_t)b * p.m_pad + row] = FIN ? (float)(D * (double)p.ws) : finish_z(p, b, D);
                         } else {
                             __stcg(p.partials + ((size_t)split * p.B + b) * p.m_pad + row, D);
                         }
@@ -251,49 +564,86 @@ __global__ void __launch_bounds__(gemv_warps(NT) * 32, 1) gemv_kernel(GemvParams
                 }
             }
         }
-        if (p.splits == 1) continue;
 
         // 4. band completion: the last split to finish reduces the band.  The
         // CTA barrier orders every thread's partial stores before thread 0's
         // release-acquire increment; the barrier after it hands the acquire to
         // the threads that read the other CTAs' partials.
-        __syncthreads();
-        if (tid == 0) {
-            const unsigned prev = atom_add_acq_rel_gpu(&p.counters[band], 1u);
-            s_last = prev == (unsigned)(p.splits - 1);
-        }
-        __syncthreads();
-        if (s_last) {
-            const int r_base = band * BAND_ROWS;
-            const int rows = min(BAND_ROWS, p.m_pad - r_base);
-            for (int e = tid; e < rows * p.B; e += WARPS * 32) {
-                const int b = e / rows, row = r_base + (e - b * rows);
-                double D = 0.0;
-                for (int s = 0; s < p.splits; ++s)  // fixed order
-                    D += __ldcg(p.partials + ((size_t)s * p.B + b) * p.m_pad + row);
-                p.z[(size_t)b * p.m_pad + row] = finish_z(p, b, D);
+        bool band_done = true;
+        if (p.splits > 1) {
+            __syncthreads();
+            if (tid == 0) {
+                const unsigned prev = atom_add_acq_rel_gpu(&p.counters[band], 1u);
+                s_last = prev == (unsigned)(p.splits - 1);
             }
-            if (tid == 0) p.counters[band] = 0u;
+            __syncthreads();
+            band_done = s_last;
+            if (band_done) {
+                const int r_base = band * BAND_ROWS;
+                const int rows = min(BAND_ROWS, p.m_pad - r_base);
+                for (int e = tid; e < rows * p.B; e += THREADS) {
+                    const int b = e / rows, row = r_base + (e - b * rows);
+                    double D = 0.0;
+                    for (int s = 0; s < p.splits; ++s)  // fixed order
+                        D += __ldcg(p.partials + ((size_t)s * p.B + b) * p.m_pad + row);
+                    p.z[(size_t)b * p.m_pad + row] = FIN ? (float)(D * (double)p.ws) : finish_z(p, b, D);
+                }
+                if (tid == 0) p.counters[band] = 0u;
+            }
         }
-        __syncthreads();  // s_last is reused by the next task
+        // 5. output blocks: the band whose z completes a Hadamard block of m
+        // queues that block's transform for the end of this CTA's tasks
+        if (p.fuse_out && band_done) {
+            __syncthreads();  // the band's z is written
+            if (tid == 0) {
+                __threadfence();
+                const int r0 = band * BAND_ROWS, r1 = min(r0 + BAND_ROWS, p.m);
+                for (int bi = 0; bi < p.nblk_m; ++bi) {
+                    const int o = p.blk_off_m[bi], N = p.blk_len_m[bi];
+                    if (r0 < o + N && o < r1) {
+                        const unsigned prev = atom_add_acq_rel_gpu(&p.blk_cnt[bi], 1u);
+                        if (prev == (unsigned)(p.blk_bands[bi] - 1)) {
+                            s_pending[s_npending++] = bi;
+                            p.blk_cnt[bi] = 0u;
+                        }
+                    }
+                }
+            }
+        }
+        __syncthreads();  // s_last and the shared activations are reused by the next task
+    }
+    if (p.fuse_out) {
+        __syncthreads();
+        const int np = s_npending;
+        // the table is no longer needed: its shared memory holds the block
+        for (int i = 0; i < np; ++i) {
+            fused_output<THREADS>(p, s_pending[i], reinterpret_cast<float *>(smem_u4));
+            __syncthreads();
+        }
     }
 }
 
-template <int BPW, int NT>
+template <int BPW, int NT, bool FIN>
 cudaError_t launch_t(const GemvParams &p, int grid, cudaStream_t s, bool pdl) {
-    const size_t smem = gemv_smem_bytes(p.table_words, BPW);
-    // raised once to the largest table the library accepts (never lowered:
+    const size_t smem = FIN ? gemv_fused_smem_bytes(p.table_words, BPW, p.B, min(p.cps, p.KC) * GLQ_CHUNK_K)
+                            : gemv_smem_bytes(p.table_words, BPW);
+    // raised once to the largest the library launches with (never lowered:
     // captured graphs replay against the attribute value at replay time)
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<BPW, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)gemv_smem_bytes(GLQ_TABLE_MAX_WORDS, BPW));
+        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<BPW, NT, FIN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)GEMV_SMEM_LIMIT);
         if (e != cudaSuccess) return e;
         configured = true;
     }
+    if (smem > GEMV_SMEM_LIMIT) return cudaErrorInvalidValue;
+    if (p.fuse_out) {  // the output block is transformed in the table's shared memory
+        for (int bi = 0; bi < p.nblk_m; ++bi)
+            if ((size_t)p.B * p.blk_len_m[bi] * sizeof(float) > smem) return cudaErrorInvalidValue;
+    }
     GemvParams q = p;
     void *args[] = {&q};
-    return launch_ex((const void *)gemv_kernel<BPW, NT>, dim3(grid), dim3(gemv_warps(NT) * 32), smem, s,
+    return launch_ex((const void *)gemv_kernel<BPW, NT, FIN>, dim3(grid), dim3(gemv_warps(NT) * 32), smem, s,
                      pdl, args);
 }
 
@@ -302,25 +652,33 @@ cudaError_t launch_t(const GemvParams &p, int grid, cudaStream_t s, bool pdl) {
 // Split of the chunk range so that (bands x splits) tasks spread over the
 // persistent grid with the least makespan (in chunks per CTA), with a small
 // charge per task for the band reduction.
-GemvPlan plan_gemv(int RT, int KC, int num_sms, int warps) {
+GemvPlan plan_gemv(int RT, int KC, int num_sms, int warps, bool pow2, int max_cps, int max_splits) {
     GemvPlan pl{};
     pl.bands = (RT + warps - 1) / warps;
-    int best_s = 1;
+    int best_cps = 0;
     double best = 1e30;
-    for (int s = 1; s <= KC; ++s) {
-        const int cps = (KC + s - 1) / s;
-        const int used = (KC + cps - 1) / cps;  // splits actually populated
-        if (used != s) continue;
+    // candidate chunk counts per split: every count that populates all its
+    // splits, or the powers of two (the last split may be short)
+    for (int cps = 1; cps <= (pow2 ? 2 * KC : KC); cps = pow2 ? 2 * cps : cps + 1) {
+        const int s = (KC + cps - 1) / cps;
+        if (!pow2 && (KC + s - 1) / s != cps) continue;
+        if (cps > max_cps || s > max_splits) continue;
         const long long tasks = (long long)pl.bands * s;
         const long long waves = (tasks + num_sms - 1) / num_sms;
-        const double cost = (double)waves * (cps + (s > 1 ? 0.5 : 0.0)) + 0.02 * s;
+        const int work = cps < KC ? cps : KC;
+        const double cost = (double)waves * (work + (s > 1 ? 0.5 : 0.0)) + 0.02 * s;
         if (cost < best) {
             best = cost;
-            best_s = s;
+            best_cps = cps;
         }
+        if (s == 1) break;
     }
-    pl.splits = best_s;
-    pl.cps = (KC + best_s - 1) / best_s;
+    if (best_cps == 0) {  // nothing within the bounds: the fewest splits the bound allows
+        best_cps = 1;
+        while ((KC + best_cps - 1) / best_cps > max_splits) best_cps = pow2 ? 2 * best_cps : best_cps + 1;
+    }
+    pl.cps = best_cps;
+    pl.splits = (KC + best_cps - 1) / best_cps;
     const long long tasks = (long long)pl.bands * pl.splits;
     pl.grid = (int)(tasks < num_sms ? tasks : num_sms);
     return pl;
@@ -330,14 +688,24 @@ size_t gemv_smem_bytes(int table_words, int bpw) {
     return (size_t)table_words * 4 + (bpw == 3 ? 256 * 16 : 0);
 }
 
-cudaError_t launch_gemv(const GemvParams &p, int bpw, int grid, cudaStream_t s, bool pdl) {
+size_t gemv_fused_smem_bytes(int table_words, int bpw, int B, int klen) {
+    // the table is a multiple of 4 words, so the activation area is 16-byte aligned
+    return gemv_smem_bytes(table_words, bpw) + (size_t)B * klen * (2 + (bpw == 3 ? 2 : 0) + 4);
+}
+
+template <bool FIN>
+cudaError_t launch_sel(const GemvParams &p, int bpw, int grid, cudaStream_t s, bool pdl) {
     const bool two = p.B > 8;
     switch (bpw) {
-        case 2: return two ? launch_t<2, 2>(p, grid, s, pdl) : launch_t<2, 1>(p, grid, s, pdl);
-        case 3: return two ? launch_t<3, 2>(p, grid, s, pdl) : launch_t<3, 1>(p, grid, s, pdl);
-        case 4: return two ? launch_t<4, 2>(p, grid, s, pdl) : launch_t<4, 1>(p, grid, s, pdl);
+        case 2: return two ? launch_t<2, 2, FIN>(p, grid, s, pdl) : launch_t<2, 1, FIN>(p, grid, s, pdl);
+        case 3: return two ? launch_t<3, 2, FIN>(p, grid, s, pdl) : launch_t<3, 1, FIN>(p, grid, s, pdl);
+        case 4: return two ? launch_t<4, 2, FIN>(p, grid, s, pdl) : launch_t<4, 1, FIN>(p, grid, s, pdl);
         default: return cudaErrorInvalidValue;
     }
+}
+
+cudaError_t launch_gemv(const GemvParams &p, int bpw, int grid, cudaStream_t s, bool pdl, bool fused_in) {
+    return fused_in ? launch_sel<true>(p, bpw, grid, s, pdl) : launch_sel<false>(p, bpw, grid, s, pdl);
 }
 
 }  // namespace glq

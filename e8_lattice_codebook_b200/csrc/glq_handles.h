@@ -44,6 +44,13 @@ struct glq_workspace {
     unsigned *cnt = nullptr;      // [bands], zero between calls
 };
 
+// Hadamard block decomposition of a size (descending powers of two)
+struct glq_hblocks {
+    int count = 0;
+    int off[GLQ_MAX_BLOCKS] = {};
+    int len[GLQ_MAX_BLOCKS] = {};
+};
+
 struct glq_layer_s {
     int64_t m = 0, n = 0, m_pad = 0, n_pad = 0;
     int bpw = 0, RT = 0, KC = 0, G = 0;
@@ -64,18 +71,42 @@ struct glq_layer_s {
     int64_t last_prefill_B = 0;  // batch of the last tensor-core call (glq_prefill_replay)
     glq_workspace wsp;
     glq_prefill_ws pws;
+    glq_hblocks hb_n, hb_m;
+    unsigned *d_blk_cnt = nullptr;  // [GLQ_MAX_BLOCKS] output-block counters, zero between calls
+    int fusion = -1;                // GLQ_FUSE_* bits, or -1: the library default (glq_layer_set_fusion)
+    // the last decode launch (glq_gemv_replay)
+    const void *last_x = nullptr;
+    void *last_y = nullptr;
+    int last_x_bf16 = 0, last_y_dtype = 0;
+    bool last_fin = false, last_fout = false;
+    glq::GemvPlan last_plan{};
     size_t device_bytes = 0;
 };
 
 namespace glq {
 
-// Input RHT -> codebook GEMV -> output RHT for nb <= 16 tokens, in the
-// buffers of `w`, with the GEMV split plan (splits, cps, grid).
-cudaError_t run_decode(glq_layer L, const glq_workspace &w, const GemvPlan &plan, const void *x,
-                       bool x_bf16, void *y, int y_dtype, int nb, cudaStream_t s);
+// How one decode call of nb <= 16 tokens runs: the GEMV split plan and
+// whether the input / output transforms are fused into the GEMV launch.
+struct DecodeCfg {
+    GemvPlan plan{};
+    bool fin = false, fout = false;
+};
 
-GemvParams gemv_params(glq_layer L, const glq_workspace &w, const GemvPlan &plan, int nb);
+// max_cps bounds the chunks per split (callers with a small partial-sum
+// buffer); x and y decide the fused paths' alignment condition.
+DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y_dtype, int max_cps = 1 << 30);
+
+// (input RHT ->) codebook GEMV (-> output RHT) for nb <= 16 tokens, in the
+// buffers of `w`.
+cudaError_t run_decode(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg, const void *x, bool x_bf16,
+                       void *y, int y_dtype, int nb, cudaStream_t s);
+
+GemvParams gemv_params(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg, int nb, const void *x,
+                       bool x_bf16, void *y, int y_dtype);
 
 inline const GemvPlan &plan_for(glq_layer L, int nb) { return L->plan[nb > 8 ? 1 : 0]; }
+
+// largest split count any decode configuration of nb tokens can use
+int max_decode_splits(glq_layer L, int nb);
 
 }  // namespace glq

@@ -72,6 +72,24 @@ struct GemvParams {
     float *z;              // [B][m_pad]
     int m_pad;
     unsigned *err;
+    // ---- fused transforms (small B) ----
+    // input: every task rotates, scales and quantises its own column range
+    // of x in shared memory (no separate input-RHT launch)
+    const void *x;         // [B][n] fp16 / bf16, rows 16-byte aligned
+    int x_bf16, n;
+    const uint32_t *sin_bits;
+    int nblk_n;            // Hadamard blocks of n: descending powers of two
+    int blk_off_n[GLQ_MAX_BLOCKS], blk_len_n[GLQ_MAX_BLOCKS];
+    // output: the last band to finish a Hadamard block of m transforms it
+    // in shared memory and writes y (no separate output-RHT launch)
+    int fuse_out;
+    void *y;               // [B][m]
+    int y_dtype, m;
+    const uint32_t *sout_bits;
+    int nblk_m;
+    int blk_off_m[GLQ_MAX_BLOCKS], blk_len_m[GLQ_MAX_BLOCKS];
+    int blk_bands[GLQ_MAX_BLOCKS];  // bands whose rows meet block i
+    unsigned *blk_cnt;     // [GLQ_MAX_BLOCKS], zero between launches
 };
 
 struct PrefillParams {
@@ -122,13 +140,22 @@ inline cudaError_t launch_ex(const void *fn, dim3 grid, dim3 block, size_t smem,
 // programmatic dependent launch on the stream.
 cudaError_t launch_rht_in(const RhtInParams &p, cudaStream_t s, bool pdl);
 cudaError_t launch_rht_out(const RhtOutParams &p, cudaStream_t s, bool pdl);
-cudaError_t launch_gemv(const GemvParams &p, int bpw, int grid, cudaStream_t s, bool pdl);
+cudaError_t launch_gemv(const GemvParams &p, int bpw, int grid, cudaStream_t s, bool pdl, bool fused_in = false);
+// dynamic shared memory of a launch with the input transform fused
+// (the table, the residual table, the task's activations and scratch)
+size_t gemv_fused_smem_bytes(int table_words, int bpw, int B, int klen);
+// (227 KB per block, less room for the kernel's static shared memory)
+constexpr size_t GEMV_SMEM_LIMIT = 226 * 1024;
 
 // GEMV work split: bands of row tiles x splits of the chunk range.
 struct GemvPlan {
     int bands, splits, cps, grid;
 };
-GemvPlan plan_gemv(int RT, int KC, int num_sms, int warps);
+// Work split of the GEMV over a persistent grid.  pow2: chunks per split a
+// power of two (aligned column ranges, required by the fused input
+// transform), at most max_cps chunks per split and max_splits splits.
+GemvPlan plan_gemv(int RT, int KC, int num_sms, int warps, bool pow2 = false, int max_cps = 1 << 30,
+                   int max_splits = 1 << 30);
 cudaError_t launch_dequant(const DequantParams &p, cudaStream_t s);
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &xmap, int grid, cudaStream_t s, bool pdl);
 size_t prefill_smem_bytes();

@@ -67,6 +67,8 @@ extern "C" glq_status glq_linear_noalloc(glq_layer L, const void *x_dev, glq_dty
     if (y_dtype != x_dtype && y_dtype != GLQ_F32) return GLQ_ERR_DTYPE;
     if (B == 0) return GLQ_OK;
     if (!x_dev || !y_dev) return GLQ_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(x_dev) & 15) || (reinterpret_cast<uintptr_t>(y_dev) & 15))
+        return GLQ_ERR_INVALID_ARG;
 
     int prev = -1;
     if (cudaGetDevice(&prev) != cudaSuccess) {
@@ -86,22 +88,21 @@ extern "C" glq_status glq_linear_noalloc(glq_layer L, const void *x_dev, glq_dty
     const size_t xh_b = L->bpw == 3 ? align256((size_t)B * L->n_pad * sizeof(__half)) : 0;
     const size_t info_b = align256((size_t)B * sizeof(glq_rowinfo));
     const size_t z_b = align256((size_t)B * L->m_pad * sizeof(float));
-    glq::GemvPlan plan = glq::plan_for(L, (int)B);
-    const size_t cnt_b = align256((size_t)plan.bands * sizeof(unsigned));
+    const int max_bands = std::max(L->plan[0].bands, L->plan[1].bands);
+    const size_t cnt_b = align256((size_t)max_bands * sizeof(unsigned));
     const size_t fixed = xq_b + xh_b + info_b + z_b + cnt_b;
     const size_t per_split = (size_t)B * L->m_pad * sizeof(double);
+    glq::DecodeCfg cfg;
     if (st == GLQ_OK) {
         if (fixed > GLQ_NOALLOC_SCRATCH_BYTES) {
             st = GLQ_ERR_SHAPE;  // the activations and outputs alone do not fit
         } else {
-            // narrow the split-K plan until its partial sums fit (one split
+            // bound the split-K plan so that its partial sums fit (one split
             // needs none: the GEMV then writes z directly)
             const size_t room = GLQ_NOALLOC_SCRATCH_BYTES - fixed;
-            while (plan.splits > 1 && (size_t)plan.splits * per_split > room) {
-                plan.cps = plan.cps + 1;
-                plan.splits = (L->KC + plan.cps - 1) / plan.cps;
-            }
-            plan.grid = (int)std::min<int64_t>((int64_t)plan.bands * plan.splits, L->num_sms);
+            const int max_splits = (int)std::max<size_t>(1, std::min<size_t>(room / per_split, 1u << 30));
+            cfg = glq::decode_config(L, (int)B, x_dev, y_dev, (int)y_dtype, max_splits);
+            if (cfg.plan.splits > 1 && (size_t)cfg.plan.splits * per_split > room) st = GLQ_ERR_SHAPE;
         }
     }
     if (st == GLQ_OK) {
@@ -112,12 +113,12 @@ extern "C" glq_status glq_linear_noalloc(glq_layer L, const void *x_dev, glq_dty
         w.info = reinterpret_cast<glq_rowinfo *>(p + xq_b + xh_b);
         w.z = reinterpret_cast<float *>(p + xq_b + xh_b + info_b);
         w.cnt = reinterpret_cast<unsigned *>(p + xq_b + xh_b + info_b + z_b);
-        w.part = plan.splits > 1 ? reinterpret_cast<double *>(p + fixed) : nullptr;
+        w.part = cfg.plan.splits > 1 ? reinterpret_cast<double *>(p + fixed) : nullptr;
         cudaStream_t s = static_cast<cudaStream_t>(stream);
         // the band counters must start at zero (the array keeps whatever the
         // previous call, of any layer, left there)
-        if (cudaMemsetAsync(w.cnt, 0, (size_t)plan.bands * sizeof(unsigned), s) != cudaSuccess ||
-            glq::run_decode(L, w, plan, x_dev, x_dtype == GLQ_BF16, y_dev, (int)y_dtype, (int)B, s) !=
+        if (cudaMemsetAsync(w.cnt, 0, (size_t)cfg.plan.bands * sizeof(unsigned), s) != cudaSuccess ||
+            glq::run_decode(L, w, cfg, x_dev, x_dtype == GLQ_BF16, y_dev, (int)y_dtype, (int)B, s) !=
                 cudaSuccess) {
             cudaGetLastError();
             st = GLQ_ERR_CUDA;

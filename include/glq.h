@@ -150,18 +150,45 @@ GLQ_API glq_status glq_layer_reserve(glq_layer layer, int64_t max_B);
  * Definition: the layer formula above (glq 0.5.1 PyPI page, "How it works",
  * "Inference kernels"; GLQ v0.3.2 release notes, input_rht ->
  * fused_linear_block_diag -> output_rht).
- * x_dev: device [B][n] row-major, dtype x_dtype (GLQ_F16 or GLQ_BF16).
- * y_dev: device [B][m] row-major, dtype y_dtype (== x_dtype, or GLQ_F32).
+ * x_dev: device [B][n] row-major, dtype x_dtype (GLQ_F16 or GLQ_BF16),
+ *   16-byte aligned.
+ * y_dev: device [B][m] row-major, dtype y_dtype (== x_dtype, or GLQ_F32),
+ *   16-byte aligned.
  * B >= 0 (B == 0 is a no-op).  stream: cudaStream_t.
- * Paths: B <= 16 runs the decode kernels (input RHT, codebook GEMV on the
- *   legacy warp MMA with an on-chip codebook, output RHT); B > 16 runs the
- *   tensor-core path (input RHT, tcgen05/TMEM GEMM with a dequantising
- *   producer, output RHT).  Accumulation is fp32 on every path.
- * Errors: GLQ_ERR_INVALID_ARG, GLQ_ERR_DTYPE, GLQ_ERR_SHAPE, GLQ_ERR_OOM
- *   (workspace growth), GLQ_ERR_CUDA (launch failure).  Asynchronous.
+ * Paths: B <= 16 runs the decode path: the codebook GEMV on the legacy warp
+ *   MMA with an on-chip codebook, with both transforms fused into the same
+ *   launch when B times the largest Hadamard block is at most 32768 values
+ *   (one kernel per call), else input RHT, GEMV and output RHT as three
+ *   kernels (see glq_layer_set_fusion); B > 16 runs the tensor-core path
+ *   (input RHT, tcgen05/TMEM GEMM with a dequantising producer, output RHT).
+ *   The GEMV accumulates exactly in integers (fp64 across splits); the
+ *   tensor-core path accumulates in fp32.
+ * Errors: GLQ_ERR_INVALID_ARG (null or misaligned pointer), GLQ_ERR_DTYPE,
+ *   GLQ_ERR_SHAPE, GLQ_ERR_OOM (workspace growth), GLQ_ERR_CUDA (launch
+ *   failure).  Asynchronous.
  */
 GLQ_API glq_status glq_linear(glq_layer layer, const void *x_dev, glq_dtype x_dtype, void *y_dev,
                       glq_dtype y_dtype, int64_t B, void *stream);
+
+/*
+ * glq_layer_set_fusion -- choose how decode calls (B <= 16) run their two
+ * transforms.  flags is a bit set: GLQ_FUSE_INPUT fuses the input RHT into
+ * the GEMV launch (each task rotates its own aligned column range of x)
+ * whenever B times the largest Hadamard block of n is at most 32768 values;
+ * GLQ_FUSE_OUTPUT lets the last band of each Hadamard block of m rotate that
+ * block in the same launch when B times the largest block of m fits the
+ * library's bound; a cleared bit runs that transform as its own kernel.  The
+ * default is the library's fastest setting (GLQ_FUSE_DEFAULT).  With both bits
+ * cleared, every token's output is bitwise independent of the batch size for
+ * B <= 16; otherwise that holds among batch sizes that take the same path.
+ * All settings are bitwise reproducible run to run ("Bit-exact
+ * determinism", glq 0.5.1 PyPI page, "Inference kernels") and agree within
+ * the parity bound.  Errors: GLQ_ERR_INVALID_ARG (unknown bits).
+ */
+#define GLQ_FUSE_INPUT 1
+#define GLQ_FUSE_OUTPUT 2
+#define GLQ_FUSE_DEFAULT (-1)
+GLQ_API glq_status glq_layer_set_fusion(glq_layer layer, int32_t flags);
 
 /*
  * glq_dequant_reference -- materialise W^ (fp32, no Hadamards, ws included)

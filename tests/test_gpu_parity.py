@@ -133,17 +133,60 @@ def test_linear_workloads_full_size(dev, key, li):
 
 
 def test_determinism_and_batch_invariance(dev):
+    """Run to run: bitwise on both decode paths.  Per token across batch
+    sizes: bitwise for every B <= 16 with the transforms as separate kernels;
+    with fusion on, within B <= 8 (fused here: 8 x 4096 values) and within
+    9 <= B <= 16 (separate kernels here)."""
     wl = gi.WORKLOADS["24b-decode-4bpw"]
     L = gi.workload_layer(wl, 0)
     lay = dev.layer(L)
     xb = gi.workload_x(wl, 0, 16)
     x = to_torch_x(xb, "bf16")
-    y1 = lay(x, out_dtype=torch.float32)
-    y2 = lay(x, out_dtype=torch.float32)
-    assert torch.equal(y1, y2)
-    for B in (1, 2, 4, 8):
-        yb = lay(x[:B].contiguous(), out_dtype=torch.float32)
-        assert torch.equal(yb, y1[:B]), B
+    y16 = lay(x, out_dtype=torch.float32)
+    assert torch.equal(y16, lay(x, out_dtype=torch.float32))
+    y8 = lay(x[:8].contiguous(), out_dtype=torch.float32)
+    assert torch.equal(y8, lay(x[:8].contiguous(), out_dtype=torch.float32))
+    for B in (1, 2, 4):
+        assert torch.equal(lay(x[:B].contiguous(), out_dtype=torch.float32), y8[:B]), B
+    for B in (9, 12):
+        assert torch.equal(lay(x[:B].contiguous(), out_dtype=torch.float32), y16[:B]), B
+    lay.set_fusion(0)
+    try:
+        s16 = lay(x, out_dtype=torch.float32)
+        assert torch.equal(s16, y16)  # B = 16 took the separate kernels before too
+        for B in (1, 2, 4, 8):
+            assert torch.equal(lay(x[:B].contiguous(), out_dtype=torch.float32), s16[:B]), B
+    finally:
+        lay.set_fusion(-1)
+
+
+FUSION_CASES = [  # m, n, bpw, B, x dtype: fused input and output transforms when aligned
+    (2048, 2048, 4, 1, "bf16"), (11008, 2048, 4, 1, "bf16"), (2048, 11008, 4, 1, "bf16"),
+    (960, 2560, 3, 2, "f16"), (2560, 960, 3, 8, "f16"), (1024, 1024, 2, 16, "f16"),
+    (4096, 5120, 4, 4, "bf16"), (5120, 32768, 2, 1, "bf16"), (32768, 1024, 2, 1, "f16"),
+    (136, 8200, 4, 3, "bf16"),
+]
+
+
+@pytest.mark.parametrize("m,n,bpw,B,xdt", FUSION_CASES)
+def test_fused_and_separate_transforms(dev, m, n, bpw, B, xdt):
+    """The same layer with the transforms fused into the GEMV launch and as
+    separate kernels, and each one alone (glq_layer_set_fusion): all within
+    the bound of the oracle, every token and output."""
+    L = gi.make_layer(m + 3 * n, 2, m, n, bpw)
+    xb = gi.make_x(m + 3 * n, 2, B, n, xdt)
+    lay = dev.layer(L)
+    ref = oracle_y(L, xb, xdt)
+    x = to_torch_x(xb, xdt)
+    errs = []
+    for flags in (3, 1, 2, 0):  # both fused, input only, output only, neither
+        lay.set_fusion(flags)
+        y = lay(x, out_dtype=torch.float32).cpu().numpy().astype(np.float64)
+        errs.append(np.max(np.abs(y - ref)))
+        assert errs[-1] <= tolerance(ref), (flags, errs[-1], tolerance(ref))
+    lay.set_fusion(-1)
+    print(f"\nFUSION {m}x{n} bpw {bpw} B={B}: ratios to tol (both, in, out, none) "
+          + " ".join(f"{e / tolerance(ref):.3f}" for e in errs))
 
 
 def test_empty_batch_and_errors(dev):
@@ -158,5 +201,11 @@ def test_empty_batch_and_errors(dev):
     with pytest.raises(glq.GlqError) as e:
         glq.glq_linear(lay.handle, xx.data_ptr(), glq.GLQ_F16, yy.data_ptr(), glq.GLQ_BF16, 2,
                        torch.cuda.current_stream().cuda_stream)
+    # a pointer that is not 16-byte aligned is rejected before any launch
+    yh = torch.zeros((2, 64), dtype=torch.float16, device="cuda")
+    with pytest.raises(glq.GlqError) as e2:
+        glq.glq_linear(lay.handle, xx.data_ptr() + 2, glq.GLQ_F16, yh.data_ptr(), glq.GLQ_F16, 1,
+                       torch.cuda.current_stream().cuda_stream)
+    assert e2.value.status == 1  # INVALID_ARG
     assert e.value.status == 3  # DTYPE
     lay.check()
