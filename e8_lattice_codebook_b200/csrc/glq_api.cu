@@ -150,7 +150,7 @@ glq_status grow_prefill_ws(glq_layer L, int64_t rows) {
 }
 
 // TMA descriptor of the fp16 activations [B][n_pad]: boxes of 64 columns x
-// 256 tokens, 128-byte swizzle, zero fill past the last token.
+// 128 tokens, 128-byte swizzle, zero fill past the last token.
 bool encode_x_map(CUtensorMap *map, const __half *xh, int64_t n_pad, int64_t B) {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
@@ -165,7 +165,7 @@ bool encode_x_map(CUtensorMap *map, const __half *xh, int64_t n_pad, int64_t B) 
     }
     const cuuint64_t dims[2] = {(cuuint64_t)n_pad, (cuuint64_t)B};
     const cuuint64_t strides[1] = {(cuuint64_t)n_pad * sizeof(__half)};
-    const cuuint32_t box[2] = {64, 256};
+    const cuuint32_t box[2] = {64, 128};
     const cuuint32_t estr[2] = {1, 1};
     return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half *>(xh), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -192,11 +192,12 @@ cudaError_t launch_prefill_gemm(glq_layer L, int64_t B, cudaStream_t s, bool pdl
     pp.m_pad = (int)L->m_pad;
     pp.KC = L->KC;
     pp.RT = L->RT;
-    const int tiles_m = (int)((L->m_pad + 127) / 128);
+    const int tr = glq::prefill_tile_rows();
+    const int tiles_m = (int)((L->m_pad + tr - 1) / tr);
     pp.tiles_tok = (int)((B + glq::prefill_tile_tokens() - 1) / glq::prefill_tile_tokens());
     pp.ntiles = tiles_m * pp.tiles_tok;
     pp.err = L->d_err;
-    const int grid = std::min(pp.ntiles, L->num_sms);
+    const int grid = 2 * std::min(pp.ntiles, L->num_sms / 2);  // CTA pairs
     return glq::launch_prefill(pp, xmap, grid, s, pdl);
 }
 
@@ -468,7 +469,6 @@ glq_status glq_codebook_upload(const uint16_t *host_fp16_bits, int32_t entries, 
                 f16[e * 8 + j] = glq::half_bits_of_half_integer(neg ? -y2 : y2);
             }
         }
-        cb->code_f16_entries = (int)ncodes;
         st = dmalloc(&cb->d_table_f16, f16.size() * 2, nullptr);
         if (st == GLQ_OK && cudaMemcpy(cb->d_table_f16, f16.data(), f16.size() * 2, cudaMemcpyHostToDevice) !=
                                 cudaSuccess)

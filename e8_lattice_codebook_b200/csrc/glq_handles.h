@@ -22,8 +22,7 @@ struct glq_codebook_s {
     glq::FoldedTable fold;
     uint32_t *d_table = nullptr;  // table_words words
     int table_words = 0;          // nb rounded up to a multiple of 4
-    uint4 *d_table_f16 = nullptr; // fp16 codewords by folded code [code_f16_entries][8] (tensor-core path)
-    int code_f16_entries = 0;
+    uint4 *d_table_f16 = nullptr; // fp16 codewords by folded code [2 nb - 1][8] (tensor-core path gathers)
 };
 
 // Device buffers of the tensor-core path (B > 16 tokens).

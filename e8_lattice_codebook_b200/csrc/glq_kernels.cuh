@@ -159,7 +159,8 @@ GemvPlan plan_gemv(int RT, int KC, int num_sms, int warps, bool pow2 = false, in
 cudaError_t launch_dequant(const DequantParams &p, cudaStream_t s);
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &xmap, int grid, cudaStream_t s, bool pdl);
 size_t prefill_smem_bytes();
-int prefill_tile_tokens();
+int prefill_tile_tokens();  // tokens of one output tile (a multiple of the TMA box height)
+int prefill_tile_rows();    // weight rows of one output tile (one CTA pair)
 
 // warps per GEMV CTA (one 16-row tile each): 24 for one 8-column MMA tile
 // (B <= 8), 16 for two (B <= 16, more live registers per lane)

@@ -4,26 +4,29 @@
 // that matmuls against codebook-reconstructed weights without materialising
 // W in memory).
 //
-// Design (B200, sm_100a), one CTA per SM, persistent over output tiles of
-// 128 weight rows x 512 tokens:
-//   * warp 0 loads activation tiles (256 tokens x 64 columns, fp16, 128-byte
-//     swizzle) with TMA;
-//   * warp 1 issues tcgen05.mma (kind::f16, M = 128 rows, N = 256 tokens,
-//     K = 16) into two TMEM accumulators (512 columns), so every dequantised
-//     W step serves 512 tokens;
-//   * warps 2-5 are the dequantising producer: for each 64-column step they
-//     read the 16-bit codes of the tile's 128 rows, gather the fp16 codewords
-//     from the L2-resident table (indexed by folded code), form
-//     c = cb1 + rs cb2 and write each 8-weight group as one 16-byte chunk of
-//     the swizzled K-major A operand in shared memory.  The gathers of step
-//     k+1 and the code loads of step k+2 are in flight while step k is
-//     stored, so each step waits on at most one memory round trip;
-//   * warps 6-9 drain each accumulator as soon as its last MMA completes
-//     (tcgen05.ld), apply ws * 2^-e per token and store z (fp32), while the
-//     producer already works on the next tile.
-// Stages are handed over with mbarriers (TMA transaction bytes, producer
-// arrivals, tcgen05.commit); every wait is bounded in time and a timeout
-// aborts the CTA with an error flag instead of hanging.
+// Design (B200, sm_100a): persistent clusters of two CTAs (one per SM)
+// share each tcgen05 MMA (cta_group::2, M = 256 = 128 rows per CTA,
+// N = 256 tokens = 128 per CTA, K = 16), over output tiles of 256 weight rows
+// x 512 tokens (two TMEM accumulators of 256 columns in each CTA), with a
+// four-stage ring of 64-column steps (48 KB per CTA: its 128 rows of W and
+// its 2 x 128 tokens of x):
+//   * warp 0 of each CTA loads its half of the activations with TMA (128
+//     tokens x 64 columns, fp16, 128-byte swizzle), completing on the first
+//     CTA's barrier;
+//   * warps 2-9 (dequantising producer) gather the fp16 codewords of the
+//     CTA's 128 rows x 64 columns from the L2-resident table (16 bytes per
+//     codeword, indexed by folded code), form c = cb1 + rs cb2 and write the
+//     swizzled K-major A tile, then arrive on the first CTA's barrier; the
+//     gathers of the next step and the code loads of the next chunk are in
+//     flight while the current step is stored;
+//   * warp 1 of the first CTA issues the pair's MMAs and commits to both
+//     CTAs' barriers;
+//   * warps 10-13 and 14-17 drain accumulators 0 and 1 with tcgen05.ld as
+//     soon as the tile's last MMA completes and store z = acc ws 2^-e (fp32);
+//     each accumulator is released on its own.
+// Every wait is bounded (4e9 SM clock cycles, about 2 s); a timeout sets the
+// layer's error flag, lets in-flight TMA loads and MMAs land, frees TMEM and
+// returns.
 #include "glq_kernels.cuh"
 #include "glq_sm100.cuh"
 
@@ -31,16 +34,20 @@ namespace glq {
 
 namespace {
 
-constexpr int BM = 128;       // weight rows per tile (MMA M)
-constexpr int BN = 256;       // tokens per accumulator (MMA N)
-constexpr int NACC = 2;       // accumulators per tile (512 tokens)
-constexpr int BK = 64;        // columns per stage (one 128-byte swizzle row of fp16)
-constexpr int STAGES = 2;
-constexpr int W_BYTES = BM * BK * 2;              // 16 KB
-constexpr int X_BYTES = BN * BK * 2;              // 32 KB
-constexpr int STAGE_BYTES = W_BYTES + NACC * X_BYTES;  // 80 KB
-constexpr int THREADS = 320;  // 10 warps: TMA, MMA, 4 producer, 4 epilogue
-constexpr uint64_t WAIT_NS = 2000000000ull;  // wait limit, ns (2 s)
+constexpr int BM = 128;        // weight rows per CTA (the pair's MMA has M = 256)
+constexpr int BN = 256;        // tokens per accumulator (the pair's MMA has N = 256)
+constexpr int BNH = BN / 2;    // tokens per accumulator loaded by one CTA
+constexpr int NACC = 2;        // accumulators per tile (512 tokens)
+constexpr int BK = 64;         // columns per stage (one 128-byte swizzle row of fp16)
+constexpr int STAGES = 4;
+constexpr int W_BYTES = BM * BK * 2;                       // 16 KB
+constexpr int X_BYTES = BNH * BK * 2;                      // 16 KB per accumulator
+constexpr int STAGE_BYTES = W_BYTES + NACC * X_BYTES;     // 48 KB
+constexpr int PRODUCER_WARPS = 8;
+constexpr int EPI_WARPS = 8;                               // four per accumulator
+constexpr int EPI_WARP0 = 2 + PRODUCER_WARPS;             // warps 10-17
+constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;     // 576
+constexpr uint64_t WAIT_CYCLES = 4000000000ull;           // wait limit: 4e9 SM cycles (about 2 s)
 
 __device__ __forceinline__ uint32_t hfma2_bits(uint32_t s, uint32_t b, uint32_t a) {  // s * b + a
     uint32_t r;
@@ -53,99 +60,35 @@ __device__ __forceinline__ uint4 hfma8(uint32_t rs2, uint4 b, uint4 a) {  // rs 
                       hfma2_bits(rs2, b.w, a.w));
 }
 
-// Producer thread pt (0..127) of a W step: rows (g, g + 8) of 16-row tile
-// rt_l = pt / 16, lanes t = 2 tp, 2 tp + 1 of the fragment-native index
-// stream (pt = 16 rt_l + 8 tp + g).  Its 8 groups are i = 4 tt + 2 s2 + hi:
-// row 16 rt_l + g + 8 hi, group 4 s2 + t of the step, t = 2 tp + tt.
-struct StepCodes {
-    uint2 c1[2];     // primary codes, words s = 2h, 2h + 1 of lanes t
-    uint2 c2[2];     // 4 bpw residual codes
-    uint32_t c3[2];  // 3 bpw residual bytes
-};
-
-template <int BPW>
-__device__ __forceinline__ void load_codes(const PrefillParams &p, size_t slot0, int kb, bool live, StepCodes &c) {
-    const int kc = kb >> 1, h = kb & 1;
-#pragma unroll
-    for (int tt = 0; tt < 2; ++tt) {
-        const size_t slot = slot0 + (size_t)kc * 32 + tt;
-        c.c1[tt] = live ? __ldg(reinterpret_cast<const uint2 *>(p.idx1 + slot) + h) : make_uint2(0, 0);
-        if (BPW == 4)
-            c.c2[tt] = live ? __ldg(reinterpret_cast<const uint2 *>(reinterpret_cast<const uint4 *>(p.idx2) + slot) + h)
-                            : make_uint2(0, 0);
-        if (BPW == 3)
-            c.c3[tt] = live ? __ldg(reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint2 *>(p.idx2) + slot) + h)
-                            : 0u;
-    }
-}
-
-struct StepWords {
-    uint4 a[8];  // primary codewords
-    uint4 b[8];  // residual codewords
-};
-
-template <int BPW>
-__device__ __forceinline__ void issue_gathers(const PrefillParams &p, const StepCodes &c, bool live, StepWords &w) {
-#pragma unroll
-    for (int tt = 0; tt < 2; ++tt)
-#pragma unroll
-        for (int s2 = 0; s2 < 2; ++s2)
-#pragma unroll
-            for (int hi = 0; hi < 2; ++hi) {
-                const int i = 4 * tt + 2 * s2 + hi;
-                const uint32_t w1 = s2 ? c.c1[tt].y : c.c1[tt].x;
-                w.a[i] = live ? __ldg(p.cb_f16 + (hi ? (w1 >> 16) : (w1 & 0xFFFFu))) : make_uint4(0, 0, 0, 0);
-                if (BPW == 4) {
-                    const uint32_t w2 = s2 ? c.c2[tt].y : c.c2[tt].x;
-                    w.b[i] = live ? __ldg(p.cb_f16 + (hi ? (w2 >> 16) : (w2 & 0xFFFFu))) : make_uint4(0, 0, 0, 0);
-                } else if (BPW == 3) {
-                    const uint32_t i2 = (c.c3[tt] >> (8 * (2 * s2 + hi))) & 0xFFu;
-                    w.b[i] = live ? __ldg(p.res8 + i2) : make_uint4(0, 0, 0, 0);
-                }
-            }
-}
-
-template <int BPW>
-__device__ __forceinline__ void store_step(const PrefillParams &p, const StepWords &w, uint8_t *wt, int rt_l, int tp,
-                                           int g) {
-#pragma unroll
-    for (int tt = 0; tt < 2; ++tt)
-#pragma unroll
-        for (int s2 = 0; s2 < 2; ++s2)
-#pragma unroll
-            for (int hi = 0; hi < 2; ++hi) {
-                const int i = 4 * tt + 2 * s2 + hi;
-                const uint4 cw = BPW == 2 ? w.a[i] : hfma8(p.rs_h2, w.b[i], w.a[i]);
-                const int row = rt_l * GLQ_ROW_TILE + g + 8 * hi;
-                const int gl = 4 * s2 + 2 * tp + tt;
-                *reinterpret_cast<uint4 *>(wt + row * 128 + ((gl ^ (row & 7)) << 4)) = cw;
-            }
-}
-
 template <int BPW>
 __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_constant__ CUtensorMap xmap,
                                                               PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
-    // x_full: TMA bytes landed; w_full: the 4 producer warps wrote W;
-    // empty: the MMAs of the stage finished (tcgen05.commit);
-    // acc_full / acc_empty: accumulator a computed / drained.
+    // (first CTA) x_full: both CTAs' TMA bytes landed; w_full: both CTAs'
+    // producer warps wrote W; acc_empty: both CTAs drained accumulator a.
+    // (both CTAs) empty: the pair's MMAs of the stage finished; acc_full:
+    // accumulator a computed (commits reach both CTAs).
     __shared__ __align__(8) uint64_t x_full[STAGES], w_full[STAGES], empty_bar[STAGES], acc_full[NACC],
         acc_empty[NACC], mma_done;
     __shared__ uint32_t tmem_holder;
     __shared__ volatile int abort_flag;
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int KB = p.KC * 2;  // 64-column steps
+    const uint32_t rank = sm100::cluster_ctarank();
+    uint32_t cid, ncl;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(cid));
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(ncl));
+    const int KB = p.KC * (GLQ_CHUNK_K / BK);  // 64-column steps
 
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&x_full[s], 1);
-            mbar_init(&w_full[s], 4);
+            mbar_init(&x_full[s], 1);                   // the first CTA's TMA thread
+            mbar_init(&w_full[s], 2 * PRODUCER_WARPS);  // producer warps of both CTAs
             mbar_init(&empty_bar[s], 1);
         }
         for (int a = 0; a < NACC; ++a) {
             mbar_init(&acc_full[a], 1);
-            mbar_init(&acc_empty[a], 4);
+            mbar_init(&acc_empty[a], 2 * (EPI_WARPS / NACC));
         }
         mbar_init(&mma_done, 1);
         abort_flag = 0;
@@ -153,60 +96,65 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
         sm100::prefetch_tensormap(&xmap);
     }
     if (warp == 1) {
-        sm100::tmem_alloc(&tmem_holder, 512);
-        sm100::tmem_relinquish();
+        sm100::tmem_alloc2(&tmem_holder, 512);
+        sm100::tmem_relinquish2();
     }
     sm100::tc_fence_before();
     __syncthreads();
+    sm100::cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive
     sm100::tc_fence_after();
     const uint32_t tmem_base = tmem_holder;
     pdl_launch_dependents();
-    pdl_wait();  // activations and row info come from the input RHT
 
     auto fail = [&]() {
         atomicOr(p.err, GLQ_DEVERR_TIMEOUT);
         abort_flag = 1;
     };
-    // live accumulators of a tile (tokens tok0 .. tok0 + 512)
     auto live_acc = [&](int tok0) { return min(NACC, (p.B - tok0 + BN - 1) / BN); };
 
     if (warp == 0) {
-        // ---------------- TMA producer of the activation tiles ----------------
+        // ---------------- TMA: this CTA's half of the activation tiles ----------------
+        pdl_wait();  // the activations come from the input RHT
         if (lane == 0) {
             uint32_t it = 0;
             int32_t last_load = -1;
-            for (int tile = blockIdx.x; tile < p.ntiles && !abort_flag; tile += gridDim.x) {
-                const int ttile = tile % p.tiles_tok;
-                const int tok0 = ttile * (BN * NACC), na = live_acc(tok0);
+            for (int tile = (int)cid; tile < p.ntiles && !abort_flag; tile += (int)ncl) {
+                const int tok0 = (tile % p.tiles_tok) * (BN * NACC);
+                const int na = live_acc(tok0);
+                int halves = 0;  // live halves of both CTAs (a half past the last token is not loaded)
+                for (int a = 0; a < na; ++a)
+                    for (int r = 0; r < 2; ++r) halves += tok0 + a * BN + r * BNH < p.B;
                 for (int kb = 0; kb < KB && !abort_flag; ++kb, ++it) {
                     const uint32_t s = it % STAGES, use = it / STAGES;
-                    if (!sm100::mbar_wait(&empty_bar[s], (use & 1) ^ 1, WAIT_NS)) {
+                    if (!sm100::mbar_wait_cluster(&empty_bar[s], (use & 1) ^ 1, WAIT_CYCLES)) {
                         fail();
                         break;
                     }
-                    uint8_t *st = smem + s * STAGE_BYTES;
-                    mbar_expect_tx(&x_full[s], na * X_BYTES);
-                    for (int a = 0; a < na; ++a)
-                        sm100::tma_load_2d(st + W_BYTES + a * X_BYTES, &xmap, &x_full[s], kb * BK, tok0 + a * BN);
+                    if (rank == 0) mbar_expect_tx(&x_full[s], (uint32_t)(halves * X_BYTES));
+                    for (int a = 0; a < na; ++a) {
+                        const int t0 = tok0 + a * BN + (int)rank * BNH;
+                        if (t0 < p.B)
+                            sm100::tma_load_2d_pair(smem + s * STAGE_BYTES + W_BYTES + a * X_BYTES, &xmap,
+                                                    &x_full[s], kb * BK, t0);
+                    }
                     last_load = (int32_t)it;
                 }
             }
-            if (abort_flag)  // let the copies in flight land before the CTA exits
+            if (abort_flag && rank == 0)  // let the copies in flight land before the CTA exits
                 for (int32_t i = max(0, last_load - (STAGES - 1)); i <= last_load; ++i)
-                    sm100::mbar_wait(&x_full[i % STAGES], (uint32_t)(i / STAGES) & 1, WAIT_NS);
+                    sm100::mbar_wait(&x_full[i % STAGES], (uint32_t)(i / STAGES) & 1, WAIT_CYCLES);
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            const uint32_t idesc = sm100::idesc_f16_f32(BM, BN);
+        if (lane == 0 && rank == 0) {
+            // ---------------- MMA issuer of the pair ----------------
+            const uint32_t idesc = sm100::idesc_f16_f32(2 * BM, BN);
             uint32_t it = 0, acc_use[NACC] = {0, 0};
-            for (int tile = blockIdx.x; tile < p.ntiles && !abort_flag; tile += gridDim.x) {
-                const int ttile = tile % p.tiles_tok;
-                const int na = live_acc(ttile * (BN * NACC));
+            for (int tile = (int)cid; tile < p.ntiles && !abort_flag; tile += (int)ncl) {
+                const int na = live_acc((tile % p.tiles_tok) * (BN * NACC));
                 for (int kb = 0; kb < KB && !abort_flag; ++kb, ++it) {
                     const uint32_t s = it % STAGES, use = it / STAGES;
-                    if (!sm100::mbar_wait(&x_full[s], use & 1, WAIT_NS) ||
-                        !sm100::mbar_wait(&w_full[s], use & 1, WAIT_NS)) {
+                    if (!sm100::mbar_wait_cluster(&x_full[s], use & 1, WAIT_CYCLES) ||
+                        !sm100::mbar_wait_cluster(&w_full[s], use & 1, WAIT_CYCLES)) {
                         fail();
                         break;
                     }
@@ -214,8 +162,8 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                     uint8_t *st = smem + s * STAGE_BYTES;
                     const uint64_t adesc = sm100::smem_desc_sw128(st);
                     for (int a = 0; a < na; ++a) {
-                        if (kb == 0) {  // the epilogue must have drained this accumulator
-                            if (!sm100::mbar_wait(&acc_empty[a], (acc_use[a] & 1) ^ 1, WAIT_NS)) {
+                        if (kb == 0) {  // both CTAs' epilogues must have drained this accumulator
+                            if (!sm100::mbar_wait_cluster(&acc_empty[a], (acc_use[a] & 1) ^ 1, WAIT_CYCLES)) {
                                 fail();
                                 break;
                             }
@@ -224,92 +172,155 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                         const uint64_t bdesc = sm100::smem_desc_sw128(st + W_BYTES + a * X_BYTES);
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk)
-                            sm100::mma_f16_ss(tmem_base + a * BN, adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                                              (kb | kk) != 0);
-                        if (kb == KB - 1) sm100::mma_commit(&acc_full[a]);
+                            sm100::mma2_f16_ss(tmem_base + a * BN, adesc + 2 * kk, bdesc + 2 * kk, idesc,
+                                               (kb | kk) != 0);
+                        if (kb == KB - 1) sm100::mma2_commit_both(&acc_full[a]);
                     }
-                    sm100::mma_commit(&empty_bar[s]);
+                    sm100::mma2_commit_both(&empty_bar[s]);
                 }
                 for (int a = 0; a < na; ++a) ++acc_use[a];
             }
-            sm100::mma_commit(&mma_done);  // every MMA of this CTA has completed
-            sm100::mbar_wait(&mma_done, 0, WAIT_NS);
+            sm100::mma2_commit_both(&mma_done);  // every MMA of the pair has completed
+            sm100::mbar_wait(&mma_done, 0, WAIT_CYCLES);
+        } else if (lane == 0) {
+            sm100::mbar_wait(&mma_done, 0, WAIT_CYCLES);  // the pair's last commit reaches both CTAs
         }
-    } else if (warp < 6) {
+    } else if (warp < EPI_WARP0) {
         // ---------------- dequantising producer of the W tiles ----------------
-        const int pt = tid - 64;
-        const int rt_l = pt >> 4, tp = (pt >> 3) & 1, g = pt & 7;
+        // warp: 16-row tile rt_l of the CTA's 128 rows; lane (g, t) = slot lane
+        // 4 g + t of the fragment-native stream: in 64-column step h of a
+        // chunk, words s = 2h, 2h + 1 hold rows (g, g + 8) of groups 4 s + t,
+        // i.e. groups t and 4 + t of the step.  Codeword i = 2 s2 + hi.
+        const int rt_l = warp - 2;
+        const int g = lane >> 2, t = lane & 3;
         uint32_t it = 0;
-        for (int tile = blockIdx.x; tile < p.ntiles && !abort_flag; tile += gridDim.x) {
+        for (int tile = (int)cid; tile < p.ntiles && !abort_flag; tile += (int)ncl) {
             const int rtile = tile / p.tiles_tok;
-            const int rt = rtile * (BM / GLQ_ROW_TILE) + rt_l;
+            const int rt = (rtile * 2 + (int)rank) * (BM / GLQ_ROW_TILE) + rt_l;
             const bool live = rt < p.RT;
-            const size_t slot0 = (size_t)rt * p.KC * 32 + 4 * g + 2 * tp;
-            StepCodes codes;
-            StepWords words;
-            load_codes<BPW>(p, slot0, 0, live, codes);
-            issue_gathers<BPW>(p, codes, live, words);
-            if (KB > 1) load_codes<BPW>(p, slot0, 1, live, codes);
+            const size_t slot0 = (size_t)rt * p.KC * 32 + lane;
+            uint4 q1 = make_uint4(0, 0, 0, 0), q2 = q1, n1 = q1, n2 = q1;
+            auto load_slot = [&](int kc, uint4 &a1, uint4 &a2) {
+                if (!live || kc >= p.KC) return;
+                a1 = ldg_nc_v4(p.idx1 + slot0 + (size_t)kc * 32);
+                if (BPW == 4) a2 = ldg_nc_v4(reinterpret_cast<const uint4 *>(p.idx2) + slot0 + (size_t)kc * 32);
+                if (BPW == 3) {
+                    const uint2 v = ldg_nc_v2(reinterpret_cast<const uint2 *>(p.idx2) + slot0 + (size_t)kc * 32);
+                    a2 = make_uint4(v.x, v.y, 0, 0);
+                }
+            };
+            // gathers of step kb's 4 codewords (primary and residual)
+            uint4 ca[4], cb[4];
+            auto gather = [&](int kb) {
+                const int h = kb & 1;
+                const uint32_t wa = h ? q1.z : q1.x, wb = h ? q1.w : q1.y;
+                const uint32_t e1[4] = {wa & 0xFFFFu, wa >> 16, wb & 0xFFFFu, wb >> 16};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) ca[i] = live ? __ldg(p.cb_f16 + e1[i]) : make_uint4(0, 0, 0, 0);
+                if (BPW == 4) {
+                    const uint32_t va = h ? q2.z : q2.x, vb = h ? q2.w : q2.y;
+                    const uint32_t e2[4] = {va & 0xFFFFu, va >> 16, vb & 0xFFFFu, vb >> 16};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) cb[i] = live ? __ldg(p.cb_f16 + e2[i]) : make_uint4(0, 0, 0, 0);
+                } else if (BPW == 3) {  // bytes 2 s + hi of the 8-byte slot, s = 2h, 2h + 1
+                    const uint32_t w = h ? q2.y : q2.x;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) cb[i] = live ? __ldg(p.res8 + ((w >> (8 * i)) & 0xFFu)) : make_uint4(0, 0, 0, 0);
+                }
+            };
+            load_slot(0, q1, q2);
+            load_slot(1, n1, n2);
+            gather(0);
             for (int kb = 0; kb < KB; ++kb, ++it) {
+                uint4 cw[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) cw[i] = BPW == 2 ? ca[i] : hfma8(p.rs_h2, cb[i], ca[i]);
+                if (kb + 1 < KB) {  // the next step's gathers are in flight while this one is stored
+                    if (((kb + 1) & 1) == 0) {
+                        q1 = n1;
+                        q2 = n2;
+                        load_slot(((kb + 1) >> 1) + 1, n1, n2);  // codes one chunk ahead
+                    }
+                    gather(kb + 1);
+                }
                 const uint32_t s = it % STAGES, use = it / STAGES;
-                if (abort_flag || !sm100::mbar_wait(&empty_bar[s], (use & 1) ^ 1, WAIT_NS)) {
+                if (abort_flag || !sm100::mbar_wait_cluster(&empty_bar[s], (use & 1) ^ 1, WAIT_CYCLES)) {
                     if (!abort_flag) fail();
                     break;
                 }
-                store_step<BPW>(p, words, smem + s * STAGE_BYTES, rt_l, tp, g);
+                uint8_t *wt = smem + s * STAGE_BYTES;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int hi = i & 1, s2 = i >> 1;
+                    const int row = rt_l * GLQ_ROW_TILE + g + 8 * hi;
+                    const int gl = 4 * s2 + t;
+                    *reinterpret_cast<uint4 *>(wt + row * 128 + ((gl ^ (row & 7)) << 4)) = cw[i];
+                }
                 sm100::fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) sm100::mbar_arrive(&w_full[s]);
-                if (kb + 1 < KB) issue_gathers<BPW>(p, codes, live, words);
-                if (kb + 2 < KB) load_codes<BPW>(p, slot0, kb + 2, live, codes);
+                if (lane == 0) {
+                    if (rank == 0) sm100::mbar_arrive(&w_full[s]);
+                    else sm100::mbar_arrive_remote(&w_full[s], 0);
+                }
             }
         }
     } else {
         // ---------------- epilogue: TMEM -> z ----------------
-        const int q = warp & 3;  // TMEM lane quadrant this warp may access
-        uint32_t acc_use[NACC] = {0, 0};
-        for (int tile = blockIdx.x; tile < p.ntiles && !abort_flag; tile += gridDim.x) {
+        pdl_wait();  // the row info comes from the input RHT
+        const int ew = warp - EPI_WARP0;   // 0..7
+        const int q = warp & 3;            // TMEM lane quadrant this warp may access
+        const int a = ew >> 2;             // the accumulator this warp drains
+        uint32_t use = 0;
+        for (int tile = (int)cid; tile < p.ntiles && !abort_flag; tile += (int)ncl) {
             const int rtile = tile / p.tiles_tok, ttile = tile - rtile * p.tiles_tok;
-            const int tok0 = ttile * (BN * NACC), na = live_acc(tok0);
-            const int row = rtile * BM + 32 * q + lane;
-            for (int a = 0; a < na; ++a) {
-                if (abort_flag || !sm100::mbar_wait(&acc_full[a], acc_use[a] & 1, WAIT_NS)) {
-                    if (!abort_flag) fail();
-                    break;
-                }
-                sm100::tc_fence_after();
-                for (int c = 0; c < BN / 16; ++c) {
-                    uint32_t r[16];
-                    sm100::tmem_ld16(tmem_base + ((uint32_t)(32 * q) << 16) + a * BN + c * 16, r);
-                    sm100::tmem_wait_ld();
-                    const int tb = tok0 + a * BN + c * 16;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int tok = tb + j;
-                        if (tok < p.B && row < p.m_pad)
-                            p.z[(size_t)tok * p.m_pad + row] = __uint_as_float(r[j]) * p.ws * p.info[tok].inv_scale;
-                    }
-                }
-                sm100::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) sm100::mbar_arrive(&acc_empty[a]);
-                ++acc_use[a];
+            const int tok0 = ttile * (BN * NACC);
+            if (a >= live_acc(tok0)) continue;
+            const int tb = tok0 + a * BN;
+            const int row = (rtile * 2 + (int)rank) * BM + 32 * q + lane;
+            if (abort_flag || !sm100::mbar_wait_cluster(&acc_full[a], use & 1, WAIT_CYCLES)) {
+                if (!abort_flag) fail();
+                break;
             }
+            sm100::tc_fence_after();
+            const int nlive = min(BN, p.B - tb);
+            for (int c = 0; c < nlive; c += 32) {
+                uint32_t r[32];
+                sm100::tmem_ld32(tmem_base + ((uint32_t)(32 * q) << 16) + a * BN + c, r);
+                // lane j holds ws 2^-e of token c + j; the warp shares it by shuffles
+                const float sc = c + lane < nlive ? p.ws * p.info[tb + c + lane].inv_scale : 0.f;
+                sm100::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float scj = __shfl_sync(0xffffffffu, sc, j);
+                    if (row < p.m_pad && c + j < nlive)
+                        p.z[(size_t)(tb + c + j) * p.m_pad + row] = __uint_as_float(r[j]) * scj;
+                }
+            }
+            sm100::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (rank == 0) sm100::mbar_arrive(&acc_empty[a]);
+                else sm100::mbar_arrive_remote(&acc_empty[a], 0);
+            }
+            ++use;
         }
     }
     sm100::tc_fence_before();
     __syncthreads();
+    sm100::cluster_sync_all();  // no CTA leaves while its pair may still touch its memory
     if (warp == 1) {
         sm100::tc_fence_after();
-        sm100::tmem_dealloc(tmem_base, 512);
+        sm100::tmem_dealloc2(tmem_base, 512);
     }
 }
 
 }  // namespace
 
-size_t prefill_smem_bytes() { return (size_t)STAGES * STAGE_BYTES + 1024; }
+size_t prefill_smem_bytes() { return 1024 + (size_t)STAGES * STAGE_BYTES; }
 
 int prefill_tile_tokens() { return BN * NACC; }
+
+int prefill_tile_rows() { return 2 * BM; }
 
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &xmap, int grid, cudaStream_t s, bool pdl) {
     const size_t smem = prefill_smem_bytes();
@@ -317,14 +328,29 @@ cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &xmap, int 
                                 : (p.bpw == 3 ? (const void *)prefill_kernel<3> : (const void *)prefill_kernel<2>);
     static bool configured[5] = {false, false, false, false, false};
     if (!configured[p.bpw]) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GEMV_SMEM_LIMIT);
         if (e != cudaSuccess) return e;
         configured[p.bpw] = true;
     }
+    if (smem > GEMV_SMEM_LIMIT || (grid & 1)) return cudaErrorInvalidValue;
     PrefillParams q = p;
     CUtensorMap m = xmap;
     void *args[] = {&m, &q};
-    return launch_ex(fn, dim3(grid), dim3(THREADS), smem, s, pdl, args);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 2 : 1;
+    return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
 }  // namespace glq

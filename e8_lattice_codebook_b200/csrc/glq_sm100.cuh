@@ -21,9 +21,9 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-__device__ __forceinline__ uint64_t globaltimer_ns() {
+__device__ __forceinline__ uint64_t clock_cycles() {
     uint64_t t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
     return t;
 }
 
@@ -38,16 +38,17 @@ __device__ __forceinline__ bool mbar_try(uint64_t *bar, uint32_t parity) {
     return done != 0;
 }
 
-// Wait on phase `parity`, bounded in wall time: false once `limit_ns` has
-// passed (read from the global timer every 64 polls).
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
+// Wait on phase `parity`, bounded: false once `limit` SM clock cycles have
+// passed (the cycle counter is read every 64 polls; it is cheap, unlike the
+// global nanosecond timer).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit) {
     if (mbar_try(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
+    const uint64_t t0 = clock_cycles();
     for (;;) {
 #pragma unroll 1
         for (int i = 0; i < 64; ++i)
             if (mbar_try(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > limit_ns) return false;
+        if (clock_cycles() - t0 > limit) return false;
     }
 }
 
@@ -152,6 +153,133 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
            | (0u << 15) | (0u << 16)       // A, B K-major
            | ((uint32_t)(N >> 3) << 17)    // N / 8
            | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+// ---------------------------------------------------------------------------
+// Clusters of two CTAs (tcgen05 cta_group::2)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrive (release, cluster scope) on the barrier at the same shared-memory
+// offset as `bar` in CTA `rank` of this cluster.
+__device__ __forceinline__ void mbar_arrive_remote(uint64_t *bar, uint32_t rank) {
+    asm volatile(
+        "{\n .reg .b32 ra;\n mapa.shared::cluster.u32 ra, %0, %1;\n"
+        " mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n}\n" ::"r"(smem_addr(bar)),
+        "r"(rank)
+        : "memory");
+}
+
+// Wait with cluster-scope acquire (barriers that receive remote arrivals).
+__device__ __forceinline__ bool mbar_try_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity, uint64_t limit) {
+    if (mbar_try_cluster(bar, parity)) return true;
+    const uint64_t t0 = clock_cycles();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_cluster(bar, parity)) return true;
+        if (clock_cycles() - t0 > limit) return false;
+    }
+}
+
+// Tensor memory of a CTA pair: one warp (same warp index) in each CTA.
+__device__ __forceinline__ void tmem_alloc2(uint32_t *dst, uint32_t cols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst)),
+                 "r"(cols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t cols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+
+// D (M = 256 over the pair) (+)= A . B; issued by one thread of the pair's
+// first CTA.  A: M/2 rows from each CTA, B: N/2 rows from each CTA, both at
+// the descriptor's offset in each CTA's shared memory.
+__device__ __forceinline__ void mma2_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n"
+        " .reg .pred p;\n"
+        " setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n"
+        "}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on `bar` (same offset) in both CTAs of the pair when this thread's
+// previously issued pair MMAs complete.
+__device__ __forceinline__ void mma2_commit_both(uint64_t *bar) {
+    asm volatile(
+        "{\n .reg .b16 m;\n mov.b16 m, 3;\n"
+        " tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n}\n" ::"r"(
+            smem_addr(bar))
+        : "memory");
+}
+
+// 2-D tiled TMA load by either CTA of a pair into its own shared memory,
+// completing (transaction bytes) on the barrier at the same offset as `bar`
+// in the pair's first CTA.  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1) {
+    asm volatile(
+        "{\n .reg .b32 rb;\n mapa.shared::cluster.u32 rb, %2, 0;\n"
+        " cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [rb];\n}\n" ::"r"(smem_addr(dst)),
+        "l"(map), "r"(smem_addr(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i gets lane (base + i).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t r[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+// Named barrier over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Shared-memory matrix descriptor, K-major, 64-byte swizzle: rows of 64 B,
+// 8-row groups 512 B apart, tile base 512-aligned.
+__device__ __forceinline__ uint64_t smem_desc_sw64(const void *tile) {
+    const uint64_t addr = smem_addr(tile);
+    uint64_t d = 0;
+    d |= (addr >> 4) & 0x3FFFull;           // start address
+    d |= (uint64_t)1 << 16;                  // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(512 >> 4) << 32;         // stride byte offset
+    d |= (uint64_t)1 << 46;                  // descriptor version (sm_100)
+    d |= (uint64_t)4 << 61;                  // layout: 64-byte swizzle
+    return d;
 }
 
 }  // namespace sm100
