@@ -201,41 +201,78 @@ cudaError_t launch_prefill_gemm(glq_layer L, int64_t B, cudaStream_t s, bool pdl
     return glq::launch_prefill(pp, xmap, grid, s, pdl);
 }
 
+glq::RowsParams rows_params(const glq_hblocks &hb, int len, int len_pad, const uint32_t *signs) {
+    glq::RowsParams r{};
+    r.len = len;
+    r.len_pad = len_pad;
+    r.nblk = hb.count;
+    r.max_blk = hb.count ? hb.len[0] : 0;
+    for (int i = 0; i < hb.count; ++i) {
+        r.blk_off[i] = hb.off[i];
+        r.blk_len[i] = hb.len[i];
+        r.blk_norm[i] = (float)(1.0 / std::sqrt((double)hb.len[i]));
+    }
+    r.sign_bits = signs;
+    return r;
+}
+
 // Tensor-core path for B > 16 tokens: input RHT (fp16 activations), tcgen05
-// GEMM with the dequantising producer, output RHT.
+// GEMM with the dequantising producer, output RHT.  Rows of up to 16384
+// values use the one-CTA-per-row transform kernels; longer rows the
+// clustered ones.
 glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_dtype, int64_t B, cudaStream_t s) {
     glq_status st = grow_prefill_ws(L, B);
     if (st != GLQ_OK) return st;
+    const bool rows_in = glq::rht_rows_supported((int)L->n_pad), rows_out = glq::rht_rows_supported((int)L->m);
     for (int64_t b0 = 0; b0 < B;) {
-        const int nb = (int)std::min<int64_t>(B - b0, 65535);  // RHT grid.y limit
-        glq::RhtInParams pin{};
-        pin.x = static_cast<const char *>(x) + (size_t)b0 * L->n * 2;
-        pin.x_bf16 = x_bf16 ? 1 : 0;
-        pin.n = (int)L->n;
-        pin.n_pad = (int)L->n_pad;
-        pin.B = nb;
-        pin.sign_bits = L->d_sin;
-        pin.plan = L->plan_n;
-        pin.xh = L->pws.xh + (size_t)b0 * L->n_pad;
-        pin.info = L->pws.info + b0;
-        pin.xh_only = 1;
-        if (glq::launch_rht_in(pin, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+        const int nb = (int)std::min<int64_t>(B - b0, 65535);  // grid limit of the clustered kernels
+        if (rows_in) {
+            glq::RowsParams r = rows_params(L->hb_n, (int)L->n, (int)L->n_pad, L->d_sin);
+            r.x = static_cast<const char *>(x) + (size_t)b0 * L->n * 2;
+            r.x_bf16 = x_bf16 ? 1 : 0;
+            r.xh = L->pws.xh + (size_t)b0 * L->n_pad;
+            r.info = L->pws.info + b0;
+            if (glq::launch_rht_rows(r, true, nb, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+        } else {
+            glq::RhtInParams pin{};
+            pin.x = static_cast<const char *>(x) + (size_t)b0 * L->n * 2;
+            pin.x_bf16 = x_bf16 ? 1 : 0;
+            pin.n = (int)L->n;
+            pin.n_pad = (int)L->n_pad;
+            pin.B = nb;
+            pin.sign_bits = L->d_sin;
+            pin.plan = L->plan_n;
+            pin.xh = L->pws.xh + (size_t)b0 * L->n_pad;
+            pin.info = L->pws.info + b0;
+            pin.xh_only = 1;
+            if (glq::launch_rht_in(pin, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+        }
         b0 += nb;
     }
     if (launch_prefill_gemm(L, B, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
     L->last_prefill_B = B;
     for (int64_t b0 = 0; b0 < B;) {
         const int nb = (int)std::min<int64_t>(B - b0, 65535);
-        glq::RhtOutParams pout{};
-        pout.m = (int)L->m;
-        pout.B = nb;
-        pout.z = L->pws.z + (size_t)b0 * L->m_pad;
-        pout.z_ld = (int)L->m_pad;
-        pout.sign_bits = L->d_sout;
-        pout.plan = L->plan_m;
-        pout.y = static_cast<char *>(y) + (size_t)b0 * L->m * (y_dtype == GLQ_F32 ? 4 : 2);
-        pout.y_dtype = y_dtype;
-        if (glq::launch_rht_out(pout, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+        void *yb = static_cast<char *>(y) + (size_t)b0 * L->m * (y_dtype == GLQ_F32 ? 4 : 2);
+        if (rows_out) {
+            glq::RowsParams r = rows_params(L->hb_m, (int)L->m, (int)L->m, L->d_sout);
+            r.z = L->pws.z + (size_t)b0 * L->m_pad;
+            r.z_ld = (int)L->m_pad;
+            r.y = yb;
+            r.y_dtype = y_dtype;
+            if (glq::launch_rht_rows(r, false, nb, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+        } else {
+            glq::RhtOutParams pout{};
+            pout.m = (int)L->m;
+            pout.B = nb;
+            pout.z = L->pws.z + (size_t)b0 * L->m_pad;
+            pout.z_ld = (int)L->m_pad;
+            pout.sign_bits = L->d_sout;
+            pout.plan = L->plan_m;
+            pout.y = yb;
+            pout.y_dtype = y_dtype;
+            if (glq::launch_rht_out(pout, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+        }
         b0 += nb;
     }
     return GLQ_OK;

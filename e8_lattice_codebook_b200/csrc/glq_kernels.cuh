@@ -52,6 +52,25 @@ struct RhtOutParams {
     int y_dtype;  // 0 f16, 1 bf16, 2 f32
 };
 
+// Row transforms of the tensor-core path (glq_rht_rows.cu): one CTA per row.
+struct RowsParams {
+    int len, len_pad;           // row length (n or m) and, input side, the padded row of xh
+    int nblk, max_blk;          // Hadamard blocks of len (descending powers of two)
+    int blk_off[GLQ_MAX_BLOCKS], blk_len[GLQ_MAX_BLOCKS];
+    float blk_norm[GLQ_MAX_BLOCKS];  // 1/sqrt(block)
+    const uint32_t *sign_bits;
+    // input: x [B][len] fp16 / bf16 -> xh [B][len_pad] fp16 (xr 2^e), info [B]
+    const void *x;
+    int x_bf16;
+    __half *xh;
+    glq_rowinfo *info;
+    // output: z [B][z_ld] fp32 -> y [B][len]
+    const float *z;
+    int z_ld;
+    void *y;
+    int y_dtype;  // 0 f16, 1 bf16, 2 f32
+};
+
 struct GemvParams {
     const uint4 *idx1;     // [RT][KC][32] 16 B
     const void *idx2;      // [RT][KC][32] 16 B (4 bpw) / 8 B (3 bpw)
@@ -140,6 +159,9 @@ inline cudaError_t launch_ex(const void *fn, dim3 grid, dim3 block, size_t smem,
 // programmatic dependent launch on the stream.
 cudaError_t launch_rht_in(const RhtInParams &p, cudaStream_t s, bool pdl);
 cudaError_t launch_rht_out(const RhtOutParams &p, cudaStream_t s, bool pdl);
+// row transforms for many rows (B up to 65535 per launch), len <= 16384
+bool rht_rows_supported(int len);
+cudaError_t launch_rht_rows(const RowsParams &p, bool input, int B, cudaStream_t s, bool pdl);
 cudaError_t launch_gemv(const GemvParams &p, int bpw, int grid, cudaStream_t s, bool pdl, bool fused_in = false);
 // dynamic shared memory of a launch with the input transform fused
 // (the table, the residual table, the task's activations and scratch)

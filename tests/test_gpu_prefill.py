@@ -7,7 +7,8 @@ cores, so it keeps the same bound as the decode path:
 max |y - y_oracle| <= 2e-3 (||y_oracle||_inf + 1).
 
 * small shapes: every token of batches that span one and several 512-token
-  tiles, with ragged row, column and token tails, all three bit rates;
+  tiles, with ragged row, column and token tails, all three bit rates, and
+  rows longer than the one-CTA-per-row transform takes (16384);
 * full-size prefill workload at its largest batch: sampled tokens, the last
   (ragged) token tile included;
 * run-to-run determinism, and per-token independence of the batch size
@@ -46,6 +47,8 @@ PREFILL_SMALL = [  # m, n, bpw, B, x dtype
     (200, 2560, 3, 300, "bf16"),    # long K (40 steps), ragged accumulator
     (8, 8, 4, 20, "f16"),           # tiny layer, most of the tile is padding
     (1024, 1024, 2, 1100, "bf16"),  # three token tiles
+    (64, 20480, 2, 33, "f16"),      # input rows above 16384: clustered transform kernel
+    (20480, 64, 3, 20, "bf16"),     # output rows above 16384: clustered transform kernel
 ]
 
 
