@@ -405,22 +405,40 @@ cudaError_t run_decode(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg
                        void *y, int y_dtype, int nb, cudaStream_t s) {
     cudaError_t e = cudaSuccess;
     if (!cfg.fin) {
-        RhtInParams pin{};
-        pin.x = x;
-        pin.x_bf16 = x_bf16 ? 1 : 0;
-        pin.n = (int)L->n;
-        pin.n_pad = (int)L->n_pad;
-        pin.B = nb;
-        pin.sign_bits = L->d_sin;
-        pin.plan = L->plan_n;
-        pin.xq = w.xq;
-        pin.xh = w.xh;
-        pin.info = w.info;
-        e = launch_rht_in(pin, s, true);
+        if (rht_rows_supported((int)L->n_pad)) {  // one CTA per token
+            RowsParams r = rows_params(L->hb_n, (int)L->n, (int)L->n_pad, L->d_sin);
+            r.x = x;
+            r.x_bf16 = x_bf16 ? 1 : 0;
+            r.xq = w.xq;
+            r.xh = w.xh;
+            r.info = w.info;
+            e = launch_rht_rows(r, true, nb, s, true);
+        } else {
+            RhtInParams pin{};
+            pin.x = x;
+            pin.x_bf16 = x_bf16 ? 1 : 0;
+            pin.n = (int)L->n;
+            pin.n_pad = (int)L->n_pad;
+            pin.B = nb;
+            pin.sign_bits = L->d_sin;
+            pin.plan = L->plan_n;
+            pin.xq = w.xq;
+            pin.xh = w.xh;
+            pin.info = w.info;
+            e = launch_rht_in(pin, s, true);
+        }
         if (e != cudaSuccess) return e;
     }
     e = launch_gemv(gemv_params(L, w, cfg, nb, x, x_bf16, y, y_dtype), L->bpw, cfg.plan.grid, s, true, cfg.fin);
     if (e != cudaSuccess || cfg.fout) return e;
+    if (rht_rows_supported((int)L->m)) {
+        RowsParams r = rows_params(L->hb_m, (int)L->m, (int)L->m, L->d_sout);
+        r.z = w.z;
+        r.z_ld = (int)L->m_pad;
+        r.y = y;
+        r.y_dtype = y_dtype;
+        return launch_rht_rows(r, false, nb, s, true);
+    }
     RhtOutParams pout{};
     pout.m = (int)L->m;
     pout.B = nb;

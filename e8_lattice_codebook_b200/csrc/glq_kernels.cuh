@@ -64,6 +64,10 @@ struct RowsParams {
     int x_bf16;
     __half *xh;
     glq_rowinfo *info;
+    // input, decode format instead (when xq is set): X = round(xr 2^e) as
+    // [B][len_pad / 8][16] high / low bytes, X as fp16 in xh (3 bpw, may be
+    // null), info [B] = {exact sum of X, 2^-e}
+    uint8_t *xq;
     // output: z [B][z_ld] fp32 -> y [B][len]
     const float *z;
     int z_ld;

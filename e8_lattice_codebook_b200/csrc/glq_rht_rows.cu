@@ -13,9 +13,10 @@
 //     barrier each;
 //   * a block smaller than 16 values (only the last block, of 8) keeps its
 //     thread's upper half as padding;
-//   * the input direction also finds the row's max |xr| (one reduction), so
-//     that the fp16 operand of the tensor-core GEMM is xr 2^e with
-//     max |xr| 2^e < 2^14, and writes 2^-e for the epilogue.
+//   * the input direction also finds the row's max |xr| (one reduction) and
+//     writes either the fp16 operand of the tensor-core GEMM, xr 2^e with
+//     max |xr| 2^e < 2^14, or the decode GEMV's operand X = round(xr 2^e) as
+//     high / low bytes with its exact row sum (a second reduction), plus 2^-e.
 #include "glq_kernels.cuh"
 
 namespace glq {
@@ -156,18 +157,54 @@ __global__ void __launch_bounds__(1024) rht_rows_kernel(RowsParams p) {
             frexpf(rowmax, &e);  // rowmax < 2^e
             scale = ldexpf(1.f, 14 - e);
         }
-        if (c0 < p.len_pad) {  // padding columns [len, len_pad) hold zeros
-            uint32_t w[8];
+        if (p.xq) {  // decode GEMV operand: X = round(xr 2^e), bytes per 8-column group
+            int sum = 0;
+            if (c0 < p.len_pad) {
+                uint32_t hb[4] = {0u, 0u, 0u, 0u}, lb[4] = {0u, 0u, 0u, 0u};
+                uint32_t hx[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const __half2 h2 = __floats2half2_rn(v[2 * j] * scale, v[2 * j + 1] * scale);
-                w[j] = *reinterpret_cast<const uint32_t *>(&h2);
+                for (int j = 0; j < VPT; ++j) {
+                    const int X = __float2int_rn(v[j] * scale);
+                    sum += X;
+                    hb[j >> 2] |= (uint32_t)((X >> 8) & 0xFF) << (8 * (j & 3));
+                    lb[j >> 2] |= (uint32_t)(X & 0xFF) << (8 * (j & 3));
+                    const __half hX = __int2half_rn(X);
+                    if (j & 1) hx[j >> 1] |= (uint32_t)__half_as_ushort(hX) << 16;
+                    else hx[j >> 1] = __half_as_ushort(hX);
+                }
+                uint4 *dst = reinterpret_cast<uint4 *>(p.xq + ((size_t)b * p.len_pad + c0) * 2);
+                dst[0] = make_uint4(hb[0], hb[1], lb[0], lb[1]);  // group c0 / 8
+                dst[1] = make_uint4(hb[2], hb[3], lb[2], lb[3]);  // group c0 / 8 + 1
+                if (p.xh) {
+                    uint4 *dh = reinterpret_cast<uint4 *>(p.xh + (size_t)b * p.len_pad + c0);
+                    dh[0] = make_uint4(hx[0], hx[1], hx[2], hx[3]);
+                    dh[1] = make_uint4(hx[4], hx[5], hx[6], hx[7]);
+                }
             }
-            uint4 *dst = reinterpret_cast<uint4 *>(p.xh + (size_t)b * p.len_pad + c0);
-            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            __syncthreads();  // s_red is reused
+            if (lane == 0) reinterpret_cast<int *>(s_red)[warp] = sum;
+            __syncthreads();
+            if (tid == 0) {
+                long long total = 0;
+                for (int w = 0; w < (int)(blockDim.x >> 5); ++w) total += reinterpret_cast<int *>(s_red)[w];
+                p.info[b] = glq_rowinfo{total, 1.f / scale, 0.f};
+            }
+        } else {
+            if (c0 < p.len_pad) {  // padding columns [len, len_pad) hold zeros
+                uint32_t w[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const __half2 h2 = __floats2half2_rn(v[2 * j] * scale, v[2 * j + 1] * scale);
+                    w[j] = *reinterpret_cast<const uint32_t *>(&h2);
+                }
+                uint4 *dst = reinterpret_cast<uint4 *>(p.xh + (size_t)b * p.len_pad + c0);
+                dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            }
+            if (tid == 0) p.info[b] = glq_rowinfo{0, 1.f / scale, 0.f};
         }
-        if (tid == 0) p.info[b] = glq_rowinfo{0, 1.f / scale, 0.f};
     } else if (valid) {
         const uint32_t sb = (p.sign_bits[c0 >> 5] >> (c0 & 31)) & 0xFFFFu;
 #pragma unroll
