@@ -123,6 +123,14 @@ __device__ __forceinline__ uint4 ldg_v4(const void *p) {
     return v;
 }
 
+// Bring a line into L2 (no register result).  Safe before the wait on a
+// producing kernel: L2 is the point of coherence, so the producer's later
+// writes replace whatever the prefetch brought in; it warms the TLB and L2
+// for data that is already final.
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned *p, unsigned v) {
     unsigned old;
     asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");

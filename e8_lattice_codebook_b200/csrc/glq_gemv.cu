@@ -239,6 +239,26 @@ __device__ void fwht_segments(float *u, int nrows, int ld, const Seg *segs, int 
     }
 }
 
+// Constant data of a task's fused input, fetched before the wait on the
+// previous kernel: the S_in sign words of every Hadamard block the task's
+// column range meets (a contiguous run of columns), into `sw` starting at
+// word `*w0`.  Every thread calls it; ends with a barrier.
+template <int THREADS>
+__device__ void fused_input_signs(const GemvParams &p, int k0, int klen, uint32_t *sw, int *w0) {
+    int lo = 1 << 30, hi = 0;
+    for (int bi = 0; bi < p.nblk_n; ++bi) {
+        const int o = p.blk_off_n[bi], N = p.blk_len_n[bi];
+        if (max(k0, o) < min(k0 + klen, o + N)) {
+            lo = min(lo, o);
+            hi = max(hi, o + N);
+        }
+    }
+    const int a = lo >> 5, e = (hi + 31) >> 5;  // at most n / 32 + 1 words
+    for (int i = threadIdx.x; i < e - a; i += THREADS) sw[i] = __ldg(p.sin_bits + a + i);
+    *w0 = a;
+    __syncthreads();
+}
+
 // The task's activations for columns [k0, k0 + klen): xr = H_n (S_in x)
 // restricted to the range, scaled per token by 2^e (max |xr| 2^e < 2^14 over
 // the range), rounded to X and stored as the GEMV consumes it: xs[b][group]
@@ -249,7 +269,7 @@ __device__ void fwht_segments(float *u, int nrows, int ld, const Seg *segs, int 
 // N/S sub-blocks t of (-1)^popc(i t) (S_in x)[t S + j], i the part's index.
 template <int BPW, int THREADS>
 __device__ void fused_input(const GemvParams &p, int k0, int klen, uint4 *xs, __half *xhs, float *u,
-                            TaskRow *rows, unsigned *s_max, Seg *segs) {
+                            TaskRow *rows, unsigned *s_max, Seg *segs, const uint32_t *sw, int w0) {
     const int tid = threadIdx.x, lane = tid & 31;
     const int B = p.B, k1 = k0 + klen;
     for (int e = tid; e < B * klen; e += THREADS) u[e] = 0.f;  // columns >= n stay zero
@@ -281,7 +301,7 @@ __device__ void fused_input(const GemvParams &p, int k0, int klen, uint4 *xs, __
                     const int col = o + jh * S + 8 * v;
                     float xv[8];
                     load8_act(p.x, (size_t)b * p.n + col, p.x_bf16, xv);
-                    const uint32_t sb = (p.sin_bits[col >> 5] >> (col & 31)) & 0xFFu;
+                    const uint32_t sb = (sw[(col >> 5) - w0] >> (col & 31)) & 0xFFu;
                     const uint32_t neg = (__popc(ihi & jh) & 1) ? 0xFFu : 0u;
                     const uint32_t flip = sb ^ neg;
 #pragma unroll
@@ -410,6 +430,8 @@ __global__ void __launch_bounds__(gemv_warps(NT) * 32, 1) gemv_kernel(GemvParams
     __shared__ unsigned s_max[GLQ_DECODE_MAX_B];
     __shared__ int s_pending[GLQ_MAX_BLOCKS];
     __shared__ Seg s_segs[GLQ_MAX_BLOCKS];
+    __shared__ uint32_t s_sign[GLQ_RHT_MAX_N / 32 + 2];  // fused input: S_in words of the task's blocks
+    __shared__ int s_sign_w0;
     __shared__ int s_npending;
     uint32_t *T = reinterpret_cast<uint32_t *>(smem_u4);
     uint4 *R8 = smem_u4 + p.table_words / 4;
@@ -465,16 +487,28 @@ __global__ void __launch_bounds__(gemv_warps(NT) * 32, 1) gemv_kernel(GemvParams
     if (task < ntasks) {
         task_geom(task);
         prefetch();
+        if (FIN) {
+            fused_input_signs<THREADS>(p, c0 * GLQ_CHUNK_K, (c1 - c0) * GLQ_CHUNK_K, s_sign, &s_sign_w0);
+            // the columns of x the first task folds: Hadamard blocks met by its range
+            const int lo = s_sign_w0 * 32;
+            const int hi = min(p.n, lo + (int)(sizeof(s_sign) / 4) * 32);
+            for (int b = 0; b < p.B; ++b)
+                for (int col = lo + 64 * tid; col < hi; col += 64 * THREADS)  // 128-byte lines of bf16 / fp16
+                    prefetch_l2(static_cast<const uint16_t *>(p.x) + (size_t)b * p.n + col);
+        }
     }
 
-    const bool ok = mbar_wait_bounded(&bar, 0, TABLE_WAIT_POLLS);
-    if (!ok) {
+    // 3. activations (and row info) come from the previous kernel; with the
+    // input transform fused, the codebook copy keeps landing meanwhile
+    pdl_wait();
+    auto wait_table = [&]() {  // every thread calls it; the verdict is the CTA's
+        const bool ok = __syncthreads_and(mbar_wait_bounded(&bar, 0, TABLE_WAIT_POLLS) ? 1 : 0) != 0;
+        if (ok) return true;
         if (tid == 0) atomicOr(p.err, GLQ_DEVERR_TIMEOUT);
         mbar_wait_bounded(&bar, 0, TABLE_WAIT_POLLS);  // let the copy land before exiting
-        return;
-    }
-    // 3. activations (and row info) come from the previous kernel
-    pdl_wait();
+        return false;
+    };
+    if (!FIN && !wait_table()) return;
 
     const bool has0 = g < p.B, has1 = (g + 8) < p.B;
     const size_t xq_row = (size_t)p.n_pad / 8;  // uint4 (one group) per 8 columns
@@ -492,7 +526,10 @@ __global__ void __launch_bounds__(gemv_warps(NT) * 32, 1) gemv_kernel(GemvParams
         const int klen = (c1 - c0) * GLQ_CHUNK_K;
         if (FIN) {
             __syncthreads();  // the previous task's activations and row info are no longer read
-            fused_input<BPW, THREADS>(p, c0 * GLQ_CHUNK_K, klen, xs, xhs, ubuf, s_rows, s_max, s_segs);
+            if (!first) fused_input_signs<THREADS>(p, c0 * GLQ_CHUNK_K, klen, s_sign, &s_sign_w0);
+            fused_input<BPW, THREADS>(p, c0 * GLQ_CHUNK_K, klen, xs, xhs, ubuf, s_rows, s_max, s_segs, s_sign,
+                                      s_sign_w0);
+            if (first && !wait_table()) return;  // the CTA's common verdict: all threads return
         }
         Acc acc1, acc2;
         zero<NT>(acc1);

@@ -170,8 +170,8 @@ cudaError_t launch_gemv(const GemvParams &p, int bpw, int grid, cudaStream_t s, 
 // dynamic shared memory of a launch with the input transform fused
 // (the table, the residual table, the task's activations and scratch)
 size_t gemv_fused_smem_bytes(int table_words, int bpw, int B, int klen);
-// (227 KB per block, less room for the kernel's static shared memory)
-constexpr size_t GEMV_SMEM_LIMIT = 226 * 1024;
+// (227 KB per block, less room for the kernels' static shared memory)
+constexpr size_t GEMV_SMEM_LIMIT = 222 * 1024;
 
 // GEMV work split: bands of row tiles x splits of the chunk range.
 struct GemvPlan {

@@ -65,6 +65,10 @@ __global__ void __launch_bounds__(1024) rht_rows_kernel(RowsParams p) {
     const int b = blockIdx.x;
     const int c0 = VPT * tid;  // first column of this thread
     pdl_launch_dependents();
+    if (c0 < p.len) {  // warm L2 and the TLB before waiting on the producer
+        if (IN) prefetch_l2(static_cast<const uint16_t *>(p.x) + (size_t)b * p.len + c0);
+        else prefetch_l2(p.z + (size_t)b * p.z_ld + c0);
+    }
     pdl_wait();  // the input comes from the previous kernel
 
     float norm;
