@@ -38,7 +38,7 @@ EXPORTS = (
     "glq_codebook_destroy", "glq_layer_create", "glq_layer_destroy", "glq_layer_reserve",
     "glq_linear", "glq_dequant_reference", "glq_rht_input", "glq_rht_output",
     "glq_layer_check", "glq_layer_info", "glq_gemv_replay", "glq_linear_noalloc",
-    "glq_prefill_replay", "glq_layer_set_fusion",
+    "glq_prefill_replay", "glq_layer_set_fusion", "glq_layer_set_prefill_reconstruct",
 )
 
 
@@ -70,6 +70,7 @@ _SIGNATURES = {
     "glq_gemv_replay": ([_vp, _i64, _vp], ctypes.c_int),
     "glq_prefill_replay": ([_vp, _i64, _vp], ctypes.c_int),
     "glq_layer_set_fusion": ([_vp, ctypes.c_int32], ctypes.c_int),
+    "glq_layer_set_prefill_reconstruct": ([_vp, _i64], ctypes.c_int),
     "glq_layer_info": ([_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i32),
                         ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
 }
@@ -195,6 +196,10 @@ def glq_layer_set_fusion(handle, flags: int) -> None:
     _ok(_L().glq_layer_set_fusion(handle, int(flags)), "glq_layer_set_fusion")
 
 
+def glq_layer_set_prefill_reconstruct(handle, min_batch: int) -> None:
+    _ok(_L().glq_layer_set_prefill_reconstruct(handle, int(min_batch)), "glq_layer_set_prefill_reconstruct")
+
+
 def glq_layer_check(handle, stream) -> None:
     _ok(_L().glq_layer_check(handle, stream), "glq_layer_check")
 
@@ -313,6 +318,10 @@ class GlqLinear:
         elif flags is False:
             flags = 0
         glq_layer_set_fusion(self.handle, flags)
+
+    def set_prefill_reconstruct(self, min_batch: int):
+        """Batches >= min_batch reconstruct W in fp16 first (-1: default)."""
+        glq_layer_set_prefill_reconstruct(self.handle, min_batch)
 
     def prefill_replay(self, B, stream=None):
         glq_prefill_replay(self.handle, B, _stream_ptr(stream))

@@ -96,6 +96,7 @@ void free_prefill_ws(glq_layer L) {
     cudaFree(L->pws.xh);
     cudaFree(L->pws.info);
     cudaFree(L->pws.z);
+    cudaFree(L->pws.w16);
     L->pws = glq_prefill_ws{};
 }
 
@@ -134,13 +135,19 @@ glq_status grow_workspace(glq_layer L, int64_t rows) {
     return GLQ_OK;
 }
 
-glq_status grow_prefill_ws(glq_layer L, int64_t rows) {
-    if (rows <= L->pws.cap) return GLQ_OK;
+glq_status grow_prefill_ws(glq_layer L, int64_t rows, bool mat) {
+    if (rows <= L->pws.cap && (!mat || L->pws.w16)) return GLQ_OK;
     if (cudaDeviceSynchronize() != cudaSuccess) return GLQ_ERR_CUDA;
+    if (rows <= L->pws.cap) {  // only the reconstructed W is missing
+        return dmalloc(&L->pws.w16, (size_t)L->m_pad * L->n_pad * sizeof(__half), nullptr);
+    }
+    const bool had_w16 = L->pws.w16 != nullptr;
     free_prefill_ws(L);
     glq_status st = dmalloc(&L->pws.xh, (size_t)rows * L->n_pad * sizeof(__half), nullptr);
     if (st == GLQ_OK) st = dmalloc(&L->pws.info, (size_t)rows * sizeof(glq_rowinfo), nullptr);
     if (st == GLQ_OK) st = dmalloc(&L->pws.z, (size_t)rows * L->m_pad * sizeof(float), nullptr);
+    if (st == GLQ_OK && (mat || had_w16))
+        st = dmalloc(&L->pws.w16, (size_t)L->m_pad * L->n_pad * sizeof(__half), nullptr);
     if (st != GLQ_OK) {
         free_prefill_ws(L);
         return st;
@@ -151,6 +158,10 @@ glq_status grow_prefill_ws(glq_layer L, int64_t rows) {
 
 // TMA descriptor of the fp16 activations [B][n_pad]: boxes of 64 columns x
 // 128 tokens, 128-byte swizzle, zero fill past the last token.
+// TMA descriptor of the reconstructed W16 [m_pad][n_pad]: boxes of 64 columns
+// x 128 rows, 128-byte swizzle.
+bool encode_w_map(CUtensorMap *map, const __half *w16, int64_t n_pad, int64_t m_pad);
+
 bool encode_x_map(CUtensorMap *map, const __half *xh, int64_t n_pad, int64_t B) {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
@@ -174,9 +185,12 @@ bool encode_x_map(CUtensorMap *map, const __half *xh, int64_t n_pad, int64_t B) 
 
 // The tcgen05 GEMM of the tensor-core path on the layer's prefill
 // workspace: z[0..B) from xh[0..B).
-cudaError_t launch_prefill_gemm(glq_layer L, int64_t B, cudaStream_t s, bool pdl) {
-    CUtensorMap xmap;
-    if (!encode_x_map(&xmap, L->pws.xh, L->n_pad, B)) return cudaErrorInvalidValue;
+bool encode_w_map(CUtensorMap *map, const __half *w16, int64_t n_pad, int64_t m_pad) {
+    // same layout rules as the activations: rows of n_pad fp16, 128-byte swizzle
+    return encode_x_map(map, w16, n_pad, m_pad);
+}
+
+glq::PrefillParams prefill_params(glq_layer L, int64_t B) {
     glq::PrefillParams pp{};
     pp.idx1 = L->d_idx1;
     pp.idx2 = L->d_idx2;
@@ -197,8 +211,21 @@ cudaError_t launch_prefill_gemm(glq_layer L, int64_t B, cudaStream_t s, bool pdl
     pp.tiles_tok = (int)((B + glq::prefill_tile_tokens() - 1) / glq::prefill_tile_tokens());
     pp.ntiles = tiles_m * pp.tiles_tok;
     pp.err = L->d_err;
+    pp.table = L->primary->d_table;
+    pp.table_words = L->primary->table_words;
+    pp.fold = glq::FoldParams{L->primary->fold.nb, L->primary->fold.neg_base};
+    return pp;
+}
+
+// The tcgen05 GEMM of the tensor-core path on the layer's prefill
+// workspace: z[0..B) from xh[0..B); mat: against the reconstructed W16.
+cudaError_t launch_prefill_gemm(glq_layer L, int64_t B, bool mat, cudaStream_t s, bool pdl) {
+    CUtensorMap xmap, wmap;
+    if (!encode_x_map(&xmap, L->pws.xh, L->n_pad, B)) return cudaErrorInvalidValue;
+    if (mat && !encode_w_map(&wmap, L->pws.w16, L->n_pad, L->m_pad)) return cudaErrorInvalidValue;
+    const glq::PrefillParams pp = prefill_params(L, B);
     const int grid = 2 * std::min(pp.ntiles, L->num_sms / 2);  // CTA pairs
-    return glq::launch_prefill(pp, xmap, grid, s, pdl);
+    return glq::launch_prefill(pp, xmap, mat ? &wmap : nullptr, grid, s, pdl);
 }
 
 glq::RowsParams rows_params(const glq_hblocks &hb, int len, int len_pad, const uint32_t *signs) {
@@ -221,7 +248,8 @@ glq::RowsParams rows_params(const glq_hblocks &hb, int len, int len_pad, const u
 // values use the one-CTA-per-row transform kernels; longer rows the
 // clustered ones.
 glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_dtype, int64_t B, cudaStream_t s) {
-    glq_status st = grow_prefill_ws(L, B);
+    const bool mat = B >= L->prefill_mat_min_b;
+    glq_status st = grow_prefill_ws(L, B, mat);
     if (st != GLQ_OK) return st;
     const bool rows_in = glq::rht_rows_supported((int)L->n_pad), rows_out = glq::rht_rows_supported((int)L->m);
     for (int64_t b0 = 0; b0 < B;) {
@@ -249,8 +277,11 @@ glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_d
         }
         b0 += nb;
     }
-    if (launch_prefill_gemm(L, B, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+    if (mat && glq::launch_wmat(prefill_params(L, B), L->pws.w16, (int)L->n_pad, L->num_sms, s, true) != cudaSuccess)
+        return GLQ_ERR_CUDA;
+    if (launch_prefill_gemm(L, B, mat, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
     L->last_prefill_B = B;
+    L->last_prefill_mat = mat;
     for (int64_t b0 = 0; b0 < B;) {
         const int nb = (int)std::min<int64_t>(B - b0, 65535);
         void *yb = static_cast<char *>(y) + (size_t)b0 * L->m * (y_dtype == GLQ_F32 ? 4 : 2);
@@ -693,6 +724,12 @@ glq_status glq_layer_set_fusion(glq_layer layer, int32_t flags) {
     return GLQ_OK;
 }
 
+glq_status glq_layer_set_prefill_reconstruct(glq_layer layer, int64_t min_batch) {
+    if (!layer) return GLQ_ERR_INVALID_ARG;
+    layer->prefill_mat_min_b = min_batch < 0 ? 256 : std::max<int64_t>(min_batch, GLQ_DECODE_MAX_B + 1);
+    return GLQ_OK;
+}
+
 glq_status glq_layer_info(glq_layer layer, int64_t *m, int64_t *n, int32_t *bpw, size_t *device_bytes) {
     if (!layer) return GLQ_ERR_INVALID_ARG;
     if (m) *m = layer->m;
@@ -817,8 +854,9 @@ glq_status glq_prefill_replay(glq_layer L, int64_t B, void *stream) {
     if (!L) return GLQ_ERR_INVALID_ARG;
     if (B <= GLQ_DECODE_MAX_B || B > L->last_prefill_B) return GLQ_ERR_SHAPE;
     DeviceGuard guard(L->device);
-    return launch_prefill_gemm(L, B, static_cast<cudaStream_t>(stream), false) == cudaSuccess ? GLQ_OK
-                                                                                            : GLQ_ERR_CUDA;
+    return launch_prefill_gemm(L, B, L->last_prefill_mat, static_cast<cudaStream_t>(stream), false) == cudaSuccess
+               ? GLQ_OK
+               : GLQ_ERR_CUDA;
 }
 
 glq_status glq_layer_check(glq_layer L, void *stream) {

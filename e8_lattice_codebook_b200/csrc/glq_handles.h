@@ -31,6 +31,7 @@ struct glq_prefill_ws {
     __half *xh = nullptr;         // [cap][n_pad]
     glq_rowinfo *info = nullptr;  // [cap]
     float *z = nullptr;           // [cap][m_pad]
+    __half *w16 = nullptr;        // [m_pad][n_pad] reconstructed W (batches >= the materialise bound)
 };
 
 // Device buffers one decode call works in (B <= 16 tokens).
@@ -68,11 +69,13 @@ struct glq_layer_s {
     int64_t cap_rows = 0;
     int64_t last_B = 0;          // batch of the last decode slice (glq_gemv_replay)
     int64_t last_prefill_B = 0;  // batch of the last tensor-core call (glq_prefill_replay)
+    bool last_prefill_mat = false;
     glq_workspace wsp;
     glq_prefill_ws pws;
     glq_hblocks hb_n, hb_m;
     unsigned *d_blk_cnt = nullptr;  // [GLQ_MAX_BLOCKS] output-block counters, zero between calls
     int fusion = -1;                // GLQ_FUSE_* bits, or -1: the library default (glq_layer_set_fusion)
+    int64_t prefill_mat_min_b = 256;  // batches from here reconstruct W16 first (glq_layer_set_prefill_mode)
     // the last decode launch (glq_gemv_replay)
     const void *last_x = nullptr;
     void *last_y = nullptr;

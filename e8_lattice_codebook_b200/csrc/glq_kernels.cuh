@@ -119,6 +119,9 @@ struct PrefillParams {
     const uint4 *idx1;       // [RT][KC][32] 16 B, fragment-native codes
     const void *idx2;        // 4 bpw: 16 B / 3 bpw: 8 B per slot
     const uint4 *cb_f16;     // E8 codewords as fp16 [folded code][8] (negated entries included)
+    const uint32_t *table;   // folded nibble table (W materialisation), table_words
+    int table_words;
+    FoldParams fold;
     const uint4 *res8;       // 3 bpw: [256][8] fp16
     int bpw;
     uint32_t rs_h2;          // residual scale as fp16x2
@@ -183,7 +186,14 @@ struct GemvPlan {
 GemvPlan plan_gemv(int RT, int KC, int num_sms, int warps, bool pow2 = false, int max_cps = 1 << 30,
                    int max_splits = 1 << 30);
 cudaError_t launch_dequant(const DequantParams &p, cudaStream_t s);
-cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &xmap, int grid, cudaStream_t s, bool pdl);
+// wmap: TMA map of the dequantised fp16 W [m_pad][n_pad] (boxes 64 x 128,
+// 128-byte swizzle), or null for the fused variant whose producer warps
+// rebuild W from the codes.
+cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &xmap, const CUtensorMap *wmap, int grid,
+                           cudaStream_t s, bool pdl);
+// W16 [m_pad][n_pad] fp16 = cb1 + rs cb2 (unscaled), for the materialised variant
+cudaError_t launch_wmat(const PrefillParams &p, __half *w16, int n_pad, int num_sms, cudaStream_t s, bool pdl);
+size_t wmat_smem_bytes(int table_words, int bpw);
 size_t prefill_smem_bytes();
 int prefill_tile_tokens();  // tokens of one output tile (a multiple of the TMA box height)
 int prefill_tile_rows();    // weight rows of one output tile (one CTA pair)

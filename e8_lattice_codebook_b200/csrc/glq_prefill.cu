@@ -43,10 +43,11 @@ constexpr int STAGES = 4;
 constexpr int W_BYTES = BM * BK * 2;                       // 16 KB
 constexpr int X_BYTES = BNH * BK * 2;                      // 16 KB per accumulator
 constexpr int STAGE_BYTES = W_BYTES + NACC * X_BYTES;     // 48 KB
-constexpr int PRODUCER_WARPS = 8;
+constexpr int PRODUCER_WARPS = 8;                         // fused variant only
 constexpr int EPI_WARPS = 8;                               // four per accumulator
-constexpr int EPI_WARP0 = 2 + PRODUCER_WARPS;             // warps 10-17
-constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;     // 576
+// warp roles: 0 TMA, 1 MMA, [2-9 dequantising producer,] then the epilogue
+__host__ __device__ constexpr int epi_warp0(bool mat) { return mat ? 2 : 2 + PRODUCER_WARPS; }
+__host__ __device__ constexpr int threads_of(bool mat) { return (epi_warp0(mat) + EPI_WARPS) * 32; }  // 320 / 576
 constexpr uint64_t WAIT_CYCLES = 4000000000ull;           // wait limit: 4e9 SM cycles (about 2 s)
 
 __device__ __forceinline__ uint32_t hfma2_bits(uint32_t s, uint32_t b, uint32_t a) {  // s * b + a
@@ -60,9 +61,14 @@ __device__ __forceinline__ uint4 hfma8(uint32_t rs2, uint4 b, uint4 a) {  // rs 
                       hfma2_bits(rs2, b.w, a.w));
 }
 
-template <int BPW>
-__global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_constant__ CUtensorMap xmap,
-                                                              PrefillParams p) {
+// MAT: W was dequantised into an fp16 matrix first; both operands are
+// loaded by TMA and there is no producer.  Otherwise the producer warps
+// rebuild each W step from the codes.
+template <int BPW, bool MAT>
+__global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __grid_constant__ CUtensorMap xmap,
+                                                                      const __grid_constant__ CUtensorMap wmap,
+                                                                      PrefillParams p) {
+    constexpr int EPI_WARP0 = epi_warp0(MAT);
     extern __shared__ uint8_t smem_raw[];
     // (first CTA) x_full: both CTAs' TMA bytes landed; w_full: both CTAs'
     // producer warps wrote W; acc_empty: both CTAs drained accumulator a.
@@ -83,7 +89,7 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&x_full[s], 1);                   // the first CTA's TMA thread
-            mbar_init(&w_full[s], 2 * PRODUCER_WARPS);  // producer warps of both CTAs
+            mbar_init(&w_full[s], MAT ? 1 : 2 * PRODUCER_WARPS);  // producer warps of both CTAs
             mbar_init(&empty_bar[s], 1);
         }
         for (int a = 0; a < NACC; ++a) {
@@ -94,6 +100,7 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
         abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         sm100::prefetch_tensormap(&xmap);
+        if (MAT) sm100::prefetch_tensormap(&wmap);
     }
     if (warp == 1) {
         sm100::tmem_alloc2(&tmem_holder, 512);
@@ -130,7 +137,12 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                         fail();
                         break;
                     }
-                    if (rank == 0) mbar_expect_tx(&x_full[s], (uint32_t)(halves * X_BYTES));
+                    const int wrow = (tile / p.tiles_tok) * (2 * BM);  // the pair's first weight row
+                    const int wparts = MAT ? (wrow < p.m_pad) + (wrow + BM < p.m_pad) : 0;
+                    if (rank == 0) mbar_expect_tx(&x_full[s], (uint32_t)(halves * X_BYTES + wparts * W_BYTES));
+                    if (MAT && wrow + (int)rank * BM < p.m_pad)  // rows past m_pad are never stored
+                        sm100::tma_load_2d_pair(smem + s * STAGE_BYTES, &wmap, &x_full[s], kb * BK,
+                                                wrow + (int)rank * BM);
                     for (int a = 0; a < na; ++a) {
                         const int t0 = tok0 + a * BN + (int)rank * BNH;
                         if (t0 < p.B)
@@ -154,7 +166,7 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
                 for (int kb = 0; kb < KB && !abort_flag; ++kb, ++it) {
                     const uint32_t s = it % STAGES, use = it / STAGES;
                     if (!sm100::mbar_wait_cluster(&x_full[s], use & 1, WAIT_CYCLES) ||
-                        !sm100::mbar_wait_cluster(&w_full[s], use & 1, WAIT_CYCLES)) {
+                        (!MAT && !sm100::mbar_wait_cluster(&w_full[s], use & 1, WAIT_CYCLES))) {
                         fail();
                         break;
                     }
@@ -185,7 +197,7 @@ __global__ void __launch_bounds__(THREADS, 1) prefill_kernel(const __grid_consta
         } else if (lane == 0) {
             sm100::mbar_wait(&mma_done, 0, WAIT_CYCLES);  // the pair's last commit reaches both CTAs
         }
-    } else if (warp < EPI_WARP0) {
+    } else if (!MAT && warp < EPI_WARP0) {
         // ---------------- dequantising producer of the W tiles ----------------
         // warp: 16-row tile rt_l of the CTA's 128 rows; lane (g, t) = slot lane
         // 4 g + t of the fragment-native stream: in 64-column step h of a
@@ -322,23 +334,35 @@ int prefill_tile_tokens() { return BN * NACC; }
 
 int prefill_tile_rows() { return 2 * BM; }
 
-cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &xmap, int grid, cudaStream_t s, bool pdl) {
+cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &xmap, const CUtensorMap *wmap, int grid,
+                           cudaStream_t s, bool pdl) {
     const size_t smem = prefill_smem_bytes();
-    const void *fn = p.bpw == 4 ? (const void *)prefill_kernel<4>
-                                : (p.bpw == 3 ? (const void *)prefill_kernel<3> : (const void *)prefill_kernel<2>);
-    static bool configured[5] = {false, false, false, false, false};
-    if (!configured[p.bpw]) {
+    const bool mat = wmap != nullptr;
+    const void *fn;
+    switch (p.bpw * 2 + (mat ? 1 : 0)) {
+        case 4: fn = (const void *)prefill_kernel<2, false>; break;
+        case 5: fn = (const void *)prefill_kernel<2, true>; break;
+        case 6: fn = (const void *)prefill_kernel<3, false>; break;
+        case 7: fn = (const void *)prefill_kernel<3, true>; break;
+        case 8: fn = (const void *)prefill_kernel<4, false>; break;
+        case 9: fn = (const void *)prefill_kernel<4, true>; break;
+        default: return cudaErrorInvalidValue;
+    }
+    static bool configured[10] = {};
+    const int key = p.bpw * 2 + (mat ? 1 : 0);
+    if (!configured[key]) {
         cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GEMV_SMEM_LIMIT);
         if (e != cudaSuccess) return e;
-        configured[p.bpw] = true;
+        configured[key] = true;
     }
     if (smem > GEMV_SMEM_LIMIT || (grid & 1)) return cudaErrorInvalidValue;
     PrefillParams q = p;
     CUtensorMap m = xmap;
-    void *args[] = {&m, &q};
+    CUtensorMap wm = mat ? *wmap : xmap;  // unused by the fused variant
+    void *args[] = {&m, &wm, &q};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(THREADS);
+    cfg.blockDim = dim3(threads_of(mat));
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];

@@ -191,6 +191,20 @@ GLQ_API glq_status glq_linear(glq_layer layer, const void *x_dev, glq_dtype x_dt
 GLQ_API glq_status glq_layer_set_fusion(glq_layer layer, int32_t flags);
 
 /*
+ * glq_layer_set_prefill_reconstruct -- how tensor-core calls (B > 16) get
+ * their weights.  Calls with B >= min_batch first reconstruct W = cb1 + rs
+ * cb2 into an fp16 matrix of m_pad x n_pad (2 bytes per weight, a workspace
+ * the layer keeps until it is destroyed) and run the TMA-fed tcgen05 GEMM on
+ * it; smaller batches rebuild each W tile in shared memory inside the GEMM
+ * and never materialise W (the pages' design: "Inference kernels", glq 0.5.1
+ * PyPI page).  Reconstructing once costs one pass over the indices, while the
+ * fused producer repeats its codeword gathers for every 512 tokens, so large
+ * batches favour it.  min_batch < 0 restores the library default (256);
+ * a value above any batch disables it.  Errors: GLQ_ERR_INVALID_ARG.
+ */
+GLQ_API glq_status glq_layer_set_prefill_reconstruct(glq_layer layer, int64_t min_batch);
+
+/*
  * glq_dequant_reference -- materialise W^ (fp32, no Hadamards, ws included)
  * into w_dev [m][n] row-major, using the same on-chip decode the GEMV uses.
  * Each value is fp32(ws * fma_f32(rs, cb2, cb1)) (single roundings).

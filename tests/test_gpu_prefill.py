@@ -52,27 +52,36 @@ PREFILL_SMALL = [  # m, n, bpw, B, x dtype
 ]
 
 
+MODES = {"fused": 1 << 40, "reconstructed": 17}  # glq_layer_set_prefill_reconstruct bound
+
+
+@pytest.mark.parametrize("mode", sorted(MODES))
 @pytest.mark.parametrize("m,n,bpw,B,xdt", PREFILL_SMALL)
-def test_prefill_small_all_tokens(dev, m, n, bpw, B, xdt):
+def test_prefill_small_all_tokens(dev, m, n, bpw, B, xdt, mode):
+    """Both ways of feeding W: rebuilt per tile in shared memory (fused) and
+    reconstructed once into an fp16 matrix (reconstructed)."""
     L = gi.make_layer(m * 11 + n, 7, m, n, bpw)
     xb = gi.make_x(m * 11 + n, 7, B, n, xdt)
     lay = dev.layer(L)
+    lay.set_prefill_reconstruct(MODES[mode])
     x = to_torch_x(xb, xdt)
     y = lay(x, out_dtype=torch.float32).cpu().numpy().astype(np.float64)
     ref = oracle_y(L, xb, xdt)
     err = np.max(np.abs(y - ref))
-    print(f"\nPREFILL {m}x{n} bpw {bpw} B={B}: max err {err:.3e} tol {tolerance(ref):.3e} "
+    print(f"\nPREFILL {mode} {m}x{n} bpw {bpw} B={B}: max err {err:.3e} tol {tolerance(ref):.3e} "
           f"ratio {err / tolerance(ref):.3f}")
     assert err <= tolerance(ref), (err, tolerance(ref))
     yp = lay(x).float().cpu().numpy().astype(np.float64)
     assert np.all(np.abs(yp - ref) <= production_tolerance(ref, xdt))
 
 
+@pytest.mark.parametrize("mode", sorted(MODES))
 @pytest.mark.parametrize("li", [0, 1])
-def test_prefill_workload_largest_batch(dev, li):
+def test_prefill_workload_largest_batch(dev, li, mode):
     wl = gi.WORKLOADS["prefill-8b-mlp-4bpw"]
     L = gi.workload_layer(wl, li)
     lay = dev.layer(L)
+    lay.set_prefill_reconstruct(MODES[mode])
     B = max(wl.batches)
     xb = gi.workload_x(wl, li, B)
     x = to_torch_x(xb, wl.x_dtype)
@@ -81,16 +90,18 @@ def test_prefill_workload_largest_batch(dev, li):
     sample = sorted(set([0, 511, 512, B - 1] + list(rng.choice(B, size=3, replace=False))))
     ref = oracle_y(L, xb[sample], wl.x_dtype)
     err = np.max(np.abs(y[sample] - ref))
-    print(f"\nPARITY prefill layer {li} ({L.m}x{L.n}) B={B}: max err {err:.3e} "
+    print(f"\nPARITY prefill {mode} layer {li} ({L.m}x{L.n}) B={B}: max err {err:.3e} "
           f"tol {tolerance(ref):.3e} ratio {err / tolerance(ref):.3f}")
     assert err <= tolerance(ref), (err, tolerance(ref))
     assert np.all(np.isfinite(y))
 
 
-def test_prefill_determinism_and_batch_independence(dev):
+@pytest.mark.parametrize("mode", sorted(MODES))
+def test_prefill_determinism_and_batch_independence(dev, mode):
     m, n, bpw = 520, 1032, 4
     L = gi.make_layer(5, 5, m, n, bpw)
     lay = dev.layer(L)
+    lay.set_prefill_reconstruct(MODES[mode])
     xb = gi.make_x(5, 5, 700, n, "bf16")
     x = to_torch_x(xb, "bf16")
     y1 = lay(x, out_dtype=torch.float32)
