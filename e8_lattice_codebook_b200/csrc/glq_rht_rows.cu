@@ -9,8 +9,8 @@
 // row with one thread per 16 consecutive values:
 //   * spans 1..8 run in registers, spans 16..256 as warp shuffles (lane bits
 //     of the thread index), and the remaining spans of blocks above 512 values
-//     as shared-memory rounds over the row (value-major, conflict-free), one
-//     barrier each;
+//     as shared-memory rounds over the row (value-major, conflict-free), two
+//     spans per round (radix 4), one barrier each;
 //   * a block smaller than 16 values (only the last block, of 8) keeps its
 //     thread's upper half as padding;
 //   * the input direction also finds the row's max |xr| (one reduction) and
@@ -127,14 +127,40 @@ __global__ void __launch_bounds__(1024) rht_rows_kernel(RowsParams p) {
 #pragma unroll
         for (int j = 0; j < VPT; ++j) srow[j * T + tid] = v[j];
         __syncthreads();
-        for (int h = 32 * VPT; h < p.max_blk; h <<= 1) {
+        int h = 32 * VPT;
+        for (; 2 * h < p.max_blk; h <<= 2) {  // spans h and 2h in one round (radix 4)
             const int dt = h / VPT;
-            if (h < bsz && (tid & dt) == 0) {  // this thread's 16 columns are the lower halves
-#pragma unroll
+            if (2 * h < bsz && (tid & (3 * dt)) == 0) {  // this thread's columns are the first quarter
+#pragma unroll 4
                 for (int j = 0; j < VPT; ++j) {
-                    const float a = srow[j * T + tid], c = srow[j * T + tid + dt];
-                    srow[j * T + tid] = a + c;
-                    srow[j * T + tid + dt] = a - c;
+                    float *r = srow + j * T + tid;
+                    const float a = r[0], b = r[dt], c = r[2 * dt], d = r[3 * dt];
+                    const float ab = a + b, amb = a - b, cd = c + d, cmd = c - d;
+                    r[0] = ab + cd;
+                    r[dt] = amb + cmd;
+                    r[2 * dt] = ab - cd;
+                    r[3 * dt] = amb - cmd;
+                }
+            } else if (h < bsz && 2 * h >= bsz && (tid & dt) == 0) {  // a block ending at span h
+#pragma unroll 4
+                for (int j = 0; j < VPT; ++j) {
+                    float *r = srow + j * T + tid;
+                    const float a = r[0], c = r[dt];
+                    r[0] = a + c;
+                    r[dt] = a - c;
+                }
+            }
+            __syncthreads();
+        }
+        if (h < p.max_blk) {  // one span left
+            const int dt = h / VPT;
+            if (h < bsz && (tid & dt) == 0) {
+#pragma unroll 4
+                for (int j = 0; j < VPT; ++j) {
+                    float *r = srow + j * T + tid;
+                    const float a = r[0], c = r[dt];
+                    r[0] = a + c;
+                    r[dt] = a - c;
                 }
             }
             __syncthreads();
