@@ -135,17 +135,21 @@ glq_status grow_workspace(glq_layer L, int64_t rows) {
     return GLQ_OK;
 }
 
-glq_status grow_prefill_ws(glq_layer L, int64_t rows, bool mat) {
-    if (rows <= L->pws.cap && (!mat || L->pws.w16)) return GLQ_OK;
+glq_status grow_prefill_ws(glq_layer L, int64_t rows, bool mat, int ksplit) {
+    // z holds ksplit slices of [rows][m_pad]
+    const int64_t zrows = rows * ksplit;
+    if (rows <= L->pws.cap && zrows <= L->pws.zcap && (!mat || L->pws.w16)) return GLQ_OK;
     if (cudaDeviceSynchronize() != cudaSuccess) return GLQ_ERR_CUDA;
-    if (rows <= L->pws.cap) {  // only the reconstructed W is missing
+    if (rows <= L->pws.cap && zrows <= L->pws.zcap) {  // only the reconstructed W is missing
         return dmalloc(&L->pws.w16, (size_t)L->m_pad * L->n_pad * sizeof(__half), nullptr);
     }
+    rows = std::max(rows, L->pws.cap);
     const bool had_w16 = L->pws.w16 != nullptr;
     free_prefill_ws(L);
     glq_status st = dmalloc(&L->pws.xh, (size_t)rows * L->n_pad * sizeof(__half), nullptr);
     if (st == GLQ_OK) st = dmalloc(&L->pws.info, (size_t)rows * sizeof(glq_rowinfo), nullptr);
-    if (st == GLQ_OK) st = dmalloc(&L->pws.z, (size_t)rows * L->m_pad * sizeof(float), nullptr);
+    const int64_t zcap = std::max(zrows, rows);
+    if (st == GLQ_OK) st = dmalloc(&L->pws.z, (size_t)zcap * L->m_pad * sizeof(float), nullptr);
     if (st == GLQ_OK && (mat || had_w16))
         st = dmalloc(&L->pws.w16, (size_t)L->m_pad * L->n_pad * sizeof(__half), nullptr);
     if (st != GLQ_OK) {
@@ -153,6 +157,7 @@ glq_status grow_prefill_ws(glq_layer L, int64_t rows, bool mat) {
         return st;
     }
     L->pws.cap = rows;
+    L->pws.zcap = zcap;
     return GLQ_OK;
 }
 
@@ -190,6 +195,28 @@ bool encode_w_map(CUtensorMap *map, const __half *w16, int64_t n_pad, int64_t m_
     return encode_x_map(map, w16, n_pad, m_pad);
 }
 
+// K splits of the tensor-core GEMM: fill the CTA pairs when the output has
+// too few tiles, unless the extra partial-sum traffic costs more than it
+// saves.  Model (B200 measurements): a pair retires 256 x 512 x n x 2 FLOP at
+// about 15 TFLOP/s; each extra split writes and reads B x m_pad fp32 at
+// about 6 TB/s.
+int choose_ksplit(glq_layer L, int64_t B, int tiles) {
+    const int pairs = std::max(1, L->num_sms / 2);
+    const double t_tile = 256.0 * 512.0 * (double)L->n_pad * 2.0 / 15e12;
+    const double t_traffic = (double)B * (double)L->m_pad * 8.0 / 6e12;
+    int best = 1;
+    double best_t = 1e30;
+    for (int S = 1; S <= 8 && S <= L->KC / 4 + (S == 1); ++S) {
+        const double waves = std::ceil((double)tiles * S / pairs);
+        const double t = waves * t_tile / S + (S - 1) * t_traffic;
+        if (t < best_t * 0.97) {  // a split must pay for itself clearly
+            best_t = t;
+            best = S;
+        }
+    }
+    return best;
+}
+
 glq::PrefillParams prefill_params(glq_layer L, int64_t B) {
     glq::PrefillParams pp{};
     pp.idx1 = L->d_idx1;
@@ -209,7 +236,9 @@ glq::PrefillParams prefill_params(glq_layer L, int64_t B) {
     const int tr = glq::prefill_tile_rows();
     const int tiles_m = (int)((L->m_pad + tr - 1) / tr);
     pp.tiles_tok = (int)((B + glq::prefill_tile_tokens() - 1) / glq::prefill_tile_tokens());
-    pp.ntiles = tiles_m * pp.tiles_tok;
+    pp.ksplit = choose_ksplit(L, B, tiles_m * pp.tiles_tok);
+    pp.ntiles = tiles_m * pp.tiles_tok * pp.ksplit;
+    pp.zs = (size_t)B * L->m_pad;
     pp.err = L->d_err;
     pp.table = L->primary->d_table;
     pp.table_words = L->primary->table_words;
@@ -240,6 +269,8 @@ glq::RowsParams rows_params(const glq_hblocks &hb, int len, int len_pad, const u
         r.blk_norm[i] = (float)(1.0 / std::sqrt((double)hb.len[i]));
     }
     r.sign_bits = signs;
+    r.zsplits = 1;
+    r.zs = 0;
     return r;
 }
 
@@ -249,7 +280,8 @@ glq::RowsParams rows_params(const glq_hblocks &hb, int len, int len_pad, const u
 // clustered ones.
 glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_dtype, int64_t B, cudaStream_t s) {
     const bool mat = B >= L->prefill_mat_min_b;
-    glq_status st = grow_prefill_ws(L, B, mat);
+    const int ksplit = prefill_params(L, B).ksplit;
+    glq_status st = grow_prefill_ws(L, B, mat, ksplit);
     if (st != GLQ_OK) return st;
     const bool rows_in = glq::rht_rows_supported((int)L->n_pad), rows_out = glq::rht_rows_supported((int)L->m);
     for (int64_t b0 = 0; b0 < B;) {
@@ -289,6 +321,8 @@ glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_d
             glq::RowsParams r = rows_params(L->hb_m, (int)L->m, (int)L->m, L->d_sout);
             r.z = L->pws.z + (size_t)b0 * L->m_pad;
             r.z_ld = (int)L->m_pad;
+            r.zsplits = ksplit;
+            r.zs = (size_t)B * L->m_pad;
             r.y = yb;
             r.y_dtype = y_dtype;
             if (glq::launch_rht_rows(r, false, nb, s, true) != cudaSuccess) return GLQ_ERR_CUDA;

@@ -27,10 +27,10 @@ struct glq_codebook_s {
 
 // Device buffers of the tensor-core path (B > 16 tokens).
 struct glq_prefill_ws {
-    int64_t cap = 0;
+    int64_t cap = 0, zcap = 0;    // rows of xh / info, rows of z (all K-split slices)
     __half *xh = nullptr;         // [cap][n_pad]
     glq_rowinfo *info = nullptr;  // [cap]
-    float *z = nullptr;           // [cap][m_pad]
+    float *z = nullptr;           // [zcap][m_pad]: K-split slices of [B][m_pad]
     __half *w16 = nullptr;        // [m_pad][n_pad] reconstructed W (batches >= the materialise bound)
 };
 

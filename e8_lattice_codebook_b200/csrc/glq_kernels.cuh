@@ -68,9 +68,12 @@ struct RowsParams {
     // [B][len_pad / 8][16] high / low bytes, X as fp16 in xh (3 bpw, may be
     // null), info [B] = {exact sum of X, 2^-e}
     uint8_t *xq;
-    // output: z [B][z_ld] fp32 -> y [B][len]
+    // output: z [B][z_ld] fp32 (summed over zsplits slices zs floats apart,
+    // in order) -> y [B][len]
     const float *z;
     int z_ld;
+    int zsplits;
+    size_t zs;
     void *y;
     int y_dtype;  // 0 f16, 1 bf16, 2 f32
 };
@@ -127,9 +130,11 @@ struct PrefillParams {
     uint32_t rs_h2;          // residual scale as fp16x2
     const glq_rowinfo *info; // [B]: inv_scale per token
     float ws;
-    float *z;                // [B][m_pad]
+    float *z;                // [ksplit][B][m_pad]: one slice of partial sums per K split
+    size_t zs;               // floats between slices
+    int ksplit;              // K splits (chunk-aligned), >= 1
     int B, m_pad, KC, RT;
-    int tiles_tok, ntiles;
+    int tiles_tok, ntiles;   // ntiles = row tiles x token tiles x ksplit
     unsigned *err;
 };
 

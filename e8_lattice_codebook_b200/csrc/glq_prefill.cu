@@ -84,7 +84,6 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
     uint32_t cid, ncl;
     asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(cid));
     asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(ncl));
-    const int KB = p.KC * (GLQ_CHUNK_K / BK);  // 64-column steps
 
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -118,6 +117,16 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
         abort_flag = 1;
     };
     auto live_acc = [&](int tok0) { return min(NACC, (p.B - tok0 + BN - 1) / BN); };
+    // tile -> (weight-row tile, token tile, K split) and its 64-column steps
+    // [kb0, kb1) (splits on 128-column chunk boundaries)
+    auto geom = [&](int tile, int &rtile, int &ttile, int &ks, int &kb0, int &kb1) {
+        ks = tile % p.ksplit;
+        const int rest = tile / p.ksplit;
+        rtile = rest / p.tiles_tok;
+        ttile = rest - rtile * p.tiles_tok;
+        kb0 = 2 * ((ks * p.KC) / p.ksplit);
+        kb1 = 2 * (((ks + 1) * p.KC) / p.ksplit);
+    };
 
     if (warp == 0) {
         // ---------------- TMA: this CTA's half of the activation tiles ----------------
@@ -126,18 +135,20 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
             uint32_t it = 0;
             int32_t last_load = -1;
             for (int tile = (int)cid; tile < p.ntiles && !abort_flag; tile += (int)ncl) {
-                const int tok0 = (tile % p.tiles_tok) * (BN * NACC);
+                int rtile, ttile, ks, kb0, kb1;
+                geom(tile, rtile, ttile, ks, kb0, kb1);
+                const int tok0 = ttile * (BN * NACC);
                 const int na = live_acc(tok0);
                 int halves = 0;  // live halves of both CTAs (a half past the last token is not loaded)
                 for (int a = 0; a < na; ++a)
                     for (int r = 0; r < 2; ++r) halves += tok0 + a * BN + r * BNH < p.B;
-                for (int kb = 0; kb < KB && !abort_flag; ++kb, ++it) {
+                for (int kb = kb0; kb < kb1 && !abort_flag; ++kb, ++it) {
                     const uint32_t s = it % STAGES, use = it / STAGES;
                     if (!sm100::mbar_wait_cluster(&empty_bar[s], (use & 1) ^ 1, WAIT_CYCLES)) {
                         fail();
                         break;
                     }
-                    const int wrow = (tile / p.tiles_tok) * (2 * BM);  // the pair's first weight row
+                    const int wrow = rtile * (2 * BM);  // the pair's first weight row
                     const int wparts = MAT ? (wrow < p.m_pad) + (wrow + BM < p.m_pad) : 0;
                     if (rank == 0) mbar_expect_tx(&x_full[s], (uint32_t)(halves * X_BYTES + wparts * W_BYTES));
                     if (MAT && wrow + (int)rank * BM < p.m_pad)  // rows past m_pad are never stored
@@ -162,8 +173,10 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
             const uint32_t idesc = sm100::idesc_f16_f32(2 * BM, BN);
             uint32_t it = 0, acc_use[NACC] = {0, 0};
             for (int tile = (int)cid; tile < p.ntiles && !abort_flag; tile += (int)ncl) {
-                const int na = live_acc((tile % p.tiles_tok) * (BN * NACC));
-                for (int kb = 0; kb < KB && !abort_flag; ++kb, ++it) {
+                int rtile, ttile, ks, kb0, kb1;
+                geom(tile, rtile, ttile, ks, kb0, kb1);
+                const int na = live_acc(ttile * (BN * NACC));
+                for (int kb = kb0; kb < kb1 && !abort_flag; ++kb, ++it) {
                     const uint32_t s = it % STAGES, use = it / STAGES;
                     if (!sm100::mbar_wait_cluster(&x_full[s], use & 1, WAIT_CYCLES) ||
                         (!MAT && !sm100::mbar_wait_cluster(&w_full[s], use & 1, WAIT_CYCLES))) {
@@ -174,7 +187,7 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
                     uint8_t *st = smem + s * STAGE_BYTES;
                     const uint64_t adesc = sm100::smem_desc_sw128(st);
                     for (int a = 0; a < na; ++a) {
-                        if (kb == 0) {  // both CTAs' epilogues must have drained this accumulator
+                        if (kb == kb0) {  // both CTAs' epilogues must have drained this accumulator
                             if (!sm100::mbar_wait_cluster(&acc_empty[a], (acc_use[a] & 1) ^ 1, WAIT_CYCLES)) {
                                 fail();
                                 break;
@@ -185,8 +198,8 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk)
                             sm100::mma2_f16_ss(tmem_base + a * BN, adesc + 2 * kk, bdesc + 2 * kk, idesc,
-                                               (kb | kk) != 0);
-                        if (kb == KB - 1) sm100::mma2_commit_both(&acc_full[a]);
+                                               (kb != kb0) || (kk != 0));
+                        if (kb == kb1 - 1) sm100::mma2_commit_both(&acc_full[a]);
                     }
                     sm100::mma2_commit_both(&empty_bar[s]);
                 }
@@ -207,7 +220,8 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
         const int g = lane >> 2, t = lane & 3;
         uint32_t it = 0;
         for (int tile = (int)cid; tile < p.ntiles && !abort_flag; tile += (int)ncl) {
-            const int rtile = tile / p.tiles_tok;
+            int rtile, ttile, ks, kb0, kb1;
+            geom(tile, rtile, ttile, ks, kb0, kb1);
             const int rt = (rtile * 2 + (int)rank) * (BM / GLQ_ROW_TILE) + rt_l;
             const bool live = rt < p.RT;
             const size_t slot0 = (size_t)rt * p.KC * 32 + lane;
@@ -240,14 +254,14 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
                     for (int i = 0; i < 4; ++i) cb[i] = live ? __ldg(p.res8 + ((w >> (8 * i)) & 0xFFu)) : make_uint4(0, 0, 0, 0);
                 }
             };
-            load_slot(0, q1, q2);
-            load_slot(1, n1, n2);
-            gather(0);
-            for (int kb = 0; kb < KB; ++kb, ++it) {
+            load_slot(kb0 >> 1, q1, q2);
+            load_slot((kb0 >> 1) + 1, n1, n2);
+            gather(kb0);
+            for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 uint4 cw[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) cw[i] = BPW == 2 ? ca[i] : hfma8(p.rs_h2, cb[i], ca[i]);
-                if (kb + 1 < KB) {  // the next step's gathers are in flight while this one is stored
+                if (kb + 1 < kb1) {  // the next step's gathers are in flight while this one is stored
                     if (((kb + 1) & 1) == 0) {
                         q1 = n1;
                         q2 = n2;
@@ -284,7 +298,9 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
         const int a = ew >> 2;             // the accumulator this warp drains
         uint32_t use = 0;
         for (int tile = (int)cid; tile < p.ntiles && !abort_flag; tile += (int)ncl) {
-            const int rtile = tile / p.tiles_tok, ttile = tile - rtile * p.tiles_tok;
+            int rtile, ttile, ks, kb0, kb1;
+            geom(tile, rtile, ttile, ks, kb0, kb1);
+            float *zk = p.z + (size_t)ks * p.zs;  // this split's partial sums
             const int tok0 = ttile * (BN * NACC);
             if (a >= live_acc(tok0)) continue;
             const int tb = tok0 + a * BN;
@@ -305,7 +321,7 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
                 for (int j = 0; j < 32; ++j) {
                     const float scj = __shfl_sync(0xffffffffu, sc, j);
                     if (row < p.m_pad && c + j < nlive)
-                        p.z[(size_t)(tb + c + j) * p.m_pad + row] = __uint_as_float(r[j]) * scj;
+                        zk[(size_t)(tb + c + j) * p.m_pad + row] = __uint_as_float(r[j]) * scj;
                 }
             }
             sm100::tc_fence_before();

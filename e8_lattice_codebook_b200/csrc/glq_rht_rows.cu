@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(1024) rht_rows_kernel(RowsParams p) {
     pdl_launch_dependents();
     if (c0 < p.len) {  // warm L2 and the TLB before waiting on the producer
         if (IN) prefetch_l2(static_cast<const uint16_t *>(p.x) + (size_t)b * p.len + c0);
-        else prefetch_l2(p.z + (size_t)b * p.z_ld + c0);
+        else prefetch_l2(p.z + (size_t)b * p.z_ld + c0);  // the first split
     }
     pdl_wait();  // the input comes from the previous kernel
 
@@ -82,15 +82,19 @@ __global__ void __launch_bounds__(1024) rht_rows_kernel(RowsParams p) {
         for (int j = 0; j < VPT; ++j)
             if ((sb >> j) & 1u) v[j] = -v[j];
     } else {
-        const float4 *src = reinterpret_cast<const float4 *>(p.z + (size_t)b * p.z_ld + c0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (4 * q < valid) r = __ldcs(src + q);
-            v[4 * q] = r.x;
-            v[4 * q + 1] = r.y;
-            v[4 * q + 2] = r.z;
-            v[4 * q + 3] = r.w;
+        for (int j = 0; j < VPT; ++j) v[j] = 0.f;
+        for (int sp = 0; sp < p.zsplits; ++sp) {  // K-split partial sums, in split order
+            const float4 *src = reinterpret_cast<const float4 *>(p.z + sp * p.zs + (size_t)b * p.z_ld + c0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (4 * q < valid) r = __ldcs(src + q);
+                v[4 * q] += r.x;
+                v[4 * q + 1] += r.y;
+                v[4 * q + 2] += r.z;
+                v[4 * q + 3] += r.w;
+            }
         }
     }
     if (valid < VPT)
