@@ -246,21 +246,92 @@ def time_replays(torch, graphs, reps: int, warm: int = 3) -> float:
     return e0.elapsed_time(e1) / reps
 
 
-def per_layer_times(torch, ws: WorkloadSet, reps: int, B=None):
+def per_layer_times(torch, ws: WorkloadSet, reps: int, B=None, per_graph: int = 20):
+    """Per layer: CUDA graphs of `per_graph` back-to-back glq_linear calls of
+    that layer (rotating the weight copies), mean over the replays; and the
+    eager latency of one call (events around it, median of 21)."""
     B = ws.B if B is None else B
     out = {}
+    nc = len(ws.copies)
     for i, spec in enumerate(ws.wl.layers):
         def fn(c, i=i):
-            lay, x, y = ws.copies[c][i]
+            for k in range(per_graph):
+                lay, x, y = ws.copies[(c + k) % nc][i]
+                lay(x[:B], out=y[:B])
+        graphs = capture_graphs(torch, fn, nc)
+        ms = time_replays(torch, graphs, max(1, reps // per_graph)) / per_graph
+        del graphs
+        eager = []
+        for k in range(21):
+            lay, x, y = ws.copies[k % nc][i]
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record()
             lay(x[:B], out=y[:B])
-        graphs = capture_graphs(torch, fn, len(ws.copies))
-        ms = time_replays(torch, graphs, reps)
+            e1.record()
+            torch.cuda.synchronize()
+            eager.append(e0.elapsed_time(e1))
         L = ws.host[i]
         b = layer_bytes(L.m, L.n, L.bpw, B, 2)
-        out[f"{spec.name} {L.m}x{L.n}"] = {"us": round(ms * 1e3, 3),
-                                           "GBps": round(b / (ms * 1e-3) / 1e9, 1)}
-        del graphs
+        out[f"{spec.name} {L.m}x{L.n}"] = {"us": round(ms * 1e3, 3), "GBps": round(b / (ms * 1e-3) / 1e9, 1),
+                                           "eager_us": round(sorted(eager)[10] * 1e3, 2)}
     return out
+
+
+def dense_reference_section(glq, torch, hbm_peak, tc_peak) -> dict:
+    """Context, not the product: the same shapes as a dense bf16 linear on
+    cuBLAS (torch.nn.functional.linear), W materialised by
+    glq_dequant_reference (16 bits per weight instead of 2-4).  Decode: the
+    3B-shaped layers at B = 1 (4 rotating copies, 600 MB, above L2); prefill:
+    the 8B MLP shapes at 8192 tokens, GEMM alone and dequantise + GEMM."""
+    import torch.nn.functional as F
+    res = {"decode_b1": {}, "prefill_b8192": {}}
+    ws = WorkloadSet(glq, torch, MAIN_WORKLOAD, 1, 1)
+    for i, spec in enumerate(ws.wl.layers):
+        lay, x, _ = ws.copies[0][i]
+        L = ws.host[i]
+        Ws = [lay.dequant().to(torch.bfloat16) for _ in range(4)]
+        xs = x[:1].to(torch.bfloat16)
+        def fn(c):
+            for k in range(20):
+                F.linear(xs, Ws[(c + k) % 4])
+        graphs = capture_graphs(torch, fn, 4)
+        ms = time_replays(torch, graphs, 10) / 20
+        del graphs
+        b = 2 * L.m * L.n + 2 * L.n + 2 * L.m
+        res["decode_b1"][f"{spec.name} {L.m}x{L.n}"] = {
+            "us": round(ms * 1e3, 2), "GBps": round(b / (ms * 1e-3) / 1e9, 1),
+            "frac_hbm": round(b / (ms * 1e-3) / 1e9 / hbm_peak, 3)}
+        del Ws
+    del ws
+    torch.cuda.empty_cache()
+    wp = WorkloadSet(glq, torch, "prefill-8b-mlp-4bpw", 8192, 1)
+    for i, (lay, x, _) in enumerate(wp.copies[0]):
+        L = wp.host[i]
+        W = lay.dequant().to(torch.bfloat16)
+        xb = x.to(torch.bfloat16)
+        F.linear(xb, W)
+        torch.cuda.synchronize()
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record()
+        for _ in range(5):
+            F.linear(xb, W)
+        e1.record()
+        for _ in range(5):
+            F.linear(xb, lay.dequant().to(torch.bfloat16))
+        e2.record()
+        torch.cuda.synchronize()
+        g_ms, dg_ms = e0.elapsed_time(e1) / 5, e1.elapsed_time(e2) / 5
+        fl = 2.0 * 8192 * L.m * L.n
+        res["prefill_b8192"][f"{L.m}x{L.n}"] = {
+            "gemm_us": round(g_ms * 1e3, 1), "gemm_TFLOPs": round(fl / (g_ms * 1e-3) / 1e12, 1),
+            "dequant_gemm_us": round(dg_ms * 1e3, 1),
+            "dequant_gemm_TFLOPs": round(fl / (dg_ms * 1e-3) / 1e12, 1)}
+        del W
+    del wp
+    torch.cuda.empty_cache()
+    res["note"] = "cuBLAS bf16 via torch; W materialised at 16 bits per weight; not the product path"
+    return res
 
 
 def gemv_kernel_time(torch, ws: WorkloadSet, layer_index: int, reps: int, B=None) -> float:
@@ -500,6 +571,7 @@ def run_glq(args):
         result["decode_24b"] = sweep
 
         result["prefill"] = prefill_section(glq, torch, tc_peak, peak_src)
+        result["dense_bf16_reference"] = dense_reference_section(glq, torch, hbm_peak, tc_peak)
 
     # fp64 oracle on the host cores (one decode step, 1 token, 5 layers)
     if world == 1 and not args.no_cpu:

@@ -388,9 +388,15 @@ DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y
             c.plan = fp;
         }
     }
+    c.warps = warps;
     if (!c.fin) {
         c.plan = plan_for(L, nb);
-        if (c.plan.splits > max_splits) c.plan = plan_gemv(L->RT, L->KC, L->num_sms, warps, false, 1 << 30, max_splits);
+        if (nt == 1 && (long long)L->RT * L->KC >= 200LL * L->num_sms) {  // large layer: wide CTAs
+            c.warps = GEMV_WIDE_WARPS;
+            c.plan = plan_gemv(L->RT, L->KC, L->num_sms, c.warps);
+        }
+        if (c.plan.splits > max_splits)
+            c.plan = plan_gemv(L->RT, L->KC, L->num_sms, c.warps, false, 1 << 30, max_splits);
     }
     return c;
 }
@@ -403,7 +409,8 @@ int max_decode_splits(glq_layer L, int nb) {
                GEMV_SMEM_LIMIT)
         cap *= 2;
     const GemvPlan f = plan_gemv(L->RT, L->KC, L->num_sms, warps, true, cap);
-    return std::max(plan_for(L, nb).splits, f.splits);
+    const GemvPlan wide = plan_gemv(L->RT, L->KC, L->num_sms, GEMV_WIDE_WARPS);
+    return std::max(std::max(plan_for(L, nb).splits, f.splits), wide.splits);
 }
 
 GemvParams gemv_params(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg, int nb, const void *x,
@@ -434,6 +441,7 @@ GemvParams gemv_params(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg
     p.z = w.z;
     p.m_pad = (int)L->m_pad;
     p.err = L->d_err;
+    p.warps = cfg.warps;
     // fused transforms
     p.x = x;
     p.x_bf16 = x_bf16 ? 1 : 0;
@@ -450,7 +458,7 @@ GemvParams gemv_params(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg
     p.m = (int)L->m;
     p.sout_bits = L->d_sout;
     p.nblk_m = L->hb_m.count;
-    const int band_rows = gemv_warps(nb > 8 ? 2 : 1) * GLQ_ROW_TILE;
+    const int band_rows = cfg.warps * GLQ_ROW_TILE;
     for (int i = 0; i < L->hb_m.count; ++i) {
         const int o = L->hb_m.off[i], N = L->hb_m.len[i];
         p.blk_off_m[i] = o;

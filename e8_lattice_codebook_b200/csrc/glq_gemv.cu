@@ -418,9 +418,8 @@ __device__ void fused_output(const GemvParams &p, int blk, float *buf) {
     }
 }
 
-template <int BPW, int NT, bool FIN>
-__global__ void __launch_bounds__(gemv_warps(NT) * 32, 1) gemv_kernel(GemvParams p) {
-    constexpr int WARPS = gemv_warps(NT);
+template <int BPW, int NT, bool FIN, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
     constexpr int THREADS = WARPS * 32;
     constexpr int BAND_ROWS = WARPS * GLQ_ROW_TILE;
     extern __shared__ __align__(16) uint4 smem_u4[];
@@ -660,7 +659,7 @@ __global__ void __launch_bounds__(gemv_warps(NT) * 32, 1) gemv_kernel(GemvParams
     }
 }
 
-template <int BPW, int NT, bool FIN>
+template <int BPW, int NT, bool FIN, int WARPS = gemv_warps(NT)>
 cudaError_t launch_t(const GemvParams &p, int grid, cudaStream_t s, bool pdl) {
     const size_t smem = FIN ? gemv_fused_smem_bytes(p.table_words, BPW, p.B, min(p.cps, p.KC) * GLQ_CHUNK_K)
                             : gemv_smem_bytes(p.table_words, BPW);
@@ -668,7 +667,7 @@ cudaError_t launch_t(const GemvParams &p, int grid, cudaStream_t s, bool pdl) {
     // captured graphs replay against the attribute value at replay time)
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<BPW, NT, FIN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<BPW, NT, FIN, WARPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)GEMV_SMEM_LIMIT);
         if (e != cudaSuccess) return e;
         configured = true;
@@ -680,7 +679,7 @@ cudaError_t launch_t(const GemvParams &p, int grid, cudaStream_t s, bool pdl) {
     }
     GemvParams q = p;
     void *args[] = {&q};
-    return launch_ex((const void *)gemv_kernel<BPW, NT, FIN>, dim3(grid), dim3(gemv_warps(NT) * 32), smem, s,
+    return launch_ex((const void *)gemv_kernel<BPW, NT, FIN, WARPS>, dim3(grid), dim3(WARPS * 32), smem, s,
                      pdl, args);
 }
 
@@ -733,6 +732,15 @@ size_t gemv_fused_smem_bytes(int table_words, int bpw, int B, int klen) {
 template <bool FIN>
 cudaError_t launch_sel(const GemvParams &p, int bpw, int grid, cudaStream_t s, bool pdl) {
     const bool two = p.B > 8;
+    if (!FIN && !two && p.warps == GEMV_WIDE_WARPS) {
+        switch (bpw) {
+            case 2: return launch_t<2, 1, false, GEMV_WIDE_WARPS>(p, grid, s, pdl);
+            case 3: return launch_t<3, 1, false, GEMV_WIDE_WARPS>(p, grid, s, pdl);
+            case 4: return launch_t<4, 1, false, GEMV_WIDE_WARPS>(p, grid, s, pdl);
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    if (p.warps != gemv_warps(two ? 2 : 1)) return cudaErrorInvalidValue;
     switch (bpw) {
         case 2: return two ? launch_t<2, 2, FIN>(p, grid, s, pdl) : launch_t<2, 1, FIN>(p, grid, s, pdl);
         case 3: return two ? launch_t<3, 2, FIN>(p, grid, s, pdl) : launch_t<3, 1, FIN>(p, grid, s, pdl);

@@ -92,6 +92,7 @@ namespace glq {
 struct DecodeCfg {
     GemvPlan plan{};
     bool fin = false, fout = false;
+    int warps = 0;  // warps per GEMV CTA
 };
 
 // max_cps bounds the chunks per split (callers with a small partial-sum
