@@ -421,6 +421,33 @@ def prefill_section(glq, torch, tc_peak, peak_src, batches=(512, 2048, 8192), re
     return pre
 
 
+def decode24_section(glq, torch, hbm_peak, batches=(1, 2, 4, 8, 16), reps=100) -> dict:
+    """24B-class decode (q 4096x5120, o 5120x4096, gate/up 32768x5120, down
+    5120x32768 at 4 bpw, bf16): per batch the five-layer step as CUDA-graph
+    replays over two weight copies (544 MB > L2); at B = 1 also the per-layer
+    times and the GEMV kernel alone on the gate layer."""
+    sweep = {}
+    w24 = WorkloadSet(glq, torch, "24b-decode-4bpw", max(batches), 2)
+    for Bd in batches:
+        g24 = capture_graphs(torch, lambda c, Bd=Bd: w24.step(c, B=Bd), 2)
+        ms24 = time_replays(torch, g24, reps=reps)
+        b24 = w24.step_bytes(Bd)
+        entry = {"ms_per_step": round(ms24, 4), "GBps": round(b24 / (ms24 * 1e-3) / 1e9, 1),
+                 "frac_hbm": round(b24 / (ms24 * 1e-3) / 1e9 / hbm_peak, 4)}
+        if Bd == 1:
+            entry["layers_us"] = per_layer_times(torch, w24, reps=reps, B=1)
+            mk = gemv_kernel_time(torch, w24, 2, reps=reps, B=1)
+            Lg = w24.host[2]
+            ach = gemv_bytes(Lg.m, Lg.n, Lg.bpw, 1) / (mk * 1e-3) / 1e9
+            entry["gemv_gate_us"] = round(mk * 1e3, 3)
+            entry["gemv_gate_frac_hbm"] = round(ach / hbm_peak, 4)
+        sweep[f"B={Bd}"] = entry
+        del g24
+    del w24
+    torch.cuda.empty_cache()
+    return sweep
+
+
 def oracle_step_seconds(ws_host, xbits, bpw, x_bf16) -> float:
     from oracle import glq_oracle as orc
     t0 = time.perf_counter()
@@ -549,26 +576,7 @@ def run_glq(args):
 
     # 24B-class decode sweep
     if not args.quick:
-        sweep = {}
-        w24 = WorkloadSet(glq, torch, "24b-decode-4bpw", 16, 2)
-        for Bd in (1, 2, 4, 8, 16):
-            g24 = capture_graphs(torch, lambda c, Bd=Bd: w24.step(c, B=Bd), 2)
-            ms24 = time_replays(torch, g24, reps=100)
-            b24 = w24.step_bytes(Bd)
-            entry = {"ms_per_step": round(ms24, 4), "GBps": round(b24 / (ms24 * 1e-3) / 1e9, 1),
-                     "frac_hbm": round(b24 / (ms24 * 1e-3) / 1e9 / hbm_peak, 4)}
-            if Bd == 1:
-                entry["layers_us"] = per_layer_times(torch, w24, reps=100, B=1)
-                mk = gemv_kernel_time(torch, w24, 2, reps=100, B=1)
-                Lg = w24.host[2]
-                ach = gemv_bytes(Lg.m, Lg.n, Lg.bpw, 1) / (mk * 1e-3) / 1e9
-                entry["gemv_gate_us"] = round(mk * 1e3, 3)
-                entry["gemv_gate_frac_hbm"] = round(ach / hbm_peak, 4)
-            sweep[f"B={Bd}"] = entry
-            del g24
-        del w24
-        torch.cuda.empty_cache()
-        result["decode_24b"] = sweep
+        result["decode_24b"] = decode24_section(glq, torch, hbm_peak)
 
         result["prefill"] = prefill_section(glq, torch, tc_peak, peak_src)
         result["dense_bf16_reference"] = dense_reference_section(glq, torch, hbm_peak, tc_peak)
@@ -633,6 +641,17 @@ def run_prefill_only(args):
                                                             reps=max(1, min(args.steps, 20)))}
 
 
+def run_decode24_only(args):
+    """The 24B-class decode timings alone, one JSON object (not the bench line)."""
+    import torch
+    import e8_lattice_codebook_b200 as glq
+    torch.cuda.set_device(0)
+    hbm_peak = read_peaks()[0]
+    batches = (args.decode_batch,) if args.decode_batch else (1, 2, 4, 8, 16)
+    return {"section": "decode24", "decode_24b": decode24_section(glq, torch, hbm_peak, batches,
+                                                                  reps=max(20, min(args.steps, 400)))}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -641,15 +660,19 @@ def main():
     ap.add_argument("--impl", choices=["glq", "reference"], default="glq")
     ap.add_argument("--quick", action="store_true", help="skip the 24B sweep and prefill")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle baseline")
-    ap.add_argument("--section", choices=["all", "prefill"], default="all",
-                    help="prefill: time only the prefill workload (profiling runs)")
+    ap.add_argument("--section", choices=["all", "prefill", "decode24"], default="all",
+                    help="prefill / decode24: time only that workload (profiling runs)")
     ap.add_argument("--prefill-batch", type=int, default=0,
                     help="with --section prefill: one batch instead of 512, 2048, 8192")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="with --section decode24: one batch instead of 1, 2, 4, 8, 16")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.section == "prefill":
         res = run_prefill_only(args)
+    elif args.section == "decode24":
+        res = run_decode24_only(args)
     else:
         res = run_reference(args) if args.impl == "reference" else run_glq(args)
     if res is not None:

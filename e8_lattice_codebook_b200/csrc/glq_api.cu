@@ -422,6 +422,7 @@ GemvParams gemv_params(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg
     p.table = L->primary->d_table;
     p.table_words = L->primary->table_words;
     p.fold = FoldParams{L->primary->fold.nb, L->primary->fold.neg_base};
+    p.kc = LookupConsts{4u, 16u, 0xFFFFFFFFu};
     p.res8 = (L->bpw == 3) ? reinterpret_cast<const uint4 *>(L->residual->d_fp16) : nullptr;
     p.xq = w.xq;
     p.xh = w.xh;

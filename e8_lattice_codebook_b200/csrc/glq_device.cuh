@@ -40,6 +40,36 @@ __device__ __forceinline__ uint32_t table_word(const uint32_t *T, uint32_t e, Fo
     return w;
 }
 
+// Multipliers the GEMV's lookups take at run time (4, 16 and -1): given as
+// kernel parameters, the compiler cannot turn the multiply-adds that use them
+// into shifts or logic, so address, negation and scaling run on the integer
+// multiply-add (FMA) pipe beside the logic ops on the ALU pipe.
+struct LookupConsts {
+    uint32_t four, sixteen, neg_one;
+};
+
+// The two A-fragment registers of code e scaled by 16: lo16 = 16 (v0..v3),
+// hi16 = 16 (v4..v7) as u8 (16 v <= 192).  tbase / tneg are the shared
+// addresses of T[0] and T[-neg_base].
+__device__ __forceinline__ void table_a16(uint32_t tbase, uint32_t tneg, uint32_t e, uint32_t nb,
+                                          LookupConsts k, uint32_t &lo16, uint32_t &hi16) {
+    asm("{\n"
+        " .reg .pred p;\n"
+        " .reg .u32 a, w, t;\n"
+        " setp.ge.u32 p, %2, %3;\n"
+        " mad.lo.u32 a, %2, %4, %5;\n"
+        " @p mad.lo.u32 a, %2, %4, %6;\n"
+        " ld.shared.u32 w, [a];\n"
+        " @p mad.lo.u32 w, w, %7, %8;\n"
+        " and.b32 %1, w, 0xF0F0F0F0;\n"
+        " mul.lo.u32 t, w, %9;\n"
+        " and.b32 %0, t, 0xF0F0F0F0;\n"
+        "}\n"
+        : "=r"(lo16), "=r"(hi16)
+        : "r"(e), "r"(nb), "r"(k.four), "r"(tbase), "r"(tneg), "r"(k.neg_one), "r"(0xCCCCCCCCu),
+          "r"(k.sixteen));
+}
+
 // The same lookup from a global-memory table (reference decode).
 __device__ __forceinline__ uint32_t table_word_global(const uint32_t *T, uint32_t e, FoldParams f) {
     const bool neg = e >= (uint32_t)f.nb;

@@ -50,13 +50,25 @@ __device__ __forceinline__ void zero(Acc &a) {
         for (int j = 0; j < 4; ++j) a.hi[i][j] = a.lo[i][j] = 0;
 }
 
+// Shared addresses of the folded table: T[0] and T[-neg_base].
+struct TableRef {
+    uint32_t base, neg;
+};
+
+__device__ __forceinline__ TableRef table_ref(const uint32_t *T, FoldParams fold) {
+    const uint32_t b = (uint32_t)__cvta_generic_to_shared(T);
+    return TableRef{b, b - 4u * (uint32_t)fold.neg_base};
+}
+
 // One stage (one code per row) of one super-tile: codes of rows g and g+8.
+// The A operands are 16 v (see table_a16), so the int32 sums are 16 sum v X:
+// at most 16 * 12 * 255 * 32768 < 2^31 for the low bytes over the longest row.
 template <int NT>
-__device__ __forceinline__ void stage_int(const uint32_t *T, FoldParams fold, uint32_t codes,
+__device__ __forceinline__ void stage_int(TableRef T, FoldParams fold, LookupConsts kc, uint32_t codes,
                                           const uint4 &x0, const uint4 &x1, Acc &acc) {
-    const uint32_t wg = table_word(T, codes & 0xFFFFu, fold);
-    const uint32_t wg8 = table_word(T, codes >> 16, fold);
-    const uint32_t a[4] = {nib_lo(wg), nib_lo(wg8), nib_hi(wg), nib_hi(wg8)};
+    uint32_t a[4];
+    table_a16(T.base, T.neg, codes & 0xFFFFu, (uint32_t)fold.nb, kc, a[0], a[2]);
+    table_a16(T.base, T.neg, codes >> 16, (uint32_t)fold.nb, kc, a[1], a[3]);
     mma_u8s8(acc.hi[0], a, x0.x, x0.y);
     mma_u8u8(acc.lo[0], a, x0.z, x0.w);
     if (NT == 2) {
@@ -73,7 +85,7 @@ __device__ __forceinline__ uint4 ld_x(const void *p) {
 }
 
 template <int BPW, int NT, bool XS>
-__device__ __forceinline__ void process_chunk(const uint32_t *T, const uint4 *R8, FoldParams fold,
+__device__ __forceinline__ void process_chunk(TableRef T, const uint4 *R8, FoldParams fold, LookupConsts kc,
                                               const uint4 &q1, const uint4 &q2, const uint4 *xq0,
                                               const uint4 *xq1, const __half *xh0, const __half *xh1,
                                               bool has0, bool has1, Acc &acc1, Acc &acc2,
@@ -85,8 +97,8 @@ __device__ __forceinline__ void process_chunk(const uint32_t *T, const uint4 *R8
         uint4 x0 = make_uint4(0, 0, 0, 0), x1 = make_uint4(0, 0, 0, 0);
         if (has0) x0 = ld_x<XS>(xq0 + 4 * s);
         if (NT == 2 && has1) x1 = ld_x<XS>(xq1 + 4 * s);
-        stage_int<NT>(T, fold, p1[s], x0, x1, acc1);
-        if (BPW == 4) stage_int<NT>(T, fold, p2[s], x0, x1, acc2);
+        stage_int<NT>(T, fold, kc, p1[s], x0, x1, acc1);
+        if (BPW == 4) stage_int<NT>(T, fold, kc, p2[s], x0, x1, acc2);
         if (BPW == 3) {
             // bytes 2s (row g) and 2s+1 (row g+8) of the 8-byte payload
             const uint32_t word = (s < 2) ? q2.x : q2.y;
@@ -118,8 +130,9 @@ __device__ __forceinline__ uint4 load_q2(const void *idx2, size_t i) {
     return make_uint4(0, 0, 0, 0);
 }
 
+// sum v X of one accumulator pair from its 16 v sums (exact: a multiple of 16)
 __device__ __forceinline__ double exact_sum(int hi, int lo) {
-    return (double)((long long)hi * 256 + (long long)lo);
+    return (double)((long long)hi * 256 + (long long)lo) * 0.0625;
 }
 
 // z of (token b, any row) from D = sum over splits of the partials:
@@ -433,6 +446,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
     __shared__ int s_sign_w0;
     __shared__ int s_npending;
     uint32_t *T = reinterpret_cast<uint32_t *>(smem_u4);
+    const TableRef tref = table_ref(T, p.fold);
     uint4 *R8 = smem_u4 + p.table_words / 4;
     // fused input: [xs: B x klen/8 uint4][xhs: B x klen halves (3 bpw)][u: B x klen floats]
     const int klen_max = min(p.cps, p.KC) * GLQ_CHUNK_K;
@@ -564,7 +578,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
                         }
                         pq1 += 32;
                         ++ahead;
-                        process_chunk<BPW, NT, FIN>(T, R8, p.fold, q1, q2, px0, px1, ph0, ph1, has0, has1,
+                        process_chunk<BPW, NT, FIN>(tref, R8, p.fold, p.kc, q1, q2, px0, px1, ph0, ph1, has0, has1,
                                                     acc1, acc2, accr);
                         px0 += GLQ_GROUPS_PER_CHUNK;
                         px1 += GLQ_GROUPS_PER_CHUNK;

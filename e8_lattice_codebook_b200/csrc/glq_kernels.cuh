@@ -84,6 +84,7 @@ struct GemvParams {
     const uint32_t *table; // folded nibble table (global), table_words (multiple of 4)
     int table_words;
     FoldParams fold;
+    LookupConsts kc;       // 4, 16, -1 (see LookupConsts)
     const uint4 *res8;     // 3 bpw: [256] x 8 fp16
     const uint8_t *xq;     // [B][n_pad/8][16]
     const __half *xh;      // [B][n_pad] (3 bpw)
