@@ -198,7 +198,7 @@ __device__ __forceinline__ float flip(float v, uint32_t sb, int j) {
 // bf16 activations, or 16 fp32 partial sums of the first K split) with
 // asynchronous copies into its own slots of a staging buffer while the
 // current row is transformed.
-template <bool IN, int L>
+template <bool IN, bool XQ, int L>
 __global__ void __launch_bounds__(1 << (L - 4)) rht_rows_kernel(RowsParams p, int B) {
     constexpr int NPH = (L + 3) / 4;  // phases of (up to) four position bits
     constexpr int NCH = IN ? 2 : 4;   // 16-byte chunks of raw input per thread
@@ -274,8 +274,9 @@ __global__ void __launch_bounds__(1 << (L - 4)) rht_rows_kernel(RowsParams p, in
                     }
                 }
             }
+            const uint32_t sbr = opaque(sb);  // sign masks rebuilt per row, not kept live
 #pragma unroll
-            for (int j = 0; j < VPT; ++j) v[j] = flip(v[j], sb, j);
+            for (int j = 0; j < VPT; ++j) v[j] = flip(v[j], sbr, j);
         } else {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -334,7 +335,7 @@ __global__ void __launch_bounds__(1 << (L - 4)) rht_rows_kernel(RowsParams p, in
                 scale = ldexpf(1.f, 14 - e);
             }
             const float f = norm * scale;  // scale is a power of two: one rounding, as xr 2^e
-            if (p.xq) {  // decode GEMV operand: X = round(xr 2^e), bytes per 8-column group
+            if (XQ) {  // decode GEMV operand: X = round(xr 2^e), bytes per 8-column group
                 int sum = 0;
                 if (c0 < p.len_pad) {
                     uint32_t hb[4] = {0u, 0u, 0u, 0u}, lb[4] = {0u, 0u, 0u, 0u};
@@ -383,8 +384,9 @@ __global__ void __launch_bounds__(1 << (L - 4)) rht_rows_kernel(RowsParams p, in
             }
         } else if (valid) {
             float y[VPT];
+            const uint32_t sbr = opaque(sb);  // sign masks rebuilt per row, not kept live
 #pragma unroll
-            for (int j = 0; j < VPT; ++j) y[j] = flip(v[j] * norm, sb, j);
+            for (int j = 0; j < VPT; ++j) y[j] = flip(v[j] * norm, sbr, j);
             const size_t off = (size_t)b * p.len + c0;
             for (int q = 0; q < valid / 8; ++q) {
                 const float *r = y + 8 * q;
@@ -425,9 +427,9 @@ int rows_log2(int cover) {
     return L;
 }
 
-template <bool IN, int L>
+template <bool IN, bool XQ, int L>
 cudaError_t launch_rows_t(const RowsParams &p, int B, cudaStream_t s, bool pdl) {
-    const void *fn = (const void *)rht_rows_kernel<IN, L>;
+    const void *fn = (const void *)rht_rows_kernel<IN, XQ, L>;
     const int threads = 1 << (L - 4);
     // the row buffer and the staging buffer of the next row's raw input
     const size_t smem = (sizeof(float) << L) + (size_t)threads * (IN ? 32 : 64);
@@ -450,16 +452,17 @@ cudaError_t launch_rows_t(const RowsParams &p, int B, cudaStream_t s, bool pdl) 
     return launch_ex(fn, dim3(grid), dim3(threads), smem, s, pdl, args);
 }
 
-template <bool IN>
+// IN: input side; XQ: the decode operand (bytes of X) instead of fp16 xr 2^e
+template <bool IN, bool XQ>
 cudaError_t launch_rows_sel(const RowsParams &p, int B, cudaStream_t s, bool pdl) {
     const int cover = IN ? p.len_pad : p.len;
     switch (rows_log2(cover)) {
-        case 9: return launch_rows_t<IN, 9>(p, B, s, pdl);
-        case 10: return launch_rows_t<IN, 10>(p, B, s, pdl);
-        case 11: return launch_rows_t<IN, 11>(p, B, s, pdl);
-        case 12: return launch_rows_t<IN, 12>(p, B, s, pdl);
-        case 13: return launch_rows_t<IN, 13>(p, B, s, pdl);
-        case 14: return launch_rows_t<IN, 14>(p, B, s, pdl);
+        case 9: return launch_rows_t<IN, XQ, 9>(p, B, s, pdl);
+        case 10: return launch_rows_t<IN, XQ, 10>(p, B, s, pdl);
+        case 11: return launch_rows_t<IN, XQ, 11>(p, B, s, pdl);
+        case 12: return launch_rows_t<IN, XQ, 12>(p, B, s, pdl);
+        case 13: return launch_rows_t<IN, XQ, 13>(p, B, s, pdl);
+        case 14: return launch_rows_t<IN, XQ, 14>(p, B, s, pdl);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -468,7 +471,8 @@ cudaError_t launch_rows_sel(const RowsParams &p, int B, cudaStream_t s, bool pdl
 
 cudaError_t launch_rht_rows(const RowsParams &p, bool input, int B, cudaStream_t s, bool pdl) {
     if (B <= 0) return cudaErrorInvalidValue;
-    return input ? launch_rows_sel<true>(p, B, s, pdl) : launch_rows_sel<false>(p, B, s, pdl);
+    if (!input) return launch_rows_sel<false, false>(p, B, s, pdl);
+    return p.xq ? launch_rows_sel<true, true>(p, B, s, pdl) : launch_rows_sel<true, false>(p, B, s, pdl);
 }
 
 }  // namespace glq
