@@ -37,7 +37,7 @@ EXPORTS = (
     "glq_status_str", "glq_version", "glq_e8_codebook", "glq_codebook_upload",
     "glq_codebook_destroy", "glq_layer_create", "glq_layer_destroy", "glq_layer_reserve",
     "glq_linear", "glq_dequant_reference", "glq_rht_input", "glq_rht_output",
-    "glq_layer_check", "glq_layer_info", "glq_gemv_replay", "glq_linear_noalloc",
+    "glq_layer_check", "glq_layer_info", "glq_gemv_replay", "glq_linear_noalloc", "glq_decode_plan",
     "glq_prefill_replay", "glq_layer_set_fusion", "glq_layer_set_prefill_reconstruct",
 )
 
@@ -71,6 +71,8 @@ _SIGNATURES = {
     "glq_prefill_replay": ([_vp, _i64, _vp], ctypes.c_int),
     "glq_layer_set_fusion": ([_vp, ctypes.c_int32], ctypes.c_int),
     "glq_layer_set_prefill_reconstruct": ([_vp, _i64], ctypes.c_int),
+    "glq_decode_plan": ([_vp, _i64, ctypes.POINTER(_i32), ctypes.POINTER(_i32), ctypes.POINTER(_i32),
+                         ctypes.POINTER(_i32), ctypes.POINTER(_i32)], ctypes.c_int),
     "glq_layer_info": ([_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i32),
                         ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
 }
@@ -189,7 +191,7 @@ def glq_prefill_replay(handle, B, stream) -> None:
     _ok(_L().glq_prefill_replay(handle, B, stream), "glq_prefill_replay")
 
 
-GLQ_FUSE_INPUT, GLQ_FUSE_OUTPUT, GLQ_FUSE_DEFAULT = 1, 2, -1
+GLQ_FUSE_INPUT, GLQ_FUSE_OUTPUT, GLQ_SPLITK_CLUSTER, GLQ_FUSE_DEFAULT = 1, 2, 4, -1
 
 
 def glq_layer_set_fusion(handle, flags: int) -> None:
@@ -202,6 +204,12 @@ def glq_layer_set_prefill_reconstruct(handle, min_batch: int) -> None:
 
 def glq_layer_check(handle, stream) -> None:
     _ok(_L().glq_layer_check(handle, stream), "glq_layer_check")
+
+
+def glq_decode_plan(handle, B: int) -> dict:
+    vals = [_i32() for _ in range(5)]
+    _ok(_L().glq_decode_plan(handle, int(B), *[ctypes.byref(v) for v in vals]), "glq_decode_plan")
+    return dict(zip(("warps", "bands", "splits", "cluster", "fused_input"), (v.value for v in vals)))
 
 
 def glq_layer_info(handle):
@@ -307,6 +315,9 @@ class GlqLinear:
         glq_rht_output(self.handle, z.data_ptr(), y.data_ptr(), dtype_code(y.dtype), z.shape[0],
                        _stream_ptr(stream))
         return y
+
+    def decode_plan(self, B: int) -> dict:
+        return glq_decode_plan(self.handle, B)
 
     def gemv_replay(self, B, stream=None):
         glq_gemv_replay(self.handle, B, _stream_ptr(stream))

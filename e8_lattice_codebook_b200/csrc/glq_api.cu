@@ -355,7 +355,7 @@ constexpr long long FUSED_OUT_MAX_VALUES = 32768;
 // saves a launch when every CTA has one short task (below); the output
 // transform done by one CTA at the end of the GEMV is slower than the
 // separate, parallel kernel at every size measured, so it is off by default.
-constexpr int FUSE_DEFAULT_FLAGS = GLQ_FUSE_INPUT;
+constexpr int FUSE_DEFAULT_FLAGS = GLQ_FUSE_INPUT | GLQ_SPLITK_CLUSTER;
 
 DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y_dtype, int max_splits) {
     DecodeCfg c;
@@ -397,6 +397,21 @@ DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y
         }
         if (c.plan.splits > max_splits)
             c.plan = plan_gemv(L->RT, L->KC, L->num_sms, c.warps, false, 1 << 30, max_splits);
+    }
+    // split-K through a thread-block cluster: one task per CTA, the band's
+    // splits in one cluster (at most 16), all clusters resident at once
+    const int S = c.plan.splits;
+    if ((flags & GLQ_SPLITK_CLUSTER) && S > 1 && S <= 16 && !c.fout &&
+        (long long)c.plan.bands * S == (long long)c.plan.grid) {
+        const size_t base = c.fin ? gemv_fused_smem_bytes(L->primary->table_words, L->bpw, nb,
+                                                          std::min(c.plan.cps, L->KC) * GLQ_CHUNK_K)
+                                  : gemv_smem_bytes(L->primary->table_words, L->bpw);
+        const size_t off = (base + 255) & ~(size_t)255;
+        const size_t need = off + gemv_cluster_partials_bytes(c.warps, nb);
+        if (need <= GEMV_SMEM_LIMIT && gemv_max_clusters(L->bpw, nt, c.fin, c.warps, S, need) >= c.plan.bands) {
+            c.clu = S;
+            c.spart_off = off;
+        }
     }
     return c;
 }
@@ -454,6 +469,8 @@ GemvParams gemv_params(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg
         p.blk_len_n[i] = L->hb_n.len[i];
     }
     p.fuse_out = cfg.fout ? 1 : 0;
+    p.clu = cfg.clu;
+    p.spart_off = cfg.spart_off;
     p.y = y;
     p.y_dtype = y_dtype;
     p.m = (int)L->m;
@@ -762,9 +779,25 @@ glq_status glq_layer_reserve(glq_layer layer, int64_t max_B) {
     return grow_workspace(layer, std::min<int64_t>(std::max<int64_t>(max_B, 1), GLQ_DECODE_MAX_B));
 }
 
+glq_status glq_decode_plan(glq_layer layer, int64_t B, int32_t *warps, int32_t *bands, int32_t *splits,
+                           int32_t *cluster, int32_t *fused_input) {
+    if (!layer) return GLQ_ERR_INVALID_ARG;
+    if (B < 1 || B > GLQ_DECODE_MAX_B) return GLQ_ERR_SHAPE;
+    DeviceGuard guard(layer->device);
+    const void *aligned = reinterpret_cast<const void *>(static_cast<uintptr_t>(256));
+    const glq::DecodeCfg c = glq::decode_config(layer, (int)B, aligned, aligned, GLQ_F32);
+    if (warps) *warps = c.warps;
+    if (bands) *bands = c.plan.bands;
+    if (splits) *splits = c.plan.splits;
+    if (cluster) *cluster = c.clu;
+    if (fused_input) *fused_input = c.fin ? 1 : 0;
+    return GLQ_OK;
+}
+
 glq_status glq_layer_set_fusion(glq_layer layer, int32_t flags) {
     if (!layer) return GLQ_ERR_INVALID_ARG;
-    if (flags != GLQ_FUSE_DEFAULT && (flags & ~(GLQ_FUSE_INPUT | GLQ_FUSE_OUTPUT))) return GLQ_ERR_INVALID_ARG;
+    if (flags != GLQ_FUSE_DEFAULT && (flags & ~(GLQ_FUSE_INPUT | GLQ_FUSE_OUTPUT | GLQ_SPLITK_CLUSTER)))
+        return GLQ_ERR_INVALID_ARG;
     layer->fusion = flags;
     return GLQ_OK;
 }

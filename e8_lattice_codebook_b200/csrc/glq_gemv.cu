@@ -23,14 +23,24 @@
 //     fp16 operands with fp32 accumulation;
 //   * per task, partial sums go to a workspace in fp64; the last CTA to
 //     finish a band (atomic counter, no waiting) adds the splits in fixed
-//     order and writes the band's final z;
+//     order and writes the band's final z.  When every CTA has one task and
+//     a band's splits fit one thread-block cluster, the partials stay in
+//     shared memory instead and the cluster's CTAs add them through
+//     distributed shared memory, each for its share of the band's rows, in
+//     the same fixed order (no global round trip, no last arriver);
 //   * small batches fuse both transforms (one launch per layer): each task
 //     rotates, scales and quantises its own aligned column range of x in
 //     shared memory (a Hadamard block of size N = 2^a S restricted to an
 //     aligned range of S outputs is H_S applied to the 2^a-term signed fold
 //     of the block), and the last band to finish a Hadamard block of m
 //     transforms that block of z in shared memory and writes y.
+#include <cooperative_groups.h>
+
+#include <algorithm>
+
 #include "glq_kernels.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace glq {
 
@@ -453,6 +463,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
     uint4 *xs = R8 + (BPW == 3 ? 256 : 0);
     __half *xhs = reinterpret_cast<__half *>(xs + (size_t)p.B * klen_max / 8);
     float *ubuf = reinterpret_cast<float *>(xhs + (BPW == 3 ? (size_t)p.B * klen_max : 0));
+    // cluster reduction: this CTA's partial sums [B][BAND_ROWS] (fp64)
+    double *spart = reinterpret_cast<double *>(reinterpret_cast<char *>(smem_u4) + p.spart_off);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int ntasks = p.bands * p.splits;
@@ -519,6 +531,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
         if (ok) return true;
         if (tid == 0) atomicOr(p.err, GLQ_DEVERR_TIMEOUT);
         mbar_wait_bounded(&bar, 0, TABLE_WAIT_POLLS);  // let the copy land before exiting
+        if (p.clu) {  // leaving early: still take the cluster's two barriers of the reduction
+            cg::cluster_group cluster = cg::this_cluster();
+            cluster.sync();
+            cluster.sync();
+        }
         return false;
     };
     if (!FIN && !wait_table()) return;
@@ -607,6 +624,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
                         }
                         if (p.splits == 1) {
                             p.z[(size_t)b * p.m_pad + row] = FIN ? (float)(D * (double)p.ws) : finish_z(p, b, D);
+                        } else if (p.clu) {
+                            spart[(size_t)b * BAND_ROWS + warp * GLQ_ROW_TILE + g + (j >> 1) * 8] = D;
                         } else {
                             __stcg(p.partials + ((size_t)split * p.B + b) * p.m_pad + row, D);
                         }
@@ -620,7 +639,24 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
         // release-acquire increment; the barrier after it hands the acquire to
         // the threads that read the other CTAs' partials.
         bool band_done = true;
-        if (p.splits > 1) {
+        if (p.splits > 1 && p.clu) {
+            // one task per CTA; the cluster's CTAs are the band's splits, rank = split
+            cg::cluster_group cluster = cg::this_cluster();
+            cluster.sync();  // every split's partials are in its CTA's shared memory
+            const int S = p.clu, rank = (int)cluster.block_rank();
+            const int r_base = band * BAND_ROWS;
+            const int rows = min(BAND_ROWS, p.m_pad - r_base);
+            const int total = rows * p.B, per = (total + S - 1) / S;
+            const int e1 = min(total, (rank + 1) * per);
+            for (int e = rank * per + tid; e < e1; e += THREADS) {
+                const int b = e / rows, row = e - b * rows;
+                double D = 0.0;
+                for (int sp = 0; sp < S; ++sp)  // fixed order, as the global reduction
+                    D += cluster.map_shared_rank(spart, sp)[(size_t)b * BAND_ROWS + row];
+                p.z[(size_t)b * p.m_pad + r_base + row] = FIN ? (float)(D * (double)p.ws) : finish_z(p, b, D);
+            }
+            cluster.sync();  // no CTA leaves while a peer still reads its partials
+        } else if (p.splits > 1) {
             __syncthreads();
             if (tid == 0) {
                 const unsigned prev = atom_add_acq_rel_gpu(&p.counters[band], 1u);
@@ -675,8 +711,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
 
 template <int BPW, int NT, bool FIN, int WARPS = gemv_warps(NT)>
 cudaError_t launch_t(const GemvParams &p, int grid, cudaStream_t s, bool pdl) {
-    const size_t smem = FIN ? gemv_fused_smem_bytes(p.table_words, BPW, p.B, min(p.cps, p.KC) * GLQ_CHUNK_K)
-                            : gemv_smem_bytes(p.table_words, BPW);
+    const size_t smem = gemv_launch_smem_bytes(p, BPW, FIN, WARPS);
     // raised once to the largest the library launches with (never lowered:
     // captured graphs replay against the attribute value at replay time)
     static bool configured = false;
@@ -693,8 +728,49 @@ cudaError_t launch_t(const GemvParams &p, int grid, cudaStream_t s, bool pdl) {
     }
     GemvParams q = p;
     void *args[] = {&q};
+    if (p.clu > 1) {
+        if (grid != p.bands * p.splits || p.clu != p.splits) return cudaErrorInvalidValue;
+        static bool nonportable = false;  // clusters above 8 CTAs
+        if (!nonportable) {
+            cudaError_t e = cudaFuncSetAttribute(gemv_kernel<BPW, NT, FIN, WARPS>,
+                                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            if (e != cudaSuccess) return e;
+            nonportable = true;
+        }
+        return launch_ex((const void *)gemv_kernel<BPW, NT, FIN, WARPS>, dim3(grid), dim3(WARPS * 32), smem, s,
+                         pdl, args, p.clu);
+    }
     return launch_ex((const void *)gemv_kernel<BPW, NT, FIN, WARPS>, dim3(grid), dim3(WARPS * 32), smem, s,
                      pdl, args);
+}
+
+// Largest number of clusters of `csize` CTAs of this kernel that can be
+// resident at once (0 if the cluster does not fit).
+template <int BPW, int NT, bool FIN, int WARPS = gemv_warps(NT)>
+int max_clusters_t(int csize, size_t smem) {
+    const void *fn = (const void *)gemv_kernel<BPW, NT, FIN, WARPS>;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GEMV_SMEM_LIMIT) != cudaSuccess ||
+        cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(csize);
+    cfg.blockDim = dim3(WARPS * 32);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
 }
 
 }  // namespace
@@ -736,6 +812,47 @@ GemvPlan plan_gemv(int RT, int KC, int num_sms, int warps, bool pow2, int max_cp
 
 size_t gemv_smem_bytes(int table_words, int bpw) {
     return (size_t)table_words * 4 + (bpw == 3 ? 256 * 16 : 0);
+}
+
+size_t gemv_launch_smem_bytes(const GemvParams &p, int bpw, bool fin, int warps) {
+    const size_t base = fin ? gemv_fused_smem_bytes(p.table_words, bpw, p.B, std::min(p.cps, p.KC) * GLQ_CHUNK_K)
+                            : gemv_smem_bytes(p.table_words, bpw);
+    return p.clu ? std::max(base, p.spart_off + gemv_cluster_partials_bytes(warps, p.B)) : base;
+}
+
+size_t gemv_cluster_partials_bytes(int warps, int B) {
+    return (size_t)warps * GLQ_ROW_TILE * B * sizeof(double);
+}
+
+int gemv_max_clusters(int bpw, int nt, bool fin, int warps, int csize, size_t smem) {
+    // memoised per kernel, cluster size and shared-memory size (host-side)
+    struct Key {
+        int bpw, nt, fin, warps, csize;
+        size_t smem;
+        int n;
+    };
+    static Key cache[64];
+    static int ncache = 0;
+    for (int i = 0; i < ncache; ++i) {
+        const Key &k = cache[i];
+        if (k.bpw == bpw && k.nt == nt && k.fin == (int)fin && k.warps == warps && k.csize == csize && k.smem == smem)
+            return k.n;
+    }
+    int n = 0;
+    if (fin) {
+        if (nt == 1) n = bpw == 2 ? max_clusters_t<2, 1, true>(csize, smem) : bpw == 3 ? max_clusters_t<3, 1, true>(csize, smem) : max_clusters_t<4, 1, true>(csize, smem);
+        else n = bpw == 2 ? max_clusters_t<2, 2, true>(csize, smem) : bpw == 3 ? max_clusters_t<3, 2, true>(csize, smem) : max_clusters_t<4, 2, true>(csize, smem);
+    } else if (nt == 1 && warps == GEMV_WIDE_WARPS) {
+        n = bpw == 2 ? max_clusters_t<2, 1, false, GEMV_WIDE_WARPS>(csize, smem)
+          : bpw == 3 ? max_clusters_t<3, 1, false, GEMV_WIDE_WARPS>(csize, smem)
+                     : max_clusters_t<4, 1, false, GEMV_WIDE_WARPS>(csize, smem);
+    } else if (nt == 1) {
+        n = bpw == 2 ? max_clusters_t<2, 1, false>(csize, smem) : bpw == 3 ? max_clusters_t<3, 1, false>(csize, smem) : max_clusters_t<4, 1, false>(csize, smem);
+    } else {
+        n = bpw == 2 ? max_clusters_t<2, 2, false>(csize, smem) : bpw == 3 ? max_clusters_t<3, 2, false>(csize, smem) : max_clusters_t<4, 2, false>(csize, smem);
+    }
+    if (ncache < 64) cache[ncache++] = Key{bpw, nt, (int)fin, warps, csize, smem, n};
+    return n;
 }
 
 size_t gemv_fused_smem_bytes(int table_words, int bpw, int B, int klen) {

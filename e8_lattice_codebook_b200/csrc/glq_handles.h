@@ -93,6 +93,8 @@ struct DecodeCfg {
     GemvPlan plan{};
     bool fin = false, fout = false;
     int warps = 0;  // warps per GEMV CTA
+    int clu = 0;    // split-K through a cluster of this many CTAs (0: global reduction)
+    size_t spart_off = 0;  // shared-memory offset of the cluster partial sums
 };
 
 // max_cps bounds the chunks per split (callers with a small partial-sum

@@ -118,6 +118,11 @@ struct GemvParams {
     int blk_off_m[GLQ_MAX_BLOCKS], blk_len_m[GLQ_MAX_BLOCKS];
     int blk_bands[GLQ_MAX_BLOCKS];  // bands whose rows meet block i
     unsigned *blk_cnt;     // [GLQ_MAX_BLOCKS], zero between launches
+    // split-K in a thread-block cluster (one task per CTA, the band's
+    // splits form one cluster): clu = cluster size (= splits) or 0, and the
+    // byte offset of the partial sums in dynamic shared memory
+    int clu;
+    size_t spart_off;
 };
 
 struct PrefillParams {
@@ -153,19 +158,31 @@ struct DequantParams {
     float *w;  // [m][n]
 };
 
-// cudaLaunchKernelExC with optional programmatic stream serialisation.
+// cudaLaunchKernelExC with optional programmatic stream serialisation and
+// an optional 1-D thread-block cluster of `cluster` CTAs.
 inline cudaError_t launch_ex(const void *fn, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                             bool pdl, void **args) {
+                             bool pdl, void **args, int cluster = 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    if (cluster > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = cluster;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
+    cfg.numAttrs = na;
     return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
@@ -180,6 +197,12 @@ cudaError_t launch_gemv(const GemvParams &p, int bpw, int grid, cudaStream_t s, 
 // dynamic shared memory of a launch with the input transform fused
 // (the table, the residual table, the task's activations and scratch)
 size_t gemv_fused_smem_bytes(int table_words, int bpw, int B, int klen);
+// dynamic shared memory of a launch with these parameters
+size_t gemv_launch_smem_bytes(const GemvParams &p, int bpw, bool fin, int warps);
+// partial sums of one CTA in the cluster reduction
+size_t gemv_cluster_partials_bytes(int warps, int B);
+// clusters of csize CTAs of the selected GEMV kernel that fit at once
+int gemv_max_clusters(int bpw, int nt, bool fin, int warps, int csize, size_t smem);
 // (227 KB per block, less room for the kernels' static shared memory)
 constexpr size_t GEMV_SMEM_LIMIT = 222 * 1024;
 

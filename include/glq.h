@@ -181,12 +181,18 @@ GLQ_API glq_status glq_linear(glq_layer layer, const void *x_dev, glq_dtype x_dt
  * default is the library's fastest setting (GLQ_FUSE_DEFAULT).  With both bits
  * cleared, every token's output is bitwise independent of the batch size for
  * B <= 16; otherwise that holds among batch sizes that take the same path.
+ * GLQ_SPLITK_CLUSTER lets the split-K partial sums of a band of rows be
+ * added through the distributed shared memory of a thread-block cluster (the
+ * band's splits) instead of a global workspace and a last-arriving CTA,
+ * whenever every CTA has one task and the splits fit a cluster; the
+ * summation order is the same, so the results are bitwise identical.
  * All settings are bitwise reproducible run to run ("Bit-exact
  * determinism", glq 0.5.1 PyPI page, "Inference kernels") and agree within
  * the parity bound.  Errors: GLQ_ERR_INVALID_ARG (unknown bits).
  */
 #define GLQ_FUSE_INPUT 1
 #define GLQ_FUSE_OUTPUT 2
+#define GLQ_SPLITK_CLUSTER 4
 #define GLQ_FUSE_DEFAULT (-1)
 GLQ_API glq_status glq_layer_set_fusion(glq_layer layer, int32_t flags);
 
@@ -280,6 +286,19 @@ GLQ_API glq_status glq_linear_noalloc(glq_layer layer, const void *x_dev, glq_dt
  * Returns GLQ_OK, GLQ_ERR_TIMEOUT, GLQ_ERR_DEVICE_CHECK or GLQ_ERR_CUDA.
  */
 GLQ_API glq_status glq_layer_check(glq_layer layer, void *stream);
+
+/*
+ * glq_decode_plan -- measurement / test entry point: the launch plan a
+ * decode call of B tokens (1 <= B <= 16) with 16-byte aligned x and y takes
+ * under the layer's current settings: warps per GEMV CTA, row bands, K
+ * splits per band, the thread-block cluster size of the split-K reduction
+ * (0: global workspace and last-arriving CTA) and whether the input RHT is
+ * fused into the GEMV launch (1) or runs as its own kernel (0).  Any output
+ * may be NULL.  Errors: GLQ_ERR_INVALID_ARG, GLQ_ERR_SHAPE (B out of range).
+ * No counterpart in the pages (a view of this library's scheduling).
+ */
+GLQ_API glq_status glq_decode_plan(glq_layer layer, int64_t B, int32_t *warps, int32_t *bands,
+                                   int32_t *splits, int32_t *cluster, int32_t *fused_input);
 
 /* Layer geometry, for callers sizing buffers.  Any output may be NULL. */
 GLQ_API glq_status glq_layer_info(glq_layer layer, int64_t *m, int64_t *n, int32_t *bpw,

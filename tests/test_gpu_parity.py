@@ -189,6 +189,58 @@ def test_fused_and_separate_transforms(dev, m, n, bpw, B, xdt):
           + " ".join(f"{e / tolerance(ref):.3f}" for e in errs))
 
 
+CLUSTER_CASES = [  # m, n, bpw, B, x dtype
+    (2048, 2048, 4, 1, "bf16"), (11008, 2048, 4, 1, "bf16"), (2048, 11008, 4, 1, "bf16"),
+    (4096, 5120, 4, 1, "bf16"), (32768, 5120, 4, 1, "bf16"), (960, 2560, 3, 2, "f16"),
+    (2560, 960, 3, 8, "f16"), (1024, 1024, 2, 16, "f16"), (1000, 968, 4, 9, "bf16"),
+    (5120, 4096, 4, 16, "bf16"),
+]
+
+
+@pytest.mark.parametrize("m,n,bpw,B,xdt", CLUSTER_CASES)
+def test_cluster_splitk_matches_global_reduction(dev, m, n, bpw, B, xdt):
+    """Split-K partial sums added through a thread-block cluster's distributed
+    shared memory (GLQ_SPLITK_CLUSTER) give the same bits as the global
+    workspace and last-arriving CTA (the summation order is the same), with
+    the input transform fused and as its own kernel; the result is within the
+    oracle bound."""
+    L = gi.make_layer(7 * m + n, 3, m, n, bpw)
+    xb = gi.make_x(7 * m + n, 3, B, n, xdt)
+    lay = dev.layer(L)
+    x = to_torch_x(xb, xdt)
+    plans = []
+    for fin in (1, 0):
+        lay.set_fusion(fin | 4)
+        plans.append(lay.decode_plan(B))
+        yc = lay(x, out_dtype=torch.float32)
+        lay.set_fusion(fin)
+        assert lay.decode_plan(B)["cluster"] == 0
+        yg = lay(x, out_dtype=torch.float32)
+        assert torch.equal(yc, yg), (fin, plans[-1])
+    lay.set_fusion(-1)
+    y = lay(x, out_dtype=torch.float32).cpu().numpy().astype(np.float64)
+    ref = oracle_y(L, xb, xdt)
+    assert np.max(np.abs(y - ref)) <= tolerance(ref)
+    print(f"\nCLUSTER {m}x{n} bpw {bpw} B={B}: plans (fused, separate) {plans}, default {lay.decode_plan(B)}")
+
+
+def test_decode_plans_of_the_workloads(dev):
+    """The decode plans of the SmolLM3-3B-shaped and 24B-class layers at 1 and
+    16 tokens are consistent (a cluster, when used, holds a band's splits)
+    and the cluster reduction is in use on some of them."""
+    clustered = 0
+    for key in ("smollm3-3b-4bpw", "24b-decode-4bpw"):
+        wl = gi.WORKLOADS[key]
+        for li in range(len(wl.layers)):
+            lay = dev.layer(gi.workload_layer(wl, li))
+            for B in (1, 16):
+                plan = lay.decode_plan(B)
+                assert plan["cluster"] in (0, plan["splits"]) and plan["cluster"] != 1, (key, li, B, plan)
+                clustered += plan["cluster"] > 0
+                print(f"\nPLAN {key} layer {li} B={B}: {plan}")
+    assert clustered > 0
+
+
 def test_empty_batch_and_errors(dev):
     import e8_lattice_codebook_b200 as glq
     L = gi.make_layer(0, 0, 64, 64, 2)
