@@ -368,6 +368,7 @@ DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y
     const int flags = L->fusion < 0 ? FUSE_DEFAULT_FLAGS : L->fusion;
     c.fout = (flags & GLQ_FUSE_OUTPUT) && y_al && (long long)nb * L->hb_m.len[0] <= FUSED_OUT_MAX_VALUES &&
              (size_t)nb * L->hb_m.len[0] * sizeof(float) <= base;
+    c.warps = warps;
     if ((flags & GLQ_FUSE_INPUT) && x_al && (long long)nb * L->hb_n.len[0] <= FUSED_IN_MAX_VALUES) {
         int cap = 1;  // largest power-of-two chunk count whose activations fit shared memory
         while (cap < L->KC &&
@@ -380,7 +381,10 @@ DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y
         // Measured: the fold pays for the launch it saves when every CTA has
         // one task and a short range (<= 1024 columns, <= 4096 values in
         // all); a 4096-column range per CTA is slower than the separate
-        // transform kernel.  An explicit setting always fuses.
+        // transform kernel.  An explicit setting always fuses.  (Narrower
+        // CTAs of 16 or 20 warps that fill more SMs made the 3B-shaped step
+        // slower, 74 -> 82 us: no SM was left for the next kernel's early
+        // launch.)
         const int klen = std::min(fp.cps, L->KC) * GLQ_CHUNK_K;
         const bool cheap = (long long)fp.bands * fp.splits <= L->num_sms && klen <= 1024 && nb * klen <= 4096;
         if (need <= GEMV_SMEM_LIMIT && (cheap || L->fusion >= 0)) {
@@ -388,7 +392,6 @@ DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y
             c.plan = fp;
         }
     }
-    c.warps = warps;
     if (!c.fin) {
         c.plan = plan_for(L, nb);
         if (nt == 1 && (long long)L->RT * L->KC >= 200LL * L->num_sms) {  // large layer: wide CTAs
@@ -423,9 +426,9 @@ int max_decode_splits(glq_layer L, int nb) {
            gemv_fused_smem_bytes(L->primary->table_words, L->bpw, nb, std::min(cap * 2, L->KC) * GLQ_CHUNK_K) <=
                GEMV_SMEM_LIMIT)
         cap *= 2;
-    const GemvPlan f = plan_gemv(L->RT, L->KC, L->num_sms, warps, true, cap);
+    const int fs = plan_gemv(L->RT, L->KC, L->num_sms, warps, true, cap).splits;
     const GemvPlan wide = plan_gemv(L->RT, L->KC, L->num_sms, GEMV_WIDE_WARPS);
-    return std::max(std::max(plan_for(L, nb).splits, f.splits), wide.splits);
+    return std::max(std::max(plan_for(L, nb).splits, fs), wide.splits);
 }
 
 GemvParams gemv_params(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg, int nb, const void *x,

@@ -24,10 +24,11 @@
 //   * per task, partial sums go to a workspace in fp64; the last CTA to
 //     finish a band (atomic counter, no waiting) adds the splits in fixed
 //     order and writes the band's final z.  When every CTA has one task and
-//     a band's splits fit one thread-block cluster, the partials stay in
-//     shared memory instead and the cluster's CTAs add them through
-//     distributed shared memory, each for its share of the band's rows, in
-//     the same fixed order (no global round trip, no last arriver);
+//     a band's splits fit one thread-block cluster, each split stores its
+//     partials into the shared memory of the CTA that owns that share of the
+//     band (distributed shared memory), and after one cluster barrier every
+//     CTA adds its share in the same fixed order (no global round trip, no
+//     last arriver);
 //   * small batches fuse both transforms (one launch per layer): each task
 //     rotates, scales and quantises its own aligned column range of x in
 //     shared memory (a Hadamard block of size N = 2^a S restricted to an
@@ -162,9 +163,8 @@ struct TaskRow {  // per token, over the task's column range
     float inv_scale;  // 2^-e
 };
 
-// 8 consecutive activations (16-byte aligned) as float
-__device__ __forceinline__ void load8_act(const void *x, size_t i, int bf16, float v[8]) {
-    const uint4 r = ldg_v4(static_cast<const uint16_t *>(x) + i);
+// 8 activations (fp16 or bf16 bits) as float
+__device__ __forceinline__ void unpack8_act(const uint4 &r, int bf16, float v[8]) {
     const uint32_t w[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -282,6 +282,92 @@ __device__ void fused_input_signs(const GemvParams &p, int k0, int klen, uint32_
     __syncthreads();
 }
 
+// Warp-per-token tail of the input transform for the common task shape:
+// the range [k0, k0 + 32V) (V = 4, 8 or 16) meets one Hadamard block of n,
+// as an aligned part of it or as the whole block followed by padding past n.
+// u holds the token's folded values f (positions past S, the range's
+// columns inside the block, are not read: zeros).  Lane l holds positions
+// l V .. l V + V - 1: spans below V in registers, V .. 16 V as shuffles, then
+// the row max, the scale and X, with no CTA barrier.
+template <int BPW, int V>
+__device__ __forceinline__ void warp_transform(const GemvParams &p, int b, int N, int S, const float *u,
+                                               uint4 *xs, __half *xhs, TaskRow *rows) {
+    const int lane = threadIdx.x & 31;
+    const int klen = 32 * V, p0 = lane * V;
+    float v[V];
+#pragma unroll
+    for (int q = 0; q < V / 4; ++q) {
+        float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (p0 + 4 * q < S) r = *reinterpret_cast<const float4 *>(u + (size_t)b * klen + p0 + 4 * q);
+        v[4 * q] = r.x;
+        v[4 * q + 1] = r.y;
+        v[4 * q + 2] = r.z;
+        v[4 * q + 3] = r.w;
+    }
+    // a span applies iff it is below S (positions past S hold zeros)
+#pragma unroll
+    for (int h = 1; h < V; h <<= 1)
+        if (h < S)
+#pragma unroll
+            for (int j = 0; j < V; ++j)
+                if ((j & h) == 0) {
+                    const float a = v[j], c = v[j + h];
+                    v[j] = a + c;
+                    v[j + h] = a - c;
+                }
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+        if ((V << k) >= S) break;
+        const bool upper = (lane >> k) & 1;
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+            const float o = __shfl_xor_sync(0xffffffffu, v[j], 1 << k);
+            v[j] = upper ? o - v[j] : v[j] + o;
+        }
+    }
+    const float nrm = __frsqrt_rn((float)N);
+    float mx = 0.f;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+        v[j] *= nrm;
+        mx = fmaxf(mx, fabsf(v[j]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float scale = 1.f;
+    if (mx > 0.f && isfinite(mx)) {
+        int ex;
+        frexpf(mx, &ex);
+        scale = ldexpf(1.f, 14 - ex);
+    }
+    int sum = 0;
+    uint32_t hb[V / 4], lb[V / 4];
+#pragma unroll
+    for (int q = 0; q < V / 4; ++q) hb[q] = lb[q] = 0u;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+        const int X = __float2int_rn(v[j] * scale);
+        sum += X;
+        hb[j >> 2] |= (uint32_t)((X >> 8) & 0xFF) << (8 * (j & 3));
+        lb[j >> 2] |= (uint32_t)(X & 0xFF) << (8 * (j & 3));
+        if (BPW == 3) xhs[(size_t)b * klen + p0 + j] = __int2half_rn(X);
+    }
+    // per 8-column group: 8 high bytes, then 8 low bytes
+    uint32_t *xw = reinterpret_cast<uint32_t *>(xs + (size_t)b * (klen / 8));
+#pragma unroll
+    for (int q = 0; q < V / 4; ++q) {
+        const int c4 = p0 / 4 + q;  // 4-column quarter of the range
+        xw[(c4 >> 1) * 4 + (c4 & 1)] = hb[q];
+        xw[(c4 >> 1) * 4 + 2 + (c4 & 1)] = lb[q];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) {
+        rows[b].sum_x = sum;
+        rows[b].inv_scale = 1.f / scale;
+    }
+}
+
 // The task's activations for columns [k0, k0 + klen): xr = H_n (S_in x)
 // restricted to the range, scaled per token by 2^e (max |xr| 2^e < 2^14 over
 // the range), rounded to X and stored as the GEMV consumes it: xs[b][group]
@@ -295,12 +381,28 @@ __device__ void fused_input(const GemvParams &p, int k0, int klen, uint4 *xs, __
                             TaskRow *rows, unsigned *s_max, Seg *segs, const uint32_t *sw, int w0) {
     const int tid = threadIdx.x, lane = tid & 31;
     const int B = p.B, k1 = k0 + klen;
-    for (int e = tid; e < B * klen; e += THREADS) u[e] = 0.f;  // columns >= n stay zero
-    if (tid < GLQ_DECODE_MAX_B) {
-        s_max[tid] = 0u;
-        rows[tid].sum_x = 0;
+    // The warp-per-token tail (warp_transform) applies when the range meets
+    // one Hadamard block, from the range's first column, and spans 128, 256
+    // or 512 columns; the condition is the same in every thread.
+    int wo = 0, wN = 0, wseg = 0;
+    for (int bi = 0; bi < p.nblk_n; ++bi) {
+        const int o = p.blk_off_n[bi], N = p.blk_len_n[bi];
+        if (max(k0, o) < min(k1, o + N)) {
+            wo = o;
+            wN = N;
+            ++wseg;
+        }
     }
-    __syncthreads();
+    const bool warp_tail = B <= THREADS / 32 && (klen == 128 || klen == 256 || klen == 512) && wseg == 1 &&
+                           max(k0, wo) == k0;
+    if (!warp_tail) {
+        for (int e = tid; e < B * klen; e += THREADS) u[e] = 0.f;  // columns >= n stay zero
+        if (tid < GLQ_DECODE_MAX_B) {
+            s_max[tid] = 0u;
+            rows[tid].sum_x = 0;
+        }
+        __syncthreads();
+    }
     int nseg = 0;  // the task's segments (identical in every thread)
     for (int bi = 0; bi < p.nblk_n; ++bi) {
         const int o = p.blk_off_n[bi], N = p.blk_len_n[bi];
@@ -320,15 +422,29 @@ __device__ void fused_input(const GemvParams &p, int k0, int klen, uint4 *xs, __
             const int b = valid ? item / nv : 0, v = valid ? item - b * nv : 0;
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             if (valid) {
-                for (int jh = grp; jh < A; jh += G) {
-                    const int col = o + jh * S + 8 * v;
-                    float xv[8];
-                    load8_act(p.x, (size_t)b * p.n + col, p.x_bf16, xv);
-                    const uint32_t sb = (sw[(col >> 5) - w0] >> (col & 31)) & 0xFFu;
-                    const uint32_t neg = (__popc(ihi & jh) & 1) ? 0xFFu : 0u;
-                    const uint32_t flip = sb ^ neg;
+                // four terms per round: their loads are all in flight before any is used
+                for (int jh0 = grp; jh0 < A; jh0 += 4 * G) {
+                    uint4 r[4];
+                    uint32_t flip[4];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) acc[j] += ((flip >> j) & 1u) ? -xv[j] : xv[j];
+                    for (int q = 0; q < 4; ++q) {
+                        const int jh = jh0 + q * G;
+                        const int col = o + jh * S + 8 * v;
+                        r[q] = make_uint4(0, 0, 0, 0);
+                        flip[q] = 0u;
+                        if (jh < A) {
+                            r[q] = ldg_v4(static_cast<const uint16_t *>(p.x) + (size_t)b * p.n + col);
+                            const uint32_t sb = (sw[(col >> 5) - w0] >> (col & 31)) & 0xFFu;
+                            flip[q] = sb ^ ((__popc(ihi & jh) & 1) ? 0xFFu : 0u);
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float xv[8];
+                        unpack8_act(r[q], p.x_bf16, xv);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) acc[j] += ((flip[q] >> j) & 1u) ? -xv[j] : xv[j];
+                    }
                 }
             }
             // fixed-order reduction over the G lanes of a vector
@@ -336,7 +452,7 @@ __device__ void fused_input(const GemvParams &p, int k0, int klen, uint4 *xs, __
 #pragma unroll
                 for (int j = 0; j < 8; ++j) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
             if (valid && grp == 0) {
-                fwht8(acc);
+                if (!warp_tail) fwht8(acc);
                 float *dst = u + (size_t)b * klen + (lo - k0) + 8 * v;
                 *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
                 *reinterpret_cast<float4 *>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
@@ -344,6 +460,17 @@ __device__ void fused_input(const GemvParams &p, int k0, int klen, uint4 *xs, __
         }
     }
     __syncthreads();
+    if (warp_tail) {
+        const int S = min(k1, wo + wN) - k0;  // klen, or the whole block followed by padding
+        const int warp = tid >> 5;
+        if (warp < B) {
+            if (klen == 128) warp_transform<BPW, 4>(p, warp, wN, S, u, xs, xhs, rows);
+            else if (klen == 256) warp_transform<BPW, 8>(p, warp, wN, S, u, xs, xhs, rows);
+            else warp_transform<BPW, 16>(p, warp, wN, S, u, xs, xhs, rows);
+        }
+        __syncthreads();
+        return;
+    }
     fwht_segments<THREADS>(u, B, klen, segs, nseg);
     // normalise per block, row max per token
     const int nvec = klen / 8;
@@ -463,7 +590,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
     uint4 *xs = R8 + (BPW == 3 ? 256 : 0);
     __half *xhs = reinterpret_cast<__half *>(xs + (size_t)p.B * klen_max / 8);
     float *ubuf = reinterpret_cast<float *>(xhs + (BPW == 3 ? (size_t)p.B * klen_max : 0));
-    // cluster reduction: this CTA's partial sums [B][BAND_ROWS] (fp64)
+    // cluster reduction: the partial sums of this CTA's share of the band,
+    // [split][share] (fp64), stored by every split of the cluster
     double *spart = reinterpret_cast<double *>(reinterpret_cast<char *>(smem_u4) + p.spart_off);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
@@ -512,6 +640,21 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
     if (task < ntasks) {
         task_geom(task);
         prefetch();
+        // The rest of the first task's index range (constant data) into L2
+        // now, so that the chunks the loop reads after the wait hit L2
+        // instead of paying a DRAM round trip each (short tasks, where the
+        // one-chunk register prefetch cannot cover the latency).
+        if (rt < p.RT && c1 - c0 <= 8) {
+            const size_t base = ((size_t)rt * p.KC) * 32 + lane;
+            for (int c = c0 + GEMV_PREFETCH; c < c1; ++c) {
+                if ((lane & 7) == 0) {  // one request per 128-byte line
+                    prefetch_l2(p.idx1 + base + (size_t)c * 32);
+                    if (BPW == 4) prefetch_l2(static_cast<const uint4 *>(p.idx2) + base + (size_t)c * 32);
+                    if (BPW == 3 && (lane & 15) == 0)
+                        prefetch_l2(static_cast<const uint2 *>(p.idx2) + base + (size_t)c * 32);
+                }
+            }
+        }
         if (FIN) {
             fused_input_signs<THREADS>(p, c0 * GLQ_CHUNK_K, (c1 - c0) * GLQ_CHUNK_K, s_sign, &s_sign_w0);
             // the columns of x the first task folds: Hadamard blocks met by its range
@@ -531,11 +674,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
         if (ok) return true;
         if (tid == 0) atomicOr(p.err, GLQ_DEVERR_TIMEOUT);
         mbar_wait_bounded(&bar, 0, TABLE_WAIT_POLLS);  // let the copy land before exiting
-        if (p.clu) {  // leaving early: still take the cluster's two barriers of the reduction
-            cg::cluster_group cluster = cg::this_cluster();
-            cluster.sync();
-            cluster.sync();
-        }
+        if (p.clu) cg::this_cluster().sync();  // leaving early: still take the reduction's cluster barrier
         return false;
     };
     if (!FIN && !wait_table()) return;
@@ -625,7 +764,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
                         if (p.splits == 1) {
                             p.z[(size_t)b * p.m_pad + row] = FIN ? (float)(D * (double)p.ws) : finish_z(p, b, D);
                         } else if (p.clu) {
-                            spart[(size_t)b * BAND_ROWS + warp * GLQ_ROW_TILE + g + (j >> 1) * 8] = D;
+                            // to the cluster CTA that owns element (b, row) of the band, slot `split`
+                            const int rows_b = min(BAND_ROWS, p.m_pad - band * BAND_ROWS);
+                            const int per = (rows_b * p.B + p.clu - 1) / p.clu;
+                            const int e = b * rows_b + (row - band * BAND_ROWS), owner = e / per;
+                            cg::this_cluster().map_shared_rank(spart, owner)[split * per + (e - owner * per)] = D;
                         } else {
                             __stcg(p.partials + ((size_t)split * p.B + b) * p.m_pad + row, D);
                         }
@@ -640,22 +783,23 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
         // the threads that read the other CTAs' partials.
         bool band_done = true;
         if (p.splits > 1 && p.clu) {
-            // one task per CTA; the cluster's CTAs are the band's splits, rank = split
+            // one task per CTA; the cluster's CTAs are the band's splits, rank =
+            // split.  The band's (token, row) elements are dealt out in
+            // contiguous shares; every split has stored its partial of each
+            // element into the owner's shared memory, slot `split`.
             cg::cluster_group cluster = cg::this_cluster();
-            cluster.sync();  // every split's partials are in its CTA's shared memory
+            cluster.sync();  // all partials are in their owners' shared memory
             const int S = p.clu, rank = (int)cluster.block_rank();
             const int r_base = band * BAND_ROWS;
             const int rows = min(BAND_ROWS, p.m_pad - r_base);
             const int total = rows * p.B, per = (total + S - 1) / S;
-            const int e1 = min(total, (rank + 1) * per);
-            for (int e = rank * per + tid; e < e1; e += THREADS) {
+            const int e0 = rank * per, e1 = min(total, e0 + per);
+            for (int e = e0 + tid; e < e1; e += THREADS) {
                 const int b = e / rows, row = e - b * rows;
                 double D = 0.0;
-                for (int sp = 0; sp < S; ++sp)  // fixed order, as the global reduction
-                    D += cluster.map_shared_rank(spart, sp)[(size_t)b * BAND_ROWS + row];
+                for (int sp = 0; sp < S; ++sp) D += spart[sp * per + (e - e0)];  // fixed order
                 p.z[(size_t)b * p.m_pad + r_base + row] = FIN ? (float)(D * (double)p.ws) : finish_z(p, b, D);
             }
-            cluster.sync();  // no CTA leaves while a peer still reads its partials
         } else if (p.splits > 1) {
             __syncthreads();
             if (tid == 0) {
@@ -821,7 +965,8 @@ size_t gemv_launch_smem_bytes(const GemvParams &p, int bpw, bool fin, int warps)
 }
 
 size_t gemv_cluster_partials_bytes(int warps, int B) {
-    return (size_t)warps * GLQ_ROW_TILE * B * sizeof(double);
+    // splits x ceil(rows x B / splits) slots, splits <= 16
+    return ((size_t)warps * GLQ_ROW_TILE * B + 16) * sizeof(double);
 }
 
 int gemv_max_clusters(int bpw, int nt, bool fin, int warps, int csize, size_t smem) {
