@@ -925,7 +925,7 @@ glq_status glq_gemv_replay(glq_layer L, int64_t B, void *stream) {
     const glq::DecodeCfg cfg = glq::decode_config(L, (int)B, L->last_x, L->last_y, L->last_y_dtype);
     glq::GemvParams pg = glq::gemv_params(L, L->wsp, cfg, (int)B, L->last_x, L->last_x_bf16 != 0, L->last_y,
                                           L->last_y_dtype);
-    return glq::launch_gemv(pg, L->bpw, cfg.plan.grid, static_cast<cudaStream_t>(stream), false, cfg.fin) ==
+    return glq::launch_gemv(pg, L->bpw, cfg.plan.grid, static_cast<cudaStream_t>(stream), true, cfg.fin) ==
                    cudaSuccess
                ? GLQ_OK
                : GLQ_ERR_CUDA;

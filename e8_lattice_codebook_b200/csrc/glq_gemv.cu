@@ -644,17 +644,6 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
         // now, so that the chunks the loop reads after the wait hit L2
         // instead of paying a DRAM round trip each (short tasks, where the
         // one-chunk register prefetch cannot cover the latency).
-        if (rt < p.RT && c1 - c0 <= 8) {
-            const size_t base = ((size_t)rt * p.KC) * 32 + lane;
-            for (int c = c0 + GEMV_PREFETCH; c < c1; ++c) {
-                if ((lane & 7) == 0) {  // one request per 128-byte line
-                    prefetch_l2(p.idx1 + base + (size_t)c * 32);
-                    if (BPW == 4) prefetch_l2(static_cast<const uint4 *>(p.idx2) + base + (size_t)c * 32);
-                    if (BPW == 3 && (lane & 15) == 0)
-                        prefetch_l2(static_cast<const uint2 *>(p.idx2) + base + (size_t)c * 32);
-                }
-            }
-        }
         if (FIN) {
             fused_input_signs<THREADS>(p, c0 * GLQ_CHUNK_K, (c1 - c0) * GLQ_CHUNK_K, s_sign, &s_sign_w0);
             // the columns of x the first task folds: Hadamard blocks met by its range

@@ -235,7 +235,10 @@ GLQ_API glq_status glq_rht_output(glq_layer layer, const float *z_dev, void *y_d
  * GEMV of the most recent glq_linear call on this layer (same activations
  * already in the layer's workspace, batch B <= min(16, that call's B)),
  * writing the same split-K partial sums.  Lets a caller time the GEMV kernel
- * alone with events on `stream`.  The decode path's GEMV is the one of
+ * alone with events on `stream`.  Like glq_linear, it launches the GEMV with
+ * programmatic dependent launch, so back-to-back replays overlap one launch's
+ * prologue (codebook copy, first index loads) with the previous one's tail,
+ * as the product path does.  The decode path's GEMV is the one of
  * "Inference kernels" on the glq 0.5.1 PyPI page (matmul against indices).
  * Errors: GLQ_ERR_INVALID_ARG, GLQ_ERR_SHAPE (B out of range or no previous
  * call), GLQ_ERR_CUDA.  Asynchronous.
