@@ -439,12 +439,23 @@ cudaError_t launch_rows_t(const RowsParams &p, int B, cudaStream_t s, bool pdl) 
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    // persistent grid: every CTA that fits on the device at once, at most one per row
-    int dev = 0, sms = 0, per_sm = 0;
+    // persistent grid: every CTA that fits on the device at once, at most one
+    // per row (SM count and occupancy queried once per device, not per call)
+    constexpr int MAX_DEV = 64;
+    static int sms_of[MAX_DEV] = {}, per_sm_of[MAX_DEV] = {};
+    int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem);
     if (e != cudaSuccess) return e;
+    int sms = dev < MAX_DEV ? sms_of[dev] : 0, per_sm = dev < MAX_DEV ? per_sm_of[dev] : 0;
+    if (sms <= 0 || per_sm <= 0) {
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem);
+        if (e != cudaSuccess) return e;
+        if (dev < MAX_DEV) {
+            sms_of[dev] = sms;
+            per_sm_of[dev] = per_sm;
+        }
+    }
     const int grid = (int)std::min<long long>((long long)B, (long long)std::max(1, sms) * std::max(1, per_sm));
     RowsParams q = p;
     int nrows = B;
