@@ -214,6 +214,17 @@ class WorkloadSet:
         return sum(2 * B * L.m * L.n for L in self.host)
 
 
+def launches_per_step(ws: "WorkloadSet", B: int) -> int:
+    """Kernels one decode step launches: per layer the GEMV, plus the input
+    transform unless it is fused into the GEMV, plus the output transform
+    (glq_decode_plan reports the plan the library takes)."""
+    n = 0
+    for lay, _, _ in ws.copies[0]:
+        plan = lay.decode_plan(B)
+        n += 2 + (0 if plan["fused_input"] else 1)
+    return n
+
+
 def capture_graphs(torch, fn_per_copy, ncopy):
     graphs = []
     s = torch.cuda.Stream()
@@ -522,7 +533,7 @@ def run_glq(args):
                   f"({NCOPY * sum(L.m * L.n // 2 for L in ws.host) / 1e6:.0f} MB > 126 MB L2)",
             "timing": "CUDA-graph replay, CUDA events, max over ranks",
         },
-        "gpu_launches": 3 * len(ws.host) * args.steps,
+        "gpu_launches": launches_per_step(ws, B) * args.steps,
         "clocks": clocks,
     }
     if rank != 0:
