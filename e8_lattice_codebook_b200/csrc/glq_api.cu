@@ -702,7 +702,11 @@ glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *i
     cudaDeviceGetAttribute(&L->num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (L->num_sms <= 0) L->num_sms = 1;
     L->plan[0] = glq::plan_gemv(L->RT, L->KC, L->num_sms, glq::gemv_warps(1));
-    L->plan[1] = glq::plan_gemv(L->RT, L->KC, L->num_sms, glq::gemv_warps(2));
+    // two token tiles: a band's split-K partials are twice as many, and
+    // with several tasks per CTA they go through the global workspace;
+    // charging 2 chunks per split (measured: 24B-class step at 16 tokens
+    // 424 -> 266 us, the 32768-row layers then take one split)
+    L->plan[1] = glq::plan_gemv(L->RT, L->KC, L->num_sms, glq::gemv_warps(2), false, 1 << 30, 1 << 30, 2.0);
     const int max_bands = std::max(L->plan[0].bands, L->plan[1].bands);
     L->hb_n = hadamard_blocks_of(n);
     L->hb_m = hadamard_blocks_of(m);

@@ -909,9 +909,9 @@ int max_clusters_t(int csize, size_t smem) {
 }  // namespace
 
 // Split of the chunk range so that (bands x splits) tasks spread over the
-// persistent grid with the least makespan (in chunks per CTA), with a small
-// charge per task for the band reduction.
-GemvPlan plan_gemv(int RT, int KC, int num_sms, int warps, bool pow2, int max_cps, int max_splits) {
+// persistent grid with the least makespan (in chunks per CTA), with a
+// charge per task for the band reduction (`charge` chunks when split).
+GemvPlan plan_gemv(int RT, int KC, int num_sms, int warps, bool pow2, int max_cps, int max_splits, double charge) {
     GemvPlan pl{};
     pl.bands = (RT + warps - 1) / warps;
     int best_cps = 0;
@@ -925,7 +925,7 @@ GemvPlan plan_gemv(int RT, int KC, int num_sms, int warps, bool pow2, int max_cp
         const long long tasks = (long long)pl.bands * s;
         const long long waves = (tasks + num_sms - 1) / num_sms;
         const int work = cps < KC ? cps : KC;
-        const double cost = (double)waves * (work + (s > 1 ? 0.5 : 0.0)) + 0.02 * s;
+        const double cost = (double)waves * (work + (s > 1 ? charge : 0.0)) + 0.02 * s;
         if (cost < best) {
             best = cost;
             best_cps = cps;

@@ -212,9 +212,10 @@ struct GemvPlan {
 };
 // Work split of the GEMV over a persistent grid.  pow2: chunks per split a
 // power of two (aligned column ranges, required by the fused input
-// transform), at most max_cps chunks per split and max_splits splits.
+// transform), at most max_cps chunks per split and max_splits splits;
+// charge: the cost of a split task's band reduction, in chunks.
 GemvPlan plan_gemv(int RT, int KC, int num_sms, int warps, bool pow2 = false, int max_cps = 1 << 30,
-                   int max_splits = 1 << 30);
+                   int max_splits = 1 << 30, double charge = 0.5);
 cudaError_t launch_dequant(const DequantParams &p, cudaStream_t s);
 // wmap: TMA map of the dequantised fp16 W [m_pad][n_pad] (boxes 64 x 128,
 // 128-byte swizzle), or null for the fused variant whose producer warps
