@@ -12,16 +12,29 @@
 //   * a row of up to 2^L values (9 <= L <= 14) is held 16 values per thread;
 //     the butterflies run in registers, four position bits per phase, and the
 //     row changes layout between phases through shared memory (one store,
-//     one barrier, one load per value and phase) under an XOR swizzle that
-//     keeps every access free of bank conflicts; no warp shuffles;
+//     one barrier, one load per value and phase); no warp shuffles;
+//   * the row sits in shared memory under the padded layout word(p) = p +
+//     (p >> 5), which is additive over disjoint position bits, so every
+//     access is a per-thread base plus an immediate offset; which position
+//     bits the lanes of a warp own in each phase is chosen so that their
+//     words fall in 32 distinct banks;
+//   * the stages of a Hadamard transform commute, so the last phase carries
+//     the lowest position bits along as "fill" and writes its values straight
+//     to global memory in runs of consecutive columns; rows alternate between
+//     two buffers, so no barrier protects a buffer from the next row;
 //   * butterflies on register pairs use the packed f32x2 add / subtract of
 //     sm_100a (same IEEE rounding as scalar adds);
 //   * Hadamard blocks of a size that is not a power of two are handled by
-//     testing, per butterfly, whether both ends lie in one block;
+//     testing, per butterfly, whether both ends lie in one block; the block
+//     norm 1/sqrt(block) is applied on load, where a thread's 16 values share
+//     one block;
 //   * the input direction also finds the row's max |xr| (one reduction) and
 //     writes either the fp16 operand of the tensor-core GEMM, xr 2^e with
 //     max |xr| 2^e < 2^14, or the decode GEMV's operand X = round(xr 2^e) as
-//     high / low bytes with its exact row sum (a second reduction), plus 2^-e.
+//     high / low bytes with its exact row sum (a second reduction), plus 2^-e;
+//     the decode operand needs 8 consecutive columns per thread, so that
+//     variant returns the row to the load layout first and applies the norm
+//     there, as one product with the power-of-two scale.
 #include <algorithm>
 
 #include "glq_kernels.cuh"
@@ -48,36 +61,31 @@ __device__ __forceinline__ int block_size_at(const RowsParams &p, int c, float *
 //
 // Phase q owns the position bits 4q .. 4q+3 (those below L).  In it a thread
 // holds 16 values whose positions differ exactly in four "register" bits:
-// the phase's own bits, filled up with the lowest other bits when fewer than
-// four remain; the bits of the thread index give the other position bits in
-// increasing order.  Phase 0 is the layout of the global loads and stores
-// (16 consecutive values per thread); the later phases read and write the
-// row through shared memory.
+// the phase's own bits, filled up with the lowest position bits when fewer
+// than four remain.  The 32 lanes of a warp give five further position bits
+// and the warp index the rest, in increasing order.  The lane bits are chosen
+// per phase so that their word offsets under word(p) = p + (p >> 5) are 1, 2,
+// 4, 8 and 16 modulo 32 in some order: bits 0..4 weigh 2^b and bits 5..9 weigh
+// 2^b + 2^(b-5), i.e. 2^(b-5) modulo 32.
+//   phase 0 (bits 0..3):      lanes on bits 4..8 (16 consecutive values per
+//                             thread: the layout of the global loads);
+//   phase 1 (bits 4..7):      lanes on bits 0..3 and 9 (bit 8 when L = 9,
+//                             which leaves one two-way bank conflict);
+//   a full later phase:       lanes on bits 0..4;
+//   a last phase with f fill bits 0..f-1: lanes on bits f..f+4.
 // ---------------------------------------------------------------------------
 
-// Word of position p in shared memory: p with its bank bits (0..4) XORed by a
-// linear function of bits 5..13.  The table was found by exhaustive check:
-// with it, every access of the phases below (a warp's 32 lanes at one
-// register index) meets 32 distinct banks for every L from 9 to 14.
-__host__ __device__ constexpr uint32_t swz(uint32_t p) {
-    constexpr uint32_t M[9] = {9u, 26u, 22u, 24u, 20u, 7u, 21u, 0u, 20u};
-    uint32_t t = 0u;
-    for (int k = 0; k < 9; ++k)
-        if ((p >> (5 + k)) & 1u) t ^= M[k];
-    return p ^ t;
-}
+__host__ __device__ constexpr uint32_t word_of(uint32_t p) { return p + (p >> 5); }
+
+// shared-memory words of one row buffer (a multiple of 4: 16-byte aligned)
+__host__ __device__ constexpr int row_words(int L) { return (1 << L) + (1 << (L - 5)); }
+
+// position bits of phase q that are butterflied (the rest of the four are fill)
+__host__ __device__ constexpr int phase_na(int L, int q) { return (L - 4 * q) < 4 ? (L - 4 * q) : 4; }
 
 // position bit of register bit r (0..3) in phase q
 __host__ __device__ constexpr int reg_bit(int L, int q, int r) {
-    const int na = (L - 4 * q) < 4 ? (L - 4 * q) : 4;
-    if (r < na) return 4 * q + r;
-    int k = r - na;
-    for (int b = 0; b < L; ++b) {
-        if (b >= 4 * q && b < 4 * q + na) continue;
-        if (k == 0) return b;
-        --k;
-    }
-    return 0;
+    return r < phase_na(L, q) ? 4 * q + r : r - phase_na(L, q);
 }
 
 // position bits of register index j (0..15) in phase q
@@ -88,14 +96,67 @@ __host__ __device__ constexpr uint32_t jpos(int L, int q, int j) {
     return p;
 }
 
-// position bits given by thread index t (< 2^(L-4)) in phase q: around the
-// four register bits 4q..4q+3, or, in a last phase with fill bits, above
-// the fill bits
-template <int L>
-__device__ __forceinline__ uint32_t tpos(int q, uint32_t t) {
-    const int na = (L - 4 * q) < 4 ? (L - 4 * q) : 4;
-    if (na == 4) return (t & ((1u << (4 * q)) - 1u)) | ((t >> (4 * q)) << (4 * q + 4));
-    return t << (4 - na);
+// position bit of lane bit i (0..4) in phase q
+__host__ __device__ constexpr int lane_bit(int L, int q, int i) {
+    if (q == 0) return 4 + i;
+    if (q == 1) return i < 4 ? i : (L >= 10 ? 9 : 8);
+    const int f = 4 - phase_na(L, q);
+    return f + i;
+}
+
+__host__ __device__ constexpr bool is_reg_or_lane_bit(int L, int q, int b) {
+    for (int r = 0; r < 4; ++r)
+        if (reg_bit(L, q, r) == b) return true;
+    for (int i = 0; i < 5; ++i)
+        if (lane_bit(L, q, i) == b) return true;
+    return false;
+}
+
+// position bit of thread-index bit s (0 .. L-5): lanes first, then the warp
+// index on the remaining bits in increasing order
+__host__ __device__ constexpr int thread_bit(int L, int q, int s) {
+    if (s < 5) return lane_bit(L, q, s);
+    int k = s - 5;
+    for (int b = 0; b < L; ++b) {
+        if (is_reg_or_lane_bit(L, q, b)) continue;
+        if (k == 0) return b;
+        --k;
+    }
+    return 0;
+}
+
+// The thread-index bits of phase q as runs that land on consecutive position
+// bits: run i moves len[i] bits from src[i] to dst[i].  Built at compile
+// time, so that tpos is one shift and mask per run.
+struct TposRuns {
+    int n;
+    int src[10], dst[10], len[10];
+};
+
+__host__ __device__ constexpr TposRuns tpos_runs(int L, int q) {
+    TposRuns r{};
+    int s = 0;
+    while (s < L - 4) {
+        int n = 1;
+        while (s + n < L - 4 && thread_bit(L, q, s + n) == thread_bit(L, q, s) + n) ++n;
+        r.src[r.n] = s;
+        r.dst[r.n] = thread_bit(L, q, s);
+        r.len[r.n] = n;
+        ++r.n;
+        s += n;
+    }
+    return r;
+}
+
+// position bits given by thread index t (< 2^(L-4)) in phase q
+template <int L, int Q>
+__device__ __forceinline__ uint32_t tpos(uint32_t t) {
+    constexpr TposRuns R = tpos_runs(L, Q);
+    uint32_t p = 0u;
+#pragma unroll
+    for (int i = 0; i < 10; ++i)
+        if (i < R.n) p |= ((t >> R.src[i]) & ((1u << R.len[i]) - 1u)) << R.dst[i];
+    return p;
 }
 
 // a value the compiler must treat as new on every use, so that loop-invariant
@@ -165,19 +226,57 @@ __device__ __forceinline__ void phase_stages(float v[VPT], uint32_t X, unsigned 
     }
 }
 
-// Phase Q >= 1: load the thread's 16 values of the phase from shared memory,
-// apply its butterflies, store them back, then a CTA barrier.  Every thread
-// reads and writes only its own 16 positions within a phase.
+// Phase Q >= 1 (not the last): load the thread's 16 values of the phase
+// from shared memory, apply its butterflies, store them back, then a CTA
+// barrier.  Every thread reads and writes only its own 16 positions within a
+// phase.
 template <int L, int Q>
 __device__ __forceinline__ void phase_pass(float v[VPT], float *srow, uint32_t base, uint32_t len, unsigned full) {
-    const uint32_t b0 = opaque(base);
+    const float *r = srow + opaque(base);
 #pragma unroll
-    for (int j = 0; j < VPT; ++j) v[j] = srow[b0 ^ swz(jpos(L, Q, j))];
-    phase_stages<L, Q>(v, tpos<L>(Q, opaque(threadIdx.x)) ^ len, full);
-    const uint32_t b1 = opaque(base);
+    for (int j = 0; j < VPT; ++j) v[j] = r[word_of(jpos(L, Q, j))];
+    phase_stages<L, Q>(v, tpos<L, Q>(opaque(threadIdx.x)) ^ len, full);
+    float *w = srow + opaque(base);
 #pragma unroll
-    for (int j = 0; j < VPT; ++j) srow[b1 ^ swz(jpos(L, Q, j))] = v[j];
+    for (int j = 0; j < VPT; ++j) w[word_of(jpos(L, Q, j))] = v[j];
     __syncthreads();
+}
+
+// R consecutive output values (R = 1, 2, 4, 8) of one run, converted and
+// stored with one vector store per 16 bytes: dtype 0 fp16, 1 bf16, 2 fp32
+template <int R, int DT>
+__device__ __forceinline__ void store_run(void *dst, const float *r) {
+    if constexpr (DT == 2) {
+        float *d = static_cast<float *>(dst);
+        if constexpr (R == 1) {
+            d[0] = r[0];
+        } else if constexpr (R == 2) {
+            *reinterpret_cast<float2 *>(d) = make_float2(r[0], r[1]);
+        } else {
+#pragma unroll
+            for (int k = 0; k < R; k += 4)
+                *reinterpret_cast<float4 *>(d + k) = make_float4(r[k], r[k + 1], r[k + 2], r[k + 3]);
+        }
+    } else if constexpr (R == 1) {
+        const uint16_t h = DT == 1 ? __bfloat16_as_ushort(__float2bfloat16_rn(r[0]))
+                                      : __half_as_ushort(__float2half_rn(r[0]));
+        *static_cast<uint16_t *>(dst) = h;
+    } else {
+        uint32_t w[R / 2];
+#pragma unroll
+        for (int k = 0; k < R / 2; ++k) {
+            if constexpr (DT == 1) {
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(r[2 * k], r[2 * k + 1]);
+                w[k] = *reinterpret_cast<const uint32_t *>(&h2);
+            } else {
+                const __half2 h2 = __floats2half2_rn(r[2 * k], r[2 * k + 1]);
+                w[k] = *reinterpret_cast<const uint32_t *>(&h2);
+            }
+        }
+        if constexpr (R == 2) *static_cast<uint32_t *>(dst) = w[0];
+        else if constexpr (R == 4) *static_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
+        else *static_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
 }
 
 // 16-byte asynchronous copy from global to shared memory; with src_bytes = 0
@@ -198,17 +297,20 @@ __device__ __forceinline__ float flip(float v, uint32_t sb, int j) {
 // bf16 activations, or 16 fp32 partial sums of the first K split) with
 // asynchronous copies into its own slots of a staging buffer while the
 // current row is transformed.
-template <bool IN, bool XQ, int L>
-__global__ void __launch_bounds__(1 << (L - 4)) rht_rows_kernel(RowsParams p, int B) {
+// DT: the output dtype of the output direction (0 fp16, 1 bf16, 2 fp32)
+template <bool IN, bool XQ, int L, int DT>
+__global__ void __launch_bounds__(1 << (L - 4), L >= 14 ? 0 : (1024 >> (L - 4))) rht_rows_kernel(RowsParams p, int B) {
     constexpr int NPH = (L + 3) / 4;  // phases of (up to) four position bits
+    constexpr int QL = NPH - 1;       // the last phase
+    constexpr int NAL = phase_na(L, QL), RUN = 1 << (4 - NAL);  // its butterflied bits; run of fill values
     constexpr int NCH = IN ? 2 : 4;   // 16-byte chunks of raw input per thread
-    extern __shared__ __align__(16) float smem_rows[];
-    float *srow = smem_rows;  // the row, 2^L words, swizzled
-    const uint4 *stage = reinterpret_cast<const uint4 *>(smem_rows + (1 << L));
+    constexpr int WORDS = row_words(L);
+    extern __shared__ __align__(16) float smem_rows[];  // [2][WORDS] row buffers, then the staging slots
+    const uint4 *stage = reinterpret_cast<const uint4 *>(smem_rows + 2 * WORDS);
     __shared__ float s_red[2][32];  // per-warp row max, by row parity
     __shared__ int s_sum[2][32];    // per-warp sums of X, by row parity
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int c0 = VPT * tid;  // first column of this thread
+    const int c0 = VPT * tid;  // first column of this thread in the load layout (phase 0)
     const uint32_t len = (uint32_t)p.len;
     const int valid = max(0, min(VPT, p.len - c0));  // 16, 8 (last block of 8) or 0
     pdl_launch_dependents();
@@ -219,17 +321,32 @@ __global__ void __launch_bounds__(1 << (L - 4)) rht_rows_kernel(RowsParams p, in
     }
 
     // row-independent data of this thread
-    float norm = 0.f;
+    float norm = 0.f;  // of the block holding its 16 load-layout columns
     if (c0 < p.len) block_size_at(p, c0, &norm);
     const uint32_t sb = valid ? (p.sign_bits[c0 >> 5] >> (c0 & 31)) & 0xFFFFu : 0u;
-    uint32_t base[NPH];
-    unsigned full = 0u;
+    uint32_t sb_out = 0u;  // output direction: S_out of the last phase's 16 positions
+    if (!IN) {
+        const uint32_t tl = tpos<L, QL>((uint32_t)tid);
 #pragma unroll
-    for (int q = 0; q < NPH; ++q) {
-        const uint32_t tp = tpos<L>(q, (uint32_t)tid);
-        base[q] = swz(tp);
-        const int top = (4 * q + 4 < L ? 4 * q + 4 : L);  // one past the phase's highest bit
-        if (((tp ^ len) >> top) != 0u) full |= 1u << q;
+        for (int j = 0; j < VPT; ++j) {
+            const uint32_t pj = tl | jpos(L, QL, j);
+            if (pj < len) sb_out |= ((p.sign_bits[pj >> 5] >> (pj & 31)) & 1u) << j;
+        }
+    }
+    uint32_t base[NPH];  // word of the thread's position bits, per phase
+    unsigned full = 0u;  // per phase: every butterfly of the thread lies within one block
+    {
+        uint32_t tp[NPH];
+        tp[0] = tpos<L, 0>((uint32_t)tid);
+        if (NPH > 1) tp[NPH > 1 ? 1 : 0] = tpos<L, (NPH > 1 ? 1 : 0)>((uint32_t)tid);
+        if (NPH > 2) tp[NPH > 2 ? 2 : 0] = tpos<L, (NPH > 2 ? 2 : 0)>((uint32_t)tid);
+        if (NPH > 3) tp[NPH > 3 ? 3 : 0] = tpos<L, (NPH > 3 ? 3 : 0)>((uint32_t)tid);
+#pragma unroll
+        for (int q = 0; q < NPH; ++q) {
+            base[q] = word_of(tp[q]);
+            const int top = (4 * q + 4 < L ? 4 * q + 4 : L);  // one past the phase's highest bit
+            if (((tp[q] ^ len) >> top) != 0u) full |= 1u << q;
+        }
     }
     // staging slots, swizzled so that the 16-byte reads of 8 consecutive
     // threads meet 8 distinct bank groups
@@ -252,11 +369,14 @@ __global__ void __launch_bounds__(1 << (L - 4)) rht_rows_kernel(RowsParams p, in
     pdl_wait();  // the input comes from the previous kernel
     if (b < B) issue(b);
     for (int par = 0; b < B; b += gridDim.x, par ^= 1) {
+        float *srow = smem_rows + par * WORDS;  // rows alternate between the two buffers
         cp_async_wait_all();
         uint4 raw[NCH];
 #pragma unroll
         for (int c = 0; c < NCH; ++c) raw[c] = stage[slot(c)];
         if (b + (int)gridDim.x < B) issue(b + gridDim.x);  // this thread's slots are free again
+        // the block norm now (all but the decode operand, which scales once at the end)
+        const float nl = XQ ? 1.f : norm;
         float v[VPT];
         if (IN) {
 #pragma unroll
@@ -276,7 +396,7 @@ __global__ void __launch_bounds__(1 << (L - 4)) rht_rows_kernel(RowsParams p, in
             }
             const uint32_t sbr = opaque(sb);  // sign masks rebuilt per row, not kept live
 #pragma unroll
-            for (int j = 0; j < VPT; ++j) v[j] = flip(v[j], sbr, j);
+            for (int j = 0; j < VPT; ++j) v[j] = flip(v[j], sbr, j) * nl;
         } else {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -297,25 +417,39 @@ __global__ void __launch_bounds__(1 << (L - 4)) rht_rows_kernel(RowsParams p, in
                     v[4 * q + 3] += r.w;
                 }
             }
+#pragma unroll
+            for (int j = 0; j < VPT; ++j) v[j] *= nl;
         }
 
         // the butterflies, phase by phase (phase 0 on the values as loaded)
         phase_stages<L, 0>(v, opaque((uint32_t)c0) ^ len, full & 1u);
-        if (NPH > 1) {
-            const uint32_t b0 = opaque(base[0]);
+        {
+            float *w = srow + opaque(base[0]);
 #pragma unroll
-            for (int j = 0; j < VPT; ++j) srow[b0 ^ swz(jpos(L, 0, j))] = v[j];
+            for (int j = 0; j < VPT; ++j) w[word_of(jpos(L, 0, j))] = v[j];
             __syncthreads();
-            if (NPH > 1) phase_pass<L, (NPH > 1 ? 1 : 0)>(v, srow, base[NPH > 1 ? 1 : 0], len, (full >> 1) & 1u);
-            if (NPH > 2) phase_pass<L, (NPH > 2 ? 2 : 0)>(v, srow, base[NPH > 2 ? 2 : 0], len, (full >> 2) & 1u);
-            if (NPH > 3) phase_pass<L, (NPH > 3 ? 3 : 0)>(v, srow, base[NPH > 3 ? 3 : 0], len, (full >> 3) & 1u);
-            const uint32_t b1 = opaque(base[0]);
+        }
+        if (NPH > 2) phase_pass<L, (NPH > 2 ? 1 : 0)>(v, srow, base[NPH > 2 ? 1 : 0], len, (full >> 1) & 1u);
+        if (NPH > 3) phase_pass<L, (NPH > 3 ? 2 : 0)>(v, srow, base[NPH > 3 ? 2 : 0], len, (full >> 2) & 1u);
+        {  // the last phase
+            const float *r = srow + opaque(base[QL]);
 #pragma unroll
-            for (int j = 0; j < VPT; ++j) v[j] = srow[b1 ^ swz(jpos(L, 0, j))];
+            for (int j = 0; j < VPT; ++j) v[j] = r[word_of(jpos(L, QL, j))];
+            phase_stages<L, QL>(v, tpos<L, QL>(opaque(threadIdx.x)) ^ len, (full >> QL) & 1u);
         }
 
-        if (IN) {
-            // row max of |xr| = |v| norm (norm is one per thread: all 16 values share a block)
+        if (XQ) {
+            // back to the load layout (8 consecutive columns per group), then
+            // X = round(xr 2^e) with the norm and the scale as one product
+            {
+                float *w = srow + opaque(base[QL]);
+#pragma unroll
+                for (int j = 0; j < VPT; ++j) w[word_of(jpos(L, QL, j))] = v[j];
+                __syncthreads();
+                const float *r = srow + opaque(base[0]);
+#pragma unroll
+                for (int j = 0; j < VPT; ++j) v[j] = r[word_of(jpos(L, 0, j))];
+            }
             float mx = 0.f;
 #pragma unroll
             for (int j = 0; j < VPT; ++j) mx = fmaxf(mx, fabsf(v[j]));
@@ -324,7 +458,6 @@ __global__ void __launch_bounds__(1 << (L - 4)) rht_rows_kernel(RowsParams p, in
             for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
             if (lane == 0) s_red[par][warp] = mx;
             __syncthreads();
-            // every warp reduces the per-warp maxima (one load per lane)
             float rowmax = lane < (int)(blockDim.x >> 5) ? s_red[par][lane] : 0.f;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) rowmax = fmaxf(rowmax, __shfl_xor_sync(0xffffffffu, rowmax, o));
@@ -335,79 +468,85 @@ __global__ void __launch_bounds__(1 << (L - 4)) rht_rows_kernel(RowsParams p, in
                 scale = ldexpf(1.f, 14 - e);
             }
             const float f = norm * scale;  // scale is a power of two: one rounding, as xr 2^e
-            if (XQ) {  // decode GEMV operand: X = round(xr 2^e), bytes per 8-column group
-                int sum = 0;
-                if (c0 < p.len_pad) {
-                    uint32_t hb[4] = {0u, 0u, 0u, 0u}, lb[4] = {0u, 0u, 0u, 0u};
-                    uint32_t hx[8];
+            int sum = 0;
+            if (c0 < p.len_pad) {
+                uint32_t hb[4] = {0u, 0u, 0u, 0u}, lb[4] = {0u, 0u, 0u, 0u};
+                uint32_t hx[8];
 #pragma unroll
-                    for (int j = 0; j < VPT; ++j) {
-                        const int X = __float2int_rn(v[j] * f);
-                        sum += X;
-                        hb[j >> 2] |= (uint32_t)((X >> 8) & 0xFF) << (8 * (j & 3));
-                        lb[j >> 2] |= (uint32_t)(X & 0xFF) << (8 * (j & 3));
-                        const __half hX = __int2half_rn(X);
-                        if (j & 1) hx[j >> 1] |= (uint32_t)__half_as_ushort(hX) << 16;
-                        else hx[j >> 1] = __half_as_ushort(hX);
-                    }
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.xq + ((size_t)b * p.len_pad + c0) * 2);
-                    dst[0] = make_uint4(hb[0], hb[1], lb[0], lb[1]);  // group c0 / 8
-                    dst[1] = make_uint4(hb[2], hb[3], lb[2], lb[3]);  // group c0 / 8 + 1
-                    if (p.xh) {
-                        uint4 *dh = reinterpret_cast<uint4 *>(p.xh + (size_t)b * p.len_pad + c0);
-                        dh[0] = make_uint4(hx[0], hx[1], hx[2], hx[3]);
-                        dh[1] = make_uint4(hx[4], hx[5], hx[6], hx[7]);
-                    }
+                for (int j = 0; j < VPT; ++j) {
+                    const int X = __float2int_rn(v[j] * f);
+                    sum += X;
+                    hb[j >> 2] |= (uint32_t)((X >> 8) & 0xFF) << (8 * (j & 3));
+                    lb[j >> 2] |= (uint32_t)(X & 0xFF) << (8 * (j & 3));
+                    const __half hX = __int2half_rn(X);
+                    if (j & 1) hx[j >> 1] |= (uint32_t)__half_as_ushort(hX) << 16;
+                    else hx[j >> 1] = __half_as_ushort(hX);
                 }
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-                if (lane == 0) s_sum[par][warp] = sum;
-                __syncthreads();
-                if (tid == 0) {
-                    long long total = 0;
-                    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) total += s_sum[par][w];
-                    p.info[b] = glq_rowinfo{total, 1.f / scale, 0.f};
+                uint4 *dst = reinterpret_cast<uint4 *>(p.xq + ((size_t)b * p.len_pad + c0) * 2);
+                dst[0] = make_uint4(hb[0], hb[1], lb[0], lb[1]);  // group c0 / 8
+                dst[1] = make_uint4(hb[2], hb[3], lb[2], lb[3]);  // group c0 / 8 + 1
+                if (p.xh) {
+                    uint4 *dh = reinterpret_cast<uint4 *>(p.xh + (size_t)b * p.len_pad + c0);
+                    dh[0] = make_uint4(hx[0], hx[1], hx[2], hx[3]);
+                    dh[1] = make_uint4(hx[4], hx[5], hx[6], hx[7]);
                 }
-            } else {
-                if (c0 < p.len_pad) {  // padding columns [len, len_pad) hold zeros
-                    uint32_t w[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const __half2 h2 = __floats2half2_rn(v[2 * j] * f, v[2 * j + 1] * f);
-                        w[j] = *reinterpret_cast<const uint32_t *>(&h2);
-                    }
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.xh + (size_t)b * p.len_pad + c0);
-                    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-                }
-                if (tid == 0) p.info[b] = glq_rowinfo{0, 1.f / scale, 0.f};
             }
-        } else if (valid) {
-            float y[VPT];
-            const uint32_t sbr = opaque(sb);  // sign masks rebuilt per row, not kept live
 #pragma unroll
-            for (int j = 0; j < VPT; ++j) y[j] = flip(v[j] * norm, sbr, j);
-            const size_t off = (size_t)b * p.len + c0;
-            for (int q = 0; q < valid / 8; ++q) {
-                const float *r = y + 8 * q;
-                if (p.y_dtype == 2) {
-                    float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.y) + off + 8 * q);
-                    dst[0] = make_float4(r[0], r[1], r[2], r[3]);
-                    dst[1] = make_float4(r[4], r[5], r[6], r[7]);
-                } else {
-                    uint32_t w[4];
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            if (lane == 0) s_sum[par][warp] = sum;
+            __syncthreads();
+            if (tid == 0) {
+                long long total = 0;
+                for (int w = 0; w < (int)(blockDim.x >> 5); ++w) total += s_sum[par][w];
+                p.info[b] = glq_rowinfo{total, 1.f / scale, 0.f};
+            }
+            continue;
+        }
+
+        // the last phase's values, straight to global memory: runs of RUN
+        // consecutive columns (the fill bits), one run per real register index
+        const uint32_t tl = tpos<L, QL>(opaque(threadIdx.x));
+        if (IN) {  // fp16 xr 2^e; padding columns [len, len_pad) hold zeros
+            float mx = 0.f;
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if (p.y_dtype == 1) {
-                            const __nv_bfloat162 h2 = __floats2bfloat162_rn(r[2 * j], r[2 * j + 1]);
-                            w[j] = *reinterpret_cast<const uint32_t *>(&h2);
-                        } else {
-                            const __half2 h2 = __floats2half2_rn(r[2 * j], r[2 * j + 1]);
-                            w[j] = *reinterpret_cast<const uint32_t *>(&h2);
-                        }
-                    }
-                    *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.y) + off + 8 * q) =
-                        make_uint4(w[0], w[1], w[2], w[3]);
+            for (int j = 0; j < VPT; ++j) mx = fmaxf(mx, fabsf(v[j]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (lane == 0) s_red[par][warp] = mx;
+            __syncthreads();
+            float rowmax = lane < (int)(blockDim.x >> 5) ? s_red[par][lane] : 0.f;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) rowmax = fmaxf(rowmax, __shfl_xor_sync(0xffffffffu, rowmax, o));
+            float scale = 1.f;
+            if (rowmax > 0.f && isfinite(rowmax)) {
+                int e;
+                frexpf(rowmax, &e);  // rowmax < 2^e
+                scale = ldexpf(1.f, 14 - e);
+            }
+            __half *xrow = p.xh + (size_t)b * p.len_pad;
+#pragma unroll
+            for (int j0 = 0; j0 < (1 << NAL); ++j0) {
+                const uint32_t pj = tl | jpos(L, QL, j0);
+                if (pj < (uint32_t)p.len_pad) {
+                    float r[RUN];
+#pragma unroll
+                    for (int k = 0; k < RUN; ++k) r[k] = v[j0 + (k << NAL)] * scale;  // exact: a power of two
+                    store_run<RUN, 0>(xrow + pj, r);
+                }
+            }
+            if (tid == 0) p.info[b] = glq_rowinfo{0, 1.f / scale, 0.f};
+        } else {
+            const uint32_t sbr = opaque(sb_out);
+            constexpr size_t esz = DT == 2 ? 4 : 2;
+            char *yrow = static_cast<char *>(p.y) + (size_t)b * p.len * esz;
+#pragma unroll
+            for (int j0 = 0; j0 < (1 << NAL); ++j0) {
+                const uint32_t pj = tl | jpos(L, QL, j0);
+                if (pj < len) {
+                    float r[RUN];
+#pragma unroll
+                    for (int k = 0; k < RUN; ++k) r[k] = flip(v[j0 + (k << NAL)], sbr, j0 + (k << NAL));
+                    store_run<RUN, DT>(yrow + pj * esz, r);
                 }
             }
         }
@@ -427,12 +566,12 @@ int rows_log2(int cover) {
     return L;
 }
 
-template <bool IN, bool XQ, int L>
+template <bool IN, bool XQ, int L, int DT>
 cudaError_t launch_rows_t(const RowsParams &p, int B, cudaStream_t s, bool pdl) {
-    const void *fn = (const void *)rht_rows_kernel<IN, XQ, L>;
+    const void *fn = (const void *)rht_rows_kernel<IN, XQ, L, DT>;
     const int threads = 1 << (L - 4);
-    // the row buffer and the staging buffer of the next row's raw input
-    const size_t smem = (sizeof(float) << L) + (size_t)threads * (IN ? 32 : 64);
+    // two row buffers and the staging buffer of the next row's raw input
+    const size_t smem = 2 * sizeof(float) * (size_t)row_words(L) + (size_t)threads * (IN ? 32 : 64);
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -464,16 +603,16 @@ cudaError_t launch_rows_t(const RowsParams &p, int B, cudaStream_t s, bool pdl) 
 }
 
 // IN: input side; XQ: the decode operand (bytes of X) instead of fp16 xr 2^e
-template <bool IN, bool XQ>
+template <bool IN, bool XQ, int DT>
 cudaError_t launch_rows_sel(const RowsParams &p, int B, cudaStream_t s, bool pdl) {
     const int cover = IN ? p.len_pad : p.len;
     switch (rows_log2(cover)) {
-        case 9: return launch_rows_t<IN, XQ, 9>(p, B, s, pdl);
-        case 10: return launch_rows_t<IN, XQ, 10>(p, B, s, pdl);
-        case 11: return launch_rows_t<IN, XQ, 11>(p, B, s, pdl);
-        case 12: return launch_rows_t<IN, XQ, 12>(p, B, s, pdl);
-        case 13: return launch_rows_t<IN, XQ, 13>(p, B, s, pdl);
-        case 14: return launch_rows_t<IN, XQ, 14>(p, B, s, pdl);
+        case 9: return launch_rows_t<IN, XQ, 9, DT>(p, B, s, pdl);
+        case 10: return launch_rows_t<IN, XQ, 10, DT>(p, B, s, pdl);
+        case 11: return launch_rows_t<IN, XQ, 11, DT>(p, B, s, pdl);
+        case 12: return launch_rows_t<IN, XQ, 12, DT>(p, B, s, pdl);
+        case 13: return launch_rows_t<IN, XQ, 13, DT>(p, B, s, pdl);
+        case 14: return launch_rows_t<IN, XQ, 14, DT>(p, B, s, pdl);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -482,8 +621,15 @@ cudaError_t launch_rows_sel(const RowsParams &p, int B, cudaStream_t s, bool pdl
 
 cudaError_t launch_rht_rows(const RowsParams &p, bool input, int B, cudaStream_t s, bool pdl) {
     if (B <= 0) return cudaErrorInvalidValue;
-    if (!input) return launch_rows_sel<false, false>(p, B, s, pdl);
-    return p.xq ? launch_rows_sel<true, true>(p, B, s, pdl) : launch_rows_sel<true, false>(p, B, s, pdl);
+    if (!input) {
+        switch (p.y_dtype) {
+            case 0: return launch_rows_sel<false, false, 0>(p, B, s, pdl);
+            case 1: return launch_rows_sel<false, false, 1>(p, B, s, pdl);
+            case 2: return launch_rows_sel<false, false, 2>(p, B, s, pdl);
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    return p.xq ? launch_rows_sel<true, true, 0>(p, B, s, pdl) : launch_rows_sel<true, false, 0>(p, B, s, pdl);
 }
 
 }  // namespace glq
