@@ -160,7 +160,7 @@ __device__ __forceinline__ uint32_t tpos(uint32_t t) {
 }
 
 // a value the compiler must treat as new on every use, so that loop-invariant
-// shared-memory addresses are recomputed (one XOR) rather than kept live
+// shared-memory addresses and masks are recomputed rather than kept live
 __device__ __forceinline__ uint32_t opaque(uint32_t x) {
     uint32_t y;
     asm volatile("mov.b32 %0, %1;" : "=r"(y) : "r"(x));
@@ -180,6 +180,26 @@ __device__ __forceinline__ void bfly2(float &a0, float &a1, float &b0, float &b1
         " mov.b64 {%2, %3}, D;\n"
         "}\n"
         : "+f"(a0), "+f"(a1), "+f"(b0), "+f"(b1));
+}
+
+// (a0, a1) *= s as one packed f32x2 multiply (IEEE rounding, as two scalar ones)
+__device__ __forceinline__ void mul2(float &a0, float &a1, float s) {
+    asm("{\n"
+        " .reg .b64 A, S, D;\n"
+        " mov.b64 A, {%0, %1};\n"
+        " mov.b64 S, {%2, %2};\n"
+        " mul.rn.f32x2 D, A, S;\n"
+        " mov.b64 {%0, %1}, D;\n"
+        "}\n"
+        : "+f"(a0), "+f"(a1)
+        : "f"(s));
+}
+
+// Sign bits of two 16-bit values packed in word u (0..7) of a thread, laid
+// out as bit u (low half) and bit u + 16 (high half) of m: the XOR mask that
+// flips those halves' sign bits.
+__device__ __forceinline__ uint32_t half2_sign_mask(uint32_t m, int u) {
+    return (m << (15 - u)) & 0x80008000u;
 }
 
 // The butterflies of phase Q on a thread's 16 values (register bit r of the
@@ -210,18 +230,24 @@ __device__ __forceinline__ void phase_stages(float v[VPT], uint32_t X, unsigned 
                     bfly2(v[j], v[j + 1], v[k], v[k + 1]);
                 }
     } else {
+        // only the position bits above the span matter; for r >= 1 the
+        // neighbours j and j + 1 differ in a bit below the span, so one test
+        // covers a packed pair of butterflies
 #pragma unroll
-        for (int r = 0; r < na; ++r)
+        for (int j = 0; j < VPT; j += 2)
+            if ((X >> (4 * Q + 1)) != (jpos(L, Q, j) >> (4 * Q + 1))) {
+                const float a = v[j], c = v[j + 1];
+                v[j] = a + c;
+                v[j + 1] = a - c;
+            }
 #pragma unroll
-            for (int j = 0; j < VPT; ++j)
+        for (int r = 1; r < na; ++r)
+#pragma unroll
+            for (int j = 0; j < VPT; j += 2)
                 if (((j >> r) & 1) == 0) {
                     const int k = j | (1 << r);
-                    // only the position bits above the span matter
-                    if ((X >> (4 * Q + r + 1)) != (jpos(L, Q, j) >> (4 * Q + r + 1))) {
-                        const float a = v[j], c = v[k];
-                        v[j] = a + c;
-                        v[k] = a - c;
-                    }
+                    if ((X >> (4 * Q + r + 1)) != (jpos(L, Q, j) >> (4 * Q + r + 1)))
+                        bfly2(v[j], v[j + 1], v[k], v[k + 1]);
                 }
     }
 }
@@ -243,9 +269,11 @@ __device__ __forceinline__ void phase_pass(float v[VPT], float *srow, uint32_t b
 }
 
 // R consecutive output values (R = 1, 2, 4, 8) of one run, converted and
-// stored with one vector store per 16 bytes: dtype 0 fp16, 1 bf16, 2 fp32
+// stored with one vector store per 16 bytes: DT 0 fp16, 1 bf16, 2 fp32.
+// 16-bit pairs (R >= 2) get their sign bits flipped by half2_sign_mask(m,
+// u0 + k) for word k; single values and fp32 arrive with their signs.
 template <int R, int DT>
-__device__ __forceinline__ void store_run(void *dst, const float *r) {
+__device__ __forceinline__ void store_run(void *dst, const float *r, uint32_t m, int u0) {
     if constexpr (DT == 2) {
         float *d = static_cast<float *>(dst);
         if constexpr (R == 1) {
@@ -272,6 +300,7 @@ __device__ __forceinline__ void store_run(void *dst, const float *r) {
                 const __half2 h2 = __floats2half2_rn(r[2 * k], r[2 * k + 1]);
                 w[k] = *reinterpret_cast<const uint32_t *>(&h2);
             }
+            w[k] ^= half2_sign_mask(m, u0 + k);
         }
         if constexpr (R == 2) *static_cast<uint32_t *>(dst) = w[0];
         else if constexpr (R == 4) *static_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
@@ -299,14 +328,20 @@ __device__ __forceinline__ float flip(float v, uint32_t sb, int j) {
 // current row is transformed.
 // DT: the output dtype of the output direction (0 fp16, 1 bf16, 2 fp32)
 template <bool IN, bool XQ, int L, int DT>
-__global__ void __launch_bounds__(1 << (L - 4), L >= 14 ? 0 : (1024 >> (L - 4))) rht_rows_kernel(RowsParams p, int B) {
+__global__ void __launch_bounds__(1 << (L - 4), L >= 14 ? (IN && !XQ ? 2 : 0) : (1024 >> (L - 4))) rht_rows_kernel(RowsParams p, int B) {
     constexpr int NPH = (L + 3) / 4;  // phases of (up to) four position bits
     constexpr int QL = NPH - 1;       // the last phase
     constexpr int NAL = phase_na(L, QL), RUN = 1 << (4 - NAL);  // its butterflied bits; run of fill values
     constexpr int NCH = IN ? 2 : 4;   // 16-byte chunks of raw input per thread
     constexpr int WORDS = row_words(L);
-    extern __shared__ __align__(16) float smem_rows[];  // [2][WORDS] row buffers, then the staging slots
-    const uint4 *stage = reinterpret_cast<const uint4 *>(smem_rows + 2 * WORDS);
+    // Row buffers: the output direction alternates two, so that no barrier
+    // protects a buffer from the next row; the input direction needs one,
+    // since its max reduction already puts a barrier between the last
+    // phase's loads and the next row's stores.
+    constexpr int NBUF = IN ? 1 : 2;
+    constexpr bool PACKED_OUT = !IN && DT != 2 && RUN >= 2;  // output signs on packed 16-bit words
+    extern __shared__ __align__(16) float smem_rows[];  // [NBUF][WORDS] row buffers, then the staging slots
+    const uint4 *stage = reinterpret_cast<const uint4 *>(smem_rows + NBUF * WORDS);
     __shared__ float s_red[2][32];  // per-warp row max, by row parity
     __shared__ int s_sum[2][32];    // per-warp sums of X, by row parity
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -323,14 +358,34 @@ __global__ void __launch_bounds__(1 << (L - 4), L >= 14 ? 0 : (1024 >> (L - 4)))
     // row-independent data of this thread
     float norm = 0.f;  // of the block holding its 16 load-layout columns
     if (c0 < p.len) block_size_at(p, c0, &norm);
-    const uint32_t sb = valid ? (p.sign_bits[c0 >> 5] >> (c0 & 31)) & 0xFFFFu : 0u;
-    uint32_t sb_out = 0u;  // output direction: S_out of the last phase's 16 positions
-    if (!IN) {
+    // signs as XOR masks: input, S_in of the 16 load-layout columns per
+    // packed word (word u = columns 2u, 2u + 1); output, S_out of the last
+    // phase's 16 positions, per value (bit j) or per packed 16-bit word
+    uint32_t smask = 0u;
+    if (IN) {
+        const uint32_t sb = valid ? (p.sign_bits[c0 >> 5] >> (c0 & 31)) & 0xFFFFu : 0u;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            smask |= ((sb >> (2 * u)) & 1u) << u | ((sb >> (2 * u + 1)) & 1u) << (u + 16);
+    } else {
         const uint32_t tl = tpos<L, QL>((uint32_t)tid);
+        uint32_t sbj = 0u;
 #pragma unroll
         for (int j = 0; j < VPT; ++j) {
             const uint32_t pj = tl | jpos(L, QL, j);
-            if (pj < len) sb_out |= ((p.sign_bits[pj >> 5] >> (pj & 31)) & 1u) << j;
+            if (pj < len) sbj |= ((p.sign_bits[pj >> 5] >> (pj & 31)) & 1u) << j;
+        }
+        if (PACKED_OUT) {
+#pragma unroll
+            for (int j0 = 0; j0 < (1 << NAL); ++j0)
+#pragma unroll
+                for (int w = 0; w < RUN / 2; ++w) {
+                    const int u = j0 * (RUN / 2) + w;
+                    smask |= ((sbj >> (j0 + ((2 * w) << NAL))) & 1u) << u |
+                             ((sbj >> (j0 + ((2 * w + 1) << NAL))) & 1u) << (u + 16);
+                }
+        } else {
+            smask = sbj;
         }
     }
     uint32_t base[NPH];  // word of the thread's position bits, per phase
@@ -369,34 +424,36 @@ __global__ void __launch_bounds__(1 << (L - 4), L >= 14 ? 0 : (1024 >> (L - 4)))
     pdl_wait();  // the input comes from the previous kernel
     if (b < B) issue(b);
     for (int par = 0; b < B; b += gridDim.x, par ^= 1) {
-        float *srow = smem_rows + par * WORDS;  // rows alternate between the two buffers
+        float *srow = smem_rows + (NBUF == 2 ? par * WORDS : 0);
         cp_async_wait_all();
         uint4 raw[NCH];
 #pragma unroll
         for (int c = 0; c < NCH; ++c) raw[c] = stage[slot(c)];
         if (b + (int)gridDim.x < B) issue(b + gridDim.x);  // this thread's slots are free again
         // the block norm now (all but the decode operand, which scales once at the end)
-        const float nl = XQ ? 1.f : norm;
         float v[VPT];
         if (IN) {
+            const uint32_t sm = opaque(smask);
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 const uint32_t w[4] = {raw[q].x, raw[q].y, raw[q].z, raw[q].w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
+                    const uint32_t ws = w[j] ^ half2_sign_mask(sm, 4 * q + j);  // S_in on the raw halves
                     if (p.x_bf16) {
-                        v[8 * q + 2 * j] = __uint_as_float(w[j] << 16);
-                        v[8 * q + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+                        v[8 * q + 2 * j] = __uint_as_float(ws << 16);
+                        v[8 * q + 2 * j + 1] = __uint_as_float(ws & 0xFFFF0000u);
                     } else {
-                        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[j]));
+                        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&ws));
                         v[8 * q + 2 * j] = f.x;
                         v[8 * q + 2 * j + 1] = f.y;
                     }
                 }
             }
-            const uint32_t sbr = opaque(sb);  // sign masks rebuilt per row, not kept live
+            if (!XQ) {
 #pragma unroll
-            for (int j = 0; j < VPT; ++j) v[j] = flip(v[j], sbr, j) * nl;
+                for (int j = 0; j < VPT; j += 2) mul2(v[j], v[j + 1], norm);
+            }
         } else {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -418,7 +475,7 @@ __global__ void __launch_bounds__(1 << (L - 4), L >= 14 ? 0 : (1024 >> (L - 4)))
                 }
             }
 #pragma unroll
-            for (int j = 0; j < VPT; ++j) v[j] *= nl;
+            for (int j = 0; j < VPT; j += 2) mul2(v[j], v[j + 1], norm);
         }
 
         // the butterflies, phase by phase (phase 0 on the values as loaded)
@@ -531,12 +588,12 @@ __global__ void __launch_bounds__(1 << (L - 4), L >= 14 ? 0 : (1024 >> (L - 4)))
                     float r[RUN];
 #pragma unroll
                     for (int k = 0; k < RUN; ++k) r[k] = v[j0 + (k << NAL)] * scale;  // exact: a power of two
-                    store_run<RUN, 0>(xrow + pj, r);
+                    store_run<RUN, 0>(xrow + pj, r, 0u, 0);
                 }
             }
             if (tid == 0) p.info[b] = glq_rowinfo{0, 1.f / scale, 0.f};
         } else {
-            const uint32_t sbr = opaque(sb_out);
+            const uint32_t sm = opaque(smask);
             constexpr size_t esz = DT == 2 ? 4 : 2;
             char *yrow = static_cast<char *>(p.y) + (size_t)b * p.len * esz;
 #pragma unroll
@@ -545,8 +602,9 @@ __global__ void __launch_bounds__(1 << (L - 4), L >= 14 ? 0 : (1024 >> (L - 4)))
                 if (pj < len) {
                     float r[RUN];
 #pragma unroll
-                    for (int k = 0; k < RUN; ++k) r[k] = flip(v[j0 + (k << NAL)], sbr, j0 + (k << NAL));
-                    store_run<RUN, DT>(yrow + pj * esz, r);
+                    for (int k = 0; k < RUN; ++k)
+                        r[k] = PACKED_OUT ? v[j0 + (k << NAL)] : flip(v[j0 + (k << NAL)], sm, j0 + (k << NAL));
+                    store_run<RUN, DT>(yrow + pj * esz, r, PACKED_OUT ? sm : 0u, j0 * (RUN / 2));
                 }
             }
         }
@@ -570,8 +628,9 @@ template <bool IN, bool XQ, int L, int DT>
 cudaError_t launch_rows_t(const RowsParams &p, int B, cudaStream_t s, bool pdl) {
     const void *fn = (const void *)rht_rows_kernel<IN, XQ, L, DT>;
     const int threads = 1 << (L - 4);
-    // two row buffers and the staging buffer of the next row's raw input
-    const size_t smem = 2 * sizeof(float) * (size_t)row_words(L) + (size_t)threads * (IN ? 32 : 64);
+    // the row buffers (two on the output side) and the staging buffer of the
+    // next row's raw input
+    const size_t smem = (IN ? 1 : 2) * sizeof(float) * (size_t)row_words(L) + (size_t)threads * (IN ? 32 : 64);
     static bool configured = false;
     if (!configured) {
         cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
