@@ -197,12 +197,13 @@ bool encode_w_map(CUtensorMap *map, const __half *w16, int64_t n_pad, int64_t m_
 
 // K splits of the tensor-core GEMM: fill the CTA pairs when the output has
 // too few tiles, unless the extra partial-sum traffic costs more than it
-// saves.  Model (B200 measurements): a pair retires 256 x 512 x n x 2 FLOP at
-// about 15 TFLOP/s; each extra split writes and reads B x m_pad fp32 at
-// about 6 TB/s.
+// saves.  Model (B200 measurements): a pair retires a tile's rows x tokens x
+// n x 2 FLOP at about 15 TFLOP/s; each extra split writes and reads B x m_pad
+// fp32 at about 6 TB/s.
 int choose_ksplit(glq_layer L, int64_t B, int tiles) {
     const int pairs = std::max(1, L->num_sms / 2);
-    const double t_tile = 256.0 * 512.0 * (double)L->n_pad * 2.0 / 15e12;
+    const double t_tile = (double)glq::prefill_tile_rows() * (double)glq::prefill_tile_tokens() *
+                          (double)L->n_pad * 2.0 / 15e12;
     const double t_traffic = (double)B * (double)L->m_pad * 8.0 / 6e12;
     int best = 1;
     double best_t = 1e30;
