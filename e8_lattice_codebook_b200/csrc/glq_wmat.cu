@@ -9,14 +9,16 @@
 // a fold fix-up, and four byte permutes plus four fp16 FMAs: the nibble v
 // becomes the fp16 1024 + v, and (1024 + v) / 2 - 515 = v/2 - 3 exactly.  A
 // warp takes one (16-row tile, 128-column chunk) of the fragment-native index
-// stream: 512 coalesced bytes of codes per stream, 4 KB of W16 out.
+// stream at a time: 512 coalesced bytes of codes per stream, 4 KB of W16
+// out; the codes of its next item are already in flight meanwhile (16 warps
+// per SM, so that enough loads are outstanding to cover the DRAM latency).
 #include "glq_kernels.cuh"
 
 namespace glq {
 
 namespace {
 
-constexpr int WARPS = 8;
+constexpr int WARPS = 16;
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;
@@ -82,16 +84,24 @@ __global__ void __launch_bounds__(WARPS * 32, 1) wmat_kernel(PrefillParams p, __
     }
     pdl_wait();  // the previous user of w16 (the GEMM of an earlier call) has finished
     const long long items = (long long)p.RT * p.KC;
-    for (long long it = (long long)blockIdx.x * WARPS + warp; it < items; it += (long long)gridDim.x * WARPS) {
-        const int rt = (int)(it / p.KC), kc = (int)(it - (long long)rt * p.KC);
+    const long long stride = (long long)gridDim.x * WARPS;
+    auto load_codes = [&](long long it, uint4 &a1, uint4 &a2) {
         const size_t slot = it * 32 + lane;  // [RT][KC][32]
-        const uint4 q1 = ldg_nc_v4(p.idx1 + slot);
-        uint4 q2 = make_uint4(0, 0, 0, 0);
-        if (BPW == 4) q2 = ldg_nc_v4(reinterpret_cast<const uint4 *>(p.idx2) + slot);
+        a1 = ldg_nc_v4(p.idx1 + slot);
+        a2 = make_uint4(0, 0, 0, 0);
+        if (BPW == 4) a2 = ldg_nc_v4(reinterpret_cast<const uint4 *>(p.idx2) + slot);
         if (BPW == 3) {
             const uint2 v = ldg_nc_v2(reinterpret_cast<const uint2 *>(p.idx2) + slot);
-            q2 = make_uint4(v.x, v.y, 0, 0);
+            a2 = make_uint4(v.x, v.y, 0, 0);
         }
+    };
+    long long it = (long long)blockIdx.x * WARPS + warp;
+    uint4 n1 = make_uint4(0, 0, 0, 0), n2 = n1;  // the codes of the warp's next item
+    if (it < items) load_codes(it, n1, n2);
+    for (; it < items; it += stride) {
+        const uint4 q1 = n1, q2 = n2;
+        if (it + stride < items) load_codes(it + stride, n1, n2);
+        const int rt = (int)(it / p.KC), kc = (int)(it - (long long)rt * p.KC);
         const uint32_t c1[4] = {q1.x, q1.y, q1.z, q1.w}, c2[4] = {q2.x, q2.y, q2.z, q2.w};
 #pragma unroll
         for (int s = 0; s < 4; ++s)
