@@ -910,6 +910,18 @@ glq_status glq_rht_output(glq_layer L, const float *z_dev, void *y_dev, glq_dtyp
     if (!z_dev || !y_dev) return GLQ_ERR_INVALID_ARG;
     if (B > 65535) return GLQ_ERR_SHAPE;
     DeviceGuard guard(L->device);
+    // the kernel glq_linear's output stage takes for this batch: one CTA per
+    // row, except for one or two rows longer than 8192
+    if (glq::rht_rows_supported((int)L->m) && (B > 2 || L->m <= 8192)) {
+        glq::RowsParams r = rows_params(L->hb_m, (int)L->m, (int)L->m, L->d_sout);
+        r.z = z_dev;
+        r.z_ld = (int)L->m;
+        r.y = y_dev;
+        r.y_dtype = (int)y_dtype;
+        return glq::launch_rht_rows(r, false, (int)B, static_cast<cudaStream_t>(stream), false) == cudaSuccess
+                   ? GLQ_OK
+                   : GLQ_ERR_CUDA;
+    }
     glq::RhtOutParams p{};
     p.m = (int)L->m;
     p.B = (int)B;

@@ -223,7 +223,8 @@ GLQ_API glq_status glq_dequant_reference(glq_layer layer, float *w_dev, void *st
  * testing and composition (GLQ v0.3.2 release notes: input_rht,
  * output_rht).  glq_rht_input: xr[B][n] (fp32, device) = H_n (S_in . x).
  * glq_rht_output: y[B][m] (device, y_dtype) = S_out . H_m z, z fp32 device
- * [B][m].  Errors as glq_linear.  Asynchronous.
+ * [B][m], with the kernel glq_linear's output stage uses at this batch.
+ * Errors as glq_linear.  Asynchronous.
  */
 GLQ_API glq_status glq_rht_input(glq_layer layer, const void *x_dev, glq_dtype x_dtype, float *xr_dev,
                          int64_t B, void *stream);

@@ -82,17 +82,28 @@ def test_rht_input_matches_dense_hadamard(dev, n):
         np.testing.assert_allclose(xr[b], ref, rtol=0, atol=1e-5 * (np.abs(ref).max() + 1))
 
 
-@pytest.mark.parametrize("m", [8, 24, 56, 64, 200, 960, 2048, 11008, 14336, 32768])
-def test_rht_output_matches_dense_hadamard(dev, m):
+@pytest.mark.parametrize("B", [2, 5])
+@pytest.mark.parametrize("m", [8, 24, 56, 64, 200, 960, 2048, 4096, 5120, 11008, 14336, 32768])
+def test_rht_output_matches_dense_hadamard(dev, m, B):
+    """The output stage as glq_linear runs it at this batch (the row kernel
+    for rows up to 16384, except one or two rows longer than 8192): fp32
+    output within 1e-5 of the dense fp64 transform, 16-bit outputs within one
+    rounding of that."""
     n = 8
     L = gi.make_layer(m, 0, m, n, 2)
-    rng = np.random.default_rng(m)
-    z = rng.standard_normal((2, m)).astype(np.float32)
+    rng = np.random.default_rng(m + B)
+    z = rng.standard_normal((B, m)).astype(np.float32)
     lay = dev.layer(L)
-    y = lay.rht_output(torch.from_numpy(z).cuda()).cpu().numpy().astype(np.float64)
-    for b in range(2):
-        ref = orc.hadamard_apply(z[b].astype(np.float64)) * L.s_out
-        np.testing.assert_allclose(y[b], ref, rtol=0, atol=1e-5 * (np.abs(ref).max() + 1))
+    zc = torch.from_numpy(z).cuda()
+    y = lay.rht_output(zc).cpu().numpy().astype(np.float64)
+    refs = [orc.hadamard_apply(z[b].astype(np.float64)) * L.s_out for b in range(B)]
+    for b in range(B):
+        np.testing.assert_allclose(y[b], refs[b], rtol=0, atol=1e-5 * (np.abs(refs[b]).max() + 1))
+    for dt, u in ((torch.bfloat16, 2.0 ** -8), (torch.float16, 2.0 ** -11)):
+        yh = lay.rht_output(zc, out_dtype=dt).float().cpu().numpy().astype(np.float64)
+        for b in range(B):
+            bound = u * np.abs(refs[b]) + 2e-5 * (np.abs(refs[b]).max() + 1)
+            assert np.all(np.abs(yh[b] - refs[b]) <= bound), (dt, b)
 
 
 def _workload_cases():
