@@ -1,12 +1,14 @@
-// glq_rht_rows.cu -- the input and output randomized Hadamard transforms of
-// the tensor-core (many-token) path: xr = H_n (S_in x) and y = S_out (H_m z),
-// H block-diagonal over the binary decomposition of the size, each block a
-// Sylvester-ordered FWHT normalised by 1/sqrt(block) (glq 0.5.1 PyPI page,
-// "How it works" 2 and "Bit widths": block-diagonal FHT for sizes that are
-// not powers of two; GLQ v0.3.2 release notes, input_rht / output_rht).
+// glq_rht_rows.cu -- the input and output randomized Hadamard transforms,
+// xr = H_n (S_in x) and y = S_out (H_m z), for rows of up to 16384 values: all
+// of the tensor-core (many-token) path, the decode output stage, and the
+// decode input stage when it is not fused into the GEMV.  H is block-diagonal
+// over the binary decomposition of the size, each block a Sylvester-ordered
+// FWHT normalised by 1/sqrt(block) (glq 0.5.1 PyPI page, "How it works" 2 and
+// "Bit widths": block-diagonal FHT for sizes that are not powers of two;
+// GLQ v0.3.2 release notes, input_rht / output_rht).
 //
-// Design (B200): throughput over many rows, sizes up to 16384, bound by the
-// per-value instruction count rather than by DRAM.  A persistent grid of CTAs
+// Design (B200): throughput over many rows, bound by the per-value
+// instruction count rather than by DRAM.  A persistent grid of CTAs
 // transforms one row at a time per CTA, with the next row already streaming
 // into a shared-memory staging buffer (16-byte asynchronous copies):
 //   * a row of up to 2^L values (9 <= L <= 14) is held 16 values per thread;
@@ -20,10 +22,14 @@
 //     words fall in 32 distinct banks;
 //   * the stages of a Hadamard transform commute, so the last phase carries
 //     the lowest position bits along as "fill" and writes its values straight
-//     to global memory in runs of consecutive columns; rows alternate between
-//     two buffers, so no barrier protects a buffer from the next row;
-//   * butterflies on register pairs use the packed f32x2 add / subtract of
-//     sm_100a (same IEEE rounding as scalar adds);
+//     to global memory in runs of consecutive columns;
+//   * the output side alternates two row buffers, so that no barrier protects
+//     a buffer from the next row; the input side keeps one (its row-max
+//     reduction already separates rows), which at 2^14 values lets two
+//     1024-thread CTAs share an SM;
+//   * butterflies and the norm use the packed f32x2 add / subtract / multiply
+//     of sm_100a (same IEEE rounding as scalar operations); signs are XOR
+//     masks on packed 16-bit words where the data is 16-bit;
 //   * Hadamard blocks of a size that is not a power of two are handled by
 //     testing, per butterfly, whether both ends lie in one block; the block
 //     norm 1/sqrt(block) is applied on load, where a thread's 16 values share
