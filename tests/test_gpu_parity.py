@@ -238,16 +238,22 @@ def test_cluster_splitk_matches_global_reduction(dev, m, n, bpw, B, xdt):
 def test_decode_plans_of_the_workloads(dev):
     """The decode plans of the SmolLM3-3B-shaped and 24B-class layers at 1 and
     16 tokens are consistent (a cluster, when used, holds a band's splits)
-    and the cluster reduction is in use on some of them."""
+    and the cluster reduction is in use on some of them.  At 16 tokens the
+    32768-row gate / up layers (128 bands of 16-warp CTAs on 148 SMs) take one
+    split: charged too little for the global reduction of two token tiles,
+    the planner chose 8 splits over 7 waves there, 1.6x slower per step."""
     clustered = 0
     for key in ("smollm3-3b-4bpw", "24b-decode-4bpw"):
         wl = gi.WORKLOADS[key]
         for li in range(len(wl.layers)):
-            lay = dev.layer(gi.workload_layer(wl, li))
+            L = gi.workload_layer(wl, li)
+            lay = dev.layer(L)
             for B in (1, 16):
                 plan = lay.decode_plan(B)
                 assert plan["cluster"] in (0, plan["splits"]) and plan["cluster"] != 1, (key, li, B, plan)
                 clustered += plan["cluster"] > 0
+                if B == 16 and L.m == 32768 and torch.cuda.get_device_properties(0).multi_processor_count == 148:
+                    assert plan["splits"] == 1, (key, li, plan)
                 print(f"\nPLAN {key} layer {li} B={B}: {plan}")
     assert clustered > 0
 
