@@ -38,6 +38,7 @@
 #include <cooperative_groups.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "glq_kernels.cuh"
 
@@ -845,15 +846,14 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
 template <int BPW, int NT, bool FIN, int WARPS = gemv_warps(NT)>
 cudaError_t launch_t(const GemvParams &p, int grid, cudaStream_t s, bool pdl) {
     const size_t smem = gemv_launch_smem_bytes(p, BPW, FIN, WARPS);
-    // raised once to the largest the library launches with (never lowered:
-    // captured graphs replay against the attribute value at replay time)
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<BPW, NT, FIN, WARPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)GEMV_SMEM_LIMIT);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    // raised once per device to the largest the library launches with (never
+    // lowered: captured graphs replay against the attribute value at replay time)
+    static std::atomic<uint64_t> configured{0};
+    cudaError_t e = once_per_device(configured, [] {
+        return cudaFuncSetAttribute(gemv_kernel<BPW, NT, FIN, WARPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)GEMV_SMEM_LIMIT);
+    });
+    if (e != cudaSuccess) return e;
     if (smem > GEMV_SMEM_LIMIT) return cudaErrorInvalidValue;
     if (p.fuse_out) {  // the output block is transformed in the table's shared memory
         for (int bi = 0; bi < p.nblk_m; ++bi)
@@ -863,13 +863,12 @@ cudaError_t launch_t(const GemvParams &p, int grid, cudaStream_t s, bool pdl) {
     void *args[] = {&q};
     if (p.clu > 1) {
         if (grid != p.bands * p.splits || p.clu != p.splits) return cudaErrorInvalidValue;
-        static bool nonportable = false;  // clusters above 8 CTAs
-        if (!nonportable) {
-            cudaError_t e = cudaFuncSetAttribute(gemv_kernel<BPW, NT, FIN, WARPS>,
-                                                 cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-            if (e != cudaSuccess) return e;
-            nonportable = true;
-        }
+        static std::atomic<uint64_t> nonportable{0};  // clusters above 8 CTAs
+        e = once_per_device(nonportable, [] {
+            return cudaFuncSetAttribute(gemv_kernel<BPW, NT, FIN, WARPS>,
+                                        cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        });
+        if (e != cudaSuccess) return e;
         return launch_ex((const void *)gemv_kernel<BPW, NT, FIN, WARPS>, dim3(grid), dim3(WARPS * 32), smem, s,
                          pdl, args, p.clu);
     }
@@ -959,17 +958,23 @@ size_t gemv_cluster_partials_bytes(int warps, int B) {
 }
 
 int gemv_max_clusters(int bpw, int nt, bool fin, int warps, int csize, size_t smem) {
-    // memoised per kernel, cluster size and shared-memory size (host-side)
+    // memoised per device, kernel, cluster size and shared-memory size
+    // (host-side, under a lock: layers may be created from several threads)
     struct Key {
-        int bpw, nt, fin, warps, csize;
+        int dev, bpw, nt, fin, warps, csize;
         size_t smem;
         int n;
     };
     static Key cache[64];
     static int ncache = 0;
+    static std::mutex lock;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> guard(lock);
     for (int i = 0; i < ncache; ++i) {
         const Key &k = cache[i];
-        if (k.bpw == bpw && k.nt == nt && k.fin == (int)fin && k.warps == warps && k.csize == csize && k.smem == smem)
+        if (k.dev == dev && k.bpw == bpw && k.nt == nt && k.fin == (int)fin && k.warps == warps &&
+            k.csize == csize && k.smem == smem)
             return k.n;
     }
     int n = 0;
@@ -985,7 +990,7 @@ int gemv_max_clusters(int bpw, int nt, bool fin, int warps, int csize, size_t sm
     } else {
         n = bpw == 2 ? max_clusters_t<2, 2, false>(csize, smem) : bpw == 3 ? max_clusters_t<3, 2, false>(csize, smem) : max_clusters_t<4, 2, false>(csize, smem);
     }
-    if (ncache < 64) cache[ncache++] = Key{bpw, nt, (int)fin, warps, csize, smem, n};
+    if (ncache < 64) cache[ncache++] = Key{dev, bpw, nt, (int)fin, warps, csize, smem, n};
     return n;
 }
 

@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "glq_device.cuh"
 #include "glq_internal.h"
 
@@ -184,6 +186,22 @@ inline cudaError_t launch_ex(const void *fn, dim3 grid, dim3 block, size_t smem,
     cfg.attrs = attr;
     cfg.numAttrs = na;
     return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+// Runs set() -- the cudaFuncSetAttribute calls of one kernel -- once per
+// device (devices 0..63; attributes apply to the current device only), with
+// `done` the kernel's static bit mask of devices already set.  A race only
+// repeats set(), which is harmless.
+template <typename F>
+inline cudaError_t once_per_device(std::atomic<uint64_t> &done, F set) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev < 64 ? 1ull << dev : 0ull;
+    if (bit && (done.load(std::memory_order_relaxed) & bit)) return cudaSuccess;
+    e = set();
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_relaxed);
+    return e;
 }
 
 // Launchers (return cudaError_t of the launch).  `pdl` enables

@@ -364,13 +364,12 @@ cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &xmap, cons
         case 9: fn = (const void *)prefill_kernel<4, true>; break;
         default: return cudaErrorInvalidValue;
     }
-    static bool configured[10] = {};
+    static std::atomic<uint64_t> configured[10];  // per variant: devices set
     const int key = p.bpw * 2 + (mat ? 1 : 0);
-    if (!configured[key]) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GEMV_SMEM_LIMIT);
-        if (e != cudaSuccess) return e;
-        configured[key] = true;
-    }
+    const cudaError_t e = once_per_device(configured[key], [fn] {
+        return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GEMV_SMEM_LIMIT);
+    });
+    if (e != cudaSuccess) return e;
     if (smem > GEMV_SMEM_LIMIT || (grid & 1)) return cudaErrorInvalidValue;
     PrefillParams q = p;
     CUtensorMap m = xmap;

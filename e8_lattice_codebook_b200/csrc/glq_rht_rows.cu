@@ -637,18 +637,17 @@ cudaError_t launch_rows_t(const RowsParams &p, int B, cudaStream_t s, bool pdl) 
     // the row buffers (two on the output side) and the staging buffer of the
     // next row's raw input
     const size_t smem = (IN ? 1 : 2) * sizeof(float) * (size_t)row_words(L) + (size_t)threads * (IN ? 32 : 64);
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    static std::atomic<uint64_t> configured{0};  // devices set
+    cudaError_t e = once_per_device(configured, [fn, smem] {
+        return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    });
+    if (e != cudaSuccess) return e;
     // persistent grid: every CTA that fits on the device at once, at most one
     // per row (SM count and occupancy queried once per device, not per call)
     constexpr int MAX_DEV = 64;
     static int sms_of[MAX_DEV] = {}, per_sm_of[MAX_DEV] = {};
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     int sms = dev < MAX_DEV ? sms_of[dev] : 0, per_sm = dev < MAX_DEV ? per_sm_of[dev] : 0;
     if (sms <= 0 || per_sm <= 0) {

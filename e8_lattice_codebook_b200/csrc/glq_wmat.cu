@@ -128,13 +128,12 @@ size_t wmat_smem_bytes(int table_words, int bpw) { return (size_t)table_words * 
 cudaError_t launch_wmat(const PrefillParams &p, __half *w16, int n_pad, int num_sms, cudaStream_t s, bool pdl) {
     const void *fn = p.bpw == 4 ? (const void *)wmat_kernel<4>
                                 : (p.bpw == 3 ? (const void *)wmat_kernel<3> : (const void *)wmat_kernel<2>);
-    static bool configured[5] = {};
-    if (!configured[p.bpw]) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)wmat_smem_bytes(GLQ_TABLE_MAX_WORDS, 3));
-        if (e != cudaSuccess) return e;
-        configured[p.bpw] = true;
-    }
+    static std::atomic<uint64_t> configured[5];  // per bit width: devices set
+    const cudaError_t e = once_per_device(configured[p.bpw], [fn] {
+        return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)wmat_smem_bytes(GLQ_TABLE_MAX_WORDS, 3));
+    });
+    if (e != cudaSuccess) return e;
     const long long items = (long long)p.RT * p.KC;
     const int grid = (int)std::min<long long>(num_sms, (items + WARPS - 1) / WARPS);
     PrefillParams q = p;
