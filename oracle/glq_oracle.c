@@ -1,6 +1,8 @@
 /*
- * glq_oracle.c -- plain, slow, single-threaded fp64 CPU oracle for the GLQ
- * compressed-weight linear layer  y = S_out . H_m . W^ . H_n . (S_in . x).
+ * glq_oracle.c -- plain, slow fp64 CPU oracle for the GLQ compressed-weight
+ * linear layer  y = S_out . H_m . W^ . H_n . (S_in . x).  Single-threaded,
+ * except that the rows of the middle product may be dealt out to threads
+ * (glq_oracle_linear_mt; every output element is the same loop either way).
  *
  * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the package entry point's
  * smoke check and the benchmark's CPU-baseline leg may load this file.  The
@@ -34,6 +36,7 @@
  * Parity pins live in the test-suite; none of the functions here is unpinned.
  */
 #include <math.h>
+#include <pthread.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -263,22 +266,64 @@ int glq_oracle_decode_rows(int64_t m, int64_t n, int bpw, const uint16_t *idx1,
 /* The layer:  y = S_out . H_m . W^ . H_n . (S_in . x)                  */
 /* ------------------------------------------------------------------ */
 
+/* The middle product z = W^ xr for rows [r0, r1): W^ is decoded one row at
+ * a time (explicitly) and multiplied by a naive dot product. */
+typedef struct {
+    int64_t m, n, B, r0, r1;
+    int bpw;
+    const uint16_t *idx1;
+    const void *idx2;
+    const double *cb1, *cb2;
+    float ws, rs;
+    const double *xr;
+    double *z;
+    int rc;
+} rows_job;
+
+static void *rows_product(void *arg) {
+    rows_job *j = (rows_job *)arg;
+    double *w = (double *)malloc(sizeof(double) * (size_t)j->n);
+    if (!w) {
+        j->rc = -1;
+        return 0;
+    }
+    for (int64_t r = j->r0; r < j->r1; r++) {
+        glq_oracle_decode_rows(j->m, j->n, j->bpw, j->idx1, j->idx2, j->cb1, j->cb2, j->ws, j->rs, r, r + 1, w);
+        for (int64_t b = 0; b < j->B; b++) {
+            double acc = 0.0;
+            const double *xb = j->xr + b * j->n;
+            for (int64_t k = 0; k < j->n; k++) acc += w[k] * xb[k];
+            j->z[b * j->m + r] = acc;
+        }
+    }
+    free(w);
+    j->rc = 0;
+    return 0;
+}
+
 /* x[B][n] as fp16 (x_is_bf16 == 0) or bf16 bits; y[B][m] in double.
  * W^ is decoded one row at a time (explicitly) and multiplied by a naive
- * dot product.  Returns 0 or -1 on bad arguments / allocation failure. */
-int glq_oracle_linear(int64_t m, int64_t n, int bpw, const uint16_t *idx1, const void *idx2,
-                      const double *cb1, const double *cb2, float ws, float rs,
-                      const int8_t *s_in, const int8_t *s_out, const uint16_t *x, int x_is_bf16,
-                      int64_t B, double *y) {
+ * dot product.  The rows of the middle product are dealt out in contiguous
+ * ranges to `nthreads` POSIX threads (each output element is computed by
+ * the same loop whatever the thread count, so the result is identical).
+ * Returns 0 or -1 on bad arguments / allocation failure. */
+int glq_oracle_linear_mt(int64_t m, int64_t n, int bpw, const uint16_t *idx1, const void *idx2,
+                         const double *cb1, const double *cb2, float ws, float rs,
+                         const int8_t *s_in, const int8_t *s_out, const uint16_t *x, int x_is_bf16,
+                         int64_t B, double *y, int nthreads) {
     if (m <= 0 || n <= 0 || n % 8 != 0 || B < 0) return -1;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (nthreads > m) nthreads = (int)m;
     double *xs = (double *)malloc(sizeof(double) * (size_t)n);
     double *xr = (double *)malloc(sizeof(double) * (size_t)(B * n + 1));
     double *z = (double *)malloc(sizeof(double) * (size_t)(B * m + 1));
-    double *w = (double *)malloc(sizeof(double) * (size_t)n);
     double *zb = (double *)malloc(sizeof(double) * (size_t)m);
     double *hb = (double *)malloc(sizeof(double) * (size_t)m);
-    if (!xs || !xr || !z || !w || !zb || !hb) {
-        free(xs); free(xr); free(z); free(w); free(zb); free(hb);
+    rows_job *jobs = (rows_job *)malloc(sizeof(rows_job) * (size_t)nthreads);
+    pthread_t *tid = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!xs || !xr || !z || !zb || !hb || !jobs || !tid) {
+        free(xs); free(xr); free(z); free(zb); free(hb); free(jobs); free(tid);
         return -1;
     }
     /* input RHT: sign, then H_n */
@@ -290,22 +335,38 @@ int glq_oracle_linear(int64_t m, int64_t n, int bpw, const uint16_t *idx1, const
         }
         glq_oracle_hadamard_apply(n, xs, xr + b * n, 0);
     }
-    /* z = W^ xr, one decoded row at a time */
-    for (int64_t r = 0; r < m; r++) {
-        glq_oracle_decode_rows(m, n, bpw, idx1, idx2, cb1, cb2, ws, rs, r, r + 1, w);
-        for (int64_t b = 0; b < B; b++) {
-            double acc = 0.0;
-            const double *xb = xr + b * n;
-            for (int64_t j = 0; j < n; j++) acc += w[j] * xb[j];
-            z[b * m + r] = acc;
-        }
+    /* z = W^ xr, one decoded row at a time, rows split over the threads */
+    int rc = 0, started = 0;
+    for (int t = 0; t < nthreads; t++) {
+        rows_job *j = &jobs[t];
+        j->m = m; j->n = n; j->B = B; j->bpw = bpw;
+        j->r0 = m * t / nthreads;
+        j->r1 = m * (t + 1) / nthreads;
+        j->idx1 = idx1; j->idx2 = idx2; j->cb1 = cb1; j->cb2 = cb2;
+        j->ws = ws; j->rs = rs; j->xr = xr; j->z = z; j->rc = -1;
     }
+    for (int t = 1; t < nthreads; t++) {
+        if (pthread_create(&tid[t], 0, rows_product, &jobs[t]) != 0) break;
+        started = t;
+    }
+    rows_product(&jobs[0]);
+    for (int t = 1; t <= started; t++) pthread_join(tid[t], 0);
+    for (int t = started + 1; t < nthreads; t++) rows_product(&jobs[t]); /* threads that did not start */
+    for (int t = 0; t < nthreads; t++) rc |= jobs[t].rc;
     /* output RHT: H_m, then sign */
-    for (int64_t b = 0; b < B; b++) {
+    for (int64_t b = 0; b < B && rc == 0; b++) {
         memcpy(zb, z + b * m, sizeof(double) * (size_t)m);
         glq_oracle_hadamard_apply(m, zb, hb, 0);
         for (int64_t r = 0; r < m; r++) y[b * m + r] = (double)s_out[r] * hb[r];
     }
-    free(xs); free(xr); free(z); free(w); free(zb); free(hb);
-    return 0;
+    free(xs); free(xr); free(z); free(zb); free(hb); free(jobs); free(tid);
+    return rc;
+}
+
+/* The single-threaded form of the layer. */
+int glq_oracle_linear(int64_t m, int64_t n, int bpw, const uint16_t *idx1, const void *idx2,
+                      const double *cb1, const double *cb2, float ws, float rs,
+                      const int8_t *s_in, const int8_t *s_out, const uint16_t *x, int x_is_bf16,
+                      int64_t B, double *y) {
+    return glq_oracle_linear_mt(m, n, bpw, idx1, idx2, cb1, cb2, ws, rs, s_in, s_out, x, x_is_bf16, B, y, 1);
 }

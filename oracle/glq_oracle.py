@@ -35,7 +35,7 @@ def build(force: bool = False) -> str:
     # explicit fmaf() of the residual reconstruction.
     subprocess.check_call([
         "gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
-        "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        "-shared", "-fPIC", "-pthread", "-o", tmp, _SRC, "-lm"])
     os.replace(tmp, _LIB)
     return _LIB
 
@@ -69,6 +69,10 @@ def _load():
     lib.glq_oracle_linear.argtypes = [
         c_i64, c_i64, c_int, vp, vp, vp, vp, ctypes.c_float, ctypes.c_float,
         vp, vp, vp, c_int, c_i64, vp]
+    lib.glq_oracle_linear_mt.restype = c_int
+    lib.glq_oracle_linear_mt.argtypes = [
+        c_i64, c_i64, c_int, vp, vp, vp, vp, ctypes.c_float, ctypes.c_float,
+        vp, vp, vp, c_int, c_i64, vp, c_int]
     _lib = lib
     return lib
 
@@ -181,11 +185,23 @@ def decode_rows(m, n, bpw, idx1, idx2, ws, rs, r0=0, r1=None, cb2=None) -> np.nd
     return w
 
 
-def linear(m, n, bpw, idx1, idx2, ws, rs, s_in, s_out, x_bits, x_is_bf16, cb2=None) -> np.ndarray:
+def default_threads() -> int:
+    """Host threads the oracle uses when asked for all of them."""
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:
+        return max(1, os.cpu_count() or 1)
+
+
+def linear(m, n, bpw, idx1, idx2, ws, rs, s_in, s_out, x_bits, x_is_bf16, cb2=None,
+           threads: int = 1) -> np.ndarray:
     """y[B][m] (float64) = S_out . H_m . W^ . H_n . (S_in . x).
 
     x_bits: uint16 [B][n] holding fp16 (x_is_bf16 False) or bf16 bit patterns.
+    threads: POSIX threads the rows of W^ xr are split over (0: every host
+    core); the result does not depend on it.
     """
+    threads = default_threads() if threads == 0 else int(threads)
     idx1, idx2 = _check_idx(m, n, bpw, idx1, idx2)
     x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16).reshape(-1, n)
     B = x_bits.shape[0]
@@ -194,9 +210,9 @@ def linear(m, n, bpw, idx1, idx2, ws, rs, s_in, s_out, x_bits, x_is_bf16, cb2=No
     cb1 = e8_codebook()
     cb2 = _residual_table(bpw, cb2)
     y = np.zeros((B, m), dtype=np.float64)
-    rc = _load().glq_oracle_linear(m, n, bpw, _ptr(idx1), _ptr(idx2), _ptr(cb1), _ptr(cb2),
-                                   float(ws), float(rs), _ptr(s_in), _ptr(s_out),
-                                   _ptr(x_bits), int(bool(x_is_bf16)), B, _ptr(y))
+    rc = _load().glq_oracle_linear_mt(m, n, bpw, _ptr(idx1), _ptr(idx2), _ptr(cb1), _ptr(cb2),
+                                      float(ws), float(rs), _ptr(s_in), _ptr(s_out),
+                                      _ptr(x_bits), int(bool(x_is_bf16)), B, _ptr(y), threads)
     if rc != 0:
         raise ValueError("oracle linear rejected its arguments")
     return y

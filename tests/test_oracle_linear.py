@@ -178,3 +178,16 @@ def test_two_bpw_rate():
         L = gi.make_layer(0, 0, m, n, 2)
         assert L.idx2 is None
         assert L.idx1.nbytes * 8 == 2 * m * n
+
+
+@pytest.mark.parametrize("m,n,bpw,B,threads", [(37, 64, 4, 3, 4), (200, 136, 3, 2, 7), (8, 8, 2, 1, 16)])
+def test_threaded_oracle_is_bitwise_single_threaded(m, n, bpw, B, threads):
+    """The rows of W^ xr dealt out to POSIX threads give the same bits as the
+    single-threaded loop (each output element is computed by the same code);
+    more threads than rows are capped."""
+    L = gi.make_layer(m + n + bpw, 4, m, n, bpw)
+    xb = gi.make_x(m + n + bpw, 4, B, n, "bf16")
+    args = (m, n, bpw, L.idx1, L.idx2, L.weight_scale, L.resid_scale, L.s_in, L.s_out, xb, True)
+    y1 = orc.linear(*args, cb2=L.cb2_f16)
+    yt = orc.linear(*args, cb2=L.cb2_f16, threads=threads)
+    assert np.array_equal(y1, yt)
