@@ -97,9 +97,9 @@ struct DecodeCfg {
     size_t spart_off = 0;  // shared-memory offset of the cluster partial sums
 };
 
-// max_cps bounds the chunks per split (callers with a small partial-sum
-// buffer); x and y decide the fused paths' alignment condition.
-DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y_dtype, int max_cps = 1 << 30);
+// max_splits: at most this many K splits (callers whose partial-sum buffer
+// is small); x and y decide the fused paths' alignment condition.
+DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y_dtype, int max_splits = 1 << 30);
 
 // (input RHT ->) codebook GEMV (-> output RHT) for nb <= 16 tokens, in the
 // buffers of `w`.

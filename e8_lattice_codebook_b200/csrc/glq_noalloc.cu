@@ -12,7 +12,8 @@
 //
 // The kernels are the ones glq_linear launches (input RHT, codebook GEMV,
 // output RHT); only the workspace pointers differ, and the split-K plan is
-// narrowed, if needed, so that the partial sums fit the array.
+// narrowed, when its partial sums would not fit the array, to a split
+// count whose partial sums do.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -27,7 +28,10 @@
 // GEMV, the per-band counters and the split-K partial sums of one call.
 // Every GPU that loads the library holds it until the process exits.  Calls
 // share it: two calls whose kernels overlap on the GPU (different streams,
-// or different layers without ordering) race on it.
+// or different layers without ordering) race on it.  A call also uses the
+// layer's own device words (its error flag and the output-block counters of
+// the fused output transform), so calls on one layer must not overlap on
+// the GPU whichever entry point they use.
 static __device__ __align__(256) unsigned char g_glq_noalloc_scratch[GLQ_NOALLOC_SCRATCH_BYTES];
 
 namespace {
@@ -97,12 +101,21 @@ extern "C" glq_status glq_linear_noalloc(glq_layer L, const void *x_dev, glq_dty
         if (fixed > GLQ_NOALLOC_SCRATCH_BYTES) {
             st = GLQ_ERR_SHAPE;  // the activations and outputs alone do not fit
         } else {
-            // bound the split-K plan so that its partial sums fit (one split
-            // needs none: the GEMV then writes z directly)
+            // glq_linear's plan, unless its partial sums would not fit: only
+            // a split plan without the cluster reduction keeps them in global
+            // memory (one split writes z directly; the cluster reduction adds
+            // them in distributed shared memory).  Then the split count is
+            // bounded by the room left.
             const size_t room = GLQ_NOALLOC_SCRATCH_BYTES - fixed;
-            const int max_splits = (int)std::max<size_t>(1, std::min<size_t>(room / per_split, 1u << 30));
-            cfg = glq::decode_config(L, (int)B, x_dev, y_dev, (int)y_dtype, max_splits);
-            if (cfg.plan.splits > 1 && (size_t)cfg.plan.splits * per_split > room) st = GLQ_ERR_SHAPE;
+            auto global_partials = [&](const glq::DecodeCfg &c) {
+                return c.plan.splits > 1 && c.clu == 0 ? (size_t)c.plan.splits * per_split : (size_t)0;
+            };
+            cfg = glq::decode_config(L, (int)B, x_dev, y_dev, (int)y_dtype);
+            if (global_partials(cfg) > room) {
+                const int max_splits = (int)std::max<size_t>(1, std::min<size_t>(room / per_split, 1u << 30));
+                cfg = glq::decode_config(L, (int)B, x_dev, y_dev, (int)y_dtype, max_splits);
+                if (global_partials(cfg) > room) st = GLQ_ERR_SHAPE;
+            }
         }
     }
     if (st == GLQ_OK) {

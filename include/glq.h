@@ -274,8 +274,13 @@ GLQ_API glq_status glq_prefill_replay(glq_layer layer, int64_t B, void *stream);
  * (cudaGetSymbolAddress); make that first call before any stream capture.
  * Calls share the array and it keeps the last call's contents: two calls
  * whose work overlaps on the GPU (other streams, unordered layers) race.
- * Results equal glq_linear's up to the order of fp32 sums (the split-K
- * plan is narrowed when its partial sums would not fit the array).
+ * A call also writes the layer's own device words (error flag, output-block
+ * counters), so calls on one layer must not overlap on the GPU whichever
+ * entry point (glq_linear or this one) they use.
+ * Results equal glq_linear's, except when glq_linear's split-K partial
+ * sums would not fit the array: then the split count is narrowed (possibly
+ * to a plan without the fused input transform), and the results agree
+ * within the parity bound instead of bitwise.
  * Errors: GLQ_ERR_INVALID_ARG, GLQ_ERR_DTYPE, GLQ_ERR_SHAPE (B > 16, or a
  *   layer whose activations plus one split of partial sums exceed the
  *   array), GLQ_ERR_CUDA.  Asynchronous.
