@@ -29,7 +29,7 @@ GLQ_F16, GLQ_BF16, GLQ_F32 = 0, 1, 2
 STATUS = {
     0: "GLQ_OK", 1: "GLQ_ERR_INVALID_ARG", 2: "GLQ_ERR_SHAPE", 3: "GLQ_ERR_DTYPE",
     4: "GLQ_ERR_BPW", 5: "GLQ_ERR_NO_CODEBOOK", 6: "GLQ_ERR_OOM", 7: "GLQ_ERR_CUDA",
-    8: "GLQ_ERR_DEVICE_CHECK", 9: "GLQ_ERR_TIMEOUT", 10: "GLQ_ERR_UNSUPPORTED",
+    8: "GLQ_ERR_DEVICE_CHECK", 9: "GLQ_ERR_TIMEOUT", 10: "GLQ_ERR_UNSUPPORTED", 11: "GLQ_ERR_CAPTURE",
 }
 
 # every symbol include/glq.h declares
@@ -39,6 +39,7 @@ EXPORTS = (
     "glq_linear", "glq_dequant_reference", "glq_rht_input", "glq_rht_output",
     "glq_layer_check", "glq_layer_info", "glq_gemv_replay", "glq_linear_noalloc", "glq_decode_plan",
     "glq_prefill_replay", "glq_layer_set_fusion", "glq_layer_set_prefill_reconstruct",
+    "glq_workspace_info", "glq_workspace_release",
 )
 
 
@@ -75,6 +76,8 @@ _SIGNATURES = {
                          ctypes.POINTER(_i32), ctypes.POINTER(_i32)], ctypes.c_int),
     "glq_layer_info": ([_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i32),
                         ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
+    "glq_workspace_info": ([_i32, ctypes.POINTER(ctypes.c_size_t)], ctypes.c_int),
+    "glq_workspace_release": ([_i32], ctypes.c_int),
 }
 
 _lib = None
@@ -210,6 +213,17 @@ def glq_decode_plan(handle, B: int) -> dict:
     vals = [_i32() for _ in range(5)]
     _ok(_L().glq_decode_plan(handle, int(B), *[ctypes.byref(v) for v in vals]), "glq_decode_plan")
     return dict(zip(("warps", "bands", "splits", "cluster", "fused_input"), (v.value for v in vals)))
+
+
+def glq_workspace_info(device: int) -> int:
+    """Bytes of the device's shared workspace (every layer's calls on it use it)."""
+    nb = ctypes.c_size_t()
+    _ok(_L().glq_workspace_info(int(device), ctypes.byref(nb)), "glq_workspace_info")
+    return nb.value
+
+
+def glq_workspace_release(device: int) -> None:
+    _ok(_L().glq_workspace_release(int(device)), "glq_workspace_release")
 
 
 def glq_layer_info(handle):

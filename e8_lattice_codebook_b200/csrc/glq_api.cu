@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -78,87 +79,130 @@ glq_status dmalloc(T **p, size_t bytes, size_t *total) {
     return GLQ_OK;
 }
 
-void free_workspace(glq_layer L) {
-    cudaFree(L->wsp.xq);
-    cudaFree(L->wsp.xh);
-    cudaFree(L->wsp.info);
-    cudaFree(L->wsp.part);
-    cudaFree(L->wsp.z);
-    L->wsp.xq = nullptr;
-    L->wsp.xh = nullptr;
-    L->wsp.info = nullptr;
-    L->wsp.part = nullptr;
-    L->wsp.z = nullptr;
-    L->cap_rows = 0;
-}
-
-void free_prefill_ws(glq_layer L) {
-    cudaFree(L->pws.xh);
-    cudaFree(L->pws.info);
-    cudaFree(L->pws.z);
-    cudaFree(L->pws.w16);
-    L->pws = glq_prefill_ws{};
-}
-
 void free_layer(glq_layer L) {
     if (!L) return;
-    free_prefill_ws(L);
     cudaFree(L->d_blk_cnt);
     cudaFree(L->d_idx1);
     cudaFree(L->d_idx2);
     cudaFree(L->d_sin);
     cudaFree(L->d_sout);
     cudaFree(L->d_err);
-    cudaFree(L->wsp.cnt);
-    free_workspace(L);
+    cudaFree(L->d_cnt);
     delete L;
 }
 
-glq_status grow_workspace(glq_layer L, int64_t rows) {
-    if (rows <= L->cap_rows) return GLQ_OK;
-    cudaError_t e = cudaDeviceSynchronize();
-    if (e != cudaSuccess) return GLQ_ERR_CUDA;
-    free_workspace(L);
-    glq_status st = dmalloc(&L->wsp.xq, (size_t)rows * L->n_pad * 2, nullptr);
-    if (st == GLQ_OK && L->bpw == 3) st = dmalloc(&L->wsp.xh, (size_t)rows * L->n_pad * sizeof(__half), nullptr);
-    if (st == GLQ_OK) st = dmalloc(&L->wsp.info, (size_t)rows * sizeof(glq_rowinfo), nullptr);
-    int max_splits = 1;
-    for (int nb = 1; nb <= rows; ++nb) max_splits = std::max(max_splits, glq::max_decode_splits(L, nb));
-    if (st == GLQ_OK && max_splits > 1)
-        st = dmalloc(&L->wsp.part, (size_t)max_splits * rows * L->m_pad * sizeof(double), nullptr);
-    if (st == GLQ_OK) st = dmalloc(&L->wsp.z, (size_t)rows * L->m_pad * sizeof(float), nullptr);
-    if (st != GLQ_OK) {
-        free_workspace(L);
-        return st;
+// ---------------------------------------------------------------------------
+// The device's shared workspace: every transient buffer of glq_linear, for
+// all layers on the device.  Each buffer grows to the largest size a call or
+// a reservation has asked for; growth synchronises the device and frees the
+// previous buffer (so work captured in a CUDA graph before a growth must not
+// be replayed after it: reserve first).  Calls that use it must be serialised
+// on the GPU (one stream, or explicit ordering).
+// ---------------------------------------------------------------------------
+
+enum WsBuf { WS_XQ, WS_XH, WS_INFO, WS_PART, WS_Z, WS_PXH, WS_PINFO, WS_PZ, WS_W16, WS_COUNT };
+
+struct DeviceWs {
+    void *buf[WS_COUNT] = {};
+    size_t cap[WS_COUNT] = {};
+};
+
+constexpr int WS_MAX_DEVICES = 128;
+std::mutex g_ws_mu;
+DeviceWs g_ws[WS_MAX_DEVICES];
+
+struct WsNeed {
+    size_t b[WS_COUNT] = {};
+};
+
+size_t ws_bytes_locked(int dev) {
+    size_t t = 0;
+    for (int i = 0; i < WS_COUNT; ++i) t += g_ws[dev].cap[i];
+    return t;
+}
+
+// Makes every buffer of `dev` (the current device) at least `need` bytes and
+// returns their addresses.  `s` is the stream of the call: if it is being
+// captured and a buffer must grow, nothing is allocated (GLQ_ERR_CAPTURE).
+glq_status ws_acquire(int dev, const WsNeed &need, cudaStream_t s, void *out[WS_COUNT]) {
+    if (dev < 0 || dev >= WS_MAX_DEVICES) return GLQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_ws_mu);
+    DeviceWs &w = g_ws[dev];
+    bool grow = false;
+    for (int i = 0; i < WS_COUNT; ++i) grow |= need.b[i] > w.cap[i];
+    if (grow) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) {
+            cudaGetLastError();
+            return GLQ_ERR_CUDA;
+        }
+        if (cs != cudaStreamCaptureStatusNone) return GLQ_ERR_CAPTURE;
+        if (cudaDeviceSynchronize() != cudaSuccess) {
+            cudaGetLastError();
+            return GLQ_ERR_CUDA;
+        }
+        for (int i = 0; i < WS_COUNT; ++i) {
+            if (need.b[i] <= w.cap[i]) continue;
+            cudaFree(w.buf[i]);
+            w.buf[i] = nullptr;
+            w.cap[i] = 0;
+            const size_t bytes = (need.b[i] + 255) & ~(size_t)255;
+            if (cudaMalloc(&w.buf[i], bytes) != cudaSuccess) {
+                cudaGetLastError();
+                w.buf[i] = nullptr;
+                return GLQ_ERR_OOM;
+            }
+            w.cap[i] = bytes;
+        }
     }
-    L->cap_rows = rows;
+    for (int i = 0; i < WS_COUNT; ++i) out[i] = w.buf[i];
     return GLQ_OK;
 }
 
-glq_status grow_prefill_ws(glq_layer L, int64_t rows, bool mat, int ksplit) {
-    // z holds ksplit slices of [rows][m_pad]
-    const int64_t zrows = rows * ksplit;
-    if (rows <= L->pws.cap && zrows <= L->pws.zcap && (!mat || L->pws.w16)) return GLQ_OK;
-    if (cudaDeviceSynchronize() != cudaSuccess) return GLQ_ERR_CUDA;
-    if (rows <= L->pws.cap && zrows <= L->pws.zcap) {  // only the reconstructed W is missing
-        return dmalloc(&L->pws.w16, (size_t)L->m_pad * L->n_pad * sizeof(__half), nullptr);
-    }
-    rows = std::max(rows, L->pws.cap);
-    const bool had_w16 = L->pws.w16 != nullptr;
-    free_prefill_ws(L);
-    glq_status st = dmalloc(&L->pws.xh, (size_t)rows * L->n_pad * sizeof(__half), nullptr);
-    if (st == GLQ_OK) st = dmalloc(&L->pws.info, (size_t)rows * sizeof(glq_rowinfo), nullptr);
-    const int64_t zcap = std::max(zrows, rows);
-    if (st == GLQ_OK) st = dmalloc(&L->pws.z, (size_t)zcap * L->m_pad * sizeof(float), nullptr);
-    if (st == GLQ_OK && (mat || had_w16))
-        st = dmalloc(&L->pws.w16, (size_t)L->m_pad * L->n_pad * sizeof(__half), nullptr);
-    if (st != GLQ_OK) {
-        free_prefill_ws(L);
-        return st;
-    }
-    L->pws.cap = rows;
-    L->pws.zcap = zcap;
-    return GLQ_OK;
+// Decode buffers for calls of up to `rows` (<= 16) tokens on layer L.
+void decode_need(glq_layer L, int64_t rows, WsNeed &n) {
+    if (rows <= 0) return;
+    rows = std::min<int64_t>(rows, GLQ_DECODE_MAX_B);
+    int max_splits = 1;
+    for (int nb = 1; nb <= rows; ++nb) max_splits = std::max(max_splits, glq::max_decode_splits(L, nb));
+    n.b[WS_XQ] = std::max(n.b[WS_XQ], (size_t)rows * L->n_pad * 2);
+    if (L->bpw == 3) n.b[WS_XH] = std::max(n.b[WS_XH], (size_t)rows * L->n_pad * sizeof(__half));
+    n.b[WS_INFO] = std::max(n.b[WS_INFO], (size_t)rows * sizeof(glq_rowinfo));
+    if (max_splits > 1)
+        n.b[WS_PART] = std::max(n.b[WS_PART], (size_t)max_splits * rows * L->m_pad * sizeof(double));
+    n.b[WS_Z] = std::max(n.b[WS_Z], (size_t)rows * L->m_pad * sizeof(float));
+}
+
+int choose_ksplit(glq_layer L, int64_t B, int tiles);
+int prefill_tiles(glq_layer L, int64_t B);
+
+// Tensor-core buffers for one call of exactly B (> 16) tokens on layer L.
+void prefill_need(glq_layer L, int64_t B, WsNeed &n) {
+    const int ks = choose_ksplit(L, B, prefill_tiles(L, B));
+    n.b[WS_PXH] = std::max(n.b[WS_PXH], (size_t)B * L->n_pad * sizeof(__half));
+    n.b[WS_PINFO] = std::max(n.b[WS_PINFO], (size_t)B * sizeof(glq_rowinfo));
+    n.b[WS_PZ] = std::max(n.b[WS_PZ], (size_t)ks * B * L->m_pad * sizeof(float));
+    if (B >= L->prefill_mat_min_b) n.b[WS_W16] = std::max(n.b[WS_W16], (size_t)L->m_pad * L->n_pad * sizeof(__half));
+}
+
+glq_workspace decode_view(glq_layer L, void *const buf[WS_COUNT]) {
+    glq_workspace w;
+    w.xq = static_cast<uint8_t *>(buf[WS_XQ]);
+    w.xh = static_cast<__half *>(buf[WS_XH]);
+    w.info = static_cast<glq_rowinfo *>(buf[WS_INFO]);
+    w.part = static_cast<double *>(buf[WS_PART]);
+    w.z = static_cast<float *>(buf[WS_Z]);
+    w.cnt = L->d_cnt;
+    return w;
+}
+
+glq_prefill_ws prefill_view(void *const buf[WS_COUNT]) {
+    glq_prefill_ws w;
+    w.xh = static_cast<__half *>(buf[WS_PXH]);
+    w.info = static_cast<glq_rowinfo *>(buf[WS_PINFO]);
+    w.z = static_cast<float *>(buf[WS_PZ]);
+    w.w16 = static_cast<__half *>(buf[WS_W16]);
+    return w;
 }
 
 // TMA descriptor of the fp16 activations [B][n_pad]: boxes of 64 columns x
@@ -218,7 +262,13 @@ int choose_ksplit(glq_layer L, int64_t B, int tiles) {
     return best;
 }
 
-glq::PrefillParams prefill_params(glq_layer L, int64_t B) {
+int prefill_tiles(glq_layer L, int64_t B) {
+    const int tr = glq::prefill_tile_rows();
+    const int tiles_m = (int)((L->m_pad + tr - 1) / tr);
+    return tiles_m * (int)((B + glq::prefill_tile_tokens() - 1) / glq::prefill_tile_tokens());
+}
+
+glq::PrefillParams prefill_params(glq_layer L, const glq_prefill_ws &ws, int64_t B) {
     glq::PrefillParams pp{};
     pp.idx1 = L->d_idx1;
     pp.idx2 = L->d_idx2;
@@ -227,9 +277,9 @@ glq::PrefillParams prefill_params(glq_layer L, int64_t B) {
     pp.bpw = L->bpw;
     const __half2 rs2 = __floats2half2_rn(L->rs, L->rs);
     pp.rs_h2 = *reinterpret_cast<const uint32_t *>(&rs2);
-    pp.info = L->pws.info;
+    pp.info = ws.info;
     pp.ws = L->ws;
-    pp.z = L->pws.z;
+    pp.z = ws.z;
     pp.B = (int)B;
     pp.m_pad = (int)L->m_pad;
     pp.KC = L->KC;
@@ -249,11 +299,12 @@ glq::PrefillParams prefill_params(glq_layer L, int64_t B) {
 
 // The tcgen05 GEMM of the tensor-core path on the layer's prefill
 // workspace: z[0..B) from xh[0..B); mat: against the reconstructed W16.
-cudaError_t launch_prefill_gemm(glq_layer L, int64_t B, bool mat, cudaStream_t s, bool pdl) {
+cudaError_t launch_prefill_gemm(glq_layer L, const glq_prefill_ws &ws, int64_t B, bool mat, cudaStream_t s,
+                                bool pdl) {
     CUtensorMap xmap, wmap;
-    if (!encode_x_map(&xmap, L->pws.xh, L->n_pad, B)) return cudaErrorInvalidValue;
-    if (mat && !encode_w_map(&wmap, L->pws.w16, L->n_pad, L->m_pad)) return cudaErrorInvalidValue;
-    const glq::PrefillParams pp = prefill_params(L, B);
+    if (!encode_x_map(&xmap, ws.xh, L->n_pad, B)) return cudaErrorInvalidValue;
+    if (mat && !encode_w_map(&wmap, ws.w16, L->n_pad, L->m_pad)) return cudaErrorInvalidValue;
+    const glq::PrefillParams pp = prefill_params(L, ws, B);
     const int grid = 2 * std::min(pp.ntiles, L->num_sms / 2);  // CTA pairs
     return glq::launch_prefill(pp, xmap, mat ? &wmap : nullptr, grid, s, pdl);
 }
@@ -281,9 +332,13 @@ glq::RowsParams rows_params(const glq_hblocks &hb, int len, int len_pad, const u
 // clustered ones.
 glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_dtype, int64_t B, cudaStream_t s) {
     const bool mat = B >= L->prefill_mat_min_b;
-    const int ksplit = prefill_params(L, B).ksplit;
-    glq_status st = grow_prefill_ws(L, B, mat, ksplit);
+    WsNeed need;
+    prefill_need(L, B, need);
+    void *buf[WS_COUNT];
+    glq_status st = ws_acquire(L->device, need, s, buf);
     if (st != GLQ_OK) return st;
+    const glq_prefill_ws ws = prefill_view(buf);
+    const int ksplit = prefill_params(L, ws, B).ksplit;
     const bool rows_in = glq::rht_rows_supported((int)L->n_pad), rows_out = glq::rht_rows_supported((int)L->m);
     for (int64_t b0 = 0; b0 < B;) {
         const int nb = (int)std::min<int64_t>(B - b0, 65535);  // grid limit of the clustered kernels
@@ -291,8 +346,8 @@ glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_d
             glq::RowsParams r = rows_params(L->hb_n, (int)L->n, (int)L->n_pad, L->d_sin);
             r.x = static_cast<const char *>(x) + (size_t)b0 * L->n * 2;
             r.x_bf16 = x_bf16 ? 1 : 0;
-            r.xh = L->pws.xh + (size_t)b0 * L->n_pad;
-            r.info = L->pws.info + b0;
+            r.xh = ws.xh + (size_t)b0 * L->n_pad;
+            r.info = ws.info + b0;
             if (glq::launch_rht_rows(r, true, nb, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
         } else {
             glq::RhtInParams pin{};
@@ -303,16 +358,16 @@ glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_d
             pin.B = nb;
             pin.sign_bits = L->d_sin;
             pin.plan = L->plan_n;
-            pin.xh = L->pws.xh + (size_t)b0 * L->n_pad;
-            pin.info = L->pws.info + b0;
+            pin.xh = ws.xh + (size_t)b0 * L->n_pad;
+            pin.info = ws.info + b0;
             pin.xh_only = 1;
             if (glq::launch_rht_in(pin, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
         }
         b0 += nb;
     }
-    if (mat && glq::launch_wmat(prefill_params(L, B), L->pws.w16, (int)L->n_pad, L->num_sms, s, true) != cudaSuccess)
+    if (mat && glq::launch_wmat(prefill_params(L, ws, B), ws.w16, (int)L->n_pad, L->num_sms, s, true) != cudaSuccess)
         return GLQ_ERR_CUDA;
-    if (launch_prefill_gemm(L, B, mat, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+    if (launch_prefill_gemm(L, ws, B, mat, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
     L->last_prefill_B = B;
     L->last_prefill_mat = mat;
     for (int64_t b0 = 0; b0 < B;) {
@@ -320,7 +375,7 @@ glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_d
         void *yb = static_cast<char *>(y) + (size_t)b0 * L->m * (y_dtype == GLQ_F32 ? 4 : 2);
         if (rows_out) {
             glq::RowsParams r = rows_params(L->hb_m, (int)L->m, (int)L->m, L->d_sout);
-            r.z = L->pws.z + (size_t)b0 * L->m_pad;
+            r.z = ws.z + (size_t)b0 * L->m_pad;
             r.z_ld = (int)L->m_pad;
             r.zsplits = ksplit;
             r.zs = (size_t)B * L->m_pad;
@@ -331,7 +386,7 @@ glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_d
             glq::RhtOutParams pout{};
             pout.m = (int)L->m;
             pout.B = nb;
-            pout.z = L->pws.z + (size_t)b0 * L->m_pad;
+            pout.z = ws.z + (size_t)b0 * L->m_pad;
             pout.z_ld = (int)L->m_pad;
             pout.sign_bits = L->d_sout;
             pout.plan = L->plan_m;
@@ -565,6 +620,7 @@ const char *glq_status_str(glq_status s) {
         case GLQ_ERR_DEVICE_CHECK: return "GLQ_ERR_DEVICE_CHECK";
         case GLQ_ERR_TIMEOUT: return "GLQ_ERR_TIMEOUT";
         case GLQ_ERR_UNSUPPORTED: return "GLQ_ERR_UNSUPPORTED";
+        case GLQ_ERR_CAPTURE: return "GLQ_ERR_CAPTURE";
     }
     return "GLQ_ERR_UNKNOWN";
 }
@@ -746,7 +802,7 @@ glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *i
     if (st == GLQ_OK) st = dmalloc(&L->d_sin, sin_bits.size() * 4, &total);
     if (st == GLQ_OK) st = dmalloc(&L->d_sout, sout_bits.size() * 4, &total);
     if (st == GLQ_OK) st = dmalloc(&L->d_err, sizeof(unsigned), &total);
-    if (st == GLQ_OK) st = dmalloc(&L->wsp.cnt, (size_t)max_bands * sizeof(unsigned), &total);
+    if (st == GLQ_OK) st = dmalloc(&L->d_cnt, (size_t)max_bands * sizeof(unsigned), &total);
     if (st == GLQ_OK) st = dmalloc(&L->d_blk_cnt, GLQ_MAX_BLOCKS * sizeof(unsigned), &total);
     if (st == GLQ_OK) {
         bool ok = cudaMemcpy(L->d_idx1, s1.data(), L->idx1_bytes, cudaMemcpyHostToDevice) == cudaSuccess;
@@ -759,7 +815,7 @@ glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *i
         ok = ok && cudaMemcpy(L->d_sout, sout_bits.data(), sout_bits.size() * 4, cudaMemcpyHostToDevice) ==
                        cudaSuccess;
         ok = ok && cudaMemset(L->d_err, 0, sizeof(unsigned)) == cudaSuccess;
-        ok = ok && cudaMemset(L->wsp.cnt, 0, (size_t)max_bands * sizeof(unsigned)) == cudaSuccess;
+        ok = ok && cudaMemset(L->d_cnt, 0, (size_t)max_bands * sizeof(unsigned)) == cudaSuccess;
         ok = ok && cudaMemset(L->d_blk_cnt, 0, GLQ_MAX_BLOCKS * sizeof(unsigned)) == cudaSuccess;
         if (!ok) st = GLQ_ERR_CUDA;
     }
@@ -784,7 +840,39 @@ glq_status glq_layer_reserve(glq_layer layer, int64_t max_B) {
     if (!layer) return GLQ_ERR_INVALID_ARG;
     if (max_B < 0) return GLQ_ERR_SHAPE;
     DeviceGuard guard(layer->device);
-    return grow_workspace(layer, std::min<int64_t>(std::max<int64_t>(max_B, 1), GLQ_DECODE_MAX_B));
+    WsNeed need;
+    decode_need(layer, std::max<int64_t>(max_B, 1), need);
+    // every tensor-core batch up to max_B (the K-split count, and with it
+    // the partial-sum slices, depends on the batch); past 65536 tokens the
+    // output has far more tiles than CTA pairs and the largest batch decides
+    for (int64_t B = GLQ_DECODE_MAX_B + 1; B <= std::min<int64_t>(max_B, 65536); ++B) prefill_need(layer, B, need);
+    if (max_B > 65536) prefill_need(layer, max_B, need);
+    void *buf[WS_COUNT];
+    return ws_acquire(layer->device, need, 0, buf);
+}
+
+glq_status glq_workspace_info(int32_t device, size_t *bytes) {
+    if (!bytes || device < 0 || device >= WS_MAX_DEVICES) return GLQ_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_ws_mu);
+    *bytes = ws_bytes_locked(device);
+    return GLQ_OK;
+}
+
+glq_status glq_workspace_release(int32_t device) {
+    if (device < 0 || device >= WS_MAX_DEVICES) return GLQ_ERR_INVALID_ARG;
+    DeviceGuard guard(device);
+    std::lock_guard<std::mutex> lock(g_ws_mu);
+    if (cudaDeviceSynchronize() != cudaSuccess) {
+        cudaGetLastError();
+        return GLQ_ERR_CUDA;
+    }
+    DeviceWs &w = g_ws[device];
+    for (int i = 0; i < WS_COUNT; ++i) {
+        cudaFree(w.buf[i]);
+        w.buf[i] = nullptr;
+        w.cap[i] = 0;
+    }
+    return GLQ_OK;
 }
 
 glq_status glq_decode_plan(glq_layer layer, int64_t B, int32_t *warps, int32_t *bands, int32_t *splits,
@@ -838,15 +926,19 @@ glq_status glq_linear(glq_layer L, const void *x_dev, glq_dtype x_dtype, void *y
     DeviceGuard guard(L->device);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (B > GLQ_DECODE_MAX_B) return run_prefill(L, x_dev, x_dtype == GLQ_BF16, y_dev, (int)y_dtype, B, s);
-    glq_status st = grow_workspace(L, std::min<int64_t>(B, GLQ_DECODE_MAX_B));
+    WsNeed need;
+    decode_need(L, B, need);
+    void *buf[WS_COUNT];
+    glq_status st = ws_acquire(L->device, need, s, buf);
     if (st != GLQ_OK) return st;
+    const glq_workspace wsp = decode_view(L, buf);
     const size_t xe = 2, ye = y_dtype == GLQ_F32 ? 4 : 2;
     for (int64_t b0 = 0; b0 < B; b0 += GLQ_DECODE_MAX_B) {
         const int nb = (int)std::min<int64_t>(GLQ_DECODE_MAX_B, B - b0);
         const void *x = static_cast<const char *>(x_dev) + (size_t)b0 * L->n * xe;
         void *y = static_cast<char *>(y_dev) + (size_t)b0 * L->m * ye;
         const glq::DecodeCfg cfg = glq::decode_config(L, nb, x, y, (int)y_dtype);
-        if (glq::run_decode(L, L->wsp, cfg, x, x_dtype == GLQ_BF16, y, (int)y_dtype, nb, s) != cudaSuccess) {
+        if (glq::run_decode(L, wsp, cfg, x, x_dtype == GLQ_BF16, y, (int)y_dtype, nb, s) != cudaSuccess) {
             cudaGetLastError();
             return GLQ_ERR_CUDA;
         }
@@ -940,8 +1032,11 @@ glq_status glq_gemv_replay(glq_layer L, int64_t B, void *stream) {
     if (B < 1 || B > L->last_B) return GLQ_ERR_SHAPE;
     DeviceGuard guard(L->device);
     const glq::DecodeCfg cfg = glq::decode_config(L, (int)B, L->last_x, L->last_y, L->last_y_dtype);
-    glq::GemvParams pg = glq::gemv_params(L, L->wsp, cfg, (int)B, L->last_x, L->last_x_bf16 != 0, L->last_y,
-                                          L->last_y_dtype);
+    void *buf[WS_COUNT];
+    glq_status st = ws_acquire(L->device, WsNeed{}, static_cast<cudaStream_t>(stream), buf);
+    if (st != GLQ_OK) return st;
+    glq::GemvParams pg = glq::gemv_params(L, decode_view(L, buf), cfg, (int)B, L->last_x, L->last_x_bf16 != 0,
+                                          L->last_y, L->last_y_dtype);
     return glq::launch_gemv(pg, L->bpw, cfg.plan.grid, static_cast<cudaStream_t>(stream), true, cfg.fin) ==
                    cudaSuccess
                ? GLQ_OK
@@ -952,7 +1047,11 @@ glq_status glq_prefill_replay(glq_layer L, int64_t B, void *stream) {
     if (!L) return GLQ_ERR_INVALID_ARG;
     if (B <= GLQ_DECODE_MAX_B || B > L->last_prefill_B) return GLQ_ERR_SHAPE;
     DeviceGuard guard(L->device);
-    return launch_prefill_gemm(L, B, L->last_prefill_mat, static_cast<cudaStream_t>(stream), false) == cudaSuccess
+    void *buf[WS_COUNT];
+    glq_status st = ws_acquire(L->device, WsNeed{}, static_cast<cudaStream_t>(stream), buf);
+    if (st != GLQ_OK) return st;
+    return launch_prefill_gemm(L, prefill_view(buf), B, L->last_prefill_mat, static_cast<cudaStream_t>(stream),
+                               false) == cudaSuccess
                ? GLQ_OK
                : GLQ_ERR_CUDA;
 }

@@ -25,16 +25,17 @@ struct glq_codebook_s {
     uint4 *d_table_f16 = nullptr; // fp16 codewords by folded code [2 nb - 1][8] (tensor-core path gathers)
 };
 
-// Device buffers of the tensor-core path (B > 16 tokens).
+// Device buffers one tensor-core call (B > 16 tokens) works in: a view of
+// the device's shared workspace.
 struct glq_prefill_ws {
-    int64_t cap = 0, zcap = 0;    // rows of xh / info, rows of z (all K-split slices)
-    __half *xh = nullptr;         // [cap][n_pad]
-    glq_rowinfo *info = nullptr;  // [cap]
-    float *z = nullptr;           // [zcap][m_pad]: K-split slices of [B][m_pad]
-    __half *w16 = nullptr;        // [m_pad][n_pad] reconstructed W (batches >= the materialise bound)
+    __half *xh = nullptr;         // [B][n_pad]
+    glq_rowinfo *info = nullptr;  // [B]
+    float *z = nullptr;           // [ksplit][B][m_pad]: K-split slices of [B][m_pad]
+    __half *w16 = nullptr;        // [m_pad][n_pad] reconstructed W (batches >= the reconstruct bound)
 };
 
-// Device buffers one decode call works in (B <= 16 tokens).
+// Device buffers one decode call works in (B <= 16 tokens): a view of the
+// device's shared workspace, except cnt, which the layer owns.
 struct glq_workspace {
     uint8_t *xq = nullptr;        // [B][n_pad * 2] activations, high / low bytes per group
     __half *xh = nullptr;         // [B][n_pad] fp16 activations (3 bpw only)
@@ -65,13 +66,12 @@ struct glq_layer_s {
     unsigned *d_err = nullptr;
     // GEMV work split for B <= 8 (plan[0]) and B <= 16 (plan[1])
     glq::GemvPlan plan[2]{};
-    // workspace (sized by glq_layer_reserve / on first use)
-    int64_t cap_rows = 0;
+    // the transient buffers live in the device's shared workspace (sized by
+    // glq_layer_reserve or on first use); the layer owns its band counters
+    unsigned *d_cnt = nullptr;   // [bands] split-K arrival counters, zero between calls
     int64_t last_B = 0;          // batch of the last decode slice (glq_gemv_replay)
     int64_t last_prefill_B = 0;  // batch of the last tensor-core call (glq_prefill_replay)
     bool last_prefill_mat = false;
-    glq_workspace wsp;
-    glq_prefill_ws pws;
     glq_hblocks hb_n, hb_m;
     unsigned *d_blk_cnt = nullptr;  // [GLQ_MAX_BLOCKS] output-block counters, zero between calls
     int fusion = -1;                // GLQ_FUSE_* bits, or -1: the library default (glq_layer_set_fusion)

@@ -29,10 +29,13 @@
  *   - input side: sign then H_n; output side: H_m then sign.
  *
  * Threading and ordering: every call that takes a cudaStream_t is
- * asynchronous and stream-ordered.  Calls on one layer must be serialised
- * (one stream, or explicit events): a layer owns one device workspace.
- * Handles are not thread-safe; distinct layers may be used concurrently on
- * distinct streams.  Every function returns a status and never throws.
+ * asynchronous and stream-ordered.  The transient device buffers of
+ * glq_linear (rotated activations, split-K partial sums, pre-rotation
+ * outputs, the reconstructed fp16 W of large batches) live in one workspace
+ * per device shared by all its layers, so the glq_linear calls of one device
+ * must be serialised on the GPU (one stream, or explicit events).  A layer
+ * itself owns only its indices, signs and a few counter words.  Handles are
+ * not thread-safe.  Every function returns a status and never throws.
  */
 #ifndef GLQ_B200_H
 #define GLQ_B200_H
@@ -61,7 +64,9 @@ typedef enum {
     GLQ_ERR_CUDA = 7,         /* a CUDA runtime call or launch failed */
     GLQ_ERR_DEVICE_CHECK = 8, /* a device-side check recorded a fault */
     GLQ_ERR_TIMEOUT = 9,      /* a bounded device-side wait gave up */
-    GLQ_ERR_UNSUPPORTED = 10  /* codebook contents the kernels cannot hold */
+    GLQ_ERR_UNSUPPORTED = 10, /* codebook contents the kernels cannot hold */
+    GLQ_ERR_CAPTURE = 11      /* the call needs a larger device workspace while its
+                                 stream is being captured: reserve first */
 } glq_status;
 
 typedef enum { GLQ_F16 = 0, GLQ_BF16 = 1, GLQ_F32 = 2 } glq_dtype;
@@ -137,13 +142,33 @@ GLQ_API glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uin
 GLQ_API glq_status glq_layer_destroy(glq_layer layer);
 
 /*
- * glq_layer_reserve -- size the layer's device workspace for batches up to
- * max_B so that later glq_linear calls with B <= max_B allocate nothing
- * (and may be captured in a CUDA graph).  glq_linear grows the workspace
- * on demand otherwise (a synchronous allocation).  Errors: GLQ_ERR_SHAPE,
+ * glq_layer_reserve -- grow the device's shared workspace so that every
+ * glq_linear call on this layer with B <= max_B (decode and tensor-core
+ * batches alike) finds its buffers already there: such calls then allocate
+ * nothing and never synchronise, so they may be captured in a CUDA graph.
+ * Reserve every layer first, then capture.  Without a reservation glq_linear
+ * grows the workspace on demand: that synchronises the device and frees the
+ * previous buffers, so graphs captured before a growth must not be replayed
+ * after it; a growth needed while the call's stream is being captured
+ * returns GLQ_ERR_CAPTURE instead.  Synchronous.  Errors: GLQ_ERR_SHAPE,
  * GLQ_ERR_OOM, GLQ_ERR_CUDA.
  */
 GLQ_API glq_status glq_layer_reserve(glq_layer layer, int64_t max_B);
+
+/*
+ * glq_workspace_info -- bytes of device memory the shared workspace of
+ * `device` holds (every layer's calls on that device use it).  Host only.
+ * Errors: GLQ_ERR_INVALID_ARG.
+ */
+GLQ_API glq_status glq_workspace_info(int32_t device, size_t *bytes);
+
+/*
+ * glq_workspace_release -- synchronise `device` and free its shared
+ * workspace; the next call that needs it allocates it again.  No captured
+ * graph that used it may be replayed afterwards.  Errors:
+ * GLQ_ERR_INVALID_ARG, GLQ_ERR_CUDA.
+ */
+GLQ_API glq_status glq_workspace_release(int32_t device);
 
 /*
  * glq_linear -- y = S_out . H_m . W^ . H_n . (S_in . x).
@@ -159,13 +184,20 @@ GLQ_API glq_status glq_layer_reserve(glq_layer layer, int64_t max_B);
  *   MMA with an on-chip codebook, with both transforms fused into the same
  *   launch when B times the largest Hadamard block is at most 32768 values
  *   (one kernel per call), else input RHT, GEMV and output RHT as three
- *   kernels (see glq_layer_set_fusion); B > 16 runs the tensor-core path
- *   (input RHT, tcgen05/TMEM GEMM with a dequantising producer, output RHT).
- *   The GEMV accumulates exactly in integers (fp64 across splits); the
- *   tensor-core path accumulates in fp32.
+ *   kernels (see glq_layer_set_fusion); B > 16 runs the tensor-core path:
+ *   input RHT, then, from 256 tokens (glq_layer_set_prefill_reconstruct),
+ *   one pass that reconstructs W = cb1 + rs cb2 as an fp16 matrix in the
+ *   device's shared workspace and a TMA-fed tcgen05/TMEM GEMM on it, below
+ *   that a tcgen05 GEMM whose producer warps rebuild each W tile in shared
+ *   memory (W never stored), then output RHT.  The GEMV accumulates exactly
+ *   in integers (fp64 across splits); the tensor-core path accumulates in
+ *   fp32.
+ * Workspace: the device's shared workspace (see glq_layer_reserve); a call
+ *   it already covers allocates nothing and does not synchronise.
  * Errors: GLQ_ERR_INVALID_ARG (null or misaligned pointer), GLQ_ERR_DTYPE,
- *   GLQ_ERR_SHAPE, GLQ_ERR_OOM (workspace growth), GLQ_ERR_CUDA (launch
- *   failure).  Asynchronous.
+ *   GLQ_ERR_SHAPE, GLQ_ERR_OOM (workspace growth), GLQ_ERR_CAPTURE (growth
+ *   needed during stream capture), GLQ_ERR_CUDA (launch failure).
+ *   Asynchronous.
  */
 GLQ_API glq_status glq_linear(glq_layer layer, const void *x_dev, glq_dtype x_dtype, void *y_dev,
                       glq_dtype y_dtype, int64_t B, void *stream);
@@ -199,9 +231,10 @@ GLQ_API glq_status glq_layer_set_fusion(glq_layer layer, int32_t flags);
 /*
  * glq_layer_set_prefill_reconstruct -- how tensor-core calls (B > 16) get
  * their weights.  Calls with B >= min_batch first reconstruct W = cb1 + rs
- * cb2 into an fp16 matrix of m_pad x n_pad (2 bytes per weight, a workspace
- * the layer keeps until it is destroyed) and run the TMA-fed tcgen05 GEMM on
- * it; smaller batches rebuild each W tile in shared memory inside the GEMM
+ * cb2 into an fp16 matrix of m_pad x n_pad (2 bytes per weight, in the
+ * device's shared workspace: one such matrix, of the largest layer that
+ * used it, per device) and run the TMA-fed tcgen05 GEMM on it; smaller
+ * batches rebuild each W tile in shared memory inside the GEMM
  * and never materialise W (the pages' design: "Inference kernels", glq 0.5.1
  * PyPI page).  Reconstructing once costs one pass over the indices, while the
  * fused producer repeats its codeword gathers for every 512 tokens, so large
@@ -233,8 +266,9 @@ GLQ_API glq_status glq_rht_output(glq_layer layer, const float *z_dev, void *y_d
 
 /*
  * glq_gemv_replay -- measurement entry point: re-launches only the codebook
- * GEMV of the most recent glq_linear call on this layer (same activations
- * already in the layer's workspace, batch B <= min(16, that call's B)),
+ * GEMV of the most recent glq_linear call on this layer (its activations
+ * are read from the device's shared workspace, so no other layer's call may
+ * come between; batch B <= min(16, that call's B)),
  * writing the same split-K partial sums.  Lets a caller time the GEMV kernel
  * alone with events on `stream`.  Like glq_linear, it launches the GEMV with
  * programmatic dependent launch, so back-to-back replays overlap one launch's
@@ -249,11 +283,13 @@ GLQ_API glq_status glq_gemv_replay(glq_layer layer, int64_t B, void *stream);
 /*
  * glq_prefill_replay -- measurement entry point: re-launches only the
  * tensor-core GEMM of the most recent glq_linear call with B > 16 on this
- * layer (its fp16 rotated activations are still in the layer's workspace),
- * for 16 < B <= that call's B, rewriting the same pre-rotation outputs z.
- * Lets a caller time the GEMM kernel alone with events on `stream`.  The
- * GEMM is the tensor-core path of "Inference kernels" on the glq 0.5.1 PyPI
- * page (matmul against codebook-reconstructed weights, W never stored).
+ * layer (its fp16 rotated activations, and its reconstructed W when that
+ * call reconstructed one, are read from the device's shared workspace, so
+ * no other layer's tensor-core call may come between), for 16 < B <= that
+ * call's B, rewriting the same pre-rotation outputs z.  Lets a caller time
+ * the GEMM kernel alone with events on `stream`.  The GEMM is the
+ * tensor-core path of "Inference kernels" on the glq 0.5.1 PyPI page
+ * (matmul against codebook-reconstructed weights).
  * Errors: GLQ_ERR_INVALID_ARG, GLQ_ERR_SHAPE (B out of range or no previous
  * call), GLQ_ERR_CUDA.  Asynchronous.
  */
@@ -266,7 +302,7 @@ GLQ_API glq_status glq_prefill_replay(glq_layer layer, int64_t B, void *stream);
  * callbacks, or under a framework that owns every device allocation.  (The
  * GLQ pages have no counterpart: this is a property of this library's
  * workspace handling.)
- * Instead of the layer's workspace it uses one fixed device array of
+ * Instead of the device's shared workspace it uses one fixed device array of
  * GLQ_NOALLOC_SCRATCH_BYTES (8 MiB) that the library defines at file scope;
  * every GPU that loads the library holds it until the process exits.
  * x_dev, y_dev, x_dtype, y_dtype, stream: as glq_linear; 0 <= B <= 16.
