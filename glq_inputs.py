@@ -6,10 +6,12 @@ the fp64 oracle consume the same host arrays it produces.
 
 Recipe (numpy PCG64, ``numpy.random.default_rng``):
   * per layer, ``rng = default_rng([seed, layer_id])`` draws, in order:
-    idx1 (uint16, uniform [0, 65536)), idx2 (uint16 uniform for 4 bpw,
-    uint8 uniform [0, 256) for 3 bpw, none for 2 bpw), the 3 bpw residual
+    idx1 (uint16, uniform [0, 65536)); the residual stages of the bit width
+    in stage order (a 16-bit E8 stage: uint16 uniform; the 8-bit stage of an
+    odd bpw: uint8 uniform [0, 256)); for an odd bpw the 256-entry residual
     codebook (256 x 8 normal draws of standard deviation 0.5, rounded to
-    fp16), S_in and S_out (Rademacher +-1, int8);
+    fp16); S_in and S_out (Rademacher +-1, int8).  Residual stage s (s = 1,
+    2, ...) has the scale 8^-s;
   * per (layer, batch), ``rng = default_rng([seed, layer_id, 1_000_000 + B])``
     draws x ~ N(0, 1) of shape [B][n] (float64), then -- when the workload
     has outliers -- floor(0.01 n) distinct columns, which are multiplied by
@@ -88,18 +90,36 @@ WORKLOADS = {
 }
 
 
+def stage_bits(bpw: int) -> list:
+    """Index widths of the residual stages of a bit width (after the 16-bit
+    primary): 16-bit E8 stages, then one 8-bit stage for an odd bpw."""
+    if not 2 <= bpw <= 8:
+        raise ValueError("bpw must be in 2..8")
+    return [16] * ((bpw - 2) // 2) + ([8] if bpw % 2 else [])
+
+
 @dataclass
 class LayerInputs:
     m: int
     n: int
     bpw: int
     idx1: np.ndarray          # uint16 [m][n/8]
-    idx2: np.ndarray | None   # uint8 (3 bpw) / uint16 (4 bpw) [m][n/8]
-    cb2_f16: np.ndarray | None  # uint16 fp16 bits [256][8] for 3 bpw
+    # residual indices: None (2 bpw); one array (3 bpw: uint8, 4 bpw: uint16);
+    # from 5 bpw a list with one array per stage (stage order)
+    idx2: object
+    cb2_f16: np.ndarray | None  # uint16 fp16 bits [256][8] for an odd bpw
     s_in: np.ndarray          # int8 [n], +-1
     s_out: np.ndarray         # int8 [m], +-1
     weight_scale: float
-    resid_scale: float
+    resid_scale: object       # float (2-4 bpw) or a list of one scale per stage
+
+    def stages(self):
+        """(list of residual index arrays, list of their scales)."""
+        if self.bpw == 2:
+            return [], []
+        if self.bpw <= 4:
+            return [self.idx2], [self.resid_scale]
+        return list(self.idx2), list(self.resid_scale)
 
 
 def _rademacher(rng, k):
@@ -110,22 +130,28 @@ def make_layer(seed: int, layer_id: int, m: int, n: int, bpw: int,
                weight_scale: float = 0.05, resid_scale: float = 0.125) -> LayerInputs:
     if n % 8:
         raise ValueError("n must be a multiple of 8")
+    bits = stage_bits(bpw)
     rng = np.random.default_rng([seed, layer_id])
     G = n // 8
     idx1 = rng.integers(0, CODEBOOK_ENTRIES, size=(m, G), dtype=np.uint16)
-    idx2 = None
+    res = []
+    for b in bits:
+        if b == 16:
+            res.append(rng.integers(0, CODEBOOK_ENTRIES, size=(m, G), dtype=np.uint16))
+        else:
+            res.append(rng.integers(0, RESIDUAL8_ENTRIES, size=(m, G), dtype=np.uint8))
     cb2 = None
-    if bpw == 4:
-        idx2 = rng.integers(0, CODEBOOK_ENTRIES, size=(m, G), dtype=np.uint16)
-    elif bpw == 3:
-        idx2 = rng.integers(0, RESIDUAL8_ENTRIES, size=(m, G), dtype=np.uint8)
+    if bpw % 2:
         cb2 = rng.normal(0.0, 0.5, size=(RESIDUAL8_ENTRIES, 8)).astype(np.float16).view(np.uint16)
-    elif bpw != 2:
-        raise ValueError("bpw must be 2, 3 or 4")
     s_in = _rademacher(rng, n)
     s_out = _rademacher(rng, m)
-    return LayerInputs(m, n, bpw, idx1, idx2, cb2, s_in, s_out,
-                       float(weight_scale), float(resid_scale))
+    if bpw <= 4:
+        idx2 = res[0] if res else None
+        rs = float(resid_scale)
+    else:
+        idx2 = res
+        rs = [float(resid_scale) ** (s + 1) for s in range(len(res))]
+    return LayerInputs(m, n, bpw, idx1, idx2, cb2, s_in, s_out, float(weight_scale), rs)
 
 
 def f64_to_bf16_bits(a: np.ndarray) -> np.ndarray:

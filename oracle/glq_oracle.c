@@ -29,6 +29,9 @@
  *   - w^ = ws * (cb1 + rs * cb2), where rs is the multiplier applied at
  *     decode; rounding: c = fmaf(rs, cb2, cb1) (single rounding), then
  *     w^ = fp32(ws * c) (single rounding);
+ *   - 5-8 bpw: the residual stages of the "Bit widths" table in its order
+ *     (16-bit E8 stages, then the 8-bit stage of an odd bpw), each with its
+ *     own scale, added one fmaf per stage in that order;
  *   - H_k[i][j] = (-1)^popcount(i & j) / sqrt(k) (Sylvester order); blocks in
  *     descending size at increasing offsets;
  *   - input side: sign, then H; output side: H, then sign.
@@ -237,29 +240,67 @@ void glq_oracle_hadamard_apply(int64_t n, const double *v, double *out, int forc
 /* "Inference kernels" (Qidxs2, codebook2, inv_resid_scale)]            */
 /* ------------------------------------------------------------------ */
 
+/* Residual stages of a bit width  [glq 0.5.1, "Bit widths"]: after the
+ * 16-bit primary index, (bpw - 2) / 2 stages of 16-bit E8 indices and, for
+ * an odd bpw, one last stage of 8-bit indices into a 256-entry table
+ * (3 = 16+8, 4 = 16+16, 5 = 16+16+8, ..., 8 = 16+16+16+16).  Writes the
+ * index width of each residual stage into bits[] and returns their number,
+ * or -1 for a bpw outside 2..8. */
+int glq_oracle_stage_bits(int bpw, int *bits) {
+    if (bpw < 2 || bpw > 8) return -1;
+    int k = 0;
+    for (int i = 0; i < (bpw - 2) / 2; i++) bits[k++] = 16;
+    if (bpw % 2) bits[k++] = 8;
+    return k;
+}
+
 /* Decodes rows [r0, r1) of W^ into w[(r - r0) * n + j] (fp32 values held
- * in double).  bpw 2: no residual; bpw 3: idx2 is uint8 into cb2[256][8];
- * bpw 4: idx2 is uint16 into cb2[65536][8].  Returns 0, or -1 on a bad bpw. */
-int glq_oracle_decode_rows(int64_t m, int64_t n, int bpw, const uint16_t *idx1,
-                           const void *idx2, const double *cb1, const double *cb2,
-                           float ws, float rs, int64_t r0, int64_t r1, double *w) {
-    if (bpw < 2 || bpw > 4 || n % 8 != 0 || r0 < 0 || r1 > m) return -1;
+ * in double).  idx_res[s] is residual stage s ([m][n/8], uint16 into cb16
+ * for a 16-bit stage, uint8 into cb8[256][8] for the 8-bit one) and rs[s]
+ * its scale.  Reconstruction, stage by stage in that order:
+ *   c = cb1[idx1][j];  c = fmaf(rs[s], cb_s[idx_s][j], c)  (one rounding each);
+ *   w^ = fp32(ws * c)  (one rounding).
+ * Returns 0, or -1 on bad arguments. */
+int glq_oracle_decode_stages(int64_t m, int64_t n, int bpw, const uint16_t *idx1,
+                             const void *const *idx_res, const double *cb1, const double *cb16,
+                             const double *cb8, float ws, const float *rs, int64_t r0, int64_t r1,
+                             double *w) {
+    int bits[4];
+    int ns = glq_oracle_stage_bits(bpw, bits);
+    if (ns < 0 || n % 8 != 0 || r0 < 0 || r1 > m) return -1;
+    for (int s = 0; s < ns; s++)
+        if (!idx_res || !idx_res[s] || (bits[s] == 16 && !cb16) || (bits[s] == 8 && !cb8)) return -1;
     int64_t G = n / 8;
     for (int64_t r = r0; r < r1; r++) {
         for (int64_t g = 0; g < G; g++) {
             const double *c1 = cb1 + (int64_t)idx1[r * G + g] * 8;
-            const double *c2 = 0;
-            if (bpw == 3) c2 = cb2 + (int64_t)((const uint8_t *)idx2)[r * G + g] * 8;
-            if (bpw == 4) c2 = cb2 + (int64_t)((const uint16_t *)idx2)[r * G + g] * 8;
             for (int j = 0; j < 8; j++) {
                 float c = (float)c1[j]; /* exact: codewords are multiples of 1/2 */
-                if (c2) c = fmaf(rs, (float)c2[j], c);
+                for (int s = 0; s < ns; s++) {
+                    const double *cs = bits[s] == 16
+                        ? cb16 + (int64_t)((const uint16_t *)idx_res[s])[r * G + g] * 8
+                        : cb8 + (int64_t)((const uint8_t *)idx_res[s])[r * G + g] * 8;
+                    c = fmaf(rs[s], (float)cs[j], c);
+                }
                 /* a binary32 x binary32 product is exact in binary64 */
                 w[(r - r0) * n + g * 8 + j] = (double)(float)((double)ws * (double)c);
             }
         }
     }
     return 0;
+}
+
+/* The two-stage form of the pages' matmul arguments (Qidxs2, codebook2,
+ * inv_resid_scale): bpw 2: no residual; bpw 3: idx2 is uint8 into
+ * cb2[256][8]; bpw 4: idx2 is uint16 into cb2[65536][8].  Returns 0, or -1
+ * on a bad bpw. */
+int glq_oracle_decode_rows(int64_t m, int64_t n, int bpw, const uint16_t *idx1,
+                           const void *idx2, const double *cb1, const double *cb2,
+                           float ws, float rs, int64_t r0, int64_t r1, double *w) {
+    if (bpw < 2 || bpw > 4) return -1;
+    const void *res[1] = {idx2};
+    return glq_oracle_decode_stages(m, n, bpw, idx1, res, cb1, bpw == 4 ? cb2 : 0, bpw == 3 ? cb2 : 0, ws,
+                                    &rs, r0, r1, w);
 }
 
 /* ------------------------------------------------------------------ */
@@ -272,9 +313,10 @@ typedef struct {
     int64_t m, n, B, r0, r1;
     int bpw;
     const uint16_t *idx1;
-    const void *idx2;
-    const double *cb1, *cb2;
-    float ws, rs;
+    const void *const *idx_res;
+    const double *cb1, *cb16, *cb8;
+    float ws;
+    const float *rs;
     const double *xr;
     double *z;
     int rc;
@@ -288,7 +330,12 @@ static void *rows_product(void *arg) {
         return 0;
     }
     for (int64_t r = j->r0; r < j->r1; r++) {
-        glq_oracle_decode_rows(j->m, j->n, j->bpw, j->idx1, j->idx2, j->cb1, j->cb2, j->ws, j->rs, r, r + 1, w);
+        if (glq_oracle_decode_stages(j->m, j->n, j->bpw, j->idx1, j->idx_res, j->cb1, j->cb16, j->cb8, j->ws,
+                                     j->rs, r, r + 1, w) != 0) {
+            free(w);
+            j->rc = -1;
+            return 0;
+        }
         for (int64_t b = 0; b < j->B; b++) {
             double acc = 0.0;
             const double *xb = j->xr + b * j->n;
@@ -307,10 +354,11 @@ static void *rows_product(void *arg) {
  * ranges to `nthreads` POSIX threads (each output element is computed by
  * the same loop whatever the thread count, so the result is identical).
  * Returns 0 or -1 on bad arguments / allocation failure. */
-int glq_oracle_linear_mt(int64_t m, int64_t n, int bpw, const uint16_t *idx1, const void *idx2,
-                         const double *cb1, const double *cb2, float ws, float rs,
-                         const int8_t *s_in, const int8_t *s_out, const uint16_t *x, int x_is_bf16,
-                         int64_t B, double *y, int nthreads) {
+int glq_oracle_linear_stages_mt(int64_t m, int64_t n, int bpw, const uint16_t *idx1,
+                                const void *const *idx_res, const double *cb1, const double *cb16,
+                                const double *cb8, float ws, const float *rs, const int8_t *s_in,
+                                const int8_t *s_out, const uint16_t *x, int x_is_bf16, int64_t B, double *y,
+                                int nthreads) {
     if (m <= 0 || n <= 0 || n % 8 != 0 || B < 0) return -1;
     if (nthreads < 1) nthreads = 1;
     if (nthreads > 256) nthreads = 256;
@@ -342,7 +390,7 @@ int glq_oracle_linear_mt(int64_t m, int64_t n, int bpw, const uint16_t *idx1, co
         j->m = m; j->n = n; j->B = B; j->bpw = bpw;
         j->r0 = m * t / nthreads;
         j->r1 = m * (t + 1) / nthreads;
-        j->idx1 = idx1; j->idx2 = idx2; j->cb1 = cb1; j->cb2 = cb2;
+        j->idx1 = idx1; j->idx_res = idx_res; j->cb1 = cb1; j->cb16 = cb16; j->cb8 = cb8;
         j->ws = ws; j->rs = rs; j->xr = xr; j->z = z; j->rc = -1;
     }
     for (int t = 1; t < nthreads; t++) {
@@ -363,7 +411,18 @@ int glq_oracle_linear_mt(int64_t m, int64_t n, int bpw, const uint16_t *idx1, co
     return rc;
 }
 
-/* The single-threaded form of the layer. */
+/* The two-stage form (bpw 2..4, see glq_oracle_decode_rows). */
+int glq_oracle_linear_mt(int64_t m, int64_t n, int bpw, const uint16_t *idx1, const void *idx2,
+                         const double *cb1, const double *cb2, float ws, float rs,
+                         const int8_t *s_in, const int8_t *s_out, const uint16_t *x, int x_is_bf16,
+                         int64_t B, double *y, int nthreads) {
+    if (bpw < 2 || bpw > 4) return -1;
+    const void *res[1] = {idx2};
+    return glq_oracle_linear_stages_mt(m, n, bpw, idx1, res, cb1, bpw == 4 ? cb2 : 0, bpw == 3 ? cb2 : 0, ws, &rs,
+                                       s_in, s_out, x, x_is_bf16, B, y, nthreads);
+}
+
+/* The single-threaded two-stage form. */
 int glq_oracle_linear(int64_t m, int64_t n, int bpw, const uint16_t *idx1, const void *idx2,
                       const double *cb1, const double *cb2, float ws, float rs,
                       const int8_t *s_in, const int8_t *s_out, const uint16_t *x, int x_is_bf16,

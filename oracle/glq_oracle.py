@@ -73,6 +73,15 @@ def _load():
     lib.glq_oracle_linear_mt.argtypes = [
         c_i64, c_i64, c_int, vp, vp, vp, vp, ctypes.c_float, ctypes.c_float,
         vp, vp, vp, c_int, c_i64, vp, c_int]
+    lib.glq_oracle_stage_bits.restype = c_int
+    lib.glq_oracle_stage_bits.argtypes = [c_int, vp]
+    lib.glq_oracle_decode_stages.restype = c_int
+    lib.glq_oracle_decode_stages.argtypes = [
+        c_i64, c_i64, c_int, vp, vp, vp, vp, vp, ctypes.c_float, vp, c_i64, c_i64, vp]
+    lib.glq_oracle_linear_stages_mt.restype = c_int
+    lib.glq_oracle_linear_stages_mt.argtypes = [
+        c_i64, c_i64, c_int, vp, vp, vp, vp, vp, ctypes.c_float, vp,
+        vp, vp, vp, c_int, c_i64, vp, c_int]
     _lib = lib
     return lib
 
@@ -138,13 +147,20 @@ def hadamard_apply(v, force_dense: bool = False) -> np.ndarray:
     return out
 
 
-def _residual_table(bpw: int, cb2):
-    if bpw == 2:
-        return None
-    if bpw == 4:
-        return e8_codebook() if cb2 is None else np.ascontiguousarray(cb2, dtype=np.float64)
+def stage_bits(bpw: int) -> list:
+    """Index widths of the residual stages of a bit width, as the oracle reads
+    the "Bit widths" table (16-bit E8 stages, then an 8-bit stage for an odd
+    bpw)."""
+    bits = np.zeros(4, dtype=np.int32)
+    k = _load().glq_oracle_stage_bits(int(bpw), _ptr(bits))
+    if k < 0:
+        raise ValueError(f"bad bpw {bpw}")
+    return [int(b) for b in bits[:k]]
+
+
+def _table8(cb2):
     if cb2 is None:
-        raise ValueError("bpw 3 needs the 256-entry residual codebook")
+        return None
     cb2 = np.asarray(cb2)
     if cb2.dtype == np.uint16:  # fp16 bits
         cb2 = f16_table_to_double(cb2)
@@ -159,27 +175,49 @@ def f16_table_to_double(bits) -> np.ndarray:
     return np.array(flat, dtype=np.float64).reshape(bits.shape)
 
 
-def _check_idx(m, n, bpw, idx1, idx2):
-    G = n // 8
-    idx1 = np.ascontiguousarray(idx1, dtype=np.uint16).reshape(m, G)
-    if bpw == 3:
-        idx2 = np.ascontiguousarray(idx2, dtype=np.uint8).reshape(m, G)
-    elif bpw == 4:
-        idx2 = np.ascontiguousarray(idx2, dtype=np.uint16).reshape(m, G)
-    else:
-        idx2 = None
-    return idx1, idx2
+class _Stages:
+    """The residual stages of a call, marshalled for the C oracle: index
+    arrays (kept alive), their pointer array and the scale array."""
+
+    def __init__(self, m, n, bpw, idx1, idx2, rs, cb2):
+        G = n // 8
+        self.bits = stage_bits(bpw)
+        self.idx1 = np.ascontiguousarray(idx1, dtype=np.uint16).reshape(m, G)
+        if not self.bits:
+            arrays, scales = [], []
+        elif bpw <= 4:
+            arrays, scales = [idx2], [rs]
+        else:
+            arrays, scales = list(idx2), list(rs)
+        if len(arrays) != len(self.bits) or len(scales) != len(self.bits):
+            raise ValueError("residual stages do not match the bit width")
+        self.arrays = [np.ascontiguousarray(a, dtype=np.uint16 if b == 16 else np.uint8).reshape(m, G)
+                       for a, b in zip(arrays, self.bits)]
+        self.ptrs = (ctypes.c_void_p * 4)(*([a.ctypes.data for a in self.arrays] + [None] * (4 - len(self.arrays))))
+        self.scales = np.zeros(4, dtype=np.float32)
+        self.scales[:len(scales)] = np.asarray(scales, dtype=np.float32)
+        self.cb1 = e8_codebook()
+        self.cb16 = self.cb1 if 16 in self.bits else None
+        if 8 in self.bits and cb2 is None:
+            raise ValueError("an odd bpw needs the 256-entry residual codebook")
+        self.cb8 = _table8(cb2) if 8 in self.bits else None
+        if bpw == 4 and cb2 is not None:  # an explicit table for the 16-bit stage
+            self.cb16 = np.ascontiguousarray(cb2, dtype=np.float64)
 
 
 def decode_rows(m, n, bpw, idx1, idx2, ws, rs, r0=0, r1=None, cb2=None) -> np.ndarray:
-    """Explicit W^ rows [r0, r1) as float64 arrays holding fp32 values."""
+    """Explicit W^ rows [r0, r1) as float64 arrays holding fp32 values.
+
+    bpw 2..4: idx2 an array (or None), rs a float; bpw 5..8: idx2 a list of
+    the residual stages' index arrays and rs a list of their scales.  cb2:
+    the 256-entry table of an odd bpw (fp16 bits or values).
+    """
     r1 = m if r1 is None else r1
-    idx1, idx2 = _check_idx(m, n, bpw, idx1, idx2)
-    cb1 = e8_codebook()
-    cb2 = _residual_table(bpw, cb2)
+    st = _Stages(m, n, bpw, idx1, idx2, rs, cb2)
     w = np.zeros((r1 - r0, n), dtype=np.float64)
-    rc = _load().glq_oracle_decode_rows(m, n, bpw, _ptr(idx1), _ptr(idx2), _ptr(cb1),
-                                        _ptr(cb2), float(ws), float(rs), r0, r1, _ptr(w))
+    rc = _load().glq_oracle_decode_stages(m, n, bpw, _ptr(st.idx1), ctypes.cast(st.ptrs, ctypes.c_void_p),
+                                          _ptr(st.cb1), _ptr(st.cb16), _ptr(st.cb8), float(ws),
+                                          _ptr(st.scales), r0, r1, _ptr(w))
     if rc != 0:
         raise ValueError("oracle decode rejected its arguments")
     return w
@@ -198,21 +236,21 @@ def linear(m, n, bpw, idx1, idx2, ws, rs, s_in, s_out, x_bits, x_is_bf16, cb2=No
     """y[B][m] (float64) = S_out . H_m . W^ . H_n . (S_in . x).
 
     x_bits: uint16 [B][n] holding fp16 (x_is_bf16 False) or bf16 bit patterns.
+    idx2 / rs / cb2 as decode_rows (per-stage lists from 5 bpw).
     threads: POSIX threads the rows of W^ xr are split over (0: every host
     core); the result does not depend on it.
     """
     threads = default_threads() if threads == 0 else int(threads)
-    idx1, idx2 = _check_idx(m, n, bpw, idx1, idx2)
+    st = _Stages(m, n, bpw, idx1, idx2, rs, cb2)
     x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16).reshape(-1, n)
     B = x_bits.shape[0]
     s_in = np.ascontiguousarray(s_in, dtype=np.int8)
     s_out = np.ascontiguousarray(s_out, dtype=np.int8)
-    cb1 = e8_codebook()
-    cb2 = _residual_table(bpw, cb2)
     y = np.zeros((B, m), dtype=np.float64)
-    rc = _load().glq_oracle_linear_mt(m, n, bpw, _ptr(idx1), _ptr(idx2), _ptr(cb1), _ptr(cb2),
-                                      float(ws), float(rs), _ptr(s_in), _ptr(s_out),
-                                      _ptr(x_bits), int(bool(x_is_bf16)), B, _ptr(y), threads)
+    rc = _load().glq_oracle_linear_stages_mt(m, n, bpw, _ptr(st.idx1), ctypes.cast(st.ptrs, ctypes.c_void_p),
+                                             _ptr(st.cb1), _ptr(st.cb16), _ptr(st.cb8), float(ws),
+                                             _ptr(st.scales), _ptr(s_in), _ptr(s_out), _ptr(x_bits),
+                                             int(bool(x_is_bf16)), B, _ptr(y), threads)
     if rc != 0:
         raise ValueError("oracle linear rejected its arguments")
     return y
