@@ -204,7 +204,7 @@ class WorkloadSet:
         self.layers = []  # [layer][copy] = (GlqLinear, x, y)
         for i, L in enumerate(self.host):
             res = None
-            if L.bpw == 3:
+            if L.bpw % 2:
                 res = glq.Codebook(L.cb2_f16.reshape(256, 8))
             elif L.bpw == 4:
                 res = self.e8
@@ -692,6 +692,10 @@ def run_glq(args):
                                                      gemv_layer=2),
             "smollm2-360m-3bpw": decode_config_section(glq, torch, "smollm2-360m-3bpw", hbm_peak),
             "single-1024-2bpw": decode_config_section(glq, torch, "single-1024-2bpw", hbm_peak),
+            # 5-8 bpw residual stages and a mixed-precision model
+            "24b-decode-5bpw": decode_config_section(glq, torch, "24b-decode-5bpw", hbm_peak, gemv_layer=2),
+            "24b-decode-6bpw": decode_config_section(glq, torch, "24b-decode-6bpw", hbm_peak, gemv_layer=2),
+            "smollm3-3b-mixed": decode_config_section(glq, torch, "smollm3-3b-mixed", hbm_peak),
         }
         result["prefill"] = prefill_section(glq, torch, tc_peak, peak_src)
         result["dense_bf16_reference"] = dense_reference_section(glq, torch, hbm_peak, tc_peak)

@@ -39,7 +39,7 @@ EXPORTS = (
     "glq_linear", "glq_dequant_reference", "glq_rht_input", "glq_rht_output",
     "glq_layer_check", "glq_layer_info", "glq_gemv_replay", "glq_linear_noalloc", "glq_decode_plan",
     "glq_prefill_replay", "glq_layer_set_fusion", "glq_layer_set_prefill_reconstruct",
-    "glq_workspace_info", "glq_workspace_release",
+    "glq_workspace_info", "glq_workspace_release", "glq_layer_create_stages",
 )
 
 
@@ -60,6 +60,8 @@ _SIGNATURES = {
     "glq_codebook_destroy": ([_vp], ctypes.c_int),
     "glq_layer_create": ([_i64, _i64, _i32, _vp, _vp, _vp, _vp, ctypes.c_float, ctypes.c_float,
                           _vp, _vp, ctypes.POINTER(_vp)], ctypes.c_int),
+    "glq_layer_create_stages": ([_i64, _i64, _i32, _vp, _vp, _vp, _vp, ctypes.c_float, _vp,
+                                 _vp, _vp, ctypes.POINTER(_vp)], ctypes.c_int),
     "glq_layer_destroy": ([_vp], ctypes.c_int),
     "glq_layer_reserve": ([_vp, _i64], ctypes.c_int),
     "glq_linear": ([_vp, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, _vp], ctypes.c_int),
@@ -153,6 +155,39 @@ def glq_layer_create(m, n, bpw, idx1, idx2, primary, residual, weight_scale, res
                           primary, residual, float(weight_scale), float(resid_scale),
                           s_in.ctypes.data, s_out.ctypes.data, ctypes.byref(h)),
         "glq_layer_create")
+    return h.value
+
+
+def stage_bits(bpw: int) -> list:
+    """Index widths of the residual stages of a bit width (glq 0.5.1 PyPI
+    page, "Bit widths"): 16-bit E8 stages, then an 8-bit stage for odd bpw."""
+    if not 2 <= bpw <= 8:
+        raise ValueError("bpw must be in 2..8")
+    return [16] * ((bpw - 2) // 2) + ([8] if bpw % 2 else [])
+
+
+def glq_layer_create_stages(m, n, bpw, idx1, idx_res, primary, residual, weight_scale, resid_scales,
+                            s_in, s_out) -> int:
+    """idx_res: one [m][n/8] index array per residual stage (stage order),
+    resid_scales: one scale per stage."""
+    bits = stage_bits(bpw)
+    idx_res = list(idx_res or [])
+    scales = np.ascontiguousarray(list(resid_scales or []), dtype=np.float32)
+    if len(idx_res) != len(bits) or scales.size != len(bits):
+        raise ValueError(f"bpw {bpw} has {len(bits)} residual stages")
+    idx1 = np.ascontiguousarray(idx1, dtype=np.uint16)
+    arrays = [np.ascontiguousarray(a, dtype=np.uint16 if b == 16 else np.uint8) for a, b in zip(idx_res, bits)]
+    s_in = np.ascontiguousarray(s_in, dtype=np.int8)
+    s_out = np.ascontiguousarray(s_out, dtype=np.int8)
+    if idx1.size != m * (n // 8) or s_in.size != n or s_out.size != m or any(a.size != idx1.size for a in arrays):
+        raise ValueError("array sizes do not match m, n")
+    ptrs = (ctypes.c_void_p * max(1, len(arrays)))(*[a.ctypes.data for a in arrays])
+    h = _vp()
+    _ok(_L().glq_layer_create_stages(m, n, bpw, idx1.ctypes.data, ctypes.cast(ptrs, ctypes.c_void_p) if arrays else None,
+                                     primary, residual, float(weight_scale),
+                                     scales.ctypes.data if arrays else None, s_in.ctypes.data,
+                                     s_out.ctypes.data, ctypes.byref(h)),
+        "glq_layer_create_stages")
     return h.value
 
 
@@ -287,11 +322,19 @@ class GlqLinear:
 
     def __init__(self, m, n, bpw, idx1, idx2, primary: Codebook, residual: Codebook | None,
                  weight_scale, resid_scale, s_in, s_out):
+        """bpw 2-4: idx2 the residual index array (or None) and resid_scale
+        a float; bpw 5-8: idx2 a list of the residual stages' index arrays
+        and resid_scale a list of their scales (stage order); residual: the
+        256-entry codebook of an odd bpw, else None (or the E8 codebook)."""
         self.m, self.n, self.bpw = int(m), int(n), int(bpw)
         self._cbs = (primary, residual)  # keep codebooks alive
-        self.handle = glq_layer_create(
-            self.m, self.n, self.bpw, idx1, idx2, primary.handle,
-            0 if residual is None else residual.handle, weight_scale, resid_scale, s_in, s_out)
+        rh = 0 if residual is None else residual.handle
+        if self.bpw <= 4:
+            self.handle = glq_layer_create(self.m, self.n, self.bpw, idx1, idx2, primary.handle, rh,
+                                           weight_scale, resid_scale, s_in, s_out)
+        else:
+            self.handle = glq_layer_create_stages(self.m, self.n, self.bpw, idx1, idx2, primary.handle, rh,
+                                                  weight_scale, resid_scale, s_in, s_out)
 
     def reserve(self, max_B: int):
         glq_layer_reserve(self.handle, max_B)

@@ -83,7 +83,8 @@ void free_layer(glq_layer L) {
     if (!L) return;
     cudaFree(L->d_blk_cnt);
     cudaFree(L->d_idx1);
-    cudaFree(L->d_idx2);
+    for (int k = 0; k < 3; ++k) cudaFree(L->d_res16[k]);
+    cudaFree(L->d_res8);
     cudaFree(L->d_sin);
     cudaFree(L->d_sout);
     cudaFree(L->d_err);
@@ -166,7 +167,7 @@ void decode_need(glq_layer L, int64_t rows, WsNeed &n) {
     int max_splits = 1;
     for (int nb = 1; nb <= rows; ++nb) max_splits = std::max(max_splits, glq::max_decode_splits(L, nb));
     n.b[WS_XQ] = std::max(n.b[WS_XQ], (size_t)rows * L->n_pad * 2);
-    if (L->bpw == 3) n.b[WS_XH] = std::max(n.b[WS_XH], (size_t)rows * L->n_pad * sizeof(__half));
+    if (L->has8) n.b[WS_XH] = std::max(n.b[WS_XH], (size_t)rows * L->n_pad * sizeof(__half));
     n.b[WS_INFO] = std::max(n.b[WS_INFO], (size_t)rows * sizeof(glq_rowinfo));
     if (max_splits > 1)
         n.b[WS_PART] = std::max(n.b[WS_PART], (size_t)max_splits * rows * L->m_pad * sizeof(double));
@@ -271,12 +272,17 @@ int prefill_tiles(glq_layer L, int64_t B) {
 glq::PrefillParams prefill_params(glq_layer L, const glq_prefill_ws &ws, int64_t B) {
     glq::PrefillParams pp{};
     pp.idx1 = L->d_idx1;
-    pp.idx2 = L->d_idx2;
+    for (int k = 0; k < 3; ++k) {
+        pp.idx16[k] = L->d_res16[k];
+        const __half2 h = __floats2half2_rn(L->rs16[k], L->rs16[k]);
+        pp.rs16_h2[k] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    pp.idx8 = L->d_res8;
+    const __half2 h8 = __floats2half2_rn(L->rs8, L->rs8);
+    pp.rs8_h2 = *reinterpret_cast<const uint32_t *>(&h8);
     pp.cb_f16 = L->primary->d_table_f16;
-    pp.res8 = L->bpw == 3 ? reinterpret_cast<const uint4 *>(L->residual->d_fp16) : nullptr;
+    pp.tab8 = L->has8 ? reinterpret_cast<const uint4 *>(L->residual->d_fp16) : nullptr;
     pp.bpw = L->bpw;
-    const __half2 rs2 = __floats2half2_rn(L->rs, L->rs);
-    pp.rs_h2 = *reinterpret_cast<const uint32_t *>(&rs2);
     pp.info = ws.info;
     pp.ws = L->ws;
     pp.z = ws.z;
@@ -416,7 +422,7 @@ constexpr int FUSE_DEFAULT_FLAGS = GLQ_FUSE_INPUT | GLQ_SPLITK_CLUSTER;
 DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y_dtype, int max_splits) {
     DecodeCfg c;
     const int nt = nb > 8 ? 2 : 1;
-    const int warps = gemv_warps(nt);
+    const int warps = gemv_warps(nt, L->bpw);
     const size_t base = gemv_smem_bytes(L->primary->table_words, L->bpw);
     const bool x_al = (reinterpret_cast<uintptr_t>(x) & 15) == 0;
     const bool y_al = (reinterpret_cast<uintptr_t>(y) & 15) == 0;
@@ -450,7 +456,7 @@ DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y
     }
     if (!c.fin) {
         c.plan = plan_for(L, nb);
-        if (nt == 1 && (long long)L->RT * L->KC >= 200LL * L->num_sms) {  // large layer: wide CTAs
+        if (nt == 1 && L->bpw <= 4 && (long long)L->RT * L->KC >= 200LL * L->num_sms) {  // large layer: wide CTAs
             c.warps = GEMV_WIDE_WARPS;
             c.plan = plan_gemv(L->RT, L->KC, L->num_sms, c.warps);
         }
@@ -476,15 +482,15 @@ DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y
 }
 
 int max_decode_splits(glq_layer L, int nb) {
-    const int warps = gemv_warps(nb > 8 ? 2 : 1);
+    const int warps = gemv_warps(nb > 8 ? 2 : 1, L->bpw);
     int cap = 1;
     while (cap < L->KC &&
            gemv_fused_smem_bytes(L->primary->table_words, L->bpw, nb, std::min(cap * 2, L->KC) * GLQ_CHUNK_K) <=
                GEMV_SMEM_LIMIT)
         cap *= 2;
     const int fs = plan_gemv(L->RT, L->KC, L->num_sms, warps, true, cap).splits;
-    const GemvPlan wide = plan_gemv(L->RT, L->KC, L->num_sms, GEMV_WIDE_WARPS);
-    return std::max(std::max(plan_for(L, nb).splits, fs), wide.splits);
+    const int ws = L->bpw <= 4 ? plan_gemv(L->RT, L->KC, L->num_sms, GEMV_WIDE_WARPS).splits : 1;
+    return std::max(std::max(plan_for(L, nb).splits, fs), ws);
 }
 
 GemvParams gemv_params(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg, int nb, const void *x,
@@ -492,12 +498,20 @@ GemvParams gemv_params(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg
     const GemvPlan &plan = cfg.plan;
     GemvParams p{};
     p.idx1 = L->d_idx1;
-    p.idx2 = L->d_idx2;
+    double rsum = 0.0;
+    for (int k = 0; k < 3; ++k) {
+        p.idx16[k] = L->d_res16[k];
+        p.rs16_d[k] = k < L->nres16 ? (double)L->rs16[k] : 0.0;
+        rsum += p.rs16_d[k];
+    }
+    p.idx8 = L->d_res8;
+    p.rs8_d = L->has8 ? 2.0 * (double)L->rs8 : 0.0;
+    p.corr_mult = 1.0 + rsum;
     p.table = L->primary->d_table;
     p.table_words = L->primary->table_words;
     p.fold = FoldParams{L->primary->fold.nb, L->primary->fold.neg_base};
     p.kc = LookupConsts{4u, 16u, 0xFFFFFFFFu};
-    p.res8 = (L->bpw == 3) ? reinterpret_cast<const uint4 *>(L->residual->d_fp16) : nullptr;
+    p.tab8 = L->has8 ? reinterpret_cast<const uint4 *>(L->residual->d_fp16) : nullptr;
     p.xq = w.xq;
     p.xh = w.xh;
     p.info = w.info;
@@ -508,8 +522,6 @@ GemvParams gemv_params(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg
     p.bands = plan.bands;
     p.splits = plan.splits;
     p.cps = plan.cps;
-    p.rs_d = L->bpw == 3 ? 2.0 * (double)L->rs : (double)L->rs;
-    p.corr_mult = L->bpw == 4 ? 1.0 + (double)L->rs : 1.0;
     p.ws = L->ws;
     p.partials = w.part;
     p.counters = w.cnt;
@@ -709,28 +721,32 @@ glq_status glq_codebook_destroy(glq_codebook cb) {
     return GLQ_OK;
 }
 
-glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *idx1, const void *idx2,
-                            glq_codebook primary, glq_codebook residual, float weight_scale,
-                            float resid_scale, const int8_t *s_in, const int8_t *s_out,
-                            glq_layer *out) {
+glq_status glq_layer_create_stages(int64_t m, int64_t n, int32_t bpw, const uint16_t *idx1,
+                                   const void *const *idx_res, glq_codebook primary, glq_codebook residual,
+                                   float weight_scale, const float *resid_scales, const int8_t *s_in,
+                                   const int8_t *s_out, glq_layer *out) {
     if (!out) return GLQ_ERR_INVALID_ARG;
     *out = nullptr;
     if (m <= 0 || n <= 0 || m % 8 || n % 8 || m > MAX_DIM || n > MAX_DIM) return GLQ_ERR_SHAPE;
-    if (bpw < 2 || bpw > 4) return GLQ_ERR_BPW;
+    if (bpw < 2 || bpw > 8) return GLQ_ERR_BPW;
+    const int n16 = glq::stages16(bpw);
+    const bool has8 = glq::stage8(bpw);
+    const int nres = n16 + (has8 ? 1 : 0);
     if (!idx1 || !s_in || !s_out) return GLQ_ERR_INVALID_ARG;
+    if (nres > 0 && (!idx_res || !resid_scales)) return GLQ_ERR_BPW;
+    for (int k = 0; k < nres; ++k)
+        if (!idx_res[k]) return GLQ_ERR_BPW;
     if (!primary) return GLQ_ERR_NO_CODEBOOK;
     if (primary->entries != GLQ_CB_ENTRIES || !primary->folded) return GLQ_ERR_NO_CODEBOOK;
-    if (bpw == 2 && (idx2 || residual)) return GLQ_ERR_BPW;
-    if (bpw == 3) {
-        if (!idx2) return GLQ_ERR_BPW;
+    if (has8) {  // the 8-bit stage indexes a 256-entry table
         if (!residual) return GLQ_ERR_NO_CODEBOOK;
         if (residual->entries != GLQ_CB8_ENTRIES) return GLQ_ERR_BPW;
+    } else if (residual && residual != primary) {  // 16-bit stages index the E8 table
+        return GLQ_ERR_BPW;
     }
-    if (bpw == 4) {
-        if (!idx2) return GLQ_ERR_BPW;
-        if (residual && residual != primary) return GLQ_ERR_BPW;
-    }
-    if (!std::isfinite(weight_scale) || !std::isfinite(resid_scale)) return GLQ_ERR_INVALID_ARG;
+    if (!std::isfinite(weight_scale)) return GLQ_ERR_INVALID_ARG;
+    for (int k = 0; k < nres; ++k)
+        if (!std::isfinite(resid_scales[k])) return GLQ_ERR_INVALID_ARG;
     if (!all_signs(s_in, n) || !all_signs(s_out, m)) return GLQ_ERR_INVALID_ARG;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -751,33 +767,36 @@ glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *i
     L->KC = (int)(L->n_pad / GLQ_CHUNK_K);
     L->device = dev;
     L->primary = primary;
-    L->residual = bpw == 4 ? primary : residual;
+    L->residual = has8 ? residual : (n16 ? primary : nullptr);
     L->ws = weight_scale;
-    L->rs = bpw == 2 ? 0.f : resid_scale;
+    L->nres16 = n16;
+    L->has8 = has8;
+    for (int k = 0; k < n16; ++k) L->rs16[k] = resid_scales[k];
+    L->rs8 = has8 ? resid_scales[n16] : 0.f;
+    // batches of the tensor-core path reconstruct W first from 256 tokens;
+    // with more than two stages always (the dequantising producer holds two)
+    L->prefill_mat_min_b = bpw <= 4 ? 256 : GLQ_DECODE_MAX_B + 1;
     L->plan_n = glq::make_rht_plan((int)n);
     L->plan_m = glq::make_rht_plan((int)m);
     cudaDeviceGetAttribute(&L->num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (L->num_sms <= 0) L->num_sms = 1;
-    L->plan[0] = glq::plan_gemv(L->RT, L->KC, L->num_sms, glq::gemv_warps(1));
+    L->plan[0] = glq::plan_gemv(L->RT, L->KC, L->num_sms, glq::gemv_warps(1, bpw));
     // two token tiles: a band's split-K partials are twice as many, and
     // with several tasks per CTA they go through the global workspace;
     // charging 2 chunks per split (measured: 24B-class step at 16 tokens
     // 424 -> 266 us, the 32768-row layers then take one split)
-    L->plan[1] = glq::plan_gemv(L->RT, L->KC, L->num_sms, glq::gemv_warps(2), false, 1 << 30, 1 << 30, 2.0);
+    L->plan[1] = glq::plan_gemv(L->RT, L->KC, L->num_sms, glq::gemv_warps(2, bpw), false, 1 << 30, 1 << 30, 2.0);
     const int max_bands = std::max(L->plan[0].bands, L->plan[1].bands);
     L->hb_n = hadamard_blocks_of(n);
     L->hb_m = hadamard_blocks_of(m);
 
-    // fragment-native index streams (layout: glq_internal.h)
+    // fragment-native index streams (layout: glq_internal.h): the primary and
+    // every 16-bit stage as folded codes, the 8-bit stage as raw indices
     const FoldedTable &F = primary->fold;
     const size_t slots = (size_t)L->RT * L->KC * 32;
-    std::vector<uint16_t> s1(slots * 8, F.zero_code);
-    std::vector<uint16_t> s2u16;
-    std::vector<uint8_t> s2u8;
-    if (bpw == 4) s2u16.assign(slots * 8, F.zero_code);
-    if (bpw == 3) s2u8.assign(slots * 8, 0);
-    const uint16_t *i2u16 = static_cast<const uint16_t *>(idx2);
-    const uint8_t *i2u8 = static_cast<const uint8_t *>(idx2);
+    std::vector<std::vector<uint16_t>> s16(1 + n16, std::vector<uint16_t>(slots * 8, F.zero_code));
+    std::vector<uint8_t> s8;
+    if (has8) s8.assign(slots * 8, 0);
     for (int64_t r = 0; r < m; ++r) {
         const int64_t rt = r / GLQ_ROW_TILE;
         const int rr = (int)(r % GLQ_ROW_TILE);
@@ -788,28 +807,29 @@ glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *i
             const int t = grp % 4;
             const size_t slot = ((size_t)rt * L->KC + kc) * 32 + (size_t)(4 * g + t);
             const size_t src = (size_t)r * L->G + grp;
-            s1[slot * 8 + 2 * s + hi] = F.code[idx1[src]];
-            if (bpw == 4) s2u16[slot * 8 + 2 * s + hi] = F.code[i2u16[src]];
-            if (bpw == 3) s2u8[slot * 8 + 2 * s + hi] = i2u8[src];
+            const size_t dst = slot * 8 + 2 * s + hi;
+            s16[0][dst] = F.code[idx1[src]];
+            for (int k = 0; k < n16; ++k) s16[1 + k][dst] = F.code[static_cast<const uint16_t *>(idx_res[k])[src]];
+            if (has8) s8[dst] = static_cast<const uint8_t *>(idx_res[n16])[src];
         }
     }
     std::vector<uint32_t> sin_bits = pack_signs(s_in, n), sout_bits = pack_signs(s_out, m);
     size_t total = 0;
-    L->idx1_bytes = s1.size() * sizeof(uint16_t);
-    L->idx2_bytes = bpw == 4 ? s2u16.size() * 2 : (bpw == 3 ? s2u8.size() : 0);
-    glq_status st = dmalloc(&L->d_idx1, L->idx1_bytes, &total);
-    if (st == GLQ_OK && bpw > 2) st = dmalloc((char **)&L->d_idx2, L->idx2_bytes, &total);
+    const size_t bytes16 = slots * 8 * sizeof(uint16_t);
+    L->idx_bytes = bytes16 * (1 + n16) + s8.size();
+    glq_status st = dmalloc(&L->d_idx1, bytes16, &total);
+    for (int k = 0; k < n16 && st == GLQ_OK; ++k) st = dmalloc(&L->d_res16[k], bytes16, &total);
+    if (st == GLQ_OK && has8) st = dmalloc(&L->d_res8, s8.size(), &total);
     if (st == GLQ_OK) st = dmalloc(&L->d_sin, sin_bits.size() * 4, &total);
     if (st == GLQ_OK) st = dmalloc(&L->d_sout, sout_bits.size() * 4, &total);
     if (st == GLQ_OK) st = dmalloc(&L->d_err, sizeof(unsigned), &total);
     if (st == GLQ_OK) st = dmalloc(&L->d_cnt, (size_t)max_bands * sizeof(unsigned), &total);
     if (st == GLQ_OK) st = dmalloc(&L->d_blk_cnt, GLQ_MAX_BLOCKS * sizeof(unsigned), &total);
     if (st == GLQ_OK) {
-        bool ok = cudaMemcpy(L->d_idx1, s1.data(), L->idx1_bytes, cudaMemcpyHostToDevice) == cudaSuccess;
-        if (ok && bpw == 4)
-            ok = cudaMemcpy(L->d_idx2, s2u16.data(), L->idx2_bytes, cudaMemcpyHostToDevice) == cudaSuccess;
-        if (ok && bpw == 3)
-            ok = cudaMemcpy(L->d_idx2, s2u8.data(), L->idx2_bytes, cudaMemcpyHostToDevice) == cudaSuccess;
+        bool ok = cudaMemcpy(L->d_idx1, s16[0].data(), bytes16, cudaMemcpyHostToDevice) == cudaSuccess;
+        for (int k = 0; k < n16 && ok; ++k)
+            ok = cudaMemcpy(L->d_res16[k], s16[1 + k].data(), bytes16, cudaMemcpyHostToDevice) == cudaSuccess;
+        if (ok && has8) ok = cudaMemcpy(L->d_res8, s8.data(), s8.size(), cudaMemcpyHostToDevice) == cudaSuccess;
         ok = ok && cudaMemcpy(L->d_sin, sin_bits.data(), sin_bits.size() * 4, cudaMemcpyHostToDevice) ==
                        cudaSuccess;
         ok = ok && cudaMemcpy(L->d_sout, sout_bits.data(), sout_bits.size() * 4, cudaMemcpyHostToDevice) ==
@@ -827,6 +847,21 @@ glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *i
     L->device_bytes = total;
     *out = L;
     return GLQ_OK;
+}
+
+glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uint16_t *idx1, const void *idx2,
+                            glq_codebook primary, glq_codebook residual, float weight_scale,
+                            float resid_scale, const int8_t *s_in, const int8_t *s_out,
+                            glq_layer *out) {
+    if (!out) return GLQ_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (bpw < 2 || bpw > 4) return GLQ_ERR_BPW;
+    if (bpw == 2 && (idx2 || residual)) return GLQ_ERR_BPW;
+    if (bpw > 2 && !idx2) return GLQ_ERR_BPW;
+    if (!std::isfinite(resid_scale)) return GLQ_ERR_INVALID_ARG;
+    const void *res[1] = {idx2};
+    return glq_layer_create_stages(m, n, bpw, idx1, bpw > 2 ? res : nullptr, primary, residual, weight_scale,
+                                   bpw > 2 ? &resid_scale : nullptr, s_in, s_out, out);
 }
 
 glq_status glq_layer_destroy(glq_layer layer) {
@@ -900,6 +935,7 @@ glq_status glq_layer_set_fusion(glq_layer layer, int32_t flags) {
 
 glq_status glq_layer_set_prefill_reconstruct(glq_layer layer, int64_t min_batch) {
     if (!layer) return GLQ_ERR_INVALID_ARG;
+    if (layer->bpw > 4) return GLQ_OK;  // always reconstructed: the dequantising producer holds two stages
     layer->prefill_mat_min_b = min_batch < 0 ? 256 : std::max<int64_t>(min_batch, GLQ_DECODE_MAX_B + 1);
     return GLQ_OK;
 }
@@ -956,17 +992,21 @@ glq_status glq_dequant_reference(glq_layer L, float *w_dev, void *stream) {
     DeviceGuard guard(L->device);
     glq::DequantParams p{};
     p.idx1 = L->d_idx1;
-    p.idx2 = L->d_idx2;
+    for (int k = 0; k < 3; ++k) {
+        p.idx16[k] = L->d_res16[k];
+        p.rs16[k] = L->rs16[k];
+    }
+    p.idx8 = L->d_res8;
+    p.rs8 = L->rs8;
     p.table = L->primary->d_table;
     p.fold = glq::FoldParams{L->primary->fold.nb, L->primary->fold.neg_base};
-    p.res8 = (L->bpw == 3) ? reinterpret_cast<const uint4 *>(L->residual->d_fp16) : nullptr;
+    p.tab8 = L->has8 ? reinterpret_cast<const uint4 *>(L->residual->d_fp16) : nullptr;
     p.bpw = L->bpw;
     p.m = L->m;
     p.n = (int)L->n;
     p.G = L->G;
     p.KC = L->KC;
     p.ws = L->ws;
-    p.rs = L->rs;
     p.w = w_dev;
     return glq::launch_dequant(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GLQ_OK : GLQ_ERR_CUDA;
 }

@@ -1,9 +1,10 @@
 // glq_dequant.cu -- explicit reconstruction of W^ (glq 0.5.1 PyPI page,
 // "How it works" 1 and "Bit widths": a 16-bit E8 index per 8-weight group,
-// an optional 8-bit / 16-bit residual stage, one global scale per layer).
-// It reads the same device index streams and folded codebook as the GEMV
-// and decodes with the same routines, then forms
-//     w = fp32(ws * fma_f32(rs, cb2, cb1))
+// then the residual stages of the bit width (16-bit E8 stages, an 8-bit
+// stage last for an odd bpw), one global scale per layer).  It reads the
+// same device index streams and folded codebook as the GEMV and decodes
+// with the same routines, then forms, stage by stage in that order,
+//     c = cb1;  c = fma_f32(rs_k, cb_k, c);  w = fp32(ws * c)
 // with explicit round-to-nearest intrinsics (no contraction changes it).
 #include "glq_kernels.cuh"
 
@@ -28,26 +29,25 @@ __global__ void dequant_kernel(DequantParams p) {
 
     const uint32_t *w1 = reinterpret_cast<const uint32_t *>(p.idx1 + slot);
     uint32_t code1 = (w1[s] >> (16 * hi)) & 0xFFFFu;
-    float c1[8], c2[8];
-    unpack_exact(table_word_global(p.table, code1, p.fold), c1);
-    if (p.bpw == 4) {
-        const uint32_t *w2 = reinterpret_cast<const uint32_t *>(reinterpret_cast<const uint4 *>(p.idx2) + slot);
-        uint32_t code2 = (w2[s] >> (16 * hi)) & 0xFFFFu;
-        unpack_exact(table_word_global(p.table, code2, p.fold), c2);
-    } else if (p.bpw == 3) {
-        const uint8_t *b2 = reinterpret_cast<const uint8_t *>(reinterpret_cast<const uint2 *>(p.idx2) + slot);
-        uint32_t i2 = b2[2 * s + hi];
-        const __half *e = reinterpret_cast<const __half *>(p.res8 + i2);
+    float c[8], cs[8];
+    unpack_exact(table_word_global(p.table, code1, p.fold), c);
+    // the residual stages in order: 16-bit E8 stages, then the 8-bit one
+    const int n16 = stages16(p.bpw);
+    for (int k = 0; k < n16; ++k) {
+        const uint32_t *wk = reinterpret_cast<const uint32_t *>(p.idx16[k] + slot);
+        unpack_exact(table_word_global(p.table, (wk[s] >> (16 * hi)) & 0xFFFFu, p.fold), cs);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) c2[j] = __half2float(e[j]);
+        for (int j = 0; j < 8; ++j) c[j] = __fmaf_rn(p.rs16[k], cs[j], c[j]);
+    }
+    if (stage8(p.bpw)) {
+        const uint8_t *b8 = reinterpret_cast<const uint8_t *>(p.idx8 + slot);
+        const __half *e = reinterpret_cast<const __half *>(p.tab8 + b8[2 * s + hi]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) c[j] = __fmaf_rn(p.rs8, __half2float(e[j]), c[j]);
     }
     float *out = p.w + r * (int64_t)p.n + (int64_t)grp * 8;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        float c = c1[j];
-        if (p.bpw > 2) c = __fmaf_rn(p.rs, c2[j], c);
-        out[j] = __fmul_rn(p.ws, c);
-    }
+    for (int j = 0; j < 8; ++j) out[j] = __fmul_rn(p.ws, c[j]);
 }
 
 }  // namespace

@@ -96,24 +96,31 @@ __device__ __forceinline__ uint4 ld_x(const void *p) {
     return ldg_v4(p);
 }
 
+// One chunk (128 columns = 4 super-tiles of 32) of a warp's row tile: q1
+// holds the primary codes, qr[k] those of 16-bit residual stage k, q8 the
+// 8-bit stage's indices (odd bpw).
 template <int BPW, int NT, bool XS>
 __device__ __forceinline__ void process_chunk(TableRef T, const uint4 *R8, FoldParams fold, LookupConsts kc,
-                                              const uint4 &q1, const uint4 &q2, const uint4 *xq0,
-                                              const uint4 *xq1, const __half *xh0, const __half *xh1,
-                                              bool has0, bool has1, Acc &acc1, Acc &acc2,
-                                              float accr[2][4]) {
+                                              const uint4 &q1, const uint4 (&qr)[Stages<BPW>::NA],
+                                              const uint2 &q8, const uint4 *xq0, const uint4 *xq1,
+                                              const __half *xh0, const __half *xh1, bool has0, bool has1,
+                                              Acc &acc1, Acc (&accs)[Stages<BPW>::NA], float accr[2][4]) {
+    constexpr int N16 = Stages<BPW>::N16;
     const uint32_t p1[4] = {q1.x, q1.y, q1.z, q1.w};
-    const uint32_t p2[4] = {q2.x, q2.y, q2.z, q2.w};
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
         uint4 x0 = make_uint4(0, 0, 0, 0), x1 = make_uint4(0, 0, 0, 0);
         if (has0) x0 = ld_x<XS>(xq0 + 4 * s);
         if (NT == 2 && has1) x1 = ld_x<XS>(xq1 + 4 * s);
         stage_int<NT>(T, fold, kc, p1[s], x0, x1, acc1);
-        if (BPW == 4) stage_int<NT>(T, fold, kc, p2[s], x0, x1, acc2);
-        if (BPW == 3) {
+#pragma unroll
+        for (int k = 0; k < N16; ++k) {
+            const uint32_t pk[4] = {qr[k].x, qr[k].y, qr[k].z, qr[k].w};
+            stage_int<NT>(T, fold, kc, pk[s], x0, x1, accs[k]);
+        }
+        if (Stages<BPW>::U8) {
             // bytes 2s (row g) and 2s+1 (row g+8) of the 8-byte payload
-            const uint32_t word = (s < 2) ? q2.x : q2.y;
+            const uint32_t word = (s < 2) ? q8.x : q8.y;
             const uint32_t sh = (s & 1) * 16;
             const uint4 ra = R8[(word >> sh) & 0xFFu];
             const uint4 rb = R8[(word >> (sh + 8)) & 0xFFu];
@@ -132,14 +139,14 @@ __device__ __forceinline__ void process_chunk(TableRef T, const uint4 *R8, FoldP
     }
 }
 
+// The index words of chunk slot i of every stage (fragment-native streams).
 template <int BPW>
-__device__ __forceinline__ uint4 load_q2(const void *idx2, size_t i) {
-    if (BPW == 4) return ldg_nc_v4(reinterpret_cast<const uint4 *>(idx2) + i);
-    if (BPW == 3) {
-        uint2 v = ldg_nc_v2(reinterpret_cast<const uint2 *>(idx2) + i);
-        return make_uint4(v.x, v.y, 0, 0);
-    }
-    return make_uint4(0, 0, 0, 0);
+__device__ __forceinline__ void load_codes(const GemvParams &p, size_t i, uint4 &q1, uint4 (&qr)[Stages<BPW>::NA],
+                                           uint2 &q8) {
+    q1 = ldg_nc_v4(p.idx1 + i);
+#pragma unroll
+    for (int k = 0; k < Stages<BPW>::N16; ++k) qr[k] = ldg_nc_v4(p.idx16[k] + i);
+    if (Stages<BPW>::U8) q8 = ldg_nc_v2(p.idx8 + i);
 }
 
 // sum v X of one accumulator pair from its 16 v sums (exact: a multiple of 16)
@@ -351,7 +358,7 @@ __device__ __forceinline__ void warp_transform(const GemvParams &p, int b, int N
         sum += X;
         hb[j >> 2] |= (uint32_t)((X >> 8) & 0xFF) << (8 * (j & 3));
         lb[j >> 2] |= (uint32_t)(X & 0xFF) << (8 * (j & 3));
-        if (BPW == 3) xhs[(size_t)b * klen + p0 + j] = __int2half_rn(X);
+        if (Stages<BPW>::U8) xhs[(size_t)b * klen + p0 + j] = __int2half_rn(X);
     }
     // per 8-column group: 8 high bytes, then 8 low bytes
     uint32_t *xw = reinterpret_cast<uint32_t *>(xs + (size_t)b * (klen / 8));
@@ -509,7 +516,7 @@ __device__ void fused_input(const GemvParams &p, int k0, int klen, uint4 *xs, __
             sum += X;
             hb[j >> 2] |= (uint32_t)((X >> 8) & 0xFF) << (8 * (j & 3));
             lb[j >> 2] |= (uint32_t)(X & 0xFF) << (8 * (j & 3));
-            if (BPW == 3) xhs[(size_t)b * klen + 8 * v + j] = __int2half_rn(X);
+            if (Stages<BPW>::U8) xhs[(size_t)b * klen + 8 * v + j] = __int2half_rn(X);
         }
         xs[(size_t)b * nvec + v] = make_uint4(hb[0], hb[1], lb[0], lb[1]);
         atomicAdd(&rows[b].sum_x, sum);
@@ -588,9 +595,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
     uint4 *R8 = smem_u4 + p.table_words / 4;
     // fused input: [xs: B x klen/8 uint4][xhs: B x klen halves (3 bpw)][u: B x klen floats]
     const int klen_max = min(p.cps, p.KC) * GLQ_CHUNK_K;
-    uint4 *xs = R8 + (BPW == 3 ? 256 : 0);
+    uint4 *xs = R8 + (Stages<BPW>::U8 ? 256 : 0);
     __half *xhs = reinterpret_cast<__half *>(xs + (size_t)p.B * klen_max / 8);
-    float *ubuf = reinterpret_cast<float *>(xhs + (BPW == 3 ? (size_t)p.B * klen_max : 0));
+    float *ubuf = reinterpret_cast<float *>(xhs + (Stages<BPW>::U8 ? (size_t)p.B * klen_max : 0));
     // cluster reduction: the partial sums of this CTA's share of the band,
     // [split][share] (fp64), stored by every split of the cluster
     double *spart = reinterpret_cast<double *>(reinterpret_cast<char *>(smem_u4) + p.spart_off);
@@ -606,7 +613,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
     __syncthreads();
     if (tid == 0) {
         const uint32_t tbytes = (uint32_t)p.table_words * 4u;
-        const uint32_t rbytes = BPW == 3 ? 256u * 16u : 0u;
+        const uint32_t rbytes = Stages<BPW>::U8 ? 256u * 16u : 0u;
         mbar_expect_tx(&bar, tbytes + rbytes);
         const uint32_t piece = 32768u;
         for (uint32_t off = 0; off < tbytes; off += piece) {
@@ -614,12 +621,14 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
             bulk_g2s(reinterpret_cast<char *>(T) + off, reinterpret_cast<const char *>(p.table) + off,
                      len, &bar);
         }
-        if (BPW == 3) bulk_g2s(R8, p.res8, rbytes, &bar);
+        if (Stages<BPW>::U8) bulk_g2s(R8, p.tab8, rbytes, &bar);
     }
     pdl_launch_dependents();
 
     // 2. index loads of the first task (constant data: before the PDL wait)
-    uint4 r1[GEMV_PREFETCH], r2[GEMV_PREFETCH];
+    constexpr int NA = Stages<BPW>::NA;
+    uint4 r1[GEMV_PREFETCH], rq[GEMV_PREFETCH][NA];
+    uint2 r8[GEMV_PREFETCH];
     int task = blockIdx.x;
     int rt = 0, c0 = 0, c1 = 0;
     auto task_geom = [&](int tk) {
@@ -632,10 +641,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
         const size_t base = ((size_t)rt * p.KC) * 32 + lane;
 #pragma unroll
         for (int i = 0; i < GEMV_PREFETCH; ++i) {
-            if (rt < p.RT && c0 + i < c1) {
-                r1[i] = ldg_nc_v4(p.idx1 + base + (size_t)(c0 + i) * 32);
-                r2[i] = load_q2<BPW>(p.idx2, base + (size_t)(c0 + i) * 32);
-            }
+            if (rt < p.RT && c0 + i < c1) load_codes<BPW>(p, base + (size_t)(c0 + i) * 32, r1[i], rq[i], r8[i]);
         }
     };
     if (task < ntasks) {
@@ -690,22 +696,22 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
                                       s_sign_w0);
             if (first && !wait_table()) return;  // the CTA's common verdict: all threads return
         }
-        Acc acc1, acc2;
+        Acc acc1, accs[NA];
         zero<NT>(acc1);
-        zero<NT>(acc2);
+#pragma unroll
+        for (int k = 0; k < NA; ++k) zero<NT>(accs[k]);
         float accr[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 
         if (rt < p.RT) {
             const size_t base = ((size_t)rt * p.KC + c0) * 32 + lane;
-            const uint4 *pq1 = p.idx1 + base + GEMV_PREFETCH * 32;  // next chunk to load
-            const size_t q2_off = base + GEMV_PREFETCH * 32;
+            size_t q_next = base + GEMV_PREFETCH * 32;  // slot of the next chunk to load
             const uint4 *px0, *px1;
             const __half *ph0, *ph1;
             if (FIN) {  // the task's range in shared memory, row stride klen
                 px0 = xs + (size_t)g * (klen / 8) + t;
                 px1 = xs + (size_t)(g + 8) * (klen / 8) + t;
-                ph0 = BPW == 3 ? xhs + (size_t)g * klen + 8 * t : nullptr;
-                ph1 = BPW == 3 ? xhs + (size_t)(g + 8) * klen + 8 * t : nullptr;
+                ph0 = Stages<BPW>::U8 ? xhs + (size_t)g * klen + 8 * t : nullptr;
+                ph1 = Stages<BPW>::U8 ? xhs + (size_t)(g + 8) * klen + 8 * t : nullptr;
             } else {
                 px0 = xq0 + (size_t)c0 * GLQ_GROUPS_PER_CHUNK;
                 px1 = xq1 + (size_t)c0 * GLQ_GROUPS_PER_CHUNK;
@@ -717,18 +723,18 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
 #pragma unroll
                 for (int i = 0; i < GEMV_PREFETCH; ++i) {
                     if (c + i < c1) {
-                        const uint4 q1 = r1[i], q2 = r2[i];
-                        if (ahead < c1) {
-                            r1[i] = ldg_nc_v4(pq1);
-                            r2[i] = load_q2<BPW>(p.idx2, q2_off + (size_t)(ahead - c0 - GEMV_PREFETCH) * 32);
-                        }
-                        pq1 += 32;
+                        uint4 q1 = r1[i], qr[NA];
+                        uint2 q8 = r8[i];
+#pragma unroll
+                        for (int k = 0; k < NA; ++k) qr[k] = rq[i][k];
+                        if (ahead < c1) load_codes<BPW>(p, q_next, r1[i], rq[i], r8[i]);
+                        q_next += 32;
                         ++ahead;
-                        process_chunk<BPW, NT, FIN>(tref, R8, p.fold, p.kc, q1, q2, px0, px1, ph0, ph1, has0, has1,
-                                                    acc1, acc2, accr);
+                        process_chunk<BPW, NT, FIN>(tref, R8, p.fold, p.kc, q1, qr, q8, px0, px1, ph0, ph1, has0,
+                                                    has1, acc1, accs, accr);
                         px0 += GLQ_GROUPS_PER_CHUNK;
                         px1 += GLQ_GROUPS_PER_CHUNK;
-                        if (BPW == 3) {
+                        if (Stages<BPW>::U8) {
                             ph0 += GLQ_CHUNK_K;
                             ph1 += GLQ_CHUNK_K;
                         }
@@ -745,8 +751,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
                     const int row = row0 + (j >> 1) * 8;
                     if (b < p.B) {
                         double D = exact_sum(acc1.hi[nt][j], acc1.lo[nt][j]);
-                        if (BPW == 4) D += p.rs_d * exact_sum(acc2.hi[nt][j], acc2.lo[nt][j]);
-                        if (BPW == 3) D += p.rs_d * (double)accr[nt][j];
+#pragma unroll
+                        for (int k = 0; k < Stages<BPW>::N16; ++k)
+                            D += p.rs16_d[k] * exact_sum(accs[k].hi[nt][j], accs[k].lo[nt][j]);
+                        if (Stages<BPW>::U8) D += p.rs8_d * (double)accr[nt][j];
                         if (FIN) {  // this range's own scale and sum: a partial of x . w
                             D = (D - (double)GLQ_NIB_OFFSET * p.corr_mult * (double)s_rows[b].sum_x) *
                                 (0.5 * (double)s_rows[b].inv_scale);
@@ -843,7 +851,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) gemv_kernel(GemvParams p) {
     }
 }
 
-template <int BPW, int NT, bool FIN, int WARPS = gemv_warps(NT)>
+template <int BPW, int NT, bool FIN, int WARPS = gemv_warps(NT, BPW)>
 cudaError_t launch_t(const GemvParams &p, int grid, cudaStream_t s, bool pdl) {
     const size_t smem = gemv_launch_smem_bytes(p, BPW, FIN, WARPS);
     // raised once per device to the largest the library launches with (never
@@ -878,7 +886,7 @@ cudaError_t launch_t(const GemvParams &p, int grid, cudaStream_t s, bool pdl) {
 
 // Largest number of clusters of `csize` CTAs of this kernel that can be
 // resident at once (0 if the cluster does not fit).
-template <int BPW, int NT, bool FIN, int WARPS = gemv_warps(NT)>
+template <int BPW, int NT, bool FIN, int WARPS = gemv_warps(NT, BPW)>
 int max_clusters_t(int csize, size_t smem) {
     const void *fn = (const void *)gemv_kernel<BPW, NT, FIN, WARPS>;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GEMV_SMEM_LIMIT) != cudaSuccess ||
@@ -943,7 +951,7 @@ GemvPlan plan_gemv(int RT, int KC, int num_sms, int warps, bool pow2, int max_cp
 }
 
 size_t gemv_smem_bytes(int table_words, int bpw) {
-    return (size_t)table_words * 4 + (bpw == 3 ? 256 * 16 : 0);
+    return (size_t)table_words * 4 + (stage8(bpw) ? 256 * 16 : 0);
 }
 
 size_t gemv_launch_smem_bytes(const GemvParams &p, int bpw, bool fin, int warps) {
@@ -955,6 +963,16 @@ size_t gemv_launch_smem_bytes(const GemvParams &p, int bpw, bool fin, int warps)
 size_t gemv_cluster_partials_bytes(int warps, int B) {
     // splits x ceil(rows x B / splits) slots, splits <= 16
     return ((size_t)warps * GLQ_ROW_TILE * B + 16) * sizeof(double);
+}
+
+// The kernel variant of (BPW, token tiles, fused input, warps) the launcher
+// selects, and its resident-cluster count.
+template <int BPW>
+int max_clusters_sel(int nt, bool fin, int warps, int csize, size_t smem) {
+    if (fin) return nt == 1 ? max_clusters_t<BPW, 1, true>(csize, smem) : max_clusters_t<BPW, 2, true>(csize, smem);
+    if (BPW <= 4 && nt == 1 && warps == GEMV_WIDE_WARPS)
+        return max_clusters_t<BPW, 1, false, (BPW <= 4 ? GEMV_WIDE_WARPS : gemv_warps(1, BPW))>(csize, smem);
+    return nt == 1 ? max_clusters_t<BPW, 1, false>(csize, smem) : max_clusters_t<BPW, 2, false>(csize, smem);
 }
 
 int gemv_max_clusters(int bpw, int nt, bool fin, int warps, int csize, size_t smem) {
@@ -978,17 +996,15 @@ int gemv_max_clusters(int bpw, int nt, bool fin, int warps, int csize, size_t sm
             return k.n;
     }
     int n = 0;
-    if (fin) {
-        if (nt == 1) n = bpw == 2 ? max_clusters_t<2, 1, true>(csize, smem) : bpw == 3 ? max_clusters_t<3, 1, true>(csize, smem) : max_clusters_t<4, 1, true>(csize, smem);
-        else n = bpw == 2 ? max_clusters_t<2, 2, true>(csize, smem) : bpw == 3 ? max_clusters_t<3, 2, true>(csize, smem) : max_clusters_t<4, 2, true>(csize, smem);
-    } else if (nt == 1 && warps == GEMV_WIDE_WARPS) {
-        n = bpw == 2 ? max_clusters_t<2, 1, false, GEMV_WIDE_WARPS>(csize, smem)
-          : bpw == 3 ? max_clusters_t<3, 1, false, GEMV_WIDE_WARPS>(csize, smem)
-                     : max_clusters_t<4, 1, false, GEMV_WIDE_WARPS>(csize, smem);
-    } else if (nt == 1) {
-        n = bpw == 2 ? max_clusters_t<2, 1, false>(csize, smem) : bpw == 3 ? max_clusters_t<3, 1, false>(csize, smem) : max_clusters_t<4, 1, false>(csize, smem);
-    } else {
-        n = bpw == 2 ? max_clusters_t<2, 2, false>(csize, smem) : bpw == 3 ? max_clusters_t<3, 2, false>(csize, smem) : max_clusters_t<4, 2, false>(csize, smem);
+    switch (bpw) {
+        case 2: n = max_clusters_sel<2>(nt, fin, warps, csize, smem); break;
+        case 3: n = max_clusters_sel<3>(nt, fin, warps, csize, smem); break;
+        case 4: n = max_clusters_sel<4>(nt, fin, warps, csize, smem); break;
+        case 5: n = max_clusters_sel<5>(nt, fin, warps, csize, smem); break;
+        case 6: n = max_clusters_sel<6>(nt, fin, warps, csize, smem); break;
+        case 7: n = max_clusters_sel<7>(nt, fin, warps, csize, smem); break;
+        case 8: n = max_clusters_sel<8>(nt, fin, warps, csize, smem); break;
+        default: n = 0;
     }
     if (ncache < 64) cache[ncache++] = Key{dev, bpw, nt, (int)fin, warps, csize, smem, n};
     return n;
@@ -996,25 +1012,28 @@ int gemv_max_clusters(int bpw, int nt, bool fin, int warps, int csize, size_t sm
 
 size_t gemv_fused_smem_bytes(int table_words, int bpw, int B, int klen) {
     // the table is a multiple of 4 words, so the activation area is 16-byte aligned
-    return gemv_smem_bytes(table_words, bpw) + (size_t)B * klen * (2 + (bpw == 3 ? 2 : 0) + 4);
+    return gemv_smem_bytes(table_words, bpw) + (size_t)B * klen * (2 + (stage8(bpw) ? 2 : 0) + 4);
+}
+
+template <int BPW, bool FIN>
+cudaError_t launch_bpw(const GemvParams &p, int grid, cudaStream_t s, bool pdl) {
+    const bool two = p.B > 8;
+    if (BPW <= 4 && !FIN && !two && p.warps == GEMV_WIDE_WARPS)
+        return launch_t<BPW, 1, false, (BPW <= 4 ? GEMV_WIDE_WARPS : gemv_warps(1, BPW))>(p, grid, s, pdl);
+    if (p.warps != gemv_warps(two ? 2 : 1, BPW)) return cudaErrorInvalidValue;
+    return two ? launch_t<BPW, 2, FIN>(p, grid, s, pdl) : launch_t<BPW, 1, FIN>(p, grid, s, pdl);
 }
 
 template <bool FIN>
 cudaError_t launch_sel(const GemvParams &p, int bpw, int grid, cudaStream_t s, bool pdl) {
-    const bool two = p.B > 8;
-    if (!FIN && !two && p.warps == GEMV_WIDE_WARPS) {
-        switch (bpw) {
-            case 2: return launch_t<2, 1, false, GEMV_WIDE_WARPS>(p, grid, s, pdl);
-            case 3: return launch_t<3, 1, false, GEMV_WIDE_WARPS>(p, grid, s, pdl);
-            case 4: return launch_t<4, 1, false, GEMV_WIDE_WARPS>(p, grid, s, pdl);
-            default: return cudaErrorInvalidValue;
-        }
-    }
-    if (p.warps != gemv_warps(two ? 2 : 1)) return cudaErrorInvalidValue;
     switch (bpw) {
-        case 2: return two ? launch_t<2, 2, FIN>(p, grid, s, pdl) : launch_t<2, 1, FIN>(p, grid, s, pdl);
-        case 3: return two ? launch_t<3, 2, FIN>(p, grid, s, pdl) : launch_t<3, 1, FIN>(p, grid, s, pdl);
-        case 4: return two ? launch_t<4, 2, FIN>(p, grid, s, pdl) : launch_t<4, 1, FIN>(p, grid, s, pdl);
+        case 2: return launch_bpw<2, FIN>(p, grid, s, pdl);
+        case 3: return launch_bpw<3, FIN>(p, grid, s, pdl);
+        case 4: return launch_bpw<4, FIN>(p, grid, s, pdl);
+        case 5: return launch_bpw<5, FIN>(p, grid, s, pdl);
+        case 6: return launch_bpw<6, FIN>(p, grid, s, pdl);
+        case 7: return launch_bpw<7, FIN>(p, grid, s, pdl);
+        case 8: return launch_bpw<8, FIN>(p, grid, s, pdl);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -57,10 +57,16 @@ struct glq_layer_s {
     int bpw = 0, RT = 0, KC = 0, G = 0;
     int device = 0, num_sms = 0;
     glq_codebook primary = nullptr, residual = nullptr;
-    float ws = 0.f, rs = 0.f;
+    float ws = 0.f;
     uint4 *d_idx1 = nullptr;
-    void *d_idx2 = nullptr;
-    size_t idx1_bytes = 0, idx2_bytes = 0;
+    // residual stages ("Bit widths"): nres16 16-bit E8 stages, then an 8-bit
+    // stage into the 256-entry table `residual` when has8 (odd bpw)
+    int nres16 = 0;
+    bool has8 = false;
+    uint4 *d_res16[3] = {};       // fragment-native code streams of the 16-bit stages
+    uint2 *d_res8 = nullptr;      // fragment-native index stream of the 8-bit stage
+    float rs16[3] = {}, rs8 = 0.f;
+    size_t idx_bytes = 0;         // all index streams on the device
     uint32_t *d_sin = nullptr, *d_sout = nullptr;
     glq::RhtPlan plan_n{}, plan_m{};
     unsigned *d_err = nullptr;

@@ -38,7 +38,7 @@ struct RhtInParams {
     const uint32_t *sign_bits;  // bit k set: S_in[k] = -1
     RhtPlan plan;
     uint8_t *xq;        // [B][n_pad/8][16]: high bytes, low bytes of X (product path)
-    __half *xh;         // [B][n_pad] fp16 X (3 bpw residual stage) or null
+    __half *xh;         // [B][n_pad] fp16 X (the 8-bit residual stage of an odd bpw) or null
     glq_rowinfo *info;  // [B] (product path)
     float *xr_f32;      // [B][n] unscaled fp32 (test entry point) or null
     int xh_only;        // tensor-core path: write xh = fp16(xr 2^e) only (no xq, no sum)
@@ -67,8 +67,8 @@ struct RowsParams {
     __half *xh;
     glq_rowinfo *info;
     // input, decode format instead (when xq is set): X = round(xr 2^e) as
-    // [B][len_pad / 8][16] high / low bytes, X as fp16 in xh (3 bpw, may be
-    // null), info [B] = {exact sum of X, 2^-e}
+    // [B][len_pad / 8][16] high / low bytes, X as fp16 in xh (odd bpw, may
+    // be null), info [B] = {exact sum of X, 2^-e}
     uint8_t *xq;
     // output: z [B][z_ld] fp32 (summed over zsplits slices zs floats apart,
     // in order) -> y [B][len]
@@ -80,28 +80,42 @@ struct RowsParams {
     int y_dtype;  // 0 f16, 1 bf16, 2 f32
 };
 
+// Residual stages of a bit width ("Bit widths", glq 0.5.1 PyPI page): after
+// the 16-bit primary, N16 16-bit E8 stages, then an 8-bit stage (U8) for an
+// odd bpw.
+template <int BPW>
+struct Stages {
+    static constexpr int N16 = (BPW - 2) / 2;
+    static constexpr bool U8 = (BPW & 1) != 0;
+    static constexpr int NA = N16 > 0 ? N16 : 1;  // extent of per-stage arrays
+};
+__host__ __device__ constexpr int stages16(int bpw) { return (bpw - 2) / 2; }
+__host__ __device__ constexpr bool stage8(int bpw) { return (bpw & 1) != 0; }
+
 struct GemvParams {
     const uint4 *idx1;     // [RT][KC][32] 16 B
-    const void *idx2;      // [RT][KC][32] 16 B (4 bpw) / 8 B (3 bpw)
+    const uint4 *idx16[3]; // 16-bit residual stages: [RT][KC][32] 16 B each
+    const uint2 *idx8;     // the 8-bit stage: [RT][KC][32] 8 B
     const uint32_t *table; // folded nibble table (global), table_words (multiple of 4)
     int table_words;
     FoldParams fold;
     LookupConsts kc;       // 4, 16, -1 (see LookupConsts)
-    const uint4 *res8;     // 3 bpw: [256] x 8 fp16
+    const uint4 *tab8;     // odd bpw: the 256-entry table, [256] x 8 fp16
     const uint8_t *xq;     // [B][n_pad/8][16]
-    const __half *xh;      // [B][n_pad] (3 bpw)
+    const __half *xh;      // [B][n_pad] (odd bpw)
     const glq_rowinfo *info;
     int B, n_pad, KC, RT;
     int bands, splits, cps;
-    double rs_d;           // weight of the residual sum in a partial: rs (4 bpw) or 2 rs (3 bpw)
-    double corr_mult;      // (1 + rs) for 4 bpw, 1 otherwise
+    double rs16_d[3];      // weights of the 16-bit stages' sums in a partial: their scales
+    double rs8_d;          // weight of the 8-bit stage's sum: 2 x its scale
+    double corr_mult;      // 1 + the sum of the 16-bit stages' scales
     float ws;
     double *partials;      // [splits][B][m_pad]
     unsigned *counters;    // [bands], zero between launches
     float *z;              // [B][m_pad]
     int m_pad;
     unsigned *err;
-    int warps;             // warps per CTA (gemv_warps(NT), or GEMV_WIDE_WARPS)
+    int warps;             // warps per CTA (gemv_warps(NT, bpw), or GEMV_WIDE_WARPS)
     // ---- fused transforms (small B) ----
     // input: every task rotates, scales and quantises its own column range
     // of x in shared memory (no separate input-RHT launch)
@@ -129,14 +143,16 @@ struct GemvParams {
 
 struct PrefillParams {
     const uint4 *idx1;       // [RT][KC][32] 16 B, fragment-native codes
-    const void *idx2;        // 4 bpw: 16 B / 3 bpw: 8 B per slot
+    const uint4 *idx16[3];   // 16-bit residual stages, 16 B per slot
+    const uint2 *idx8;       // the 8-bit stage, 8 B per slot
     const uint4 *cb_f16;     // E8 codewords as fp16 [folded code][8] (negated entries included)
     const uint32_t *table;   // folded nibble table (W materialisation), table_words
     int table_words;
     FoldParams fold;
-    const uint4 *res8;       // 3 bpw: [256][8] fp16
+    const uint4 *tab8;       // odd bpw: [256][8] fp16
     int bpw;
-    uint32_t rs_h2;          // residual scale as fp16x2
+    uint32_t rs16_h2[3];     // the 16-bit stages' scales as fp16x2
+    uint32_t rs8_h2;         // the 8-bit stage's scale as fp16x2
     const glq_rowinfo *info; // [B]: inv_scale per token
     float ws;
     float *z;                // [ksplit][B][m_pad]: one slice of partial sums per K split
@@ -149,14 +165,15 @@ struct PrefillParams {
 
 struct DequantParams {
     const uint4 *idx1;
-    const void *idx2;
+    const uint4 *idx16[3];
+    const uint2 *idx8;
     const uint32_t *table;
     FoldParams fold;
-    const uint4 *res8;
+    const uint4 *tab8;
     int bpw;
     int64_t m;
     int n, G, KC;
-    float ws, rs;
+    float ws, rs16[3], rs8;
     float *w;  // [m][n]
 };
 
@@ -240,7 +257,8 @@ cudaError_t launch_dequant(const DequantParams &p, cudaStream_t s);
 // rebuild W from the codes.
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &xmap, const CUtensorMap *wmap, int grid,
                            cudaStream_t s, bool pdl);
-// W16 [m_pad][n_pad] fp16 = cb1 + rs cb2 (unscaled), for the materialised variant
+// W16 [m_pad][n_pad] fp16 = cb1 + rs cb2 + ... (unscaled, every residual
+// stage), for the materialised variant
 cudaError_t launch_wmat(const PrefillParams &p, __half *w16, int n_pad, int num_sms, cudaStream_t s, bool pdl);
 size_t wmat_smem_bytes(int table_words, int bpw);
 size_t prefill_smem_bytes();
@@ -248,8 +266,12 @@ int prefill_tile_tokens();  // tokens of one output tile (a multiple of the TMA 
 int prefill_tile_rows();    // weight rows of one output tile (one CTA pair)
 
 // warps per GEMV CTA (one 16-row tile each): 24 for one 8-column MMA tile
-// (B <= 8), 16 for two (B <= 16, more live registers per lane)
-__host__ __device__ constexpr int gemv_warps(int nt) { return nt == 1 ? 24 : 16; }
+// (B <= 8), 16 for two (B <= 16, more live registers per lane); from 5 bpw
+// every residual stage adds its accumulators and code registers per lane,
+// so 16 and 12
+__host__ __device__ constexpr int gemv_warps(int nt, int bpw) {
+    return bpw <= 4 ? (nt == 1 ? 24 : 16) : (nt == 1 ? 16 : 12);
+}
 // warps of the wide variant (one 8-column tile) for large layers, where the
 // GEMV is bound by instruction issue and more warps hide more latency
 // (measured on the 24B-class layers: -12 % per step against 24 warps)

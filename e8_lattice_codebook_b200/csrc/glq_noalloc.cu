@@ -89,7 +89,7 @@ extern "C" glq_status glq_linear_noalloc(glq_layer L, const void *x_dev, glq_dty
 
     // carve the array: xq | xh | info | z | counters | partials
     const size_t xq_b = align256((size_t)B * L->n_pad * 2);
-    const size_t xh_b = L->bpw == 3 ? align256((size_t)B * L->n_pad * sizeof(__half)) : 0;
+    const size_t xh_b = L->has8 ? align256((size_t)B * L->n_pad * sizeof(__half)) : 0;
     const size_t info_b = align256((size_t)B * sizeof(glq_rowinfo));
     const size_t z_b = align256((size_t)B * L->m_pad * sizeof(float));
     const int max_bands = std::max(L->plan[0].bands, L->plan[1].bands);
@@ -122,7 +122,7 @@ extern "C" glq_status glq_linear_noalloc(glq_layer L, const void *x_dev, glq_dty
         char *p = static_cast<char *>(base);
         glq_workspace w;
         w.xq = reinterpret_cast<uint8_t *>(p);
-        w.xh = L->bpw == 3 ? reinterpret_cast<__half *>(p + xq_b) : nullptr;
+        w.xh = L->has8 ? reinterpret_cast<__half *>(p + xq_b) : nullptr;
         w.info = reinterpret_cast<glq_rowinfo *>(p + xq_b + xh_b);
         w.z = reinterpret_cast<float *>(p + xq_b + xh_b + info_b);
         w.cnt = reinterpret_cast<unsigned *>(p + xq_b + xh_b + info_b + z_b);

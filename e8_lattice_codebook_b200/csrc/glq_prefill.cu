@@ -229,9 +229,9 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
             auto load_slot = [&](int kc, uint4 &a1, uint4 &a2) {
                 if (!live || kc >= p.KC) return;
                 a1 = ldg_nc_v4(p.idx1 + slot0 + (size_t)kc * 32);
-                if (BPW == 4) a2 = ldg_nc_v4(reinterpret_cast<const uint4 *>(p.idx2) + slot0 + (size_t)kc * 32);
+                if (BPW == 4) a2 = ldg_nc_v4(p.idx16[0] + slot0 + (size_t)kc * 32);
                 if (BPW == 3) {
-                    const uint2 v = ldg_nc_v2(reinterpret_cast<const uint2 *>(p.idx2) + slot0 + (size_t)kc * 32);
+                    const uint2 v = ldg_nc_v2(p.idx8 + slot0 + (size_t)kc * 32);
                     a2 = make_uint4(v.x, v.y, 0, 0);
                 }
             };
@@ -251,7 +251,7 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
                 } else if (BPW == 3) {  // bytes 2 s + hi of the 8-byte slot, s = 2h, 2h + 1
                     const uint32_t w = h ? q2.y : q2.x;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) cb[i] = live ? __ldg(p.res8 + ((w >> (8 * i)) & 0xFFu)) : make_uint4(0, 0, 0, 0);
+                    for (int i = 0; i < 4; ++i) cb[i] = live ? __ldg(p.tab8 + ((w >> (8 * i)) & 0xFFu)) : make_uint4(0, 0, 0, 0);
                 }
             };
             load_slot(kb0 >> 1, q1, q2);
@@ -260,7 +260,8 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
             for (int kb = kb0; kb < kb1; ++kb, ++it) {
                 uint4 cw[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) cw[i] = BPW == 2 ? ca[i] : hfma8(p.rs_h2, cb[i], ca[i]);
+                for (int i = 0; i < 4; ++i)
+                    cw[i] = BPW == 2 ? ca[i] : hfma8(BPW == 4 ? p.rs16_h2[0] : p.rs8_h2, cb[i], ca[i]);
                 if (kb + 1 < kb1) {  // the next step's gathers are in flight while this one is stored
                     if (((kb + 1) & 1) == 0) {
                         q1 = n1;
@@ -355,17 +356,17 @@ cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &xmap, cons
     const size_t smem = prefill_smem_bytes();
     const bool mat = wmap != nullptr;
     const void *fn;
-    switch (p.bpw * 2 + (mat ? 1 : 0)) {
+    // the kernel with W reconstructed does not depend on the bit width;
+    // the dequantising producer exists for 2-4 bpw (two stages at most)
+    switch ((mat ? 4 : p.bpw) * 2 + (mat ? 1 : 0)) {
         case 4: fn = (const void *)prefill_kernel<2, false>; break;
-        case 5: fn = (const void *)prefill_kernel<2, true>; break;
         case 6: fn = (const void *)prefill_kernel<3, false>; break;
-        case 7: fn = (const void *)prefill_kernel<3, true>; break;
         case 8: fn = (const void *)prefill_kernel<4, false>; break;
         case 9: fn = (const void *)prefill_kernel<4, true>; break;
         default: return cudaErrorInvalidValue;
     }
     static std::atomic<uint64_t> configured[10];  // per variant: devices set
-    const int key = p.bpw * 2 + (mat ? 1 : 0);
+    const int key = (mat ? 4 : p.bpw) * 2 + (mat ? 1 : 0);
     const cudaError_t e = once_per_device(configured[key], [fn] {
         return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GEMV_SMEM_LIMIT);
     });

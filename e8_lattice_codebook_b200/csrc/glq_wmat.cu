@@ -1,6 +1,7 @@
 // glq_wmat.cu -- the weights of a layer reconstructed once into an fp16
-// matrix W16[m_pad][n_pad] = cb1 + rs cb2 (the per-layer scale ws is applied
-// in the GEMM epilogue), for the tensor-core path at large batches
+// matrix W16[m_pad][n_pad] = cb1 + rs_1 cb_1 + rs_2 cb_2 + ... (every
+// residual stage in order, one fp16 fma each; the per-layer scale ws is
+// applied in the GEMM epilogue), for the tensor-core path at large batches
 // (glq 0.5.1 PyPI page, "How it works" 1 and 4, "Bit widths"; the pages'
 // kernels never materialise W -- see the layer API for when this path runs).
 //
@@ -67,13 +68,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1) wmat_kernel(PrefillParams p, __
     if (tid == 0) mbar_init(&bar, 1);
     __syncthreads();
     if (tid == 0) {
-        const uint32_t tbytes = (uint32_t)p.table_words * 4u, rbytes = BPW == 3 ? 256u * 16u : 0u;
+        const uint32_t tbytes = (uint32_t)p.table_words * 4u, rbytes = Stages<BPW>::U8 ? 256u * 16u : 0u;
         mbar_expect_tx(&bar, tbytes + rbytes);
         for (uint32_t off = 0; off < tbytes; off += 32768u) {
             const uint32_t len = tbytes - off < 32768u ? tbytes - off : 32768u;
             bulk_g2s(reinterpret_cast<char *>(T) + off, reinterpret_cast<const char *>(p.table) + off, len, &bar);
         }
-        if (BPW == 3) bulk_g2s(const_cast<uint4 *>(R8), p.res8, rbytes, &bar);
+        if (Stages<BPW>::U8) bulk_g2s(const_cast<uint4 *>(R8), p.tab8, rbytes, &bar);
     }
     pdl_launch_dependents();
     const bool ok = __syncthreads_and(mbar_wait_bounded(&bar, 0, 1u << 24) ? 1 : 0) != 0;
@@ -85,34 +86,43 @@ __global__ void __launch_bounds__(WARPS * 32, 1) wmat_kernel(PrefillParams p, __
     pdl_wait();  // the previous user of w16 (the GEMM of an earlier call) has finished
     const long long items = (long long)p.RT * p.KC;
     const long long stride = (long long)gridDim.x * WARPS;
-    auto load_codes = [&](long long it, uint4 &a1, uint4 &a2) {
+    constexpr int N16 = Stages<BPW>::N16, NA = Stages<BPW>::NA;
+    auto load_codes = [&](long long it, uint4 &a1, uint4 (&ar)[NA], uint2 &a8) {
         const size_t slot = it * 32 + lane;  // [RT][KC][32]
         a1 = ldg_nc_v4(p.idx1 + slot);
-        a2 = make_uint4(0, 0, 0, 0);
-        if (BPW == 4) a2 = ldg_nc_v4(reinterpret_cast<const uint4 *>(p.idx2) + slot);
-        if (BPW == 3) {
-            const uint2 v = ldg_nc_v2(reinterpret_cast<const uint2 *>(p.idx2) + slot);
-            a2 = make_uint4(v.x, v.y, 0, 0);
-        }
+#pragma unroll
+        for (int k = 0; k < N16; ++k) ar[k] = ldg_nc_v4(p.idx16[k] + slot);
+        if (Stages<BPW>::U8) a8 = ldg_nc_v2(p.idx8 + slot);
     };
     long long it = (long long)blockIdx.x * WARPS + warp;
-    uint4 n1 = make_uint4(0, 0, 0, 0), n2 = n1;  // the codes of the warp's next item
-    if (it < items) load_codes(it, n1, n2);
+    // the codes of the warp's next item
+    uint4 n1 = make_uint4(0, 0, 0, 0), nr[NA];
+    uint2 n8 = make_uint2(0, 0);
+#pragma unroll
+    for (int k = 0; k < NA; ++k) nr[k] = n1;
+    if (it < items) load_codes(it, n1, nr, n8);
     for (; it < items; it += stride) {
-        const uint4 q1 = n1, q2 = n2;
-        if (it + stride < items) load_codes(it + stride, n1, n2);
+        uint4 q1 = n1, qr[NA];
+        const uint2 q8 = n8;
+#pragma unroll
+        for (int k = 0; k < NA; ++k) qr[k] = nr[k];
+        if (it + stride < items) load_codes(it + stride, n1, nr, n8);
         const int rt = (int)(it / p.KC), kc = (int)(it - (long long)rt * p.KC);
-        const uint32_t c1[4] = {q1.x, q1.y, q1.z, q1.w}, c2[4] = {q2.x, q2.y, q2.z, q2.w};
+        const uint32_t c1[4] = {q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
         for (int s = 0; s < 4; ++s)
 #pragma unroll
             for (int hi = 0; hi < 2; ++hi) {
                 uint4 cw = expand_word(fold_word(T, hi ? (c1[s] >> 16) : (c1[s] & 0xFFFFu), p.fold));
-                if (BPW == 4)
-                    cw = hfma8(p.rs_h2, expand_word(fold_word(T, hi ? (c2[s] >> 16) : (c2[s] & 0xFFFFu), p.fold)), cw);
-                if (BPW == 3) {  // byte 2 s + hi of the 8-byte slot
-                    const uint32_t i2 = ((s < 2 ? c2[0] : c2[1]) >> (8 * (2 * (s & 1) + hi))) & 0xFFu;
-                    cw = hfma8(p.rs_h2, R8[i2], cw);
+#pragma unroll
+                for (int k = 0; k < N16; ++k) {  // the 16-bit stages in order
+                    const uint32_t ck[4] = {qr[k].x, qr[k].y, qr[k].z, qr[k].w};
+                    cw = hfma8(p.rs16_h2[k], expand_word(fold_word(T, hi ? (ck[s] >> 16) : (ck[s] & 0xFFFFu), p.fold)),
+                               cw);
+                }
+                if (Stages<BPW>::U8) {  // the 8-bit stage last: byte 2 s + hi of the 8-byte slot
+                    const uint32_t i2 = ((s < 2 ? q8.x : q8.y) >> (8 * (2 * (s & 1) + hi))) & 0xFFu;
+                    cw = hfma8(p.rs8_h2, R8[i2], cw);
                 }
                 const int row = rt * GLQ_ROW_TILE + g + 8 * hi;
                 const int col = kc * GLQ_CHUNK_K + 8 * (4 * s + t);
@@ -123,12 +133,21 @@ __global__ void __launch_bounds__(WARPS * 32, 1) wmat_kernel(PrefillParams p, __
 
 }  // namespace
 
-size_t wmat_smem_bytes(int table_words, int bpw) { return (size_t)table_words * 4 + (bpw == 3 ? 256 * 16 : 0); }
+size_t wmat_smem_bytes(int table_words, int bpw) { return (size_t)table_words * 4 + (stage8(bpw) ? 256 * 16 : 0); }
 
 cudaError_t launch_wmat(const PrefillParams &p, __half *w16, int n_pad, int num_sms, cudaStream_t s, bool pdl) {
-    const void *fn = p.bpw == 4 ? (const void *)wmat_kernel<4>
-                                : (p.bpw == 3 ? (const void *)wmat_kernel<3> : (const void *)wmat_kernel<2>);
-    static std::atomic<uint64_t> configured[5];  // per bit width: devices set
+    const void *fn = nullptr;
+    switch (p.bpw) {
+        case 2: fn = (const void *)wmat_kernel<2>; break;
+        case 3: fn = (const void *)wmat_kernel<3>; break;
+        case 4: fn = (const void *)wmat_kernel<4>; break;
+        case 5: fn = (const void *)wmat_kernel<5>; break;
+        case 6: fn = (const void *)wmat_kernel<6>; break;
+        case 7: fn = (const void *)wmat_kernel<7>; break;
+        case 8: fn = (const void *)wmat_kernel<8>; break;
+        default: return cudaErrorInvalidValue;
+    }
+    static std::atomic<uint64_t> configured[9];  // per bit width: devices set
     const cudaError_t e = once_per_device(configured[p.bpw], [fn] {
         return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     (int)wmat_smem_bytes(GLQ_TABLE_MAX_WORDS, 3));

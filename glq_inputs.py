@@ -18,7 +18,10 @@ Recipe (numpy PCG64, ``numpy.random.default_rng``):
     20 for every token; x is then rounded to fp16 or bf16 (nearest even).
 
 The workloads mirror the shapes of the models the GLQ project pages serve
-(SmolLM2-360M, SmolLM3-3B, a 24B-class model, an 8B-class MLP prefill).
+(SmolLM2-360M, SmolLM3-3B, a 24B-class model, an 8B-class MLP prefill), plus
+the 24B-class shapes at 5 and 6 bpw and a mixed-precision SmolLM3-3B-shaped
+set (the pages' 3.5 / 4.5 bpw "mixed" checkpoints are layers of different
+bit widths).
 """
 from __future__ import annotations
 
@@ -50,6 +53,10 @@ class Workload:
     resid_scale: float = 0.125
     outliers: bool = False
     extra: dict = field(default_factory=dict)
+    layer_bpw: tuple = ()  # per-layer bit widths of a mixed-precision model (overrides bpw)
+
+    def bpw_of(self, layer_id: int) -> int:
+        return self.layer_bpw[layer_id] if self.layer_bpw else self.bpw
 
 
 WORKLOADS = {
@@ -81,6 +88,31 @@ WORKLOADS = {
                 LayerSpec("gate", 32768, 5120), LayerSpec("up", 32768, 5120),
                 LayerSpec("down", 5120, 32768)),
         batches=(1, 2, 4, 8, 16)),
+    "24b-decode-5bpw": Workload(
+        "24b-decode-5bpw",
+        "24B-class decode at 5 bpw (uint16 + uint16 E8 + uint8 residual stages, scales 1/8, 1/64), bf16 x",
+        seed=13, bpw=5, x_dtype="bf16",
+        layers=(LayerSpec("q", 4096, 5120), LayerSpec("o", 5120, 4096),
+                LayerSpec("gate", 32768, 5120), LayerSpec("up", 32768, 5120),
+                LayerSpec("down", 5120, 32768)),
+        batches=(1, 16)),
+    "24b-decode-6bpw": Workload(
+        "24b-decode-6bpw",
+        "24B-class decode at 6 bpw (uint16 + two uint16 E8 residual stages, scales 1/8, 1/64), bf16 x",
+        seed=14, bpw=6, x_dtype="bf16",
+        layers=(LayerSpec("q", 4096, 5120), LayerSpec("o", 5120, 4096),
+                LayerSpec("gate", 32768, 5120), LayerSpec("up", 32768, 5120),
+                LayerSpec("down", 5120, 32768)),
+        batches=(1, 16)),
+    "smollm3-3b-mixed": Workload(
+        "smollm3-3b-mixed",
+        "SmolLM3-3B-shaped projections, mixed precision: q, o at 4 bpw; gate, up, down at 5 bpw "
+        "(4.64 bpw by weight), bf16 x",
+        seed=15, bpw=5, x_dtype="bf16",
+        layers=(LayerSpec("q", 2048, 2048), LayerSpec("o", 2048, 2048),
+                LayerSpec("gate", 11008, 2048), LayerSpec("up", 11008, 2048),
+                LayerSpec("down", 2048, 11008)),
+        batches=(1, 4), layer_bpw=(4, 4, 5, 5, 5)),
     "prefill-8b-mlp-4bpw": Workload(
         "prefill-8b-mlp-4bpw",
         "prefill GEMM at 4 bpw, 14336x4096 and 4096x14336, bf16 x with 1% outlier columns x20",
@@ -179,7 +211,7 @@ def make_x(seed: int, layer_id: int, B: int, n: int, x_dtype: str,
 
 def workload_layer(wl: Workload, layer_id: int) -> LayerInputs:
     spec = wl.layers[layer_id]
-    return make_layer(wl.seed, layer_id, spec.m, spec.n, wl.bpw, wl.weight_scale, wl.resid_scale)
+    return make_layer(wl.seed, layer_id, spec.m, spec.n, wl.bpw_of(layer_id), wl.weight_scale, wl.resid_scale)
 
 
 def workload_x(wl: Workload, layer_id: int, B: int) -> np.ndarray:

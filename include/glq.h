@@ -23,7 +23,9 @@
  *   - codeword of group g in row r covers input columns 8g..8g+7; index
  *     arrays are row-major [m][n/8];
  *   - w^[r][8g+j] = ws * (cb1[idx1][j] + rs * cb2[idx2][j]) where rs is the
- *     multiplier applied at decode (the pages' inverse residual scale);
+ *     multiplier applied at decode (the pages' inverse residual scale); from
+ *     5 bpw every residual stage k adds rs_k * cb_k[idx_k][j], in the order
+ *     of the "Bit widths" table (16-bit E8 stages, then the 8-bit stage);
  *   - H_k[i][j] = (-1)^popcount(i & j) / sqrt(k) per block, blocks of the
  *     binary decomposition of n in descending size at increasing offsets;
  *   - input side: sign then H_n; output side: H_m then sign.
@@ -58,7 +60,7 @@ typedef enum {
     GLQ_ERR_INVALID_ARG = 1,  /* null pointer, bad sign value, bad scale */
     GLQ_ERR_SHAPE = 2,        /* m, n not positive multiples of 8; B < 0; size limits */
     GLQ_ERR_DTYPE = 3,        /* unsupported dtype combination */
-    GLQ_ERR_BPW = 4,          /* bpw not in {2,3,4} or inconsistent residual */
+    GLQ_ERR_BPW = 4,          /* bpw not in 2..8 or inconsistent residual stages */
     GLQ_ERR_NO_CODEBOOK = 5,  /* missing or wrong-sized codebook handle */
     GLQ_ERR_OOM = 6,          /* device or host allocation failed */
     GLQ_ERR_CUDA = 7,         /* a CUDA runtime call or launch failed */
@@ -139,6 +141,31 @@ GLQ_API glq_status glq_layer_create(int64_t m, int64_t n, int32_t bpw, const uin
                             const void *idx2, glq_codebook primary, glq_codebook residual,
                             float weight_scale, float resid_scale, const int8_t *s_in,
                             const int8_t *s_out, glq_layer *out);
+
+/*
+ * glq_layer_create_stages -- glq_layer_create for every bit width of the
+ * "Bit widths" table on the glq 0.5.1 PyPI page: bpw 2..8 is a 16-bit
+ * primary E8 index per 8 weights followed by (bpw - 2) / 2 residual stages of
+ * 16-bit E8 indices and, for an odd bpw, one last stage of 8-bit indices
+ * into a 256-entry table (5 = 16+16+8, 6 = 16+16+16, 7 = 16+16+16+8,
+ * 8 = 16+16+16+16).  Mixed-precision models are layers of different bpw.
+ * w^[r][8g+j] = ws * c with c = cb1[idx1][j], then for each residual stage k
+ *   in that order c = fma_f32(rs_k, cb_k[idx_k][j], c).
+ * idx_res: host array of pointers, one per residual stage in stage order:
+ *   uint16 [m][n/8] for a 16-bit stage, uint8 [m][n/8] for the 8-bit stage
+ *   (may be NULL for bpw 2).  Read during the call only.
+ * resid_scales: host float per residual stage (same order), finite.
+ * residual: the 256-entry codebook for an odd bpw; otherwise NULL or the
+ *   primary handle (16-bit stages index the E8 table).
+ * Tensor-core calls (B > 16) of a layer above 4 bpw always reconstruct W in
+ *   fp16 first (one fp16 fma per stage).
+ * Other arguments, ownership and errors as glq_layer_create.  Synchronous.
+ */
+GLQ_API glq_status glq_layer_create_stages(int64_t m, int64_t n, int32_t bpw, const uint16_t *idx1,
+                                           const void *const *idx_res, glq_codebook primary,
+                                           glq_codebook residual, float weight_scale,
+                                           const float *resid_scales, const int8_t *s_in,
+                                           const int8_t *s_out, glq_layer *out);
 GLQ_API glq_status glq_layer_destroy(glq_layer layer);
 
 /*
@@ -246,7 +273,8 @@ GLQ_API glq_status glq_layer_set_prefill_reconstruct(glq_layer layer, int64_t mi
 /*
  * glq_dequant_reference -- materialise W^ (fp32, no Hadamards, ws included)
  * into w_dev [m][n] row-major, using the same on-chip decode the GEMV uses.
- * Each value is fp32(ws * fma_f32(rs, cb2, cb1)) (single roundings).
+ * Each value is fp32(ws * fma_f32(rs, cb2, cb1)) (single roundings); from 5
+ * bpw one fma_f32 per residual stage in stage order.
  * Errors: GLQ_ERR_INVALID_ARG, GLQ_ERR_CUDA.  Asynchronous.
  */
 GLQ_API glq_status glq_dequant_reference(glq_layer layer, float *w_dev, void *stream);

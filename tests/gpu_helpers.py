@@ -27,7 +27,7 @@ class Device:
     def layer(self, L: gi.LayerInputs):
         glq = self.glq
         res = None
-        if L.bpw == 3:
+        if L.bpw % 2:
             res = glq.Codebook(L.cb2_f16.reshape(256, 8))
         elif L.bpw == 4:
             res = self.e8

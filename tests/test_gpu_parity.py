@@ -121,7 +121,10 @@ _LAYERS = {}
 
 
 def _workload_layer(dev, key, li):
-    """Host inputs and device layer of one workload layer, built once per module."""
+    """Host inputs and device layer of one workload layer, built once (the
+    layers of the previous workload are released first)."""
+    if any(k != key for k, _ in _LAYERS):
+        _LAYERS.clear()
     if (key, li) not in _LAYERS:
         L = gi.workload_layer(gi.WORKLOADS[key], li)
         _LAYERS[(key, li)] = (L, dev.layer(L))
@@ -149,7 +152,8 @@ def test_linear_workloads_full_size(dev, key, li, B):
         sample = list(range(B))
     else:
         rng = np.random.default_rng(1000 * li + B)
-        sample = sorted(set([0, 511, 512, B - 1] + [int(t) for t in rng.choice(B, size=3, replace=False)]))
+        sample = sorted(set([t for t in (0, 511, 512) if t < B] + [B - 1] +
+                            [int(t) for t in rng.choice(B, size=3, replace=False)]))
     ref = orc.linear(L.m, L.n, L.bpw, L.idx1, L.idx2, L.weight_scale, L.resid_scale, L.s_in, L.s_out,
                      xb[sample], wl.x_dtype == "bf16", cb2=L.cb2_f16, threads=0)
     err = np.max(np.abs(y[sample] - ref))
@@ -167,8 +171,6 @@ def test_linear_workloads_full_size(dev, key, li, B):
             ref_w = orc.decode_rows(L.m, L.n, L.bpw, L.idx1, L.idx2, L.weight_scale, L.resid_scale,
                                     r, r + 1, cb2=L.cb2_f16)
             np.testing.assert_array_equal(wr[i], ref_w[0])
-    if key == "24b-decode-4bpw" and li == len(wl.layers) - 1 and B == wl.batches[-1]:
-        _LAYERS.clear()  # release the 24B-class layers before the prefill workload
 
 
 def test_determinism_and_batch_invariance(dev):
