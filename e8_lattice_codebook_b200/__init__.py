@@ -40,6 +40,7 @@ EXPORTS = (
     "glq_layer_check", "glq_layer_info", "glq_gemv_replay", "glq_linear_noalloc", "glq_decode_plan",
     "glq_prefill_replay", "glq_layer_set_fusion", "glq_layer_set_prefill_reconstruct",
     "glq_workspace_info", "glq_workspace_release", "glq_layer_create_stages",
+    "glq_layer_set_batch_invariant",
 )
 
 
@@ -74,6 +75,7 @@ _SIGNATURES = {
     "glq_prefill_replay": ([_vp, _i64, _vp], ctypes.c_int),
     "glq_layer_set_fusion": ([_vp, ctypes.c_int32], ctypes.c_int),
     "glq_layer_set_prefill_reconstruct": ([_vp, _i64], ctypes.c_int),
+    "glq_layer_set_batch_invariant": ([_vp, ctypes.c_int32], ctypes.c_int),
     "glq_decode_plan": ([_vp, _i64, ctypes.POINTER(_i32), ctypes.POINTER(_i32), ctypes.POINTER(_i32),
                          ctypes.POINTER(_i32), ctypes.POINTER(_i32)], ctypes.c_int),
     "glq_layer_info": ([_vp, ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i32),
@@ -240,6 +242,10 @@ def glq_layer_set_prefill_reconstruct(handle, min_batch: int) -> None:
     _ok(_L().glq_layer_set_prefill_reconstruct(handle, int(min_batch)), "glq_layer_set_prefill_reconstruct")
 
 
+def glq_layer_set_batch_invariant(handle, enable: bool) -> None:
+    _ok(_L().glq_layer_set_batch_invariant(handle, 1 if enable else 0), "glq_layer_set_batch_invariant")
+
+
 def glq_layer_check(handle, stream) -> None:
     _ok(_L().glq_layer_check(handle, stream), "glq_layer_check")
 
@@ -390,6 +396,10 @@ class GlqLinear:
     def set_prefill_reconstruct(self, min_batch: int):
         """Batches >= min_batch reconstruct W in fp16 first (-1: default)."""
         glq_layer_set_prefill_reconstruct(self.handle, min_batch)
+
+    def set_batch_invariant(self, enable: bool):
+        """Every token's output independent of the batch size and path."""
+        glq_layer_set_batch_invariant(self.handle, enable)
 
     def prefill_replay(self, B, stream=None):
         glq_prefill_replay(self.handle, B, _stream_ptr(stream))

@@ -174,6 +174,16 @@ void decode_need(glq_layer L, int64_t rows, WsNeed &n) {
     n.b[WS_Z] = std::max(n.b[WS_Z], (size_t)rows * L->m_pad * sizeof(float));
 }
 
+// Buffers of a batch-invariant call of B tokens: activations, row info and
+// outputs for every token, split-K partial sums for one 16-token slice.
+void invariant_need(glq_layer L, int64_t B, WsNeed &n) {
+    decode_need(L, std::min<int64_t>(B, GLQ_DECODE_MAX_B), n);
+    n.b[WS_XQ] = std::max(n.b[WS_XQ], (size_t)B * L->n_pad * 2);
+    if (L->has8) n.b[WS_XH] = std::max(n.b[WS_XH], (size_t)B * L->n_pad * sizeof(__half));
+    n.b[WS_INFO] = std::max(n.b[WS_INFO], (size_t)B * sizeof(glq_rowinfo));
+    n.b[WS_Z] = std::max(n.b[WS_Z], (size_t)B * L->m_pad * sizeof(float));
+}
+
 int choose_ksplit(glq_layer L, int64_t B, int tiles);
 int prefill_tiles(glq_layer L, int64_t B);
 
@@ -189,7 +199,10 @@ void prefill_need(glq_layer L, int64_t B, WsNeed &n) {
 glq_workspace decode_view(glq_layer L, void *const buf[WS_COUNT]) {
     glq_workspace w;
     w.xq = static_cast<uint8_t *>(buf[WS_XQ]);
-    w.xh = static_cast<__half *>(buf[WS_XH]);
+    // the fp16 activations exist for the 8-bit stage only: the buffer may be
+    // held (sized by an odd-bpw layer) while this layer needs none, and a
+    // non-null pointer makes the input transform write it
+    w.xh = L->has8 ? static_cast<__half *>(buf[WS_XH]) : nullptr;
     w.info = static_cast<glq_rowinfo *>(buf[WS_INFO]);
     w.part = static_cast<double *>(buf[WS_PART]);
     w.z = static_cast<float *>(buf[WS_Z]);
@@ -419,6 +432,8 @@ constexpr long long FUSED_OUT_MAX_VALUES = 32768;
 // separate, parallel kernel at every size measured, so it is off by default.
 constexpr int FUSE_DEFAULT_FLAGS = GLQ_FUSE_INPUT | GLQ_SPLITK_CLUSTER;
 
+void choose_cluster(glq_layer L, int nb, int flags, DecodeCfg &c);
+
 DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y_dtype, int max_splits) {
     DecodeCfg c;
     const int nt = nb > 8 ? 2 : 1;
@@ -463,8 +478,15 @@ DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y
         if (c.plan.splits > max_splits)
             c.plan = plan_gemv(L->RT, L->KC, L->num_sms, c.warps, false, 1 << 30, max_splits);
     }
-    // split-K through a thread-block cluster: one task per CTA, the band's
-    // splits in one cluster (at most 16), all clusters resident at once
+    choose_cluster(L, nb, flags, c);
+    return c;
+}
+
+// Split-K through a thread-block cluster: one task per CTA, the band's
+// splits in one cluster (at most 16), all clusters resident at once.  The
+// summation order is that of the global reduction.
+void choose_cluster(glq_layer L, int nb, int flags, DecodeCfg &c) {
+    const int nt = nb > 8 ? 2 : 1;
     const int S = c.plan.splits;
     if ((flags & GLQ_SPLITK_CLUSTER) && S > 1 && S <= 16 && !c.fout &&
         (long long)c.plan.bands * S == (long long)c.plan.grid) {
@@ -478,6 +500,21 @@ DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y
             c.spart_off = off;
         }
     }
+}
+
+DecodeCfg invariant_config(glq_layer L, int nb) {
+    DecodeCfg c;
+    const int nt = nb > 8 ? 2 : 1;
+    c.warps = gemv_warps(nt, L->bpw);
+    // the chunks per split of the layer's one-token plan, for every slice
+    const int cps = L->plan[0].cps;
+    c.plan.cps = cps;
+    c.plan.splits = (L->KC + cps - 1) / cps;
+    c.plan.bands = (L->RT + c.warps - 1) / c.warps;
+    const long long tasks = (long long)c.plan.bands * c.plan.splits;
+    c.plan.grid = (int)std::min<long long>(tasks, L->num_sms);
+    const int flags = L->fusion < 0 ? FUSE_DEFAULT_FLAGS : L->fusion;
+    choose_cluster(L, nb, flags, c);
     return c;
 }
 
@@ -613,6 +650,113 @@ cudaError_t run_decode(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg
     pout.y = y;
     pout.y_dtype = y_dtype;
     return launch_rht_out(pout, s, true);
+}
+
+// The batch-invariant mode (glq_layer_set_batch_invariant): every batch
+// takes the exact decode arithmetic.  The input transform (the kernel chosen
+// by n alone) rotates and quantises every token, the GEMV runs on slices of
+// at most 16 tokens with the split plan of invariant_config (the same for
+// every slice size), and the output transform (the kernel chosen by m alone)
+// rotates every token: each token's y is the same bits whatever the batch.
+glq_status run_invariant(glq_layer L, const void *x, bool x_bf16, void *y, int y_dtype, int64_t B,
+                         cudaStream_t s, void *const buf[], size_t xq_row_bytes) {
+    glq_workspace w;
+    w.xq = static_cast<uint8_t *>(buf[0]);
+    w.xh = L->has8 ? static_cast<__half *>(buf[1]) : nullptr;  // 8-bit stage only
+    w.info = static_cast<glq_rowinfo *>(buf[2]);
+    w.part = static_cast<double *>(buf[3]);
+    w.z = static_cast<float *>(buf[4]);
+    w.cnt = L->d_cnt;
+    for (int64_t b0 = 0; b0 < B;) {  // input transform, every token
+        const int nb = (int)std::min<int64_t>(B - b0, 65535);
+        const void *xb = static_cast<const char *>(x) + (size_t)b0 * L->n * 2;
+        cudaError_t e;
+        if (rht_rows_supported((int)L->n_pad)) {
+            RowsParams r{};
+            r.len = (int)L->n;
+            r.len_pad = (int)L->n_pad;
+            r.nblk = L->hb_n.count;
+            r.max_blk = L->hb_n.count ? L->hb_n.len[0] : 0;
+            for (int i = 0; i < L->hb_n.count; ++i) {
+                r.blk_off[i] = L->hb_n.off[i];
+                r.blk_len[i] = L->hb_n.len[i];
+                r.blk_norm[i] = (float)(1.0 / std::sqrt((double)L->hb_n.len[i]));
+            }
+            r.sign_bits = L->d_sin;
+            r.zsplits = 1;
+            r.x = xb;
+            r.x_bf16 = x_bf16 ? 1 : 0;
+            r.xq = w.xq + (size_t)b0 * xq_row_bytes;
+            r.xh = w.xh ? w.xh + (size_t)b0 * L->n_pad : nullptr;
+            r.info = w.info + b0;
+            e = launch_rht_rows(r, true, nb, s, true);
+        } else {
+            RhtInParams pin{};
+            pin.x = xb;
+            pin.x_bf16 = x_bf16 ? 1 : 0;
+            pin.n = (int)L->n;
+            pin.n_pad = (int)L->n_pad;
+            pin.B = nb;
+            pin.sign_bits = L->d_sin;
+            pin.plan = L->plan_n;
+            pin.xq = w.xq + (size_t)b0 * xq_row_bytes;
+            pin.xh = w.xh ? w.xh + (size_t)b0 * L->n_pad : nullptr;
+            pin.info = w.info + b0;
+            e = launch_rht_in(pin, s, true);
+        }
+        if (e != cudaSuccess) return GLQ_ERR_CUDA;
+        b0 += nb;
+    }
+    for (int64_t b0 = 0; b0 < B; b0 += GLQ_DECODE_MAX_B) {  // GEMV, 16 tokens at a time
+        const int nb = (int)std::min<int64_t>(B - b0, GLQ_DECODE_MAX_B);
+        glq_workspace ws = w;
+        ws.xq = w.xq + (size_t)b0 * xq_row_bytes;
+        ws.xh = w.xh ? w.xh + (size_t)b0 * L->n_pad : nullptr;
+        ws.info = w.info + b0;
+        ws.z = w.z + (size_t)b0 * L->m_pad;
+        const DecodeCfg cfg = invariant_config(L, nb);
+        if (launch_gemv(gemv_params(L, ws, cfg, nb, nullptr, x_bf16, nullptr, y_dtype), L->bpw, cfg.plan.grid, s,
+                        true, false) != cudaSuccess)
+            return GLQ_ERR_CUDA;
+    }
+    for (int64_t b0 = 0; b0 < B;) {  // output transform, every token
+        const int nb = (int)std::min<int64_t>(B - b0, 65535);
+        void *yb = static_cast<char *>(y) + (size_t)b0 * L->m * (y_dtype == GLQ_F32 ? 4 : 2);
+        cudaError_t e;
+        if (rht_rows_supported((int)L->m)) {
+            RowsParams r{};
+            r.len = (int)L->m;
+            r.len_pad = (int)L->m;
+            r.nblk = L->hb_m.count;
+            r.max_blk = L->hb_m.count ? L->hb_m.len[0] : 0;
+            for (int i = 0; i < L->hb_m.count; ++i) {
+                r.blk_off[i] = L->hb_m.off[i];
+                r.blk_len[i] = L->hb_m.len[i];
+                r.blk_norm[i] = (float)(1.0 / std::sqrt((double)L->hb_m.len[i]));
+            }
+            r.sign_bits = L->d_sout;
+            r.zsplits = 1;
+            r.z = w.z + (size_t)b0 * L->m_pad;
+            r.z_ld = (int)L->m_pad;
+            r.y = yb;
+            r.y_dtype = y_dtype;
+            e = launch_rht_rows(r, false, nb, s, true);
+        } else {
+            RhtOutParams pout{};
+            pout.m = (int)L->m;
+            pout.B = nb;
+            pout.z = w.z + (size_t)b0 * L->m_pad;
+            pout.z_ld = (int)L->m_pad;
+            pout.sign_bits = L->d_sout;
+            pout.plan = L->plan_m;
+            pout.y = yb;
+            pout.y_dtype = y_dtype;
+            e = launch_rht_out(pout, s, true);
+        }
+        if (e != cudaSuccess) return GLQ_ERR_CUDA;
+        b0 += nb;
+    }
+    return GLQ_OK;
 }
 
 }  // namespace glq
@@ -877,6 +1021,7 @@ glq_status glq_layer_reserve(glq_layer layer, int64_t max_B) {
     DeviceGuard guard(layer->device);
     WsNeed need;
     decode_need(layer, std::max<int64_t>(max_B, 1), need);
+    if (layer->invariant) invariant_need(layer, std::max<int64_t>(max_B, 1), need);
     // every tensor-core batch up to max_B (the K-split count, and with it
     // the partial-sum slices, depends on the batch); past 65536 tokens the
     // output has far more tiles than CTA pairs and the largest batch decides
@@ -916,7 +1061,8 @@ glq_status glq_decode_plan(glq_layer layer, int64_t B, int32_t *warps, int32_t *
     if (B < 1 || B > GLQ_DECODE_MAX_B) return GLQ_ERR_SHAPE;
     DeviceGuard guard(layer->device);
     const void *aligned = reinterpret_cast<const void *>(static_cast<uintptr_t>(256));
-    const glq::DecodeCfg c = glq::decode_config(layer, (int)B, aligned, aligned, GLQ_F32);
+    const glq::DecodeCfg c = layer->invariant ? glq::invariant_config(layer, (int)B)
+                                              : glq::decode_config(layer, (int)B, aligned, aligned, GLQ_F32);
     if (warps) *warps = c.warps;
     if (bands) *bands = c.plan.bands;
     if (splits) *splits = c.plan.splits;
@@ -930,6 +1076,12 @@ glq_status glq_layer_set_fusion(glq_layer layer, int32_t flags) {
     if (flags != GLQ_FUSE_DEFAULT && (flags & ~(GLQ_FUSE_INPUT | GLQ_FUSE_OUTPUT | GLQ_SPLITK_CLUSTER)))
         return GLQ_ERR_INVALID_ARG;
     layer->fusion = flags;
+    return GLQ_OK;
+}
+
+glq_status glq_layer_set_batch_invariant(glq_layer layer, int32_t enable) {
+    if (!layer || (enable != 0 && enable != 1)) return GLQ_ERR_INVALID_ARG;
+    layer->invariant = enable != 0;
     return GLQ_OK;
 }
 
@@ -961,6 +1113,17 @@ glq_status glq_linear(glq_layer L, const void *x_dev, glq_dtype x_dtype, void *y
         return GLQ_ERR_INVALID_ARG;  // the kernels use 8- and 16-byte accesses
     DeviceGuard guard(L->device);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (L->invariant) {
+        WsNeed need;
+        invariant_need(L, B, need);
+        void *buf[WS_COUNT];
+        glq_status st = ws_acquire(L->device, need, s, buf);
+        if (st != GLQ_OK) return st;
+        void *const v[5] = {buf[WS_XQ], buf[WS_XH], buf[WS_INFO], buf[WS_PART], buf[WS_Z]};
+        st = glq::run_invariant(L, x_dev, x_dtype == GLQ_BF16, y_dev, (int)y_dtype, B, s, v, (size_t)L->n_pad * 2);
+        if (st != GLQ_OK) cudaGetLastError();
+        return st;
+    }
     if (B > GLQ_DECODE_MAX_B) return run_prefill(L, x_dev, x_dtype == GLQ_BF16, y_dev, (int)y_dtype, B, s);
     WsNeed need;
     decode_need(L, B, need);
@@ -1072,8 +1235,10 @@ glq_status glq_gemv_replay(glq_layer L, int64_t B, void *stream) {
     if (B < 1 || B > L->last_B) return GLQ_ERR_SHAPE;
     DeviceGuard guard(L->device);
     const glq::DecodeCfg cfg = glq::decode_config(L, (int)B, L->last_x, L->last_y, L->last_y_dtype);
+    WsNeed need;  // buffers large enough for this layer (their contents are the last call's)
+    decode_need(L, B, need);
     void *buf[WS_COUNT];
-    glq_status st = ws_acquire(L->device, WsNeed{}, static_cast<cudaStream_t>(stream), buf);
+    glq_status st = ws_acquire(L->device, need, static_cast<cudaStream_t>(stream), buf);
     if (st != GLQ_OK) return st;
     glq::GemvParams pg = glq::gemv_params(L, decode_view(L, buf), cfg, (int)B, L->last_x, L->last_x_bf16 != 0,
                                           L->last_y, L->last_y_dtype);
@@ -1087,8 +1252,11 @@ glq_status glq_prefill_replay(glq_layer L, int64_t B, void *stream) {
     if (!L) return GLQ_ERR_INVALID_ARG;
     if (B <= GLQ_DECODE_MAX_B || B > L->last_prefill_B) return GLQ_ERR_SHAPE;
     DeviceGuard guard(L->device);
+    WsNeed need;  // buffers large enough for this layer (their contents are the last call's)
+    prefill_need(L, B, need);
+    if (L->last_prefill_mat) need.b[WS_W16] = std::max(need.b[WS_W16], (size_t)L->m_pad * L->n_pad * sizeof(__half));
     void *buf[WS_COUNT];
-    glq_status st = ws_acquire(L->device, WsNeed{}, static_cast<cudaStream_t>(stream), buf);
+    glq_status st = ws_acquire(L->device, need, static_cast<cudaStream_t>(stream), buf);
     if (st != GLQ_OK) return st;
     return launch_prefill_gemm(L, prefill_view(buf), B, L->last_prefill_mat, static_cast<cudaStream_t>(stream),
                                false) == cudaSuccess

@@ -81,6 +81,7 @@ struct glq_layer_s {
     glq_hblocks hb_n, hb_m;
     unsigned *d_blk_cnt = nullptr;  // [GLQ_MAX_BLOCKS] output-block counters, zero between calls
     int fusion = -1;                // GLQ_FUSE_* bits, or -1: the library default (glq_layer_set_fusion)
+    bool invariant = false;         // every batch through the exact decode path (glq_layer_set_batch_invariant)
     int64_t prefill_mat_min_b = 256;  // batches from here reconstruct W16 first (glq_layer_set_prefill_mode)
     // the last decode launch (glq_gemv_replay)
     const void *last_x = nullptr;
@@ -119,5 +120,10 @@ inline const GemvPlan &plan_for(glq_layer L, int nb) { return L->plan[nb > 8 ? 1
 
 // largest split count any decode configuration of nb tokens can use
 int max_decode_splits(glq_layer L, int nb);
+
+// The decode configuration of the batch-invariant mode for a slice of nb
+// <= 16 tokens: separate transforms and a split of the chunk range that
+// does not depend on nb (the layer's one-token plan's chunks per split).
+DecodeCfg invariant_config(glq_layer L, int nb);
 
 }  // namespace glq

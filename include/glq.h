@@ -256,6 +256,24 @@ GLQ_API glq_status glq_linear(glq_layer layer, const void *x_dev, glq_dtype x_dt
 GLQ_API glq_status glq_layer_set_fusion(glq_layer layer, int32_t flags);
 
 /*
+ * glq_layer_set_batch_invariant -- enable (1) or disable (0, the default) a
+ * mode in which every token's output is the same bits whatever the batch
+ * size it arrives in and whichever path a batch of that size would take
+ * otherwise (the pages' claim that a prompt gives identical logits at B = 1
+ * decode and in a batched prefill: glq 0.5.1 PyPI page, "Inference kernels",
+ * "Bit-exact determinism").  In this mode every call, prefill-sized ones
+ * included, runs the exact decode arithmetic: the input transform over all
+ * tokens (the kernel chosen by n alone), the codebook GEMV on slices of at
+ * most 16 tokens with one split plan per layer that no batch size changes
+ * (integer sums of the E8 stages are exact; the fp32 sums of an 8-bit stage
+ * then follow one order), and the output transform over all tokens (the
+ * kernel chosen by m alone).  Batches above 16 tokens then run at GEMV speed
+ * (the indices are read once per 16 tokens) instead of on the tensor cores.
+ * Errors: GLQ_ERR_INVALID_ARG.
+ */
+GLQ_API glq_status glq_layer_set_batch_invariant(glq_layer layer, int32_t enable);
+
+/*
  * glq_layer_set_prefill_reconstruct -- how tensor-core calls (B > 16) get
  * their weights.  Calls with B >= min_batch first reconstruct W = cb1 + rs
  * cb2 into an fp16 matrix of m_pad x n_pad (2 bytes per weight, in the
