@@ -40,7 +40,7 @@ EXPORTS = (
     "glq_layer_check", "glq_layer_info", "glq_gemv_replay", "glq_linear_noalloc", "glq_decode_plan",
     "glq_prefill_replay", "glq_layer_set_fusion", "glq_layer_set_prefill_reconstruct",
     "glq_workspace_info", "glq_workspace_release", "glq_layer_create_stages",
-    "glq_layer_set_batch_invariant",
+    "glq_layer_set_batch_invariant", "glq_layer_create_shard", "glq_cast",
 )
 
 
@@ -63,6 +63,9 @@ _SIGNATURES = {
                           _vp, _vp, ctypes.POINTER(_vp)], ctypes.c_int),
     "glq_layer_create_stages": ([_i64, _i64, _i32, _vp, _vp, _vp, _vp, ctypes.c_float, _vp,
                                  _vp, _vp, ctypes.POINTER(_vp)], ctypes.c_int),
+    "glq_layer_create_shard": ([_i64, _i64, _i32, _vp, _vp, _vp, _vp, ctypes.c_float, _vp,
+                                _vp, _vp, _i64, _i64, ctypes.POINTER(_vp)], ctypes.c_int),
+    "glq_cast": ([_vp, _vp, ctypes.c_int, _i64, _vp], ctypes.c_int),
     "glq_layer_destroy": ([_vp], ctypes.c_int),
     "glq_layer_reserve": ([_vp, _i64], ctypes.c_int),
     "glq_linear": ([_vp, _vp, ctypes.c_int, _vp, ctypes.c_int, _i64, _vp], ctypes.c_int),
@@ -191,6 +194,40 @@ def glq_layer_create_stages(m, n, bpw, idx1, idx_res, primary, residual, weight_
                                      s_out.ctypes.data, ctypes.byref(h)),
         "glq_layer_create_stages")
     return h.value
+
+
+def _stage_args(m, n, bpw, idx1, idx_res, resid_scales, s_in, s_out):
+    bits = stage_bits(bpw)
+    idx_res = list(idx_res or [])
+    scales = np.ascontiguousarray(list(resid_scales or []), dtype=np.float32)
+    if len(idx_res) != len(bits) or scales.size != len(bits):
+        raise ValueError(f"bpw {bpw} has {len(bits)} residual stages")
+    idx1 = np.ascontiguousarray(idx1, dtype=np.uint16)
+    arrays = [np.ascontiguousarray(a, dtype=np.uint16 if b == 16 else np.uint8) for a, b in zip(idx_res, bits)]
+    s_in = np.ascontiguousarray(s_in, dtype=np.int8)
+    s_out = np.ascontiguousarray(s_out, dtype=np.int8)
+    if idx1.size != m * (n // 8) or s_in.size != n or s_out.size != m or any(a.size != idx1.size for a in arrays):
+        raise ValueError("array sizes do not match m, n")
+    ptrs = (ctypes.c_void_p * max(1, len(arrays)))(*[a.ctypes.data for a in arrays])
+    keep = (idx1, arrays, scales, s_in, s_out, ptrs)
+    return keep, (ctypes.cast(ptrs, ctypes.c_void_p) if arrays else None), (scales.ctypes.data if arrays else None)
+
+
+def glq_layer_create_shard(m, n, bpw, idx1, idx_res, primary, residual, weight_scale, resid_scales,
+                           s_in, s_out, k_begin, k_end) -> int:
+    """The row-parallel part of a layer holding input columns [k_begin, k_end)
+    (whole-layer host arrays; idx_res / resid_scales one per residual stage)."""
+    keep, pres, pscales = _stage_args(m, n, bpw, idx1, idx_res, resid_scales, s_in, s_out)
+    h = _vp()
+    _ok(_L().glq_layer_create_shard(m, n, bpw, keep[0].ctypes.data, pres, primary, residual, float(weight_scale),
+                                    pscales, keep[3].ctypes.data, keep[4].ctypes.data, int(k_begin), int(k_end),
+                                    ctypes.byref(h)),
+        "glq_layer_create_shard")
+    return h.value
+
+
+def glq_cast(src_ptr, dst_ptr, dtype, count, stream) -> None:
+    _ok(_L().glq_cast(src_ptr, dst_ptr, dtype, int(count), stream), "glq_cast")
 
 
 def glq_layer_destroy(handle: int) -> None:

@@ -168,7 +168,8 @@ void decode_need(glq_layer L, int64_t rows, WsNeed &n) {
     for (int nb = 1; nb <= rows; ++nb) max_splits = std::max(max_splits, glq::max_decode_splits(L, nb));
     n.b[WS_XQ] = std::max(n.b[WS_XQ], (size_t)rows * L->n_pad * 2);
     if (L->has8) n.b[WS_XH] = std::max(n.b[WS_XH], (size_t)rows * L->n_pad * sizeof(__half));
-    n.b[WS_INFO] = std::max(n.b[WS_INFO], (size_t)rows * sizeof(glq_rowinfo));
+    // a shard also keeps the row sums over its own columns, after 16 rows
+    n.b[WS_INFO] = std::max(n.b[WS_INFO], (L->shard ? 2 * GLQ_DECODE_MAX_B : rows) * sizeof(glq_rowinfo));
     if (max_splits > 1)
         n.b[WS_PART] = std::max(n.b[WS_PART], (size_t)max_splits * rows * L->m_pad * sizeof(double));
     n.b[WS_Z] = std::max(n.b[WS_Z], (size_t)rows * L->m_pad * sizeof(float));
@@ -193,7 +194,8 @@ void prefill_need(glq_layer L, int64_t B, WsNeed &n) {
     n.b[WS_PXH] = std::max(n.b[WS_PXH], (size_t)B * L->n_pad * sizeof(__half));
     n.b[WS_PINFO] = std::max(n.b[WS_PINFO], (size_t)B * sizeof(glq_rowinfo));
     n.b[WS_PZ] = std::max(n.b[WS_PZ], (size_t)ks * B * L->m_pad * sizeof(float));
-    if (B >= L->prefill_mat_min_b) n.b[WS_W16] = std::max(n.b[WS_W16], (size_t)L->m_pad * L->n_pad * sizeof(__half));
+    if (B >= L->prefill_mat_min_b)
+        n.b[WS_W16] = std::max(n.b[WS_W16], (size_t)L->m_pad * stream_cols(L) * sizeof(__half));
 }
 
 glq_workspace decode_view(glq_layer L, void *const buf[WS_COUNT]) {
@@ -225,7 +227,9 @@ glq_prefill_ws prefill_view(void *const buf[WS_COUNT]) {
 // x 128 rows, 128-byte swizzle.
 bool encode_w_map(CUtensorMap *map, const __half *w16, int64_t n_pad, int64_t m_pad);
 
-bool encode_x_map(CUtensorMap *map, const __half *xh, int64_t n_pad, int64_t B) {
+// cols columns of rows `ld` fp16 apart (a shard reads its column range of the
+// whole rows)
+bool encode_x_map(CUtensorMap *map, const __half *xh, int64_t cols, int64_t B, int64_t ld) {
     static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     if (!encode) {
         cudaDriverEntryPointQueryResult q;
@@ -237,8 +241,8 @@ bool encode_x_map(CUtensorMap *map, const __half *xh, int64_t n_pad, int64_t B) 
         }
         encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
-    const cuuint64_t dims[2] = {(cuuint64_t)n_pad, (cuuint64_t)B};
-    const cuuint64_t strides[1] = {(cuuint64_t)n_pad * sizeof(__half)};
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)B};
+    const cuuint64_t strides[1] = {(cuuint64_t)ld * sizeof(__half)};
     const cuuint32_t box[2] = {64, 128};
     const cuuint32_t estr[2] = {1, 1};
     return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<__half *>(xh), dims, strides, box, estr,
@@ -250,7 +254,7 @@ bool encode_x_map(CUtensorMap *map, const __half *xh, int64_t n_pad, int64_t B) 
 // workspace: z[0..B) from xh[0..B).
 bool encode_w_map(CUtensorMap *map, const __half *w16, int64_t n_pad, int64_t m_pad) {
     // same layout rules as the activations: rows of n_pad fp16, 128-byte swizzle
-    return encode_x_map(map, w16, n_pad, m_pad);
+    return encode_x_map(map, w16, n_pad, m_pad, n_pad);
 }
 
 // K splits of the tensor-core GEMM: fill the CTA pairs when the output has
@@ -261,7 +265,7 @@ bool encode_w_map(CUtensorMap *map, const __half *w16, int64_t n_pad, int64_t m_
 int choose_ksplit(glq_layer L, int64_t B, int tiles) {
     const int pairs = std::max(1, L->num_sms / 2);
     const double t_tile = (double)glq::prefill_tile_rows() * (double)glq::prefill_tile_tokens() *
-                          (double)L->n_pad * 2.0 / 15e12;
+                          (double)stream_cols(L) * 2.0 / 15e12;
     const double t_traffic = (double)B * (double)L->m_pad * 8.0 / 6e12;
     int best = 1;
     double best_t = 1e30;
@@ -321,8 +325,9 @@ glq::PrefillParams prefill_params(glq_layer L, const glq_prefill_ws &ws, int64_t
 cudaError_t launch_prefill_gemm(glq_layer L, const glq_prefill_ws &ws, int64_t B, bool mat, cudaStream_t s,
                                 bool pdl) {
     CUtensorMap xmap, wmap;
-    if (!encode_x_map(&xmap, ws.xh, L->n_pad, B)) return cudaErrorInvalidValue;
-    if (mat && !encode_w_map(&wmap, ws.w16, L->n_pad, L->m_pad)) return cudaErrorInvalidValue;
+    const int64_t k0 = (int64_t)L->kc0 * GLQ_CHUNK_K;  // a shard's first column (256-byte aligned)
+    if (!encode_x_map(&xmap, ws.xh + k0, stream_cols(L), B, L->n_pad)) return cudaErrorInvalidValue;
+    if (mat && !encode_w_map(&wmap, ws.w16, stream_cols(L), L->m_pad)) return cudaErrorInvalidValue;
     const glq::PrefillParams pp = prefill_params(L, ws, B);
     const int grid = 2 * std::min(pp.ntiles, L->num_sms / 2);  // CTA pairs
     return glq::launch_prefill(pp, xmap, mat ? &wmap : nullptr, grid, s, pdl);
@@ -384,7 +389,8 @@ glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_d
         }
         b0 += nb;
     }
-    if (mat && glq::launch_wmat(prefill_params(L, ws, B), ws.w16, (int)L->n_pad, L->num_sms, s, true) != cudaSuccess)
+    if (mat && glq::launch_wmat(prefill_params(L, ws, B), ws.w16, (int)stream_cols(L), L->num_sms, s, true) !=
+                   cudaSuccess)
         return GLQ_ERR_CUDA;
     if (launch_prefill_gemm(L, ws, B, mat, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
     L->last_prefill_B = B;
@@ -443,10 +449,10 @@ DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y
     const bool y_al = (reinterpret_cast<uintptr_t>(y) & 15) == 0;
     (void)y_dtype;
     const int flags = L->fusion < 0 ? FUSE_DEFAULT_FLAGS : L->fusion;
-    c.fout = (flags & GLQ_FUSE_OUTPUT) && y_al && (long long)nb * L->hb_m.len[0] <= FUSED_OUT_MAX_VALUES &&
+    c.fout = !L->shard && (flags & GLQ_FUSE_OUTPUT) && y_al && (long long)nb * L->hb_m.len[0] <= FUSED_OUT_MAX_VALUES &&
              (size_t)nb * L->hb_m.len[0] * sizeof(float) <= base;
     c.warps = warps;
-    if ((flags & GLQ_FUSE_INPUT) && x_al && (long long)nb * L->hb_n.len[0] <= FUSED_IN_MAX_VALUES) {
+    if (!L->shard && (flags & GLQ_FUSE_INPUT) && x_al && (long long)nb * L->hb_n.len[0] <= FUSED_IN_MAX_VALUES) {
         int cap = 1;  // largest power-of-two chunk count whose activations fit shared memory
         while (cap < L->KC &&
                gemv_fused_smem_bytes(L->primary->table_words, L->bpw, nb, std::min(cap * 2, L->KC) * GLQ_CHUNK_K) <=
@@ -549,9 +555,12 @@ GemvParams gemv_params(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg
     p.fold = FoldParams{L->primary->fold.nb, L->primary->fold.neg_base};
     p.kc = LookupConsts{4u, 16u, 0xFFFFFFFFu};
     p.tab8 = L->has8 ? reinterpret_cast<const uint4 *>(L->residual->d_fp16) : nullptr;
-    p.xq = w.xq;
-    p.xh = w.xh;
-    p.info = w.info;
+    // a shard reads its column range of the activation rows, and the row
+    // sums over that range (stored after the first 16 rows of row info)
+    const int64_t k0 = (int64_t)L->kc0 * GLQ_CHUNK_K;
+    p.xq = w.xq ? w.xq + k0 * 2 : nullptr;
+    p.xh = w.xh ? w.xh + k0 : nullptr;
+    p.info = L->shard ? w.info + GLQ_DECODE_MAX_B : w.info;
     p.B = nb;
     p.n_pad = (int)L->n_pad;
     p.KC = L->KC;
@@ -627,6 +636,13 @@ cudaError_t run_decode(glq_layer L, const glq_workspace &w, const DecodeCfg &cfg
             e = launch_rht_in(pin, s, true);
         }
         if (e != cudaSuccess) return e;
+        if (L->shard) {  // the row sums of X over the shard's columns
+            const int c0 = L->kc0 * GLQ_CHUNK_K;
+            const int c1 = (int)std::min<int64_t>(c0 + stream_cols(L), L->n);
+            e = launch_shard_rowsum(w.xq, (size_t)L->n_pad * 2, c0, c1, w.info, w.info + GLQ_DECODE_MAX_B, nb, s,
+                                    true);
+            if (e != cudaSuccess) return e;
+        }
     }
     e = launch_gemv(gemv_params(L, w, cfg, nb, x, x_bf16, y, y_dtype), L->bpw, cfg.plan.grid, s, true, cfg.fin);
     if (e != cudaSuccess || cfg.fout) return e;
@@ -865,13 +881,18 @@ glq_status glq_codebook_destroy(glq_codebook cb) {
     return GLQ_OK;
 }
 
-glq_status glq_layer_create_stages(int64_t m, int64_t n, int32_t bpw, const uint16_t *idx1,
-                                   const void *const *idx_res, glq_codebook primary, glq_codebook residual,
-                                   float weight_scale, const float *resid_scales, const int8_t *s_in,
-                                   const int8_t *s_out, glq_layer *out) {
+// A layer over input columns [k_begin, k_end) of n (the whole layer, or a
+// row-parallel shard): the index arrays are the whole layer's.
+static glq_status create_layer(int64_t m, int64_t n, int32_t bpw, const uint16_t *idx1, const void *const *idx_res,
+                        glq_codebook primary, glq_codebook residual, float weight_scale,
+                        const float *resid_scales, const int8_t *s_in, const int8_t *s_out, int64_t k_begin,
+                        int64_t k_end, glq_layer *out) {
     if (!out) return GLQ_ERR_INVALID_ARG;
     *out = nullptr;
     if (m <= 0 || n <= 0 || m % 8 || n % 8 || m > MAX_DIM || n > MAX_DIM) return GLQ_ERR_SHAPE;
+    if (k_begin < 0 || k_end > n || k_begin >= k_end || k_begin % GLQ_CHUNK_K ||
+        (k_end % GLQ_CHUNK_K && k_end != n))
+        return GLQ_ERR_SHAPE;
     if (bpw < 2 || bpw > 8) return GLQ_ERR_BPW;
     const int n16 = glq::stages16(bpw);
     const bool has8 = glq::stage8(bpw);
@@ -904,11 +925,14 @@ glq_status glq_layer_create_stages(int64_t m, int64_t n, int32_t bpw, const uint
     L->m = m;
     L->n = n;
     L->bpw = bpw;
-    L->G = (int)(n / 8);
+    const int G_full = (int)(n / 8), g0 = (int)(k_begin / 8);
+    L->G = (int)((k_end - k_begin) / 8);
     L->m_pad = (m + GLQ_ROW_TILE - 1) / GLQ_ROW_TILE * GLQ_ROW_TILE;
     L->n_pad = (n + GLQ_CHUNK_K - 1) / GLQ_CHUNK_K * GLQ_CHUNK_K;
     L->RT = (int)(L->m_pad / GLQ_ROW_TILE);
-    L->KC = (int)(L->n_pad / GLQ_CHUNK_K);
+    L->KC = (int)((k_end - k_begin + GLQ_CHUNK_K - 1) / GLQ_CHUNK_K);
+    L->kc0 = (int)(k_begin / GLQ_CHUNK_K);
+    L->shard = k_begin != 0 || k_end != n;
     L->device = dev;
     L->primary = primary;
     L->residual = has8 ? residual : (n16 ? primary : nullptr);
@@ -950,7 +974,7 @@ glq_status glq_layer_create_stages(int64_t m, int64_t n, int32_t bpw, const uint
             const int s = (grp % GLQ_GROUPS_PER_CHUNK) / 4;
             const int t = grp % 4;
             const size_t slot = ((size_t)rt * L->KC + kc) * 32 + (size_t)(4 * g + t);
-            const size_t src = (size_t)r * L->G + grp;
+            const size_t src = (size_t)r * G_full + g0 + grp;
             const size_t dst = slot * 8 + 2 * s + hi;
             s16[0][dst] = F.code[idx1[src]];
             for (int k = 0; k < n16; ++k) s16[1 + k][dst] = F.code[static_cast<const uint16_t *>(idx_res[k])[src]];
@@ -990,6 +1014,34 @@ glq_status glq_layer_create_stages(int64_t m, int64_t n, int32_t bpw, const uint
     }
     L->device_bytes = total;
     *out = L;
+    return GLQ_OK;
+}
+
+glq_status glq_layer_create_stages(int64_t m, int64_t n, int32_t bpw, const uint16_t *idx1,
+                                   const void *const *idx_res, glq_codebook primary, glq_codebook residual,
+                                   float weight_scale, const float *resid_scales, const int8_t *s_in,
+                                   const int8_t *s_out, glq_layer *out) {
+    return create_layer(m, n, bpw, idx1, idx_res, primary, residual, weight_scale, resid_scales, s_in, s_out, 0, n,
+                        out);
+}
+
+glq_status glq_layer_create_shard(int64_t m, int64_t n, int32_t bpw, const uint16_t *idx1,
+                                  const void *const *idx_res, glq_codebook primary, glq_codebook residual,
+                                  float weight_scale, const float *resid_scales, const int8_t *s_in,
+                                  const int8_t *s_out, int64_t k_begin, int64_t k_end, glq_layer *out) {
+    return create_layer(m, n, bpw, idx1, idx_res, primary, residual, weight_scale, resid_scales, s_in, s_out,
+                        k_begin, k_end, out);
+}
+
+glq_status glq_cast(const float *src_dev, void *dst_dev, glq_dtype dtype, int64_t count, void *stream) {
+    if (count < 0) return GLQ_ERR_SHAPE;
+    if (dtype != GLQ_F16 && dtype != GLQ_BF16 && dtype != GLQ_F32) return GLQ_ERR_DTYPE;
+    if (count == 0) return GLQ_OK;
+    if (!src_dev || !dst_dev) return GLQ_ERR_INVALID_ARG;
+    if (glq::launch_cast(src_dev, dst_dev, (int)dtype, count, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return GLQ_ERR_CUDA;
+    }
     return GLQ_OK;
 }
 
@@ -1081,6 +1133,7 @@ glq_status glq_layer_set_fusion(glq_layer layer, int32_t flags) {
 
 glq_status glq_layer_set_batch_invariant(glq_layer layer, int32_t enable) {
     if (!layer || (enable != 0 && enable != 1)) return GLQ_ERR_INVALID_ARG;
+    if (layer->shard && enable) return GLQ_ERR_INVALID_ARG;
     layer->invariant = enable != 0;
     return GLQ_OK;
 }
@@ -1111,6 +1164,7 @@ glq_status glq_linear(glq_layer L, const void *x_dev, glq_dtype x_dtype, void *y
     if (!x_dev || !y_dev) return GLQ_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(x_dev) & 15) || (reinterpret_cast<uintptr_t>(y_dev) & 15))
         return GLQ_ERR_INVALID_ARG;  // the kernels use 8- and 16-byte accesses
+    if (L->shard && y_dtype != GLQ_F32) return GLQ_ERR_DTYPE;  // partial sums stay fp32 until summed
     DeviceGuard guard(L->device);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (L->invariant) {
@@ -1166,7 +1220,7 @@ glq_status glq_dequant_reference(glq_layer L, float *w_dev, void *stream) {
     p.tab8 = L->has8 ? reinterpret_cast<const uint4 *>(L->residual->d_fp16) : nullptr;
     p.bpw = L->bpw;
     p.m = L->m;
-    p.n = (int)L->n;
+    p.n = L->G * 8;  // a shard's own columns
     p.G = L->G;
     p.KC = L->KC;
     p.ws = L->ws;
@@ -1254,7 +1308,8 @@ glq_status glq_prefill_replay(glq_layer L, int64_t B, void *stream) {
     DeviceGuard guard(L->device);
     WsNeed need;  // buffers large enough for this layer (their contents are the last call's)
     prefill_need(L, B, need);
-    if (L->last_prefill_mat) need.b[WS_W16] = std::max(need.b[WS_W16], (size_t)L->m_pad * L->n_pad * sizeof(__half));
+    if (L->last_prefill_mat)
+        need.b[WS_W16] = std::max(need.b[WS_W16], (size_t)L->m_pad * stream_cols(L) * sizeof(__half));
     void *buf[WS_COUNT];
     glq_status st = ws_acquire(L->device, need, static_cast<cudaStream_t>(stream), buf);
     if (st != GLQ_OK) return st;

@@ -36,6 +36,9 @@ struct glq_prefill_ws {
 
 // Device buffers one decode call works in (B <= 16 tokens): a view of the
 // device's shared workspace, except cnt, which the layer owns.
+// Columns the layer's index streams cover (n_pad for a whole layer).
+inline int64_t stream_cols(glq_layer L);
+
 struct glq_workspace {
     uint8_t *xq = nullptr;        // [B][n_pad * 2] activations, high / low bytes per group
     __half *xh = nullptr;         // [B][n_pad] fp16 activations (3 bpw only)
@@ -54,7 +57,12 @@ struct glq_hblocks {
 
 struct glq_layer_s {
     int64_t m = 0, n = 0, m_pad = 0, n_pad = 0;
-    int bpw = 0, RT = 0, KC = 0, G = 0;
+    int bpw = 0, RT = 0, KC = 0, G = 0;  // KC, G: chunks / groups of the index streams (the shard's)
+    // row-parallel shard: the layer holds input columns [kc0 * 128, kc0 * 128
+    // + KC * 128) of n (a whole layer: kc0 = 0, KC * 128 = n_pad); its output
+    // is the fp32 partial sum of those columns
+    bool shard = false;
+    int kc0 = 0;
     int device = 0, num_sms = 0;
     glq_codebook primary = nullptr, residual = nullptr;
     float ws = 0.f;
@@ -91,6 +99,8 @@ struct glq_layer_s {
     glq::GemvPlan last_plan{};
     size_t device_bytes = 0;
 };
+
+inline int64_t stream_cols(glq_layer L) { return (int64_t)L->KC * GLQ_CHUNK_K; }
 
 namespace glq {
 

@@ -252,6 +252,12 @@ struct GemvPlan {
 GemvPlan plan_gemv(int RT, int KC, int num_sms, int warps, bool pow2 = false, int max_cps = 1 << 30,
                    int max_splits = 1 << 30, double charge = 0.5);
 cudaError_t launch_dequant(const DequantParams &p, cudaStream_t s);
+// Row-parallel shards (glq_shard.cu): per token, the exact sum of X over the
+// columns [c0, c1) of the decode activations xq (rows of row_bytes bytes), with
+// the token's scale copied from `in`; and an elementwise fp32 -> dtype cast.
+cudaError_t launch_shard_rowsum(const uint8_t *xq, size_t row_bytes, int c0, int c1, const glq_rowinfo *in,
+                                glq_rowinfo *out, int B, cudaStream_t s, bool pdl);
+cudaError_t launch_cast(const float *src, void *dst, int dtype, int64_t count, cudaStream_t s);
 // wmap: TMA map of the dequantised fp16 W [m_pad][n_pad] (boxes 64 x 128,
 // 128-byte swizzle), or null for the fused variant whose producer warps
 // rebuild W from the codes.

@@ -65,7 +65,7 @@ size_t align256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 extern "C" glq_status glq_linear_noalloc(glq_layer L, const void *x_dev, glq_dtype x_dtype, void *y_dev,
                                          glq_dtype y_dtype, int64_t B, void *stream) {
-    if (!L) return GLQ_ERR_INVALID_ARG;
+    if (!L || L->shard) return GLQ_ERR_INVALID_ARG;  // a shard's row sums need the shared workspace
     if (B < 0 || B > GLQ_DECODE_MAX_B) return GLQ_ERR_SHAPE;
     if (x_dtype != GLQ_F16 && x_dtype != GLQ_BF16) return GLQ_ERR_DTYPE;
     if (y_dtype != x_dtype && y_dtype != GLQ_F32) return GLQ_ERR_DTYPE;

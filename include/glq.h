@@ -169,6 +169,37 @@ GLQ_API glq_status glq_layer_create_stages(int64_t m, int64_t n, int32_t bpw, co
 GLQ_API glq_status glq_layer_destroy(glq_layer layer);
 
 /*
+ * glq_layer_create_shard -- the part of a layer that one GPU holds when the
+ * layer is split over its input columns (row-parallel: y = sum over parts
+ * of S_out . H_m . W^[:, part] . (H_n (S_in . x))[part], because H_m and
+ * S_out are linear).  Arguments as glq_layer_create_stages, with the whole
+ * layer's host arrays (idx1 and every idx_res [m][n/8], s_in [n], s_out [m]);
+ * the shard keeps input columns [k_begin, k_end): k_begin a multiple of
+ * 128, k_end a multiple of 128 or n.  Every GPU rotates the whole input x (x
+ * is replicated) and computes its part's fp32 output; one all-reduce (sum)
+ * of the parts' y over the GPUs, then glq_cast to the caller's dtype, gives
+ * the layer's y.  glq_linear on a shard requires y_dtype == GLQ_F32; the
+ * fused transforms, the batch-invariant mode and glq_linear_noalloc are not
+ * available for shards.  glq_dequant_reference writes the shard's columns,
+ * w_dev [m][k_end - k_begin].  Errors as glq_layer_create, GLQ_ERR_SHAPE for
+ * a bad column range.  Synchronous.
+ */
+GLQ_API glq_status glq_layer_create_shard(int64_t m, int64_t n, int32_t bpw, const uint16_t *idx1,
+                                          const void *const *idx_res, glq_codebook primary,
+                                          glq_codebook residual, float weight_scale,
+                                          const float *resid_scales, const int8_t *s_in, const int8_t *s_out,
+                                          int64_t k_begin, int64_t k_end, glq_layer *out);
+
+/*
+ * glq_cast -- dst[i] = src[i] rounded to nearest even in `dtype`
+ * (GLQ_F16, GLQ_BF16 or GLQ_F32), i < count; src_dev fp32 and dst_dev on the
+ * current device.  Rounds the all-reduced fp32 output of row-parallel shards
+ * to the model's dtype.  Errors: GLQ_ERR_SHAPE, GLQ_ERR_DTYPE,
+ * GLQ_ERR_INVALID_ARG, GLQ_ERR_CUDA.  Asynchronous.
+ */
+GLQ_API glq_status glq_cast(const float *src_dev, void *dst_dev, glq_dtype dtype, int64_t count, void *stream);
+
+/*
  * glq_layer_reserve -- grow the device's shared workspace so that every
  * glq_linear call on this layer with B <= max_B (decode and tensor-core
  * batches alike) finds its buffers already there: such calls then allocate
