@@ -50,7 +50,9 @@ DECODE_DTYPE = ("u8 x s8/u8 integer MMA on int16-quantised rotated activations (
 # GEMV on the 24B-class gate layer at one token, from the ncu capture whose
 # summary is profiles/gemv_24b-gate-32768x5120_4bpw_b1.md, keyed by the
 # sha256 of the GEMV source it was taken at: a changed kernel reports null.
-PROFILED_GEMV_TRAFFIC = {}
+PROFILED_GEMV_TRAFFIC = {
+    "04b1709412df87891a6836b91e8cb3d14c24e4dcc78bc67baca85efb7a135c31": 84112640 + 3054336,
+}
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
