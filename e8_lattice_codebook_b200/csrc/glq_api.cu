@@ -392,7 +392,12 @@ glq_status run_prefill(glq_layer L, const void *x, bool x_bf16, void *y, int y_d
     if (mat && glq::launch_wmat(prefill_params(L, ws, B), ws.w16, (int)stream_cols(L), L->num_sms, s, true) !=
                    cudaSuccess)
         return GLQ_ERR_CUDA;
-    if (launch_prefill_gemm(L, ws, B, mat, s, true) != cudaSuccess) return GLQ_ERR_CUDA;
+    // The dequantising-producer variant is launched without programmatic
+    // dependent launch: started early behind the previous kernels, calls
+    // issued back to back stalled until a bounded wait gave up (measured:
+    // 8B-class layers at 17-64 tokens); launched after its predecessor
+    // completes, they do not.
+    if (launch_prefill_gemm(L, ws, B, mat, s, mat) != cudaSuccess) return GLQ_ERR_CUDA;
     L->last_prefill_B = B;
     L->last_prefill_mat = mat;
     for (int64_t b0 = 0; b0 < B;) {
@@ -941,9 +946,11 @@ static glq_status create_layer(int64_t m, int64_t n, int32_t bpw, const uint16_t
     L->has8 = has8;
     for (int k = 0; k < n16; ++k) L->rs16[k] = resid_scales[k];
     L->rs8 = has8 ? resid_scales[n16] : 0.f;
-    // batches of the tensor-core path reconstruct W first from 256 tokens;
-    // with more than two stages always (the dequantising producer holds two)
-    L->prefill_mat_min_b = bpw <= 4 ? 256 : GLQ_DECODE_MAX_B + 1;
+    // every batch of the tensor-core path reconstructs W first (measured on
+    // the 8B-class layers from 17 to 255 tokens: 70-87 us per call against
+    // 175-217 us for the dequantising producer); the producer stays available
+    // for 2-4 bpw through glq_layer_set_prefill_reconstruct
+    L->prefill_mat_min_b = GLQ_DECODE_MAX_B + 1;
     L->plan_n = glq::make_rht_plan((int)n);
     L->plan_m = glq::make_rht_plan((int)m);
     cudaDeviceGetAttribute(&L->num_sms, cudaDevAttrMultiProcessorCount, dev);
@@ -1141,7 +1148,7 @@ glq_status glq_layer_set_batch_invariant(glq_layer layer, int32_t enable) {
 glq_status glq_layer_set_prefill_reconstruct(glq_layer layer, int64_t min_batch) {
     if (!layer) return GLQ_ERR_INVALID_ARG;
     if (layer->bpw > 4) return GLQ_OK;  // always reconstructed: the dequantising producer holds two stages
-    layer->prefill_mat_min_b = min_batch < 0 ? 256 : std::max<int64_t>(min_batch, GLQ_DECODE_MAX_B + 1);
+    layer->prefill_mat_min_b = min_batch < 0 ? GLQ_DECODE_MAX_B + 1 : std::max<int64_t>(min_batch, GLQ_DECODE_MAX_B + 1);
     return GLQ_OK;
 }
 

@@ -90,7 +90,7 @@ struct glq_layer_s {
     unsigned *d_blk_cnt = nullptr;  // [GLQ_MAX_BLOCKS] output-block counters, zero between calls
     int fusion = -1;                // GLQ_FUSE_* bits, or -1: the library default (glq_layer_set_fusion)
     bool invariant = false;         // every batch through the exact decode path (glq_layer_set_batch_invariant)
-    int64_t prefill_mat_min_b = 256;  // batches from here reconstruct W16 first (glq_layer_set_prefill_mode)
+    int64_t prefill_mat_min_b = GLQ_DECODE_MAX_B + 1;  // batches from here reconstruct W16 first (glq_layer_set_prefill_reconstruct)
     // the last decode launch (glq_gemv_replay)
     const void *last_x = nullptr;
     void *last_y = nullptr;

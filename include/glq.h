@@ -243,11 +243,11 @@ GLQ_API glq_status glq_workspace_release(int32_t device);
  *   launch when B times the largest Hadamard block is at most 32768 values
  *   (one kernel per call), else input RHT, GEMV and output RHT as three
  *   kernels (see glq_layer_set_fusion); B > 16 runs the tensor-core path:
- *   input RHT, then, from 256 tokens (glq_layer_set_prefill_reconstruct),
- *   one pass that reconstructs W = cb1 + rs cb2 as an fp16 matrix in the
- *   device's shared workspace and a TMA-fed tcgen05/TMEM GEMM on it, below
- *   that a tcgen05 GEMM whose producer warps rebuild each W tile in shared
- *   memory (W never stored), then output RHT.  The GEMV accumulates exactly
+ *   input RHT, one pass that reconstructs W = cb1 + rs cb2 as an fp16 matrix
+ *   in the device's shared workspace, a TMA-fed tcgen05/TMEM GEMM on it
+ *   (or, when glq_layer_set_prefill_reconstruct raises the bound above B, a
+ *   tcgen05 GEMM whose producer warps rebuild each W tile in shared memory,
+ *   W never stored), then output RHT.  The GEMV accumulates exactly
  *   in integers (fp64 across splits); the tensor-core path accumulates in
  *   fp32.
  * Workspace: the device's shared workspace (see glq_layer_reserve); a call
@@ -310,12 +310,14 @@ GLQ_API glq_status glq_layer_set_batch_invariant(glq_layer layer, int32_t enable
  * cb2 into an fp16 matrix of m_pad x n_pad (2 bytes per weight, in the
  * device's shared workspace: one such matrix, of the largest layer that
  * used it, per device) and run the TMA-fed tcgen05 GEMM on it; smaller
- * batches rebuild each W tile in shared memory inside the GEMM
- * and never materialise W (the pages' design: "Inference kernels", glq 0.5.1
- * PyPI page).  Reconstructing once costs one pass over the indices, while the
- * fused producer repeats its codeword gathers for every 512 tokens, so large
- * batches favour it.  min_batch < 0 restores the library default (256);
- * a value above any batch disables it.  Errors: GLQ_ERR_INVALID_ARG.
+ * batches rebuild each W tile in shared memory inside the GEMM and never
+ * materialise W (the pages' design: "Inference kernels", glq 0.5.1 PyPI
+ * page).  Reconstructing once costs one pass over the indices, while the
+ * dequantising producer repeats its codeword gathers for every 512 tokens;
+ * measured on B200 the reconstruction is faster at every batch from 17
+ * tokens, so the default (min_batch < 0) is 17: every tensor-core call
+ * reconstructs.  A bound above a batch selects the producer for it (2-4 bpw;
+ * layers above 4 bpw always reconstruct).  Errors: GLQ_ERR_INVALID_ARG.
  */
 GLQ_API glq_status glq_layer_set_prefill_reconstruct(glq_layer layer, int64_t min_batch);
 

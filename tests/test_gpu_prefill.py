@@ -73,6 +73,7 @@ def test_prefill_small_all_tokens(dev, m, n, bpw, B, xdt, mode):
     assert err <= tolerance(ref), (err, tolerance(ref))
     yp = lay(x).float().cpu().numpy().astype(np.float64)
     assert np.all(np.abs(yp - ref) <= production_tolerance(ref, xdt))
+    lay.check()  # no bounded device wait gave up
 
 
 @pytest.mark.parametrize("mode", sorted(MODES))
@@ -94,6 +95,7 @@ def test_prefill_workload_largest_batch(dev, li, mode):
           f"tol {tolerance(ref):.3e} ratio {err / tolerance(ref):.3f}")
     assert err <= tolerance(ref), (err, tolerance(ref))
     assert np.all(np.isfinite(y))
+    lay.check()
 
 
 @pytest.mark.parametrize("mode", sorted(MODES))
@@ -110,3 +112,32 @@ def test_prefill_determinism_and_batch_independence(dev, mode):
     for B in (17, 300, 512, 513):
         yb = lay(x[:B].contiguous(), out_dtype=torch.float32)
         assert torch.equal(yb, y1[:B]), B
+    lay.check()
+
+
+def test_producer_back_to_back_calls_do_not_stall(dev):
+    """The dequantising-producer variant at small batches, six calls back to
+    back on one stream: each must run to completion (no bounded device wait
+    giving up).  Launched with programmatic dependent launch behind the
+    previous call's kernels, such calls stalled for seconds until a wait's
+    limit released them (GLQ_ERR_TIMEOUT); the variant now starts after its
+    predecessor completes."""
+    import time
+    wl = gi.WORKLOADS["prefill-8b-mlp-4bpw"]
+    L = gi.workload_layer(wl, 0)
+    lay = dev.layer(L)
+    lay.set_prefill_reconstruct(1 << 40)  # the producer for every batch
+    for B in (17, 64):
+        xb = gi.workload_x(wl, 0, B)
+        x = to_torch_x(xb, wl.x_dtype)
+        y = torch.empty((B, L.m), dtype=torch.float32, device="cuda")
+        lay(x, out=y)
+        torch.cuda.synchronize()
+        t0 = time.time()
+        for _ in range(6):
+            lay(x, out=y)
+        lay.check()  # raises GlqError(GLQ_ERR_TIMEOUT) if a wait gave up
+        assert time.time() - t0 < 1.0, B
+        ref = oracle_y(L, xb[[0, B - 1]], wl.x_dtype)
+        assert np.max(np.abs(y.cpu().numpy().astype(np.float64)[[0, B - 1]] - ref)) <= tolerance(ref)
+    lay.set_prefill_reconstruct(-1)
