@@ -700,6 +700,8 @@ def run_glq(args):
             "smollm3-3b-mixed": decode_config_section(glq, torch, "smollm3-3b-mixed", hbm_peak),
         }
         result["prefill"] = prefill_section(glq, torch, tc_peak, peak_src)
+        # the batches between the decode path and the 512-token tiles
+        result["prefill_mid"] = prefill_section(glq, torch, tc_peak, peak_src, batches=(32, 64, 128), reps=20)
         result["dense_bf16_reference"] = dense_reference_section(glq, torch, hbm_peak, tc_peak)
 
     # fp64 oracle on the host cores: one decode step (1 token, 5 layers) on
