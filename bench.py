@@ -51,7 +51,7 @@ DECODE_DTYPE = ("u8 x s8/u8 integer MMA on int16-quantised rotated activations (
 # summary is profiles/gemv_24b-gate-32768x5120_4bpw_b1.md, keyed by the
 # sha256 of the GEMV source it was taken at: a changed kernel reports null.
 PROFILED_GEMV_TRAFFIC = {
-    "04b1709412df87891a6836b91e8cb3d14c24e4dcc78bc67baca85efb7a135c31": 84112640 + 3054336,
+    "8ba979ed5d9f9b06b4f37ef8298de07a9693d969ba3a03536565df023ef772d1": 84113664 + 3624960,
 }
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -454,12 +454,12 @@ def gemv_source_sha256() -> str:
         return hashlib.sha256(f.read()).hexdigest()
 
 
-def prefill_section(glq, torch, tc_peak, peak_src, batches=(512, 2048, 8192), reps=5) -> dict:
+def prefill_section(glq, torch, tc_peak, peak_src, batches=(512, 2048, 8192), reps=5, hbm_peak=None) -> dict:
     """8B-class MLP prefill (14336x4096 and 4096x14336 at 4 bpw): the whole
     glq_linear step (input RHT, tensor-core GEMM, output RHT) per batch, and
-    the GEMM kernel alone (glq_prefill_replay) per layer, timed with events
-    on the stream the kernels run on.  The inputs (x 8192 x 14336 bf16 is
-    235 MB) exceed L2."""
+    the GEMM kernel alone (glq_prefill_replay) per layer, and the input
+    transform alone with either kernel, timed with events on the stream the
+    kernels run on.  The inputs (x 8192 x 14336 bf16 is 235 MB) exceed L2."""
     pre = {}
     wp = WorkloadSet(glq, torch, "prefill-8b-mlp-4bpw", max(batches), ncopy=1)
     for Bp in batches:
@@ -493,12 +493,66 @@ def prefill_section(glq, torch, tc_peak, peak_src, batches=(512, 2048, 8192), re
             gemm[f"{L.m}x{L.n}"] = {"kernel_us": round(mk * 1e3, 1), "TFLOPs": round(tk, 1),
                                     "frac": round(tk / tc_peak, 4)}
         entry["gemm_kernel"] = gemm
+        if hbm_peak:
+            entry["input_transform"] = input_transform_times(glq, torch, wp, Bp, hbm_peak, reps=reps)
         pre[f"B={Bp}"] = entry
     pre["peak"] = {"TFLOPs": tc_peak, "source": peak_src,
                    "note": "fp16 operands: measured cuBLAS bf16 peak (same nominal rate)"}
     del wp
     torch.cuda.empty_cache()
     return pre
+
+
+def input_transform_times(glq, torch, wp, Bp: int, hbm_peak: float, reps: int = 5) -> dict:
+    """The input transform of each prefill layer alone (glq_rht_input_operand),
+    the CUDA-core butterfly kernel (1) against the warp tensor-core kernel (2),
+    on row windows of the layer's activations that rotate through more than
+    L2 (the largest batch's rows).  Per layer, longest rows first: three
+    warm-up pairs (butterfly, tensor core) launched eagerly, then per kernel
+    a CUDA graph of `reps` launches, replayed three times between events.
+    Algorithmic bytes: B n (2 B in + 2 B out)."""
+    out = {}
+    for li in sorted(range(len(wp.host)), key=lambda i: -wp.host[i].n):
+        lay, x, _ = wp.layers[li][0]
+        L = wp.host[li]
+        nwin = max(1, x.shape[0] // Bp)
+        n_pad = (L.n + 127) // 128 * 128
+        xh = torch.empty((nwin * Bp, n_pad), dtype=torch.float16, device="cuda")
+        info = torch.empty((nwin * Bp, 4), dtype=torch.float32, device="cuda")
+
+        def launch(kern, w, stream):
+            glq.glq_rht_input_operand(lay.handle, x[w * Bp].data_ptr(), glq.dtype_code(x.dtype),
+                                      xh[w * Bp].data_ptr(), info[w * Bp].data_ptr(), Bp, kern,
+                                      stream.cuda_stream)
+        cur = torch.cuda.current_stream()
+        for w in range(3):
+            launch(1, w % nwin, cur)
+            launch(2, w % nwin, cur)
+        torch.cuda.synchronize()
+        alg = Bp * L.n * 4
+        entry = {"algorithmic_bytes": alg, "hbm_us": round(alg / (hbm_peak * 1e9) * 1e6, 2)}
+        for kern, name in ((1, "butterfly"), (2, "tensor_core")):
+            g = torch.cuda.CUDAGraph()
+            s = torch.cuda.Stream()
+            with torch.cuda.stream(s):
+                with torch.cuda.graph(g, stream=s):
+                    for r in range(reps):
+                        launch(kern, r % nwin, s)
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(3):
+                g.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / (3 * reps)
+            gbs = alg / (us * 1e-6) / 1e9
+            entry[name] = {"us": round(us, 2), "GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm_peak, 4)}
+            del g
+        out[f"n={L.n}"] = entry
+        del xh, info
+    return out
 
 
 def oracle_step_seconds(ws_host, xbits, x_bf16, threads: int = 1) -> float:
@@ -699,7 +753,7 @@ def run_glq(args):
             "24b-decode-6bpw": decode_config_section(glq, torch, "24b-decode-6bpw", hbm_peak, gemv_layer=2),
             "smollm3-3b-mixed": decode_config_section(glq, torch, "smollm3-3b-mixed", hbm_peak),
         }
-        result["prefill"] = prefill_section(glq, torch, tc_peak, peak_src)
+        result["prefill"] = prefill_section(glq, torch, tc_peak, peak_src, hbm_peak=hbm_peak)
         # the batches between the decode path and the 512-token tiles
         result["prefill_mid"] = prefill_section(glq, torch, tc_peak, peak_src, batches=(32, 64, 128), reps=20)
         result["dense_bf16_reference"] = dense_reference_section(glq, torch, hbm_peak, tc_peak)
@@ -769,10 +823,26 @@ def run_prefill_only(args):
     import torch
     import e8_lattice_codebook_b200 as glq
     torch.cuda.set_device(0)
-    _, tc_peak, _, peak_src = read_peaks()
+    hbm_peak, tc_peak, _, peak_src = read_peaks()
     batches = (args.prefill_batch,) if args.prefill_batch else (512, 2048, 8192)
     return {"section": "prefill", "prefill": prefill_section(glq, torch, tc_peak, peak_src, batches,
-                                                            reps=max(1, min(args.steps, 20)))}
+                                                            reps=max(1, min(args.steps, 20)),
+                                                            hbm_peak=hbm_peak)}
+
+
+def run_transforms_only(args):
+    """The prefill layers' input transforms alone, both kernels, one JSON
+    object (not the bench line; profiling runs: the launch order is that of
+    input_transform_times)."""
+    import torch
+    import e8_lattice_codebook_b200 as glq
+    torch.cuda.set_device(0)
+    hbm_peak = read_peaks()[0]
+    B = args.prefill_batch or 2048
+    wp = WorkloadSet(glq, torch, "prefill-8b-mlp-4bpw", 8192, ncopy=1)
+    return {"section": "transforms", "B": B,
+            "input_transform": input_transform_times(glq, torch, wp, B, hbm_peak,
+                                                     reps=max(1, min(args.steps, 50)))}
 
 
 def run_decode_only(args):
@@ -798,7 +868,7 @@ def main():
     ap.add_argument("--impl", choices=["glq", "reference"], default="glq")
     ap.add_argument("--quick", action="store_true", help="skip the 24B sweep and prefill")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle baseline")
-    ap.add_argument("--section", choices=["all", "prefill", "decode"], default="all",
+    ap.add_argument("--section", choices=["all", "prefill", "decode", "transforms"], default="all",
                     help="prefill / decode: time only that workload (profiling runs)")
     ap.add_argument("--workload", default="", help="with --section decode: the workload key")
     ap.add_argument("--prefill-batch", type=int, default=0,
@@ -810,6 +880,8 @@ def main():
         args.warmup = 3
     if args.section == "prefill":
         res = run_prefill_only(args)
+    elif args.section == "transforms":
+        res = run_transforms_only(args)
     elif args.section == "decode":
         res = run_decode_only(args)
     else:

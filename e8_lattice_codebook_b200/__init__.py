@@ -41,6 +41,7 @@ EXPORTS = (
     "glq_prefill_replay", "glq_layer_set_fusion", "glq_layer_set_prefill_reconstruct",
     "glq_workspace_info", "glq_workspace_release", "glq_layer_create_stages",
     "glq_layer_set_batch_invariant", "glq_layer_create_shard", "glq_cast",
+    "glq_rht_input_operand",
 )
 
 
@@ -73,6 +74,7 @@ _SIGNATURES = {
     "glq_dequant_reference": ([_vp, _vp, _vp], ctypes.c_int),
     "glq_rht_input": ([_vp, _vp, ctypes.c_int, _vp, _i64, _vp], ctypes.c_int),
     "glq_rht_output": ([_vp, _vp, _vp, ctypes.c_int, _i64, _vp], ctypes.c_int),
+    "glq_rht_input_operand": ([_vp, _vp, ctypes.c_int, _vp, _vp, _i64, ctypes.c_int, _vp], ctypes.c_int),
     "glq_layer_check": ([_vp, _vp], ctypes.c_int),
     "glq_gemv_replay": ([_vp, _i64, _vp], ctypes.c_int),
     "glq_prefill_replay": ([_vp, _i64, _vp], ctypes.c_int),
@@ -260,6 +262,11 @@ def glq_rht_output(handle, z_ptr, y_ptr, y_dtype, B, stream) -> None:
     _ok(_L().glq_rht_output(handle, z_ptr, y_ptr, y_dtype, B, stream), "glq_rht_output")
 
 
+def glq_rht_input_operand(handle, x_ptr, x_dtype, xh_ptr, info_ptr, B, kernel, stream) -> None:
+    _ok(_L().glq_rht_input_operand(handle, x_ptr, x_dtype, xh_ptr, info_ptr, B, kernel, stream),
+        "glq_rht_input_operand")
+
+
 def glq_gemv_replay(handle, B, stream) -> None:
     _ok(_L().glq_gemv_replay(handle, B, stream), "glq_gemv_replay")
 
@@ -408,6 +415,19 @@ class GlqLinear:
         glq_rht_input(self.handle, x.data_ptr(), dtype_code(x.dtype), xr.data_ptr(), x.shape[0],
                       _stream_ptr(stream))
         return xr
+
+    RHT_AUTO, RHT_BUTTERFLY, RHT_TENSOR = 0, 1, 2  # kernels of glq_rht_input_operand
+
+    def rht_input_operand(self, x, kernel=0, stream=None):
+        """(xh [B][n_pad] fp16 = xr 2^e per row, inv [B] fp32 = 2^-e): the
+        tensor-core path's input stage with the chosen kernel."""
+        torch = _torch()
+        n_pad = (self.n + 127) // 128 * 128
+        xh = torch.empty((x.shape[0], n_pad), dtype=torch.float16, device=x.device)
+        info = torch.empty((x.shape[0], 4), dtype=torch.float32, device=x.device)
+        glq_rht_input_operand(self.handle, x.data_ptr(), dtype_code(x.dtype), xh.data_ptr(), info.data_ptr(),
+                              x.shape[0], kernel, _stream_ptr(stream))
+        return xh, info[:, 2]
 
     def rht_output(self, z, out_dtype=None, stream=None):
         torch = _torch()

@@ -7,6 +7,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstddef>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -1255,6 +1256,44 @@ glq_status glq_rht_input(glq_layer L, const void *x_dev, glq_dtype x_dtype, floa
     p.xr_f32 = xr_dev;
     return glq::launch_rht_in(p, static_cast<cudaStream_t>(stream), false) == cudaSuccess ? GLQ_OK
                                                                                          : GLQ_ERR_CUDA;
+}
+
+// the row information the transform kernels write: word 2 of each 16-byte
+// record is 2^-e (the layout glq_rht_input_operand documents)
+static_assert(sizeof(glq_rowinfo) == 16 && offsetof(glq_rowinfo, inv_scale) == 8, "glq_rowinfo layout");
+
+glq_status glq_rht_input_operand(glq_layer L, const void *x_dev, glq_dtype x_dtype, void *xh_dev,
+                                 void *row_info_dev, int64_t B, int kernel, void *stream) {
+    if (!L) return GLQ_ERR_INVALID_ARG;
+    if (B < 0 || B > 65535) return GLQ_ERR_SHAPE;
+    if (x_dtype != GLQ_F16 && x_dtype != GLQ_BF16) return GLQ_ERR_DTYPE;
+    if (kernel < 0 || kernel > 2) return GLQ_ERR_INVALID_ARG;
+    if (B == 0) return GLQ_OK;
+    if (!x_dev || !xh_dev || !row_info_dev || (reinterpret_cast<uintptr_t>(x_dev) & 15u)) return GLQ_ERR_INVALID_ARG;
+    DeviceGuard guard(L->device);
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    glq::RowsParams r = rows_params(L->hb_n, (int)L->n, (int)L->n_pad, L->d_sin);
+    r.x = x_dev;
+    r.x_bf16 = x_dtype == GLQ_BF16 ? 1 : 0;
+    r.xh = static_cast<__half *>(xh_dev);
+    r.info = static_cast<glq_rowinfo *>(row_info_dev);
+    r.butterfly = kernel == 1 ? 1 : 0;
+    if (kernel == 2 && !glq::rht_in_mma_supported(r)) return GLQ_ERR_SHAPE;
+    if (glq::rht_rows_supported((int)L->n_pad))
+        return glq::launch_rht_rows(r, true, (int)B, s, false) == cudaSuccess ? GLQ_OK : GLQ_ERR_CUDA;
+    if (kernel != 0) return GLQ_ERR_SHAPE;
+    glq::RhtInParams pin{};
+    pin.x = x_dev;
+    pin.x_bf16 = r.x_bf16;
+    pin.n = (int)L->n;
+    pin.n_pad = (int)L->n_pad;
+    pin.B = (int)B;
+    pin.sign_bits = L->d_sin;
+    pin.plan = L->plan_n;
+    pin.xh = r.xh;
+    pin.info = r.info;
+    pin.xh_only = 1;
+    return glq::launch_rht_in(pin, s, false) == cudaSuccess ? GLQ_OK : GLQ_ERR_CUDA;
 }
 
 glq_status glq_rht_output(glq_layer L, const float *z_dev, void *y_dev, glq_dtype y_dtype, int64_t B,

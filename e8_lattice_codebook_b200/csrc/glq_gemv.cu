@@ -346,7 +346,7 @@ __device__ __forceinline__ void warp_transform(const GemvParams &p, int b, int N
     if (mx > 0.f && isfinite(mx)) {
         int ex;
         frexpf(mx, &ex);
-        scale = ldexpf(1.f, 14 - ex);
+        scale = ldexpf(1.f, min(14 - ex, 126));  // scale and 1 / scale normal for the tiniest rows
     }
     int sum = 0;
     uint32_t hb[V / 4], lb[V / 4];
@@ -505,7 +505,7 @@ __device__ void fused_input(const GemvParams &p, int k0, int klen, uint4 *xs, __
         if (rowmax > 0.f && isfinite(rowmax)) {
             int ex;
             frexpf(rowmax, &ex);
-            scale = ldexpf(1.f, 14 - ex);
+            scale = ldexpf(1.f, min(14 - ex, 126));  // scale and 1 / scale normal for the tiniest rows
         }
         const float *r = u + (size_t)b * klen + 8 * v;
         uint32_t hb[2] = {0u, 0u}, lb[2] = {0u, 0u};

@@ -52,6 +52,9 @@ struct RhtOutParams {
     RhtPlan plan;
     void *y;      // [B][m]
     int y_dtype;  // 0 f16, 1 bf16, 2 f32
+    // input side, fp16 operand: 0 the tensor-core kernel where it applies,
+    // 1 always the butterfly kernel
+    int butterfly;
 };
 
 // Row transforms of the tensor-core path (glq_rht_rows.cu): one CTA per row.
@@ -78,6 +81,9 @@ struct RowsParams {
     size_t zs;
     void *y;
     int y_dtype;  // 0 f16, 1 bf16, 2 f32
+    // input side, fp16 operand: 0 the tensor-core kernel where it applies,
+    // 1 always the butterfly kernel
+    int butterfly;
 };
 
 // Residual stages of a bit width ("Bit widths", glq 0.5.1 PyPI page): after
@@ -228,6 +234,10 @@ cudaError_t launch_rht_out(const RhtOutParams &p, cudaStream_t s, bool pdl);
 // row transforms for many rows (B up to 65535 per launch), len <= 16384
 bool rht_rows_supported(int len);
 cudaError_t launch_rht_rows(const RowsParams &p, bool input, int B, cudaStream_t s, bool pdl);
+// the input side on the warp tensor cores (fp16 operand of the tensor-core
+// GEMM; rows of 512 .. 16384 values, a multiple of 256, len == len_pad)
+bool rht_in_mma_supported(const RowsParams &p);
+cudaError_t launch_rht_in_mma(const RowsParams &p, int B, cudaStream_t s, bool pdl);
 cudaError_t launch_gemv(const GemvParams &p, int bpw, int grid, cudaStream_t s, bool pdl, bool fused_in = false);
 // dynamic shared memory of a launch with the input transform fused
 // (the table, the residual table, the task's activations and scratch)

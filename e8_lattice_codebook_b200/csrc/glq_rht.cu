@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(THREADS) rht_in_kernel(RhtInParams p) {
     if (rowmax > 0.f && isfinite(rowmax)) {
         int e;
         frexpf(rowmax, &e);  // rowmax < 2^e
-        scale = ldexpf(1.f, 14 - e);
+        scale = ldexpf(1.f, min(14 - e, 126));  // scale and 1 / scale normal for the tiniest rows
     }
     __half *xh = p.xh ? p.xh + (size_t)b * p.n_pad : nullptr;
     if (p.xh_only) {  // tensor-core path: fp16 activations, one rounding

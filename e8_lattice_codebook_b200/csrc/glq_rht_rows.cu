@@ -528,7 +528,7 @@ __global__ void __launch_bounds__(1 << (L - 4), L >= 14 ? (IN && !XQ ? 2 : 0) : 
             if (rowmax > 0.f && isfinite(rowmax)) {
                 int e;
                 frexpf(rowmax, &e);  // rowmax < 2^e
-                scale = ldexpf(1.f, 14 - e);
+                scale = ldexpf(1.f, min(14 - e, 126));  // scale and 1 / scale normal for the tiniest rows
             }
             const float f = norm * scale;  // scale is a power of two: one rounding, as xr 2^e
             int sum = 0;
@@ -584,7 +584,7 @@ __global__ void __launch_bounds__(1 << (L - 4), L >= 14 ? (IN && !XQ ? 2 : 0) : 
             if (rowmax > 0.f && isfinite(rowmax)) {
                 int e;
                 frexpf(rowmax, &e);  // rowmax < 2^e
-                scale = ldexpf(1.f, 14 - e);
+                scale = ldexpf(1.f, min(14 - e, 126));  // scale and 1 / scale normal for the tiniest rows
             }
             __half *xrow = p.xh + (size_t)b * p.len_pad;
 #pragma unroll
@@ -693,7 +693,9 @@ cudaError_t launch_rht_rows(const RowsParams &p, bool input, int B, cudaStream_t
             default: return cudaErrorInvalidValue;
         }
     }
-    return p.xq ? launch_rows_sel<true, true, 0>(p, B, s, pdl) : launch_rows_sel<true, false, 0>(p, B, s, pdl);
+    if (p.xq) return launch_rows_sel<true, true, 0>(p, B, s, pdl);
+    if (!p.butterfly && rht_in_mma_supported(p)) return launch_rht_in_mma(p, B, s, pdl);
+    return launch_rows_sel<true, false, 0>(p, B, s, pdl);
 }
 
 }  // namespace glq

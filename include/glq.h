@@ -344,6 +344,23 @@ GLQ_API glq_status glq_rht_output(glq_layer layer, const float *z_dev, void *y_d
                           int64_t B, void *stream);
 
 /*
+ * glq_rht_input_operand -- the input stage of the tensor-core (B > 16)
+ * path alone (GLQ v0.3.2 release notes, input_rht), as the fp16 operand
+ * the GEMM reads: xh_dev [B][n_pad] fp16 = xr_b 2^e_b, xr = H_n (S_in . x),
+ * padding columns zero; row_info_dev [B][4] 32-bit words, word 2 of row b =
+ * 2^-e_b as fp32 (the other words unspecified).  The power of two is chosen
+ * per row so that the fp16 values stay finite; which one is the kernel's
+ * choice.  kernel: 0 the kernel glq_linear runs for this layer; 1 the
+ * CUDA-core butterfly kernel (n_pad <= 16384); 2 the tensor-core kernel
+ * (512 <= n <= 16384, n a multiple of 256).  Device pointers; x_dev 16-byte
+ * aligned.  Errors: GLQ_ERR_INVALID_ARG, GLQ_ERR_DTYPE, GLQ_ERR_SHAPE (B >
+ * 65535, or a kernel that does not take this row length), GLQ_ERR_CUDA.
+ * Asynchronous.
+ */
+GLQ_API glq_status glq_rht_input_operand(glq_layer layer, const void *x_dev, glq_dtype x_dtype, void *xh_dev,
+                                         void *row_info_dev, int64_t B, int kernel, void *stream);
+
+/*
  * glq_gemv_replay -- measurement entry point: re-launches only the codebook
  * GEMV of the most recent glq_linear call on this layer (its activations
  * are read from the device's shared workspace, so no other layer's call may

@@ -7,8 +7,10 @@ cores, so it keeps the same bound as the decode path:
 max |y - y_oracle| <= 2e-3 (||y_oracle||_inf + 1).
 
 * small shapes: every token of batches that span one and several 512-token
-  tiles, with ragged row, column and token tails, all three bit rates, and
-  rows longer than the one-CTA-per-row transform takes (16384);
+  tiles, with ragged row, column and token tails, all three bit rates, rows
+  longer than the one-CTA-per-row transforms take (16384), and input rows of
+  every size the tensor-core transform takes (2^10 .. 2^14 positions, one
+  to five Hadamard blocks);
 * full-size prefill workload at its largest batch: sampled tokens, the last
   (ragged) token tile included;
 * run-to-run determinism, and per-token independence of the batch size
@@ -49,6 +51,12 @@ PREFILL_SMALL = [  # m, n, bpw, B, x dtype
     (1024, 1024, 2, 1100, "bf16"),  # three token tiles
     (64, 20480, 2, 33, "f16"),      # input rows above 16384: clustered transform kernel
     (20480, 64, 3, 20, "bf16"),     # output rows above 16384: clustered transform kernel
+    # input rows a multiple of 256: the tensor-core transform kernel
+    (48, 768, 2, 40, "bf16"),       # 2^10 positions, two Hadamard blocks
+    (40, 3840, 4, 33, "f16"),       # 2^12, four blocks
+    (24, 7936, 3, 50, "bf16"),      # 2^13 (one cross-tile bit), five blocks
+    (16, 12288, 2, 20, "f16"),      # 2^14 (two cross-tile bits), two blocks
+    (16, 16384, 4, 19, "bf16"),     # 2^14, one block
 ]
 
 

@@ -28,6 +28,7 @@ CSRC = os.path.join(ROOT, "e8_lattice_codebook_b200", "csrc")
 
 HARNESS = r"""
 #include "glq_rht_rows.cu"
+#include "glq_rht_mma.cu"  // the input side's tensor-core kernel, which glq_rht_rows.cu dispatches to
 #include <cstdio>
 #include <vector>
 
