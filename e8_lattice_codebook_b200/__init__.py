@@ -41,7 +41,7 @@ EXPORTS = (
     "glq_prefill_replay", "glq_layer_set_fusion", "glq_layer_set_prefill_reconstruct",
     "glq_workspace_info", "glq_workspace_release", "glq_layer_create_stages",
     "glq_layer_set_batch_invariant", "glq_layer_create_shard", "glq_cast",
-    "glq_rht_input_operand",
+    "glq_rht_input_operand", "glq_layer_selftest_wait",
 )
 
 
@@ -75,6 +75,7 @@ _SIGNATURES = {
     "glq_rht_input": ([_vp, _vp, ctypes.c_int, _vp, _i64, _vp], ctypes.c_int),
     "glq_rht_output": ([_vp, _vp, _vp, ctypes.c_int, _i64, _vp], ctypes.c_int),
     "glq_rht_input_operand": ([_vp, _vp, ctypes.c_int, _vp, _vp, _i64, ctypes.c_int, _vp], ctypes.c_int),
+    "glq_layer_selftest_wait": ([_vp, ctypes.c_int, ctypes.c_int, _i64, _vp], ctypes.c_int),
     "glq_layer_check": ([_vp, _vp], ctypes.c_int),
     "glq_gemv_replay": ([_vp, _i64, _vp], ctypes.c_int),
     "glq_prefill_replay": ([_vp, _i64, _vp], ctypes.c_int),
@@ -267,6 +268,10 @@ def glq_rht_input_operand(handle, x_ptr, x_dtype, xh_ptr, info_ptr, B, kernel, s
         "glq_rht_input_operand")
 
 
+def glq_layer_selftest_wait(handle, kind, arrivals, limit, stream) -> None:
+    _ok(_L().glq_layer_selftest_wait(handle, kind, arrivals, limit, stream), "glq_layer_selftest_wait")
+
+
 def glq_gemv_replay(handle, B, stream) -> None:
     _ok(_L().glq_gemv_replay(handle, B, stream), "glq_gemv_replay")
 
@@ -428,6 +433,12 @@ class GlqLinear:
         glq_rht_input_operand(self.handle, x.data_ptr(), dtype_code(x.dtype), xh.data_ptr(), info.data_ptr(),
                               x.shape[0], kernel, _stream_ptr(stream))
         return xh, info[:, 2]
+
+    def selftest_wait(self, kind: int, arrivals: int, limit: int, stream=None):
+        """One bounded device wait on a barrier `arrivals` of its two arrivals
+        reach (kind 0: cycle-bounded, 1: cluster scope, 2: poll-bounded);
+        the outcome reads back through check()."""
+        glq_layer_selftest_wait(self.handle, kind, arrivals, limit, _stream_ptr(stream))
 
     def rht_output(self, z, out_dtype=None, stream=None):
         torch = _torch()

@@ -1365,6 +1365,16 @@ glq_status glq_prefill_replay(glq_layer L, int64_t B, void *stream) {
                : GLQ_ERR_CUDA;
 }
 
+glq_status glq_layer_selftest_wait(glq_layer L, int kind, int arrivals, int64_t limit, void *stream) {
+    if (!L || kind < 0 || kind > 2 || arrivals < 1 || arrivals > 2 || limit <= 0) return GLQ_ERR_INVALID_ARG;
+    if (kind == 2 && limit > (int64_t)0xFFFFFFFFll) return GLQ_ERR_INVALID_ARG;
+    DeviceGuard guard(L->device);
+    return glq::launch_wait_selftest(L->d_err, kind, arrivals, (unsigned long long)limit,
+                                     static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? GLQ_OK
+               : GLQ_ERR_CUDA;
+}
+
 glq_status glq_layer_check(glq_layer L, void *stream) {
     if (!L) return GLQ_ERR_INVALID_ARG;
     DeviceGuard guard(L->device);

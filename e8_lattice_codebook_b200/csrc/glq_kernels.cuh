@@ -238,6 +238,10 @@ cudaError_t launch_rht_rows(const RowsParams &p, bool input, int B, cudaStream_t
 // GEMM; rows of 512 .. 16384 values, a multiple of 256, len == len_pad)
 bool rht_in_mma_supported(const RowsParams &p);
 cudaError_t launch_rht_in_mma(const RowsParams &p, int B, cudaStream_t s, bool pdl);
+// one bounded wait of kind (0 cycle-bounded, 1 its cluster-scope form, 2
+// poll-bounded) on a barrier `arrivals` of its two arrivals reach; a timeout
+// sets GLQ_DEVERR_TIMEOUT in *err
+cudaError_t launch_wait_selftest(unsigned *err, int kind, int arrivals, unsigned long long limit, cudaStream_t s);
 cudaError_t launch_gemv(const GemvParams &p, int bpw, int grid, cudaStream_t s, bool pdl, bool fused_in = false);
 // dynamic shared memory of a launch with the input transform fused
 // (the table, the residual table, the task's activations and scratch)

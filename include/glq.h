@@ -361,6 +361,22 @@ GLQ_API glq_status glq_rht_input_operand(glq_layer layer, const void *x_dev, glq
                                          void *row_info_dev, int64_t B, int kernel, void *stream);
 
 /*
+ * glq_layer_selftest_wait -- testing entry point for failure detection: runs
+ * one of the bounded device waits the layer's kernels use, on a barrier that
+ * only `arrivals` of its two expected arrivals reach (1: it never completes;
+ * 2: it completes at once), with the given limit; a wait that runs out
+ * reports a timeout through the layer's device error word, as the kernels
+ * do, without faulting or hanging the GPU.  kind: 0 the cycle-bounded wait of
+ * the tensor-core pipeline (limit in SM clock cycles), 1 its cluster-scope
+ * form (same unit), 2 the poll-bounded wait of the codebook-table loads
+ * (limit in polls, < 2^32).  Read the outcome with glq_layer_check
+ * (GLQ_ERR_TIMEOUT after a timeout, which also clears the word).
+ * Errors: GLQ_ERR_INVALID_ARG (kind, arrivals or limit out of range),
+ * GLQ_ERR_CUDA.  Asynchronous.
+ */
+GLQ_API glq_status glq_layer_selftest_wait(glq_layer layer, int kind, int arrivals, int64_t limit, void *stream);
+
+/*
  * glq_gemv_replay -- measurement entry point: re-launches only the codebook
  * GEMV of the most recent glq_linear call on this layer (its activations
  * are read from the device's shared workspace, so no other layer's call may
