@@ -313,6 +313,18 @@ glq::PrefillParams prefill_params(glq_layer L, const glq_prefill_ws &ws, int64_t
     pp.tiles_tok = (int)((B + glq::prefill_tile_tokens() - 1) / glq::prefill_tile_tokens());
     pp.ksplit = choose_ksplit(L, B, tiles_m * pp.tiles_tok);
     pp.ntiles = tiles_m * pp.tiles_tok * pp.ksplit;
+    pp.tiles_whole = pp.ntiles;
+    // A last partial wave of whole tiles (one per CTA pair) runs as half
+    // tiles of 256 tokens, twice as many items taking half the time: when it
+    // has at most half a wave of tiles, and every tile has two live halves
+    // (the last token tile holds more than 256 tokens).
+    const int pairs = std::max(1, L->num_sms / 2), tt = glq::prefill_tile_tokens();
+    const int rest = pp.ntiles % pairs;
+    if (pp.ksplit == 1 && pp.ntiles > pairs && rest > 0 && 2 * rest <= pairs &&
+        (B % tt == 0 || B % tt > tt / 2)) {
+        pp.tiles_whole = pp.ntiles - rest;
+        pp.ntiles = pp.tiles_whole + 2 * rest;
+    }
     pp.zs = (size_t)B * L->m_pad;
     pp.err = L->d_err;
     pp.table = L->primary->d_table;

@@ -165,7 +165,8 @@ struct PrefillParams {
     size_t zs;               // floats between slices
     int ksplit;              // K splits (chunk-aligned), >= 1
     int B, m_pad, KC, RT;
-    int tiles_tok, ntiles;   // ntiles = row tiles x token tiles x ksplit
+    int tiles_tok, ntiles;   // ntiles: work items (row tiles x token tiles x ksplit, halves counted twice)
+    int tiles_whole;         // items [0, tiles_whole) are whole tiles, the rest halves of the tiles after them
     unsigned *err;
 };
 

@@ -7,7 +7,8 @@
 // Design (B200, sm_100a): persistent clusters of two CTAs (one per SM)
 // share each tcgen05 MMA (cta_group::2, M = 256 = 128 rows per CTA,
 // N = 256 tokens = 128 per CTA, K = 16), over output tiles of 256 weight rows
-// x 512 tokens (two TMEM accumulators of 256 columns in each CTA), with a
+// x 512 tokens (two TMEM accumulators of 256 columns in each CTA; the tiles
+// of a last partial wave as two half tiles of 256 tokens each), with a
 // four-stage ring of 64-column steps (48 KB per CTA: its 128 rows of W and
 // its 2 x 128 tokens of x):
 //   * warp 0 of each CTA loads its half of the activations with TMA (128
@@ -117,13 +118,24 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
         abort_flag = 1;
     };
     auto live_acc = [&](int tok0) { return min(NACC, (p.B - tok0 + BN - 1) / BN); };
-    // tile -> (weight-row tile, token tile, K split) and its 64-column steps
-    // [kb0, kb1) (splits on 128-column chunk boundaries)
-    auto geom = [&](int tile, int &rtile, int &ttile, int &ks, int &kb0, int &kb1) {
+    // work item -> (weight-row tile, first token, live accumulators, K split)
+    // and its 64-column steps [kb0, kb1) (splits on 128-column chunk
+    // boundaries).  Items below tiles_whole are whole tiles; the rest are the
+    // halves (256 tokens, one accumulator) of the tiles that follow, so that
+    // a last partial wave of whole tiles takes half a tile's time.
+    auto geom = [&](int item, int &rtile, int &tok0, int &na, int &ks, int &kb0, int &kb1) {
+        int tile = item, half = -1;
+        if (item >= p.tiles_whole) {
+            const int u = item - p.tiles_whole;
+            tile = p.tiles_whole + (u >> 1);
+            half = u & 1;
+        }
         ks = tile % p.ksplit;
         const int rest = tile / p.ksplit;
         rtile = rest / p.tiles_tok;
-        ttile = rest - rtile * p.tiles_tok;
+        const int ttile = rest - rtile * p.tiles_tok;
+        tok0 = ttile * (BN * NACC) + (half > 0 ? BN : 0);
+        na = half < 0 ? live_acc(tok0) : min(1, live_acc(tok0));
         kb0 = 2 * ((ks * p.KC) / p.ksplit);
         kb1 = 2 * (((ks + 1) * p.KC) / p.ksplit);
     };
@@ -135,10 +147,8 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
             uint32_t it = 0;
             int32_t last_load = -1;
             for (int tile = (int)cid; tile < p.ntiles && !abort_flag; tile += (int)ncl) {
-                int rtile, ttile, ks, kb0, kb1;
-                geom(tile, rtile, ttile, ks, kb0, kb1);
-                const int tok0 = ttile * (BN * NACC);
-                const int na = live_acc(tok0);
+                int rtile, tok0, na, ks, kb0, kb1;
+                geom(tile, rtile, tok0, na, ks, kb0, kb1);
                 int halves = 0;  // live halves of both CTAs (a half past the last token is not loaded)
                 for (int a = 0; a < na; ++a)
                     for (int r = 0; r < 2; ++r) halves += tok0 + a * BN + r * BNH < p.B;
@@ -173,9 +183,8 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
             const uint32_t idesc = sm100::idesc_f16_f32(2 * BM, BN);
             uint32_t it = 0, acc_use[NACC] = {0, 0};
             for (int tile = (int)cid; tile < p.ntiles && !abort_flag; tile += (int)ncl) {
-                int rtile, ttile, ks, kb0, kb1;
-                geom(tile, rtile, ttile, ks, kb0, kb1);
-                const int na = live_acc(ttile * (BN * NACC));
+                int rtile, tok0, na, ks, kb0, kb1;
+                geom(tile, rtile, tok0, na, ks, kb0, kb1);
                 for (int kb = kb0; kb < kb1 && !abort_flag; ++kb, ++it) {
                     const uint32_t s = it % STAGES, use = it / STAGES;
                     if (!sm100::mbar_wait_cluster(&x_full[s], use & 1, WAIT_CYCLES) ||
@@ -220,8 +229,8 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
         const int g = lane >> 2, t = lane & 3;
         uint32_t it = 0;
         for (int tile = (int)cid; tile < p.ntiles && !abort_flag; tile += (int)ncl) {
-            int rtile, ttile, ks, kb0, kb1;
-            geom(tile, rtile, ttile, ks, kb0, kb1);
+            int rtile, tok0, na, ks, kb0, kb1;
+            geom(tile, rtile, tok0, na, ks, kb0, kb1);
             const int rt = (rtile * 2 + (int)rank) * (BM / GLQ_ROW_TILE) + rt_l;
             const bool live = rt < p.RT;
             const size_t slot0 = (size_t)rt * p.KC * 32 + lane;
@@ -299,11 +308,10 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
         const int a = ew >> 2;             // the accumulator this warp drains
         uint32_t use = 0;
         for (int tile = (int)cid; tile < p.ntiles && !abort_flag; tile += (int)ncl) {
-            int rtile, ttile, ks, kb0, kb1;
-            geom(tile, rtile, ttile, ks, kb0, kb1);
+            int rtile, tok0, na, ks, kb0, kb1;
+            geom(tile, rtile, tok0, na, ks, kb0, kb1);
             float *zk = p.z + (size_t)ks * p.zs;  // this split's partial sums
-            const int tok0 = ttile * (BN * NACC);
-            if (a >= live_acc(tok0)) continue;
+            if (a >= na) continue;
             const int tb = tok0 + a * BN;
             const int row = (rtile * 2 + (int)rank) * BM + 32 * q + lane;
             if (abort_flag || !sm100::mbar_wait_cluster(&acc_full[a], use & 1, WAIT_CYCLES)) {

@@ -57,6 +57,9 @@ PREFILL_SMALL = [  # m, n, bpw, B, x dtype
     (24, 7936, 3, 50, "bf16"),      # 2^13 (one cross-tile bit), five blocks
     (16, 12288, 2, 20, "f16"),      # 2^14 (two cross-tile bits), two blocks
     (16, 16384, 4, 19, "bf16"),     # 2^14, one block
+    # 75 row tiles: one more than a wave of the 74 CTA pairs, so the last
+    # tile runs as two half tiles (256 tokens each; the second one ragged)
+    (19200, 128, 4, 300, "bf16"),
 ]
 
 
@@ -148,4 +151,29 @@ def test_producer_back_to_back_calls_do_not_stall(dev):
         assert time.time() - t0 < 1.0, B
         ref = oracle_y(L, xb[[0, B - 1]], wl.x_dtype)
         assert np.max(np.abs(y.cpu().numpy().astype(np.float64)[[0, B - 1]] - ref)) <= tolerance(ref)
+    lay.set_prefill_reconstruct(-1)
+
+
+def test_half_tiles_keep_results_bitwise(dev):
+    """A last partial wave of whole tiles runs as half tiles (one accumulator
+    of 256 tokens each): the same K order, so a token's result does not
+    depend on whether its tile was halved.  19200 rows are 75 row tiles:
+    at 512 tokens the 75th tile is the partial wave and runs halved; at 600
+    tokens (150 tiles, a ragged second token tile of 88 tokens) nothing is
+    halved."""
+    m, n, bpw = 19200, 256, 2
+    L = gi.make_layer(41, 2, m, n, bpw)
+    lay = dev.layer(L)
+    xb = gi.make_x(41, 2, 600, n, "bf16")
+    x = to_torch_x(xb, "bf16")
+    for mode in sorted(MODES):
+        lay.set_prefill_reconstruct(MODES[mode])
+        y600 = lay(x, out_dtype=torch.float32)
+        y512 = lay(x[:512].contiguous(), out_dtype=torch.float32)
+        assert torch.equal(y512, y600[:512]), mode
+        sample = [0, 255, 256, 511]
+        ref = oracle_y(L, xb[sample], "bf16")
+        err = np.max(np.abs(y512.cpu().numpy().astype(np.float64)[sample] - ref))
+        assert err <= tolerance(ref), (mode, err)
+        lay.check()
     lay.set_prefill_reconstruct(-1)
