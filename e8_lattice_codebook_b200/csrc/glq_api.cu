@@ -481,13 +481,18 @@ DecodeCfg decode_config(glq_layer L, int nb, const void *x, const void *y, int y
             gemv_fused_smem_bytes(L->primary->table_words, L->bpw, nb, std::min(fp.cps, L->KC) * GLQ_CHUNK_K);
         // Measured: the fold pays for the launch it saves when every CTA has
         // one task and a short range (<= 1024 columns, <= 4096 values in
-        // all); a 4096-column range per CTA is slower than the separate
-        // transform kernel.  An explicit setting always fuses.  (Narrower
-        // CTAs of 16 or 20 warps that fill more SMs made the 3B-shaped step
-        // slower, 74 -> 82 us: no SM was left for the next kernel's early
-        // launch.)
+        // all), and the row is long enough (n_pad > 8192) that the separate
+        // transform is a slow one-CTA row; for shorter rows the separate
+        // transform, launched early behind the previous kernel, costs less
+        // (steps back to back: 24B-class 153.7 -> 149.8 us, SmolLM3-3B-shaped
+        // 77.3 -> 75.0 us, SmolLM2-360M-shaped at two tokens 60.7 -> 54.1 us).
+        // A 4096-column range per CTA is slower than the separate transform
+        // kernel.  An explicit setting always fuses.  (Narrower CTAs of 16 or
+        // 20 warps that fill more SMs made the 3B-shaped step slower, 74 -> 82
+        // us: no SM was left for the next kernel's early launch.)
         const int klen = std::min(fp.cps, L->KC) * GLQ_CHUNK_K;
-        const bool cheap = (long long)fp.bands * fp.splits <= L->num_sms && klen <= 1024 && nb * klen <= 4096;
+        const bool cheap = (long long)fp.bands * fp.splits <= L->num_sms && klen <= 1024 && nb * klen <= 4096 &&
+                           L->n_pad > 8192;
         if (need <= GEMV_SMEM_LIMIT && (cheap || L->fusion >= 0)) {
             c.fin = true;
             c.plan = fp;
