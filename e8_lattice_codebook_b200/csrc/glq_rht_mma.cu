@@ -18,7 +18,7 @@
 //     consecutive positions), and its fp32 result, rounded to fp16, is
 //     already the A operand of the product over bits 0-3 (no data movement);
 //   * rows of 2^13 and 2^14 positions add one or two fp32 butterflies
-//     between the 2 or 4 tiles a warp holds (position bits 8, 9);
+//     between the 4 tiles a warp holds (position bits 8, 9);
 //   * the tile is stored (stmatrix) into a row buffer and read back
 //     (ldmatrix.trans) along the remaining (up to four) position bits, whose
 //     Hadamard is one more product pair with the data as the B operand;
@@ -27,18 +27,19 @@
 //     position bits into the bank-group bits, chosen so that each 8-lane
 //     phase of every ldmatrix / stmatrix and of the copies meets 8 distinct
 //     bank groups;
-//   * the matrices carry +-2^-k (exact in fp16 and bf16); the block norm's
-//     remaining factor (1, 1/sqrt2 or sqrt2 for an odd count of bits) is one
-//     fp32 multiply before the rounding to fp16;
+//   * the matrices carry +-2^-k (exact in fp16 and bf16); what the block
+//     norm still needs (a power of sqrt2: the cross butterflies are
+//     unnormalised, a product over an odd count of active bits carries
+//     2^-ceil(a/2)) is an fp32 multiply before the next rounding to fp16;
 //   * the prescale 2^e comes from the row's max |x| (max |x| 2^e in
 //     [2^7, 2^8)), so that every intermediate, bounded by ||x||_2 2^e <=
 //     2^7 max |x| 2^e, stays below 2^15; the first product runs on the raw
 //     16-bit inputs (bf16 or fp16 kind), with the scale inside its matrix
 //     for bf16 (2^(e-2), so that its fp32 result cannot overflow) and
 //     applied to its fp32 result for fp16;
-//   * intermediates are rounded to fp16 after the first and second products
-//     (the fp32 butterflies and the last product are rounded once, at the
-//     end): three roundings instead of the butterfly kernel's one;
+//   * values are rounded to fp16 three times (after the first product,
+//     after the second product and the cross butterflies, and after the
+//     last product) instead of the butterfly kernel's once;
 //   * a persistent CTA of up to 16 warps works on three rows at once as a
 //     software pipeline (stage A of one row, stage B of the previous one, the
 //     copy-out of the one before: independent work between two barriers,
