@@ -267,8 +267,10 @@ def test_cluster_splitk_matches_global_reduction(dev, m, n, bpw, B, xdt):
 
 def test_decode_plans_of_the_workloads(dev):
     """The decode plans of the SmolLM3-3B-shaped and 24B-class layers at 1 and
-    16 tokens are consistent (a cluster, when used, holds a band's splits)
-    and the cluster reduction is in use on some of them.  At 16 tokens the
+    16 tokens are consistent (a cluster, when used, holds a band's splits),
+    the cluster reduction is in use on some of them, and at one token the
+    3B-shaped layers fuse the input transform exactly when the row is
+    longer than 8192.  At 16 tokens the
     32768-row gate / up layers (128 bands of 16-warp CTAs on 148 SMs) take one
     split: charged too little for the global reduction of two token tiles,
     the planner chose 8 splits over 7 waves there, 1.6x slower per step."""
@@ -284,6 +286,11 @@ def test_decode_plans_of_the_workloads(dev):
                 clustered += plan["cluster"] > 0
                 if B == 16 and L.m == 32768 and torch.cuda.get_device_properties(0).multi_processor_count == 148:
                     assert plan["splits"] == 1, (key, li, plan)
+                if B == 1 and key == "smollm3-3b-4bpw":
+                    # the input transform is fused only for rows longer than
+                    # 8192 (down: 11008 columns); shorter rows run it as its
+                    # own kernel, launched early behind the previous one
+                    assert plan["fused_input"] == (1 if L.n > 8192 else 0), (key, li, plan)
                 print(f"\nPLAN {key} layer {li} B={B}: {plan}")
     assert clustered > 0
 
