@@ -24,7 +24,9 @@
 //     CTAs' barriers;
 //   * warps 10-13 and 14-17 drain accumulators 0 and 1 with tcgen05.ld as
 //     soon as the tile's last MMA completes and store z = acc ws 2^-e (fp32);
-//     each accumulator is released on its own.
+//     each accumulator is released on its own.  Items of one accumulator
+//     (half tiles) alternate between the two, so that one is drained while
+//     the next item's MMAs fill the other.
 // Every wait is bounded (4e9 SM clock cycles, about 2 s); a timeout sets the
 // layer's error flag, lets in-flight TMA loads and MMAs land, frees TMEM and
 // returns.
@@ -118,6 +120,11 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
         abort_flag = 1;
     };
     auto live_acc = [&](int tok0) { return min(NACC, (p.B - tok0 + BN - 1) / BN); };
+    // The first accumulator of an item: an item with one live accumulator (a
+    // half tile, or a tile whose second 256 tokens are past the batch) takes
+    // the two in turn, counted by the CTA's earlier such items, so its MMAs
+    // run while the epilogue drains the previous one; a whole tile uses both.
+    auto acc_first = [](int na, uint32_t singles) { return na == 1 ? (int)(singles & 1u) : 0; };
     // work item -> (weight-row tile, first token, live accumulators, K split)
     // and its 64-column steps [kb0, kb1) (splits on 128-column chunk
     // boundaries).  Items below tiles_whole are whole tiles; the rest are the
@@ -181,10 +188,11 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
         if (lane == 0 && rank == 0) {
             // ---------------- MMA issuer of the pair ----------------
             const uint32_t idesc = sm100::idesc_f16_f32(2 * BM, BN);
-            uint32_t it = 0, acc_use[NACC] = {0, 0};
+            uint32_t it = 0, acc_use[NACC] = {0, 0}, singles = 0;
             for (int tile = (int)cid; tile < p.ntiles && !abort_flag; tile += (int)ncl) {
                 int rtile, tok0, na, ks, kb0, kb1;
                 geom(tile, rtile, tok0, na, ks, kb0, kb1);
+                const int abase = acc_first(na, singles);
                 for (int kb = kb0; kb < kb1 && !abort_flag; ++kb, ++it) {
                     const uint32_t s = it % STAGES, use = it / STAGES;
                     if (!sm100::mbar_wait_cluster(&x_full[s], use & 1, WAIT_CYCLES) ||
@@ -195,9 +203,10 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
                     sm100::tc_fence_after();
                     uint8_t *st = smem + s * STAGE_BYTES;
                     const uint64_t adesc = sm100::smem_desc_sw128(st);
-                    for (int a = 0; a < na; ++a) {
+                    for (int a = 0; a < na; ++a) {  // x slot a of the stage into accumulator abase + a
+                        const int ac = abase + a;
                         if (kb == kb0) {  // both CTAs' epilogues must have drained this accumulator
-                            if (!sm100::mbar_wait_cluster(&acc_empty[a], (acc_use[a] & 1) ^ 1, WAIT_CYCLES)) {
+                            if (!sm100::mbar_wait_cluster(&acc_empty[ac], (acc_use[ac] & 1) ^ 1, WAIT_CYCLES)) {
                                 fail();
                                 break;
                             }
@@ -206,13 +215,14 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
                         const uint64_t bdesc = sm100::smem_desc_sw128(st + W_BYTES + a * X_BYTES);
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk)
-                            sm100::mma2_f16_ss(tmem_base + a * BN, adesc + 2 * kk, bdesc + 2 * kk, idesc,
+                            sm100::mma2_f16_ss(tmem_base + ac * BN, adesc + 2 * kk, bdesc + 2 * kk, idesc,
                                                (kb != kb0) || (kk != 0));
-                        if (kb == kb1 - 1) sm100::mma2_commit_both(&acc_full[a]);
+                        if (kb == kb1 - 1) sm100::mma2_commit_both(&acc_full[ac]);
                     }
                     sm100::mma2_commit_both(&empty_bar[s]);
                 }
-                for (int a = 0; a < na; ++a) ++acc_use[a];
+                for (int a = 0; a < na; ++a) ++acc_use[abase + a];
+                singles += na == 1;
             }
             sm100::mma2_commit_both(&mma_done);  // every MMA of the pair has completed
             sm100::mbar_wait(&mma_done, 0, WAIT_CYCLES);
@@ -306,13 +316,15 @@ __global__ void __launch_bounds__(threads_of(MAT), 1) prefill_kernel(const __gri
         const int ew = warp - EPI_WARP0;   // 0..7
         const int q = warp & 3;            // TMEM lane quadrant this warp may access
         const int a = ew >> 2;             // the accumulator this warp drains
-        uint32_t use = 0;
+        uint32_t use = 0, singles = 0;
         for (int tile = (int)cid; tile < p.ntiles && !abort_flag; tile += (int)ncl) {
             int rtile, tok0, na, ks, kb0, kb1;
             geom(tile, rtile, tok0, na, ks, kb0, kb1);
             float *zk = p.z + (size_t)ks * p.zs;  // this split's partial sums
-            if (a >= na) continue;
-            const int tb = tok0 + a * BN;
+            const int abase = acc_first(na, singles);
+            singles += na == 1;
+            if (a < abase || a >= abase + na) continue;  // accumulator a is idle in this item
+            const int tb = tok0 + (a - abase) * BN;
             const int row = (rtile * 2 + (int)rank) * BM + 32 * q + lane;
             if (abort_flag || !sm100::mbar_wait_cluster(&acc_full[a], use & 1, WAIT_CYCLES)) {
                 if (!abort_flag) fail();

@@ -177,3 +177,29 @@ def test_half_tiles_keep_results_bitwise(dev):
         assert err <= tolerance(ref), (mode, err)
         lay.check()
     lay.set_prefill_reconstruct(-1)
+
+
+def test_single_accumulator_items_alternate_bitwise(dev):
+    """Items with one live accumulator (a batch of at most 256 tokens, or the
+    ragged 88 tokens of a second token tile) take a CTA pair's two TMEM
+    accumulators in turn, so that one drains while the next item computes.
+    38400 rows are 150 row tiles, two or three items per pair: at 200
+    tokens every item has one accumulator (the pair's items alternate 0, 1,
+    0); at 600 tokens whole tiles (both accumulators) and single ones mix.
+    A token's result does not depend on which accumulator held it."""
+    m, n, bpw = 38400, 256, 2
+    L = gi.make_layer(43, 2, m, n, bpw)
+    lay = dev.layer(L)
+    xb = gi.make_x(43, 2, 600, n, "f16")
+    x = to_torch_x(xb, "f16")
+    for mode in sorted(MODES):
+        lay.set_prefill_reconstruct(MODES[mode])
+        y600 = lay(x, out_dtype=torch.float32)
+        y200 = lay(x[:200].contiguous(), out_dtype=torch.float32)
+        assert torch.equal(y200, y600[:200]), mode
+        sample = [0, 199, 511, 512, 599]
+        ref = oracle_y(L, xb[sample], "f16")
+        err = np.max(np.abs(y600.cpu().numpy().astype(np.float64)[sample] - ref))
+        assert err <= tolerance(ref), (mode, err)
+        lay.check()
+    lay.set_prefill_reconstruct(-1)
