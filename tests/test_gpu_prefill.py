@@ -183,11 +183,12 @@ def test_single_accumulator_items_alternate_bitwise(dev):
     """Items with one live accumulator (a batch of at most 256 tokens, or the
     ragged 88 tokens of a second token tile) take a CTA pair's two TMEM
     accumulators in turn, so that one drains while the next item computes.
-    38400 rows are 150 row tiles, two or three items per pair: at 200
-    tokens every item has one accumulator (the pair's items alternate 0, 1,
-    0); at 600 tokens whole tiles (both accumulators) and single ones mix.
-    A token's result does not depend on which accumulator held it."""
-    m, n, bpw = 38400, 256, 2
+    19200 rows are 75 row tiles for 74 CTA pairs: at 200 tokens every item
+    has one accumulator and the first pair takes two of them (accumulators 0
+    then 1); at 600 tokens (150 items) whole tiles, which use both, and
+    single ones (the ragged second token tile) mix, two or three items per
+    pair.  A token's result does not depend on which accumulator held it."""
+    m, n, bpw = 19200, 256, 2
     L = gi.make_layer(43, 2, m, n, bpw)
     lay = dev.layer(L)
     xb = gi.make_x(43, 2, 600, n, "f16")
