@@ -18,7 +18,7 @@
 //     consecutive positions), and its fp32 result, rounded to fp16, is
 //     already the A operand of the product over bits 0-3 (no data movement);
 //   * rows of 2^13 and 2^14 positions add one or two fp32 butterflies
-//     between the 4 tiles a warp holds (position bits 8, 9);
+//     between the tiles a warp holds (4 or 8; position bits 8, 9);
 //   * the tile is stored (stmatrix) into a row buffer and read back
 //     (ldmatrix.trans) along the remaining (up to four) position bits, whose
 //     Hadamard is one more product pair with the data as the B operand;
@@ -40,13 +40,13 @@
 //   * values are rounded to fp16 three times (after the first product,
 //     after the second product and the cross butterflies, and after the
 //     last product) instead of the butterfly kernel's once;
-//   * a persistent CTA of up to 16 warps works on three rows at once as a
+//   * a persistent CTA of up to 8 warps works on three rows at once as a
 //     software pipeline (stage A of one row, stage B of the previous one, the
 //     copy-out of the one before: independent work between two barriers,
 //     with row and output buffers alternating by row parity), one CTA
 //     barrier per row; the next rows' raw inputs stream into a ring of three
-//     staging buffers (16-byte asynchronous copies); below 2^14 positions
-//     CTAs of at most 8 warps, two or more per SM.
+//     staging buffers (16-byte asynchronous copies); one CTA per SM at 2^14
+//     positions (224 KB of buffers), two or more below.
 #include <algorithm>
 
 #include "glq_kernels.cuh"
@@ -63,14 +63,16 @@ namespace {
 //   stage B: the remaining bits 8 + C .. L - 1 (1 to 4 of them) as the k bits
 //            of one product, filled up to four with already transformed bits
 //            7, 6, 5, 4 (identity there);
-//   warps:   2^(L-8) / T, each taking T tiles per stage: 4 from L = 13 (16
-//            warps, one CTA per SM at L = 14; 8 warps, two CTAs per SM at
-//            L = 13), else 2 (2^(L-9) warps, two or more CTAs per SM).
-//            Measured at L = 14: 32 warps of 2 tiles (the cross bits split
-//            between the stages) executed 1.5x the instructions.
+//   warps:   2^(L-8) / T, each taking T tiles per stage: 8 at L = 14 (8
+//            warps, one CTA per SM, up to 255 registers a thread), 4 at
+//            L = 13 (8 warps, two CTAs per SM), else 2 (2^(L-9) warps, two
+//            or more CTAs per SM).  Measured at L = 14 (B200, 512 - 8192
+//            rows of 14336): 16 warps of 4 tiles took about 10 % longer than
+//            8 warps of 8, and 32 warps of 2 tiles (the cross bits split
+//            between the stages) executed 1.5x the instructions of 16 of 4.
 // ---------------------------------------------------------------------------
 __host__ __device__ constexpr int mma_cross(int L) { return L > 12 ? L - 12 : 0; }
-__host__ __device__ constexpr int mma_tpw(int L) { return L >= 13 ? 4 : 2; }
+__host__ __device__ constexpr int mma_tpw(int L) { return L >= 14 ? 8 : (L >= 13 ? 4 : 2); }
 __host__ __device__ constexpr int mma_warps(int L) { return (1 << (L - 8)) / mma_tpw(L); }
 // CTAs per SM the launch bounds ask for (registers): one 16-warp CTA at
 // 2^14 positions, else at least two
@@ -140,6 +142,16 @@ __host__ __device__ constexpr uint32_t slot_o(int L, uint32_t p) {
 // Hadamard block of a row of len (blocks: aligned powers of two, descending)
 __host__ __device__ constexpr bool bfly_active(uint32_t p, int b, uint32_t len) {
     return p < len && ((p ^ len) >> (b + 1)) != 0u;
+}
+
+// S_in of a warp's stage-A fragments, one bit per 16-bit value: register q
+// of the warp's tile i at bit 4 (i & 3) + q (low half) or 16 + 4 (i & 3) + q
+// (high half) of word i >> 2; sign_xor gives the mask that flips register q
+// of tile i (the fp16 / bf16 sign bits 15 and 31)
+__host__ __device__ constexpr int mma_sign_words(int L) { return (mma_tpw(L) + 3) / 4; }
+__host__ __device__ constexpr int sign_bit_of(int i, int q, int h) { return 16 * h + 4 * (i & 3) + q; }
+__host__ __device__ constexpr uint32_t sign_xor(uint32_t w, int i, int q) {
+    return (w << (15 - (4 * (i & 3) + q))) & 0x80008000u;
 }
 
 // ---------------------------------------------------------------------------
@@ -302,13 +314,13 @@ __device__ __forceinline__ void sts128_zero(uint32_t addr) {
 //   rb_i, ob_i: row-buffer / output slot of the warp's stage-B tile i.
 template <int L>
 struct MmaTables {
-    uint32_t s_k[4], o_k[4], ra_i[4], rb_i[4], ob_i[4];
+    uint32_t s_k[8], o_k[8], ra_i[8], rb_i[8], ob_i[8];
 };
 template <int L>
 __host__ __device__ constexpr MmaTables<L> mma_tables() {
     MmaTables<L> t{};
     constexpr int T = 32 * mma_warps(L);
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < mma_tpw(L); ++k) {
         t.s_k[k] = slot_s((uint32_t)(k * T) << 3);
         t.o_k[k] = slot_o(L, (uint32_t)(k * T) << 3);
         t.ra_i[k] = slot_r(L, (uint32_t)k << 8);
@@ -410,9 +422,8 @@ __global__ void __launch_bounds__(32 * mma_warps(L), mma_min_ctas(L)) rht_in_mma
     const uint32_t lRb = slot_r(L, offB), lOb = slot_o(L, offB);
     // (tile i of the warp: its slots are the warp's first tile's XOR a
     // constant, the swizzles being linear and the tile bits disjoint)
-    // S_in of the warp's stage-A fragments, one bit per 16-bit value: word q
-    // of tile i at bit 4 i + q (low half) and 16 + 4 i + q (high half)
-    uint32_t sgn = 0u;
+    // S_in of the warp's stage-A fragments (sign_bit_of)
+    uint32_t sgn[mma_sign_words(L)] = {};
     float fA[TPW];
 #pragma unroll
     for (int i = 0; i < TPW; ++i) {
@@ -422,7 +433,7 @@ __global__ void __launch_bounds__(32 * mma_warps(L), mma_min_ctas(L)) rht_in_mma
             const uint32_t lo = frag_pos(base, lane, q, 0), hi = frag_pos(base, lane, q, 1);
             const uint32_t slo = lo < len ? (p.sign_bits[lo >> 5] >> (lo & 31)) & 1u : 0u;
             const uint32_t shi = hi < len ? (p.sign_bits[hi >> 5] >> (hi & 31)) & 1u : 0u;
-            sgn |= slo << (4 * i + q) | shi << (16 + 4 * i + q);
+            sgn[i >> 2] |= slo << sign_bit_of(i, q, 0) | shi << sign_bit_of(i, q, 1);
         }
         fA[i] = cross_norm<L>(base, len);
     }
@@ -559,8 +570,7 @@ __global__ void __launch_bounds__(32 * mma_warps(L), mma_min_ctas(L)) rht_in_mma
             for (int i = 0; i < TPW; ++i) {
                 uint32_t r[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q)  // S_in: XOR of the sign bits
-                    r[q] = rn[q] ^ ((sgn << (15 - (4 * i + q))) & 0x80008000u);
+                for (int q = 0; q < 4; ++q) r[q] = rn[q] ^ sign_xor(sgn[i >> 2], i, q);  // S_in
                 if (i + 1 < TPW && real(i + 1))
                     ldsm_x4_trans(Sb + ((uint32_t)(warp * TPW + i + 1) << 9) + lS, rn);
                 if (real(i)) {

@@ -258,15 +258,28 @@ static void check(int len, unsigned seed) {
             Pair r[32][4];
             long pos[32][4][2];
             ldsm_trans(S, Sp, addr, r, pos, "stage A load");
-            for (int l = 0; l < 32; ++l)
+            for (int l = 0; l < 32; ++l) {
+                // the lane's sign words over all the warp's tiles, packed and
+                // read back as the kernel does (sign_bit_of, sign_xor)
+                uint32_t sgn[mma_sign_words(L)] = {};
+                for (int i2 = 0; i2 < TPW; ++i2)
+                    for (int q = 0; q < 4; ++q)
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t p2 = frag_pos((uint32_t)(w * TPW + i2) << 8, l, q, h);
+                            if (p2 < (uint32_t)len && (sign_bits[p2 >> 5] >> (p2 & 31) & 1))
+                                sgn[i2 >> 2] |= 1u << sign_bit_of(i2, q, h);
+                        }
                 for (int q = 0; q < 4; ++q)
                     for (int h = 0; h < 2; ++h) {
                         const uint32_t fp = frag_pos(base, l, q, h);
                         CHECK((long)fp == pos[l][q][h], "L=%d: sign mask position %u, loaded %ld", L, fp, pos[l][q][h]);
-                        const bool neg = fp < (uint32_t)len && (sign_bits[fp >> 5] >> (fp & 31) & 1);
+                        const bool neg = (sign_xor(sgn[i >> 2], i, q) >> (15 + 16 * h)) & 1u;
+                        const bool want = fp < (uint32_t)len && (sign_bits[fp >> 5] >> (fp & 31) & 1);
+                        CHECK(neg == want, "L=%d: sign of position %u from the packed words", L, fp);
                         double &v = h ? r[l][q].hi : r[l][q].lo;
                         if (neg) v = -v;
                     }
+            }
             uint32_t a1w[32][4];
             for (int l = 0; l < 32; ++l) a_frag(l, Had16{0x3E80u}, a1w[l]);  // bf16 0.25
             double A1[16][16];
