@@ -18,7 +18,7 @@
 //     consecutive positions), and its fp32 result, rounded to fp16, is
 //     already the A operand of the product over bits 0-3 (no data movement);
 //   * rows of 2^13 and 2^14 positions add one or two fp32 butterflies
-//     between the tiles a warp holds (4 or 8; position bits 8, 9);
+//     between the 4 tiles a warp holds (position bits 8, 9);
 //   * the tile is stored (stmatrix) into a row buffer and read back
 //     (ldmatrix.trans) along the remaining (up to four) position bits, whose
 //     Hadamard is one more product pair with the data as the B operand;
@@ -40,13 +40,13 @@
 //   * values are rounded to fp16 three times (after the first product,
 //     after the second product and the cross butterflies, and after the
 //     last product) instead of the butterfly kernel's once;
-//   * a persistent CTA of up to 8 warps works on three rows at once as a
+//   * a persistent CTA of up to 16 warps works on three rows at once as a
 //     software pipeline (stage A of one row, stage B of the previous one, the
 //     copy-out of the one before: independent work between two barriers,
 //     with row and output buffers alternating by row parity), one CTA
 //     barrier per row; the next rows' raw inputs stream into a ring of three
-//     staging buffers (16-byte asynchronous copies); one CTA per SM at 2^14
-//     positions (224 KB of buffers), two or more below.
+//     staging buffers (16-byte asynchronous copies); below 2^14 positions
+//     CTAs of at most 8 warps, two or more per SM.
 #include <algorithm>
 
 #include "glq_kernels.cuh"
@@ -63,16 +63,17 @@ namespace {
 //   stage B: the remaining bits 8 + C .. L - 1 (1 to 4 of them) as the k bits
 //            of one product, filled up to four with already transformed bits
 //            7, 6, 5, 4 (identity there);
-//   warps:   2^(L-8) / T, each taking T tiles per stage: 8 at L = 14 (8
-//            warps, one CTA per SM, up to 255 registers a thread), 4 at
-//            L = 13 (8 warps, two CTAs per SM), else 2 (2^(L-9) warps, two
-//            or more CTAs per SM).  Measured at L = 14 (B200, 512 - 8192
-//            rows of 14336): 16 warps of 4 tiles took about 10 % longer than
-//            8 warps of 8, and 32 warps of 2 tiles (the cross bits split
-//            between the stages) executed 1.5x the instructions of 16 of 4.
+//   warps:   2^(L-8) / T, each taking T tiles per stage: 4 from L = 13 (16
+//            warps, one CTA per SM at L = 14; 8 warps, two CTAs per SM at
+//            L = 13), else 2 (2^(L-9) warps, two or more CTAs per SM).
+//            Measured at L = 14 (B200, 2048 rows of 14336): 32 warps of 2
+//            tiles (the cross bits split between the stages) executed 1.5x
+//            the instructions; 8 warps of 8 tiles (241 registers) executed
+//            26 % fewer but, with 8 warps on the SM, issued in 41 % of the
+//            cycles instead of 59 % and took longer (44.4 against 42.8 us).
 // ---------------------------------------------------------------------------
 __host__ __device__ constexpr int mma_cross(int L) { return L > 12 ? L - 12 : 0; }
-__host__ __device__ constexpr int mma_tpw(int L) { return L >= 14 ? 8 : (L >= 13 ? 4 : 2); }
+__host__ __device__ constexpr int mma_tpw(int L) { return L >= 13 ? 4 : 2; }
 __host__ __device__ constexpr int mma_warps(int L) { return (1 << (L - 8)) / mma_tpw(L); }
 // CTAs per SM the launch bounds ask for (registers): one 16-warp CTA at
 // 2^14 positions, else at least two
