@@ -315,7 +315,7 @@ __device__ __forceinline__ void sts128_zero(uint32_t addr) {
 //   rb_i, ob_i: row-buffer / output slot of the warp's stage-B tile i.
 template <int L>
 struct MmaTables {
-    uint32_t s_k[8], o_k[8], ra_i[8], rb_i[8], ob_i[8];
+    uint32_t s_k[mma_tpw(L)], o_k[mma_tpw(L)], ra_i[mma_tpw(L)], rb_i[mma_tpw(L)], ob_i[mma_tpw(L)];
 };
 template <int L>
 __host__ __device__ constexpr MmaTables<L> mma_tables() {
