@@ -677,13 +677,18 @@ def run_glq(args):
     ms_k = gemv_kernel_time(torch, ws, li, reps=400)
     achieved = gemv_bytes(L.m, L.n, L.bpw, B) / (ms_k * 1e-3) / 1e9
     plan = ws.layers[li][0][0].decode_plan(B)
+    sha = gemv_source_sha256()
+    traffic = PROFILED_GEMV_TRAFFIC.get(sha)
+    prof = "profiles/gemv_24b-gate-32768x5120_4bpw_b1.md"
     result["roofline"] = {
         "kernel": (f"gemv_kernel<4,1,{plan['fused_input']},{plan['warps']}> gate {L.m}x{L.n} B=1 "
                    f"({plan['bands']} bands x {plan['splits']} splits)"),
         "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
         "frac": round(achieved / hbm_peak, 4), "peak_source": f"{peak_src} hbm_gbs (burst)",
-        "traffic": PROFILED_GEMV_TRAFFIC.get(gemv_source_sha256()),
-        "traffic_source": "profiles/gemv_24b-gate-32768x5120_4bpw_b1.md (null: kernel changed since)",
+        "traffic": traffic,
+        "traffic_source": (f"{prof}: ncu capture of this kernel source (glq_gemv.cu sha256 {sha[:12]}...)"
+                           if traffic is not None else
+                           f"null: glq_gemv.cu changed since the capture in {prof}"),
         "kernel_us": round(ms_k * 1e3, 3),
         "algorithmic_bytes": gemv_bytes(L.m, L.n, L.bpw, B),
     }
