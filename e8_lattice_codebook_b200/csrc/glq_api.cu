@@ -186,12 +186,9 @@ void invariant_need(glq_layer L, int64_t B, WsNeed &n) {
     n.b[WS_Z] = std::max(n.b[WS_Z], (size_t)B * L->m_pad * sizeof(float));
 }
 
-int choose_ksplit(glq_layer L, int64_t B, int tiles);
-int prefill_tiles(glq_layer L, int64_t B);
-
 // Tensor-core buffers for one call of exactly B (> 16) tokens on layer L.
 void prefill_need(glq_layer L, int64_t B, WsNeed &n) {
-    const int ks = choose_ksplit(L, B, prefill_tiles(L, B));
+    const int ks = glq::plan_prefill(L->m_pad, L->KC, B, L->num_sms).ksplit;
     n.b[WS_PXH] = std::max(n.b[WS_PXH], (size_t)B * L->n_pad * sizeof(__half));
     n.b[WS_PINFO] = std::max(n.b[WS_PINFO], (size_t)B * sizeof(glq_rowinfo));
     n.b[WS_PZ] = std::max(n.b[WS_PZ], (size_t)ks * B * L->m_pad * sizeof(float));
@@ -258,35 +255,6 @@ bool encode_w_map(CUtensorMap *map, const __half *w16, int64_t n_pad, int64_t m_
     return encode_x_map(map, w16, n_pad, m_pad, n_pad);
 }
 
-// K splits of the tensor-core GEMM: fill the CTA pairs when the output has
-// too few tiles, unless the extra partial-sum traffic costs more than it
-// saves.  Model (B200 measurements): a pair retires a tile's rows x tokens x
-// n x 2 FLOP at about 15 TFLOP/s; each extra split writes and reads B x m_pad
-// fp32 at about 6 TB/s.
-int choose_ksplit(glq_layer L, int64_t B, int tiles) {
-    const int pairs = std::max(1, L->num_sms / 2);
-    const double t_tile = (double)glq::prefill_tile_rows() * (double)glq::prefill_tile_tokens() *
-                          (double)stream_cols(L) * 2.0 / 15e12;
-    const double t_traffic = (double)B * (double)L->m_pad * 8.0 / 6e12;
-    int best = 1;
-    double best_t = 1e30;
-    for (int S = 1; S <= 8 && S <= L->KC / 4 + (S == 1); ++S) {
-        const double waves = std::ceil((double)tiles * S / pairs);
-        const double t = waves * t_tile / S + (S - 1) * t_traffic;
-        if (t < best_t * 0.97) {  // a split must pay for itself clearly
-            best_t = t;
-            best = S;
-        }
-    }
-    return best;
-}
-
-int prefill_tiles(glq_layer L, int64_t B) {
-    const int tr = glq::prefill_tile_rows();
-    const int tiles_m = (int)((L->m_pad + tr - 1) / tr);
-    return tiles_m * (int)((B + glq::prefill_tile_tokens() - 1) / glq::prefill_tile_tokens());
-}
-
 glq::PrefillParams prefill_params(glq_layer L, const glq_prefill_ws &ws, int64_t B) {
     glq::PrefillParams pp{};
     pp.idx1 = L->d_idx1;
@@ -308,23 +276,11 @@ glq::PrefillParams prefill_params(glq_layer L, const glq_prefill_ws &ws, int64_t
     pp.m_pad = (int)L->m_pad;
     pp.KC = L->KC;
     pp.RT = L->RT;
-    const int tr = glq::prefill_tile_rows();
-    const int tiles_m = (int)((L->m_pad + tr - 1) / tr);
-    pp.tiles_tok = (int)((B + glq::prefill_tile_tokens() - 1) / glq::prefill_tile_tokens());
-    pp.ksplit = choose_ksplit(L, B, tiles_m * pp.tiles_tok);
-    pp.ntiles = tiles_m * pp.tiles_tok * pp.ksplit;
-    pp.tiles_whole = pp.ntiles;
-    // A last partial wave of whole tiles (one per CTA pair) runs as half
-    // tiles of 256 tokens, twice as many items taking half the time: when it
-    // has at most half a wave of tiles, and every tile has two live halves
-    // (the last token tile holds more than 256 tokens).
-    const int pairs = std::max(1, L->num_sms / 2), tt = glq::prefill_tile_tokens();
-    const int rest = pp.ntiles % pairs;
-    if (pp.ksplit == 1 && pp.ntiles > pairs && rest > 0 && 2 * rest <= pairs &&
-        (B % tt == 0 || B % tt > tt / 2)) {
-        pp.tiles_whole = pp.ntiles - rest;
-        pp.ntiles = pp.tiles_whole + 2 * rest;
-    }
+    const glq::PrefillSplit ps = glq::plan_prefill(L->m_pad, L->KC, B, L->num_sms);
+    pp.tiles_tok = ps.tiles_tok;
+    pp.ksplit = ps.ksplit;
+    pp.ntiles = ps.ntiles;
+    pp.tiles_whole = ps.tiles_whole;
     pp.zs = (size_t)B * L->m_pad;
     pp.err = L->d_err;
     pp.table = L->primary->d_table;

@@ -286,6 +286,18 @@ size_t prefill_smem_bytes();
 int prefill_tile_tokens();  // tokens of one output tile (a multiple of the TMA box height)
 int prefill_tile_rows();    // weight rows of one output tile (one CTA pair)
 
+// Work split of the tensor-core GEMM of an m_pad x (KC chunks of 128
+// columns) layer over B tokens on num_sms SMs (host only): the K splits
+// (chunk-aligned, chosen from a cost model of CTA-pair waves against the
+// extra partial-sum traffic) and the work items; items [0, tiles_whole)
+// are whole tiles, the rest halves (256 tokens) of the tiles after them,
+// for a last partial wave of at most half the CTA pairs whose tiles all
+// have two live halves.
+struct PrefillSplit {
+    int ksplit, tiles_tok, ntiles, tiles_whole;
+};
+PrefillSplit plan_prefill(int64_t m_pad, int KC, int64_t B, int num_sms);
+
 // warps per GEMV CTA (one 16-row tile each): 24 for one 8-column MMA tile
 // (B <= 8), 16 for two (B <= 16, more live registers per lane); from 5 bpw
 // every residual stage adds its accumulators and code registers per lane,

@@ -30,6 +30,8 @@
 // Every wait is bounded (4e9 SM clock cycles, about 2 s); a timeout sets the
 // layer's error flag, lets in-flight TMA loads and MMAs land, frees TMEM and
 // returns.
+#include <cmath>
+
 #include "glq_kernels.cuh"
 #include "glq_sm100.cuh"
 
@@ -370,6 +372,44 @@ size_t prefill_smem_bytes() { return 1024 + (size_t)STAGES * STAGE_BYTES; }
 int prefill_tile_tokens() { return BN * NACC; }
 
 int prefill_tile_rows() { return 2 * BM; }
+
+PrefillSplit plan_prefill(int64_t m_pad, int KC, int64_t B, int num_sms) {
+    PrefillSplit ps{};
+    const int tr = prefill_tile_rows(), tt = prefill_tile_tokens();
+    const int pairs = num_sms / 2 > 1 ? num_sms / 2 : 1;
+    const int tiles_m = (int)((m_pad + tr - 1) / tr);
+    ps.tiles_tok = (int)((B + tt - 1) / tt);
+    const int tiles = tiles_m * ps.tiles_tok;
+    // K splits: fill the CTA pairs when the output has too few tiles, unless
+    // the extra partial-sum traffic costs more than it saves.  Model (B200
+    // measurements): a pair retires a tile's rows x tokens x K x 2 FLOP at
+    // about 15 TFLOP/s; each extra split writes and reads B x m_pad fp32 at
+    // about 6 TB/s.
+    const double t_tile = (double)tr * (double)tt * (double)KC * GLQ_CHUNK_K * 2.0 / 15e12;
+    const double t_traffic = (double)B * (double)m_pad * 8.0 / 6e12;
+    ps.ksplit = 1;
+    double best_t = 1e30;
+    for (int S = 1; S <= 8 && S <= KC / 4 + (S == 1); ++S) {
+        const double waves = std::ceil((double)tiles * S / pairs);
+        const double t = waves * t_tile / S + (S - 1) * t_traffic;
+        if (t < best_t * 0.97) {  // a split must pay for itself clearly
+            best_t = t;
+            ps.ksplit = S;
+        }
+    }
+    ps.ntiles = tiles * ps.ksplit;
+    ps.tiles_whole = ps.ntiles;
+    // A last partial wave of whole tiles (one per CTA pair) runs as half
+    // tiles of 256 tokens, twice as many items taking half the time: when it
+    // has at most half a wave of tiles, and every tile has two live halves
+    // (the last token tile holds more than 256 tokens).
+    const int rest = ps.ntiles % pairs;
+    if (ps.ksplit == 1 && ps.ntiles > pairs && rest > 0 && 2 * rest <= pairs && (B % tt == 0 || B % tt > tt / 2)) {
+        ps.tiles_whole = ps.ntiles - rest;
+        ps.ntiles = ps.tiles_whole + 2 * rest;
+    }
+    return ps;
+}
 
 cudaError_t launch_prefill(const PrefillParams &p, const CUtensorMap &xmap, const CUtensorMap *wmap, int grid,
                            cudaStream_t s, bool pdl) {
