@@ -238,11 +238,12 @@ GLQ_API glq_status glq_workspace_release(int32_t device);
  * y_dev: device [B][m] row-major, dtype y_dtype (== x_dtype, or GLQ_F32),
  *   16-byte aligned.
  * B >= 0 (B == 0 is a no-op).  stream: cudaStream_t.
- * Paths: B <= 16 runs the decode path: the codebook GEMV on the legacy warp
- *   MMA with an on-chip codebook, with both transforms fused into the same
- *   launch when B times the largest Hadamard block is at most 32768 values
- *   (one kernel per call), else input RHT, GEMV and output RHT as three
- *   kernels (see glq_layer_set_fusion); B > 16 runs the tensor-core path:
+ * Paths: B <= 16 runs the decode path: input RHT, the codebook GEMV on the
+ *   legacy warp MMA with an on-chip codebook, and output RHT, launched back
+ *   to back with programmatic dependent launch; by default the input RHT is
+ *   folded into the GEMV launch where that measured faster (see
+ *   glq_layer_set_fusion, which also sets either fusion explicitly); B > 16
+ *   runs the tensor-core path:
  *   input RHT, one pass that reconstructs W = cb1 + rs cb2 as an fp16 matrix
  *   in the device's shared workspace, a TMA-fed tcgen05/TMEM GEMM on it
  *   (or, when glq_layer_set_prefill_reconstruct raises the bound above B, a
@@ -264,11 +265,14 @@ GLQ_API glq_status glq_linear(glq_layer layer, const void *x_dev, glq_dtype x_dt
  * glq_layer_set_fusion -- choose how decode calls (B <= 16) run their two
  * transforms.  flags is a bit set: GLQ_FUSE_INPUT fuses the input RHT into
  * the GEMV launch (each task rotates its own aligned column range of x)
- * whenever B times the largest Hadamard block of n is at most 32768 values;
- * GLQ_FUSE_OUTPUT lets the last band of each Hadamard block of m rotate that
+ * whenever B times the largest Hadamard block of n is at most 32768 values
+ * and the tasks' activations fit shared memory; GLQ_FUSE_OUTPUT lets the last band of each Hadamard block of m rotate that
  * block in the same launch when B times the largest block of m fits the
  * library's bound; a cleared bit runs that transform as its own kernel.  The
- * default is the library's fastest setting (GLQ_FUSE_DEFAULT).  With both bits
+ * default (GLQ_FUSE_DEFAULT) is the setting measured fastest on B200: cluster
+ * split-K on, the output RHT as its own kernel, and the input RHT fused only
+ * for rows longer than 8192 whose tasks are short (one task per CTA, at most
+ * 1024 columns and 4096 values of x per task).  With both bits
  * cleared, every token's output is bitwise independent of the batch size for
  * B <= 16; otherwise that holds among batch sizes that take the same path.
  * GLQ_SPLITK_CLUSTER lets the split-K partial sums of a band of rows be
